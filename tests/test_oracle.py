@@ -1,0 +1,323 @@
+"""Pins for the float64 oracle (CPU only).
+
+The oracle is the plain sequential recurrence.  These tests tie it to things other than
+itself: the pages' worked water-tank example (tests/golden/water_tank.txt), the
+attention-like quadratic (semiseparable-matrix) form, brute-force products of decays, the
+convolution form of a time-invariant SSM, the pages' diagonal-SSM recurrent = convolution
+setting, closed forms of special cases, and associativity (split/resume).  The last test
+compiles deliberately broken variants of the oracle and checks that every one of them
+fails at least one pin.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import forms
+import ssd_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "water_tank.txt")
+
+
+def _golden():
+    levels, residue, below = {}, None, None
+    limit = None
+    for line in open(GOLDEN):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        parts = line.split()
+        if parts[0] == "inf":
+            limit = float(parts[1])
+        elif parts[0] == "residue":
+            residue = (int(parts[1]), float(parts[2]))
+        elif parts[0] == "residue_below":
+            below = (int(parts[1]), float(parts[2]))
+        else:
+            levels[int(parts[0])] = float(parts[1])
+    return levels, limit, residue, below
+
+
+def _tank(x, mutation=0):
+    L = len(x)
+    xs = np.asarray(x, dtype=np.float32).reshape(1, L, 1, 1)
+    dt = np.ones((1, L, 1), dtype=np.float32)
+    A = np.array([-math.log(2.0)], dtype=np.float32)
+    one = np.ones((1, L, 1, 1), dtype=np.float32)
+    D = np.zeros(1, dtype=np.float32)
+    y, _ = oracle.scan(xs, dt, A, one, one, D, mutation=mutation)
+    return y.reshape(L)
+
+
+def _rand_case(seed, Bt=2, L=37, H=4, P=3, N=5, G=2, with_init=True, io="f32"):
+    cfg = dict(batch=Bt, seqlen=L, nheads=H, headdim=P, dstate=N, ngroups=G, chunk=16,
+               io=io, init="normal0.1" if with_init else "zeros")
+    inp = ssd_inputs.make_scan_inputs(cfg, seed=seed)
+    return inp
+
+
+def _check_water_tank(mutation=0):
+    levels, limit, residue, below = _golden()
+    n = max(levels) + 1
+    y = _tank([0.0] + [2.0] * (n - 1), mutation)
+    # float32 A = -ln 2 is not exactly -ln 2; the decay differs from 1/2 by ~1e-8 relative
+    for t, v in levels.items():
+        assert abs(y[t] - v) <= 1e-6 * max(1.0, abs(v)), (t, y[t], v)
+    y64 = _tank([0.0] + [2.0] * 63, mutation)
+    assert abs(y64[-1] - limit) <= 1e-6
+    imp = _tank([1.0] + [0.0] * 40, mutation)
+    lag, frac = residue
+    assert abs(imp[lag] - frac) <= 1e-8
+    lag, bound = below
+    assert 0.0 < imp[lag] < bound
+
+
+def test_water_tank_golden():
+    _check_water_tank()
+
+
+def test_water_tank_two_ways():
+    """The page's second route: sum the inflows, each faded by its age (2+1+0.5+0.25+0.125)."""
+    x = np.array([0.0, 2, 2, 2, 2, 2], dtype=np.float32).reshape(6, 1, 1)
+    y = forms.lti_convolution(x, np.ones(1, np.float32),
+                              np.array([-math.log(2.0)], np.float32),
+                              np.ones((1, 1), np.float32), np.ones((1, 1), np.float32))
+    assert abs(y[5, 0, 0] - (2 + 1 + 0.5 + 0.25 + 0.125)) < 1e-6
+    assert np.allclose(_tank(x.reshape(-1)), y.reshape(-1), atol=1e-12)
+
+
+@pytest.mark.parametrize("seed,shape", [
+    (1, dict()),
+    (2, dict(Bt=1, L=256, H=4, P=16, N=16, G=1, with_init=False)),   # the tiny workload's shape
+    (3, dict(Bt=1, L=64, H=6, P=2, N=8, G=3)),
+    (4, dict(Bt=2, L=50, H=4, P=2, N=4, G=4)),                       # one group per head
+    (5, dict(Bt=1, L=33, H=2, P=4, N=3, G=1, io="bf16")),
+])
+def test_quadratic_form(seed, shape):
+    inp = _rand_case(seed, **shape)
+    y, hf = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                        init=None if inp["init"] is None else inp["init"].astype(np.float64))
+    yq, hq = forms.quadratic(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                             init=inp["init"])
+    scale = np.sqrt(np.mean(yq ** 2))
+    assert np.max(np.abs(y - yq)) <= 1e-11 * scale
+    assert np.max(np.abs(hf - hq)) <= 1e-11 * max(1.0, np.sqrt(np.mean(hq ** 2)))
+
+
+def test_brute_force():
+    inp = _rand_case(7, Bt=1, L=20, H=3, P=2, N=4, G=1)
+    y, _ = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                       init=inp["init"])
+    yb = forms.brute_force(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                           init=inp["init"])
+    assert np.max(np.abs(y - yb)) <= 1e-12 * np.sqrt(np.mean(yb ** 2))
+
+
+def test_lti_convolution():
+    rng = np.random.default_rng(11)
+    L, H, P, N, G = 96, 4, 3, 8, 2
+    x = rng.standard_normal((L, H, P)).astype(np.float32)
+    dtc = rng.uniform(0.05, 0.3, H).astype(np.float32)
+    A = -rng.uniform(1, 8, H).astype(np.float32)
+    Bc = rng.standard_normal((G, N)).astype(np.float32)
+    Cc = rng.standard_normal((G, N)).astype(np.float32)
+    D = rng.standard_normal(H).astype(np.float32)
+    dt = np.broadcast_to(dtc, (1, L, H)).copy()
+    Bm = np.broadcast_to(Bc, (1, L, G, N)).copy()
+    Cm = np.broadcast_to(Cc, (1, L, G, N)).copy()
+    y, _ = oracle.scan(x[None], dt, A, Bm, Cm, D)
+    yc = forms.lti_convolution(x, dtc, A, Bc, Cc, D)
+    assert np.max(np.abs(y[0] - yc)) <= 1e-11 * np.sqrt(np.mean(yc ** 2))
+
+
+def test_diagonal_ssm_page_setting():
+    """A diagonal SSM (one decay per state, zero-order-hold input matrix) on one channel is
+    the sum of scalar-decay heads; recurrent and convolutional outputs agree (the page
+    states agreement to 1e-5; float64 gives far better).  Sizes follow the page: L=64,
+    16 states, step 0.1, A = -(U + 0.5); our own draws."""
+    rng = np.random.default_rng(2024)
+    L, Ns, delta = 64, 16, 0.1
+    x = rng.standard_normal(L)
+    Ad = -(rng.uniform(0, 1, Ns) + 0.5)
+    Bd = rng.standard_normal(Ns)
+    Cd = rng.standard_normal(Ns)
+    Abar = np.exp(delta * Ad)
+    Bbar = (Abar - 1.0) / Ad * Bd
+    y_conv = forms.diag_ssm_convolution(x, Bbar, Cd, Abar)
+    # as H=16 heads, P=1, N=1, G=H: B_in * dt must equal Bbar, so B_in = Bbar / dt
+    H = Ns
+    xs32 = np.broadcast_to(x[:, None], (L, H)).reshape(1, L, H, 1).astype(np.float32)
+    dt = np.full((1, L, H), delta, dtype=np.float32)
+    A32 = Ad.astype(np.float32)
+    Bin = np.broadcast_to((Bbar / np.float32(delta)).astype(np.float32), (1, L, H)).reshape(
+        1, L, H, 1).copy()
+    Cin = np.broadcast_to(Cd.astype(np.float32), (1, L, H)).reshape(1, L, H, 1).copy()
+    y, _ = oracle.scan(xs32, dt, A32, Bin, Cin, np.zeros(H, np.float32))
+    y_rec = y[0, :, :, 0].sum(axis=1)
+    # the kernel form on exactly the float32-rounded parameters the oracle read
+    dt64 = dt[0, 0].astype(np.float64)
+    Abar32 = np.exp(dt64 * A32.astype(np.float64))
+    Bbar32 = Bin[0, 0, :, 0].astype(np.float64) * dt64
+    y_conv32 = forms.diag_ssm_convolution(xs32[0, :, 0, 0], Bbar32,
+                                          Cin[0, 0, :, 0].astype(np.float64), Abar32)
+    assert np.allclose(y_rec, y_conv32, atol=1e-12, rtol=0)
+    assert np.allclose(y_rec, y_conv, atol=1e-5, rtol=0)  # the page's tolerance
+
+
+def test_resume_split_equals_one_shot():
+    inp = _rand_case(21, Bt=2, L=90, H=4, P=3, N=6, G=2)
+    args = (inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"])
+    y, hf = oracle.scan(inp["x"], *args, init=inp["init"])
+    for L1 in (1, 37, 89):
+        ya, ha = oracle.scan(inp["x"][:, :L1], inp["dt"][:, :L1], inp["A"], inp["B"][:, :L1],
+                             inp["C"][:, :L1], inp["D"], init=inp["init"])
+        yb, hb = oracle.scan(inp["x"][:, L1:], inp["dt"][:, L1:], inp["A"], inp["B"][:, L1:],
+                             inp["C"][:, L1:], inp["D"], init=ha)
+        assert np.allclose(np.concatenate([ya, yb], axis=1), y, rtol=0, atol=1e-13)
+        assert np.allclose(hb, hf, rtol=0, atol=1e-13)
+
+
+def test_step_equals_scan():
+    inp = _rand_case(22, Bt=2, L=12, H=4, P=3, N=5, G=2)
+    y, hf = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                        init=inp["init"])
+    st = inp["init"].astype(np.float64)
+    for t in range(12):
+        yt, st = oracle.step(st, inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["B"][:, t],
+                             inp["C"][:, t], inp["D"])
+        assert np.allclose(yt, y[:, t], rtol=0, atol=1e-13)
+    assert np.allclose(st, hf, rtol=0, atol=1e-13)
+
+
+def test_chain_subset_matches_full():
+    inp = _rand_case(23, Bt=2, L=40, H=4, P=3, N=5, G=2)
+    y, hf = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                        init=inp["init"])
+    b = np.array([0, 1, 1]); h = np.array([3, 0, 2]); p = np.array([1, 2, 0])
+    ids = oracle.chain_ids(b, h, p, 4, 3)
+    init = inp["init"][b, h, p]
+    ys, hs = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                         init=init, chains=ids)
+    assert np.array_equal(ys, y[b, :, h, p])
+    assert np.array_equal(hs, hf[b, h, p])
+
+
+def test_special_case_no_decay_is_cumulative_sum():
+    """A -> 0: nothing fades, the state is a running sum of dt*B*x."""
+    inp = _rand_case(31, Bt=1, L=50, H=2, P=2, N=4, G=1, with_init=False)
+    A = np.full(2, -1e-30, dtype=np.float32)
+    y, _ = oracle.scan(inp["x"], inp["dt"], A, inp["B"], inp["C"], inp["D"])
+    x, dt, B, C = (oracle.widen(inp[k]) if k != "dt" else inp[k].astype(np.float64)
+                   for k in ("x", "dt", "B", "C"))
+    for h in range(2):
+        for p in range(2):
+            run = np.cumsum(dt[0, :, h, None] * B[0, :, 0, :] * x[0, :, h, p, None], axis=0)
+            ref = np.sum(C[0, :, 0, :] * run, axis=1) + inp["D"][h] * x[0, :, h, p]
+            assert np.allclose(y[0, :, h, p], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_special_case_instant_decay_is_memoryless():
+    """A very negative: exp(dt*A) underflows to 0, each output sees only its own token."""
+    inp = _rand_case(32, Bt=1, L=30, H=2, P=2, N=4, G=1)
+    A = np.full(2, -1e6, dtype=np.float32)
+    y, _ = oracle.scan(inp["x"], inp["dt"], A, inp["B"], inp["C"], inp["D"], init=inp["init"])
+    x, B, C = (oracle.widen(inp[k]) for k in ("x", "B", "C"))
+    dt = inp["dt"].astype(np.float64)
+    for h in range(2):
+        cb = np.sum(C[0, :, 0, :] * B[0, :, 0, :], axis=1)
+        ref = dt[0, :, h, None] * cb[:, None] * x[0, :, h, :] + inp["D"][h] * x[0, :, h, :]
+        assert np.allclose(y[0, :, h, :], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_special_case_initial_state_only():
+    """x = 0: the output is the initial state, decayed by every token so far, read by C_t."""
+    inp = _rand_case(33, Bt=1, L=40, H=2, P=3, N=4, G=1)
+    x = np.zeros_like(inp["x"])
+    y, hf = oracle.scan(x, inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], init=inp["init"])
+    C = oracle.widen(inp["C"])
+    for h in range(2):
+        decay = np.exp(np.cumsum(inp["dt"][0, :, h].astype(np.float64) * float(inp["A"][h])))
+        h0 = inp["init"][0, h].astype(np.float64)              # [P, N]
+        ref = decay[:, None] * (C[0, :, 0, :] @ h0.T)
+        assert np.allclose(y[0, :, h, :], ref, rtol=1e-12, atol=1e-14)
+        assert np.allclose(hf[0, h], decay[-1] * h0, rtol=1e-12, atol=1e-14)
+
+
+def test_bf16_inputs_widen_exactly():
+    inp = _rand_case(41, Bt=1, L=20, H=2, P=3, N=4, G=1, io="bf16")
+    y1, h1 = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                         init=inp["init"])
+    as32 = {k: ssd_inputs.bf16_bits_to_f32(inp[k]) for k in ("x", "B", "C")}
+    y2, h2 = oracle.scan(as32["x"], inp["dt"], inp["A"], as32["B"], as32["C"], inp["D"],
+                         init=inp["init"])
+    assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+
+
+def _pins_pass(mutation):
+    """Run the pins against a (possibly broken) oracle build; True if all hold."""
+    try:
+        _check_water_tank(mutation)
+        for seed, shape in [(1, dict()), (4, dict(Bt=2, L=50, H=4, P=2, N=4, G=4))]:
+            inp = _rand_case(seed, **shape)
+            y, hf = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                init=inp["init"], mutation=mutation)
+            yq, hq = forms.quadratic(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"],
+                                     inp["D"], init=inp["init"])
+            if np.max(np.abs(y - yq)) > 1e-11 * np.sqrt(np.mean(yq ** 2)):
+                return False
+        inp = _rand_case(33, Bt=1, L=40, H=2, P=3, N=4, G=1)
+        x = np.zeros_like(inp["x"])
+        y, _ = oracle.scan(x, inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                           init=inp["init"], mutation=mutation)
+        yq, _ = forms.quadratic(x, inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                init=inp["init"])
+        if not np.allclose(y, yq, rtol=1e-12, atol=1e-14):
+            return False
+    except AssertionError:
+        return False
+    return True
+
+
+def test_pins_accept_the_oracle():
+    assert _pins_pass(0)
+
+
+@pytest.mark.parametrize("mutation,what", [
+    (1, "skip term D*x dropped"),
+    (2, "output read from the state before the update"),
+    (3, "heads mapped to groups by h % G instead of contiguous blocks"),
+    (4, "step size left out of the decay"),
+    (5, "B and C swapped"),
+    (6, "initial state not decayed by the first token"),
+])
+def test_pins_catch_planted_mistake(mutation, what):
+    assert not _pins_pass(mutation), f"pins did not catch: {what}"
+
+
+def test_inputs_are_deterministic_and_slab_independent():
+    a = ssd_inputs.make_scan_inputs(0)
+    b = ssd_inputs.make_scan_inputs(0)
+    for k in ("x", "dt", "A", "B", "C", "D"):
+        assert np.array_equal(a[k], b[k])
+    # same stream whether drawn whole or across the slab boundary
+    old = ssd_inputs.SLAB_TOKENS
+    try:
+        ssd_inputs.SLAB_TOKENS = 100
+        c = ssd_inputs.make_scan_inputs(0)
+    finally:
+        ssd_inputs.SLAB_TOKENS = old
+    assert np.array_equal(a["x"], c["x"]) and np.array_equal(a["dt"], c["dt"])
+
+
+def test_input_distributions():
+    inp = ssd_inputs.make_scan_inputs(1, seqlen=256)
+    x = ssd_inputs.bf16_bits_to_f32(inp["x"]).astype(np.float64)
+    assert abs(x.mean()) < 0.02 and abs(x.std() - 1) < 0.02
+    assert np.all(inp["dt"] > 0) and abs(inp["dt"].mean() - 0.1403) < 0.003  # E[softplus(N(-2,0.5))] = 0.1403
+    assert np.all((inp["A"] <= -1.0) & (inp["A"] >= -16.0))
+    Bv = ssd_inputs.bf16_bits_to_f32(inp["B"]).astype(np.float64)
+    assert abs(Bv.std() * math.sqrt(128) - 1) < 0.03
+    ini = ssd_inputs.make_scan_inputs(2, seqlen=128, batch=1)["init"]
+    assert abs(ini.std() - 0.1) < 0.005

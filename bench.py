@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-2 SSD layer on B200: chunked scan (prefill) and decode step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ssd_chunk_scan_fwd over the 2.7B-layer workload (batch 4, seqlen 8192, 80
+heads x 64, dstate 128, bf16 x/B/C, fp32 initial state): every row of the hot path from the
+log-decay cumsums to y and the final state.  The decode row is timed in the same run on its own
+workload (1000 ssd_step calls, batch 256, 80 x 64 x 128 fp32 state) and reported under
+"decode".  Inputs are synthetic (ssd_inputs, seed 1002 / 1004) and resident in HBM; they are
+larger than L2 (126 MB), so no flush is needed between steps.  One JSON line on stdout (rank 0).
+
+With N > 1 (torchrun, one process per GPU) every rank runs the same workload on its own GPU
+(the layer shards over batch rows and heads with no exchange): weak scaling, no collective on
+the data path; times are the max over ranks.
+
+--impl reference runs the float64 CPU oracle (the plain sequential recurrence) on the host
+cores, each step a bounded sample of the same workload (batch row 0: 80 heads x 64 channels
+x 8192 tokens), and reports the same metric.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ssd_inputs  # noqa: E402
+
+METRIC = "SSD scan tokens/s per layer at 2.7B shape, % roofline; decode steps/s"
+SCAN_CFG = 2
+DECODE_CFG = 4
+
+
+def scan_bytes(c):
+    """Algorithmic bytes of one scan: every input read once, y written once, init/final state."""
+    tok = c["batch"] * c["seqlen"]
+    es = 2 if c["io"] == "bf16" else 4
+    x = tok * c["nheads"] * c["headdim"] * es
+    bc = 2 * tok * c["ngroups"] * c["dstate"] * es
+    dt = tok * c["nheads"] * 4
+    st = c["batch"] * c["nheads"] * c["headdim"] * c["dstate"] * 4
+    init = st if c["init"] != "zeros" else 0
+    return 2 * x + bc + dt + 2 * c["nheads"] * 4 + init + st
+
+
+def scan_flops(c):
+    """Causal tensor-core work per token: G(Q+1)N + H[(Q+1)P + 4NP]."""
+    Q, N, P, H, G = c["chunk"], c["dstate"], c["headdim"], c["nheads"], c["ngroups"]
+    return c["batch"] * c["seqlen"] * (G * (Q + 1) * N + H * ((Q + 1) * P + 4 * N * P))
+
+
+def step_bytes(c):
+    es = 2
+    st = c["batch"] * c["nheads"] * c["headdim"] * c["dstate"] * 4
+    x = c["batch"] * c["nheads"] * c["headdim"] * es
+    bc = 2 * c["batch"] * c["ngroups"] * c["dstate"] * es
+    return 2 * st + 2 * x + bc + c["batch"] * c["nheads"] * 4 + 2 * c["nheads"] * 4
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region (started before, stopped after)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def to_dev(a, bf16, dev):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if bf16:
+        t = t.view(torch.bfloat16)
+    return t.to(dev)
+
+
+def run_ours(args):
+    import torch
+    import mamba_ssd_scan_03_b200 as ssd
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hbm, tflops, peak_src = peaks()
+
+    # ---------------- chunked scan (the headline) ----------------
+    inp = ssd_inputs.make_scan_inputs(SCAN_CFG)
+    c = inp["cfg"]
+    names = ("x", "dt", "A", "B", "C", "D", "init")
+    t = {k: to_dev(inp[k], k in ("x", "B", "C"), dev) for k in names}
+    y = torch.empty_like(t["x"])
+    fin = torch.empty_like(t["init"])
+    ws = torch.empty(ssd.workspace_size(c["batch"], c["seqlen"], c["nheads"], c["headdim"],
+                                        c["dstate"], c["ngroups"], c["chunk"]),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def scan_once():
+        ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], c["chunk"],
+                           init_state=t["init"], workspace=ws, out=y, final_out=fin)
+
+    for _ in range(args.warmup):
+        scan_once()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            scan_once()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world)
+    status = ssd.device_status()
+    ms_per_step = total_ms / args.steps
+    tokens = c["batch"] * c["seqlen"]
+    value = world * tokens * args.steps / (total_ms / 1e3)
+    nbytes = scan_bytes(c)
+    achieved = nbytes / (statistics.mean(per) / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "traffic": args.traffic,
+            "kernel": "ssd_chunk_scan_fwd (seg_state + seg_scan + chunk_out, one call)",
+            "algorithmic_bytes": nbytes, "flops": scan_flops(c),
+            "peak_source": peak_src,
+            "flop_frac": round(scan_flops(c) / (statistics.mean(per) / 1e3) / 1e12 / tflops, 4)}
+
+    # ---------------- e2e through the public API with host buffers ----------------
+    pinned = {k: t[k].cpu().pin_memory() for k in names}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    f_host = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    dbuf = {k: torch.empty_like(t[k]) for k in names}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * y_host.element_size() + f_host.numel() * f_host.element_size()
+
+    def e2e_once():
+        for k in names:
+            dbuf[k].copy_(pinned[k], non_blocking=True)
+        ssd.chunk_scan_fwd(dbuf["x"], dbuf["dt"], dbuf["A"], dbuf["B"], dbuf["C"], dbuf["D"],
+                           c["chunk"], init_state=dbuf["init"], workspace=ws, out=y,
+                           final_out=fin)
+        y_host.copy_(y, non_blocking=True)
+        f_host.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(2):
+        e2e_once()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_once()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = {"value": world * tokens * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+    del pinned, dbuf
+
+    # ---------------- decode workload: 1000 ssd_step calls ----------------
+    dec = ssd_inputs.make_decode_inputs(DECODE_CFG)
+    dc = dec["cfg"]
+    st = to_dev(dec["state"], False, dev)
+    A4, D4 = to_dev(dec["A"], False, dev), to_dev(dec["D"], False, dev)
+    n_dec_inputs = 8
+    steps_in = []
+    for k in range(n_dec_inputs):  # distinct per-step inputs, cycled
+        s = ssd_inputs.decode_step_inputs(dec, k)
+        steps_in.append({n: to_dev(s[n], n != "dt", dev) for n in ("x", "dt", "B", "C")})
+    ydec = torch.empty_like(steps_in[0]["x"])
+
+    def dec_once(k):
+        s = steps_in[k % n_dec_inputs]
+        ssd.step(st, s["x"], s["dt"], A4, s["B"], s["C"], D4, out=ydec)
+
+    for k in range(max(3, args.warmup)):
+        dec_once(k)
+    torch.cuda.synchronize()
+    n_dec = dc["decode_steps"]
+    barrier(world)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk_dec:
+        d0.record(stream)
+        for k in range(n_dec):
+            dec_once(k)
+        d1.record(stream)
+        torch.cuda.synchronize()
+    dec_ms = max_over_ranks(d0.elapsed_time(d1), world)
+    sb = step_bytes(dc)
+    dec_ach = sb / (dec_ms / n_dec / 1e3) / 1e9
+    decode = {"metric": "decode steps/s", "value": world * n_dec / (dec_ms / 1e3),
+              "unit": "steps/s", "tokens_per_s": world * dc["batch"] * n_dec / (dec_ms / 1e3),
+              "steps": n_dec, "ms_per_step": dec_ms / n_dec,
+              "config": {"workload": dc["name"], "batch": dc["batch"], "nheads": dc["nheads"],
+                         "headdim": dc["headdim"], "dstate": dc["dstate"]},
+              "roofline": {"bound": "hbm", "achieved": round(dec_ach, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(dec_ach / hbm, 4),
+                           "traffic": args.decode_traffic, "kernel": "step_n128_kernel",
+                           "algorithmic_bytes": sb, "peak_source": peak_src},
+              "clocks": clk_dec.summary(), "gpu_launches": n_dec}
+
+    # ---------------- CPU baseline: the float64 oracle on a bounded sample -----------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, args.cpu_rows)
+
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic",
+           "config": {"workload": c["name"], "batch": c["batch"], "seqlen": c["seqlen"],
+                      "nheads": c["nheads"], "headdim": c["headdim"], "dstate": c["dstate"],
+                      "ngroups": c["ngroups"], "chunk": c["chunk"], "init_state": c["init"],
+                      "parallelism": f"replicas{world}" if world > 1 else "single",
+                      "l2": "inputs larger than L2 (719 MB per step > 126 MB), no flush"},
+           "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+           "gpu_launches": 3 * args.steps, "decode": decode, "device_status": status,
+           "path": "tcgen05" if ssd.path(c["batch"], c["seqlen"], c["nheads"], c["headdim"],
+                                        c["dstate"], c["ngroups"], c["chunk"]) == 1 else "simt"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(inp, rows=1):
+    """The oracle as it stands, all host cores, on batch rows [0, rows) of the workload."""
+    import oracle
+    c = inp["cfg"]
+    H, P, L = c["nheads"], c["headdim"], c["seqlen"]
+    b = np.repeat(np.arange(rows), H * P)
+    h = np.tile(np.repeat(np.arange(H), P), rows)
+    p = np.tile(np.arange(P), rows * H)
+    ids = oracle.chain_ids(b, h, p, H, P)
+    init = None if inp["init"] is None else inp["init"][b, h, p]
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], init=init,
+                chains=ids, nthreads=cores)
+    sec = time.perf_counter() - t0
+    return {"value": rows * L / sec, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"batch rows 0..{rows - 1} of {c['batch']} (all {H} heads x {P} channels, "
+                      f"{L} tokens), float64 sequential recurrence, {sec:.2f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = ssd_inputs.make_scan_inputs(SCAN_CFG)
+    c = inp["cfg"]
+    for _ in range(args.warmup):
+        cpu_baseline(inp, 1)
+    runs = [cpu_baseline(inp, 1) for _ in range(args.steps)]
+    tok_s = statistics.mean(r["value"] for r in runs)
+    sec = c["seqlen"] / tok_s
+    out = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": c["name"], "batch": c["batch"], "seqlen": c["seqlen"],
+                      "nheads": c["nheads"], "headdim": c["headdim"], "dstate": c["dstate"],
+                      "ngroups": c["ngroups"], "chunk": c["chunk"]},
+           "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "kind": "oracle",
+                            "cores": runs[0]["cores"], "sample": runs[0]["sample"]},
+           "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per scan call (null when not measured)")
+    ap.add_argument("--decode-traffic", type=float, default=None)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

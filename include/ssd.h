@@ -1,0 +1,152 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) Mamba-2 SSD layer library (libssd.so).
+ *
+ * The layer (per batch row b and head h, scalar decay A_h, input-dependent dt, B, C):
+ *
+ *   h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * B_t x_t^T        (state h: dstate x headdim)
+ *   y_t = C_t^T h_t + D_h * x_t
+ *
+ * equivalently y_t = sum_{s<=t} C_t^T (prod_{k=s+1..t} exp(dt_k A_h)) B_s dt_s x_s + D_h x_t,
+ * the lower-triangular semiseparable matrix of "Mamba-2 (2024): SSM e attention sono la
+ * stessa cosa" (paithon.it), section "Due modi di guardare la stessa matrice".  The
+ * recurrence is the one of "State Space Model" (book.paithon.it), sections "Un sistema
+ * che riassume il passato" (decay exp(Delta A), input term Delta B) and "Due strade, una
+ * meta" (h_t = A_t h_{t-1} + b_t with a scalar transition); the D x skip term is from
+ * "Puntata 205 -- State Space Models e Mamba" (aiperbabbani.it), "Cos'e un SSM".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor pointers are CUDA device pointers owned by the caller (device or managed
+ *    memory; anything else is rejected with SSD_ERR_INVALID_ARG before any launch).  The
+ *    library never allocates device memory; scratch comes from the caller's workspace.
+ *  - Layouts are dense row-major (contiguous):
+ *        x, y         [batch, seqlen, nheads, headdim]   io dtype
+ *        dt           [batch, seqlen, nheads]            float32 (used as given, > 0)
+ *        A, D         [nheads]                           float32 (A < 0; D may be NULL = 0)
+ *        B, C         [batch, seqlen, ngroups, dstate]   io dtype
+ *        states       [batch, nheads, headdim, dstate]   float32; element [b,h,p,n] is h[n,p]
+ *    Head h reads group g = h / (nheads / ngroups).
+ *  - io dtype (x, B, C, y): SSD_F32 or SSD_BF16.  Arithmetic is float32 with float32
+ *    accumulation; y is rounded to the io dtype (nearest even).
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument errors are
+ *    reported synchronously and nothing is launched.  A launch failure returns
+ *    SSD_ERR_CUDA.  Errors found by the kernels themselves (a bounded wait that expired)
+ *    are latched in a device status word and reported by ssd_get_device_status().
+ *  - Not thread-safe per stream: two calls that share a workspace must be ordered.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSD_OK = 0,
+  SSD_ERR_INVALID_ARG = 1,    /* NULL required pointer, non-device pointer, bad size, aliasing */
+  SSD_ERR_UNSUPPORTED = 2,    /* valid but outside what the kernels are built for */
+  SSD_ERR_WORKSPACE = 3,      /* workspace NULL or smaller than the query returned */
+  SSD_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  SSD_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait expired (see ssd_get_device_status) */
+} ssd_status;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/* Which kernels ssd_chunk_scan_fwd uses for a shape. */
+typedef enum { SSD_PATH_SIMT = 0, SSD_PATH_TCGEN05 = 1 } ssd_path;
+
+/*
+ * Bytes of device workspace ssd_chunk_scan_fwd needs for this shape (0 is possible).
+ * Returns 0 as well for invalid arguments; ssd_chunk_scan_fwd then reports the error.
+ */
+size_t ssd_chunk_scan_workspace_size(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                     int dstate, int ngroups, int chunk, ssd_dtype io);
+
+/* The path ssd_chunk_scan_fwd takes for this shape.  On the tensor-core path x, B, C and y
+ * must be 16-byte aligned (TMA tiles); a misaligned pointer there returns
+ * SSD_ERR_UNSUPPORTED (ssd_chunk_scan_fwd_simt accepts any element-aligned pointers). */
+ssd_path ssd_chunk_scan_path(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                             int dstate, int ngroups, int chunk, ssd_dtype io);
+
+/*
+ * Chunked forward scan (prefill / training forward): y over the whole sequence and the
+ * state after its last token.  The sequence is cut into contiguous blocks; inside a block
+ * the output is the masked quadratic (attention-like) form, and only a state summary is
+ * passed from block to block ("Il trucco a blocchi" of the Mamba-2 page above; block
+ * sizes 64 or 128 per "Rewolucja Mamba-2 i teoria State Space Duality SSD" of the
+ * tech.tersel.eu article).  The result does not depend on the block size.
+ *
+ *   x, dt, A, B, C, D : inputs as above (D may be NULL).
+ *   init_state        : [batch, nheads, headdim, dstate] float32, the state before token 0
+ *                       (token 0 decays it once); NULL means zeros.
+ *   y                 : output [batch, seqlen, nheads, headdim], io dtype; must not overlap
+ *                       any input.
+ *   final_state       : output state after token seqlen-1, float32; NULL = not written.
+ *                       May equal init_state (in-place streaming prefill).
+ *   chunk             : 64, 128 or 256.  The SIMT path uses it as its block length; the
+ *                       tensor-core path evaluates 128-token blocks (the tcgen05 M=128
+ *                       tile) for every admissible chunk.
+ *   seqlen            : >= 1; need not be a multiple of chunk.
+ *   Path: io = BF16, headdim = 64, dstate = 128 and an even number of heads per group ->
+ *         tcgen05 tensor cores (TMA, TMEM); everything else (including every F32 call) ->
+ *         float32 SIMT kernels (headdim <= 256, dstate <= 2048, batch*nheads <= 65535;
+ *         larger shapes return SSD_ERR_UNSUPPORTED).
+ *   workspace         : device scratch of at least ssd_chunk_scan_workspace_size() bytes,
+ *                       256-byte aligned; contents on entry are ignored.
+ */
+ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
+                              const void* C, const float* D, const float* init_state, void* y,
+                              float* final_state, int64_t batch, int64_t seqlen, int nheads,
+                              int headdim, int dstate, int ngroups, int chunk, ssd_dtype io,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The same operation forced onto the float32 SIMT kernels (any supported shape), with its
+ * own workspace query.  Used as a second GPU reference and for float32 io. */
+size_t ssd_chunk_scan_simt_workspace_size(int64_t batch, int64_t seqlen, int nheads,
+                                          int headdim, int dstate, int ngroups, int chunk,
+                                          ssd_dtype io);
+ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* A,
+                                   const void* B, const void* C, const float* D,
+                                   const float* init_state, void* y, float* final_state,
+                                   int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                   int dstate, int ngroups, int chunk, ssd_dtype io,
+                                   void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+
+/*
+ * One recurrent step (generation / decode), updating `state` in place:
+ *   alpha = exp(dt[b,h] * A[h]);  state[b,h,p,n] = alpha*state[b,h,p,n] + dt[b,h]*x[b,h,p]*B[b,g,n]
+ *   y[b,h,p] = sum_n C[b,g,n] * state[b,h,p,n] (updated) + D[h] * x[b,h,p]
+ * "State Space Models (SSM)" (ultralytics.com glossary), section "Come funzionano gli SSM":
+ * the recurrent form used during generation, constant memory per token.
+ *   state [batch, nheads, headdim, dstate] float32 (read and written once per call);
+ *   x, y [batch, nheads, headdim] io dtype; dt [batch, nheads] float32;
+ *   B, C [batch, ngroups, dstate] io dtype; A, D [nheads] float32 (D may be NULL).
+ *   y must not overlap state or any input.  No workspace, no allocation.
+ */
+ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A,
+                    const void* B, const void* C, const float* D, void* y, int64_t batch,
+                    int nheads, int headdim, int dstate, int ngroups, ssd_dtype io,
+                    cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* ssd_status_string(ssd_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that kernels latch
+ * when a bounded wait expires (for the current device).  Returns SSD_OK,
+ * SSD_ERR_DEVICE_TIMEOUT, or SSD_ERR_CUDA if the synchronisation itself failed.
+ */
+ssd_status ssd_get_device_status(cudaStream_t stream);
+
+/* Library version string, e.g. "ssd-b200 0.1 sm_100a". */
+const char* ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSD_H_ */

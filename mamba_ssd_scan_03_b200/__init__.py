@@ -1,0 +1,212 @@
+"""B200 (sm_100a) Mamba-2 SSD layer: thin Python binding over the C ABI in include/ssd.h.
+
+Every step of the computation runs in the CUDA kernels of ``libssd.so``; this module only
+checks tensors, allocates outputs and workspace with PyTorch (device memory and streams are
+PyTorch's job here), and passes raw pointers plus the current CUDA stream.  There is no CPU
+path: if the library is missing or no CUDA device is present, the calls raise.
+
+    y, final_state = chunk_scan_fwd(x, dt, A, B, C, D, chunk, init_state=None)
+    y = step(state, x, dt, A, B, C, D)          # updates `state` in place
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssd.so")
+
+SSD_F32, SSD_BF16 = 0, 1
+SSD_PATH_SIMT, SSD_PATH_TCGEN05 = 0, 1
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
+          3: "SSD_ERR_WORKSPACE", 4: "SSD_ERR_CUDA", 5: "SSD_ERR_DEVICE_TIMEOUT"}
+
+# The symbols include/ssd.h declares (tests check that the library exports each one).
+EXPORTS = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path", "ssd_chunk_scan_fwd",
+           "ssd_chunk_scan_simt_workspace_size", "ssd_chunk_scan_fwd_simt", "ssd_step",
+           "ssd_status_string", "ssd_get_device_status", "ssd_version")
+
+
+class SSDError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({_status_string(code)})")
+
+
+_lib = None
+
+_vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_SHAPE = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32]  # batch .. chunk, io
+_SCAN = [_vp] * 9 + [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
+
+
+def load():
+    """Load libssd.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m mamba_ssd_scan_03_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.ssd_chunk_scan_workspace_size.restype = _sz
+    lib.ssd_chunk_scan_workspace_size.argtypes = _SHAPE
+    lib.ssd_chunk_scan_simt_workspace_size.restype = _sz
+    lib.ssd_chunk_scan_simt_workspace_size.argtypes = _SHAPE
+    lib.ssd_chunk_scan_path.restype = _i32
+    lib.ssd_chunk_scan_path.argtypes = _SHAPE
+    for fn in (lib.ssd_chunk_scan_fwd, lib.ssd_chunk_scan_fwd_simt):
+        fn.restype = _i32
+        fn.argtypes = _SCAN
+    lib.ssd_step.restype = _i32
+    lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_status_string.argtypes = [_i32]
+    lib.ssd_get_device_status.restype = _i32
+    lib.ssd_get_device_status.argtypes = [_vp]
+    lib.ssd_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _status_string(code):
+    try:
+        return load().ssd_status_string(code).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _check(code, what):
+    if code != 0:
+        raise SSDError(code, what)
+
+
+def _io(t):
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    if t.dtype == torch.float32:
+        return SSD_F32
+    raise TypeError(f"x/B/C must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _scan_shape(x, B, chunk):
+    Bt, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    return Bt, L, H, P, N, G, int(chunk), _io(x)
+
+
+def workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io=SSD_BF16,
+                   simt=False):
+    fn = load().ssd_chunk_scan_simt_workspace_size if simt else \
+        load().ssd_chunk_scan_workspace_size
+    return fn(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io)
+
+
+def path(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io=SSD_BF16):
+    return load().ssd_chunk_scan_path(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io)
+
+
+def _scan(entry, simt, x, dt, A, B, C, D, chunk, init_state, want_final, workspace, out,
+          final_out):
+    lib = load()
+    _need(x, "x")
+    dev = x.device
+    Bt, L, H, P, N, G, Q, io = _scan_shape(x, B, chunk)
+    _need(B, "B", x.dtype, (Bt, L, G, N), dev)
+    _need(C, "C", x.dtype, (Bt, L, G, N), dev)
+    _need(dt, "dt", torch.float32, (Bt, L, H), dev)
+    _need(A, "A", torch.float32, (H,), dev)
+    if D is not None:
+        _need(D, "D", torch.float32, (H,), dev)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (Bt, H, P, N), dev)
+    y = out if out is not None else torch.empty_like(x)
+    _need(y, "out", x.dtype, x.shape, dev)
+    fin = None
+    if want_final:
+        fin = final_out if final_out is not None else torch.empty(
+            (Bt, H, P, N), dtype=torch.float32, device=dev)
+        _need(fin, "final_state", torch.float32, (Bt, H, P, N), dev)
+    need = workspace_size(Bt, L, H, P, N, G, Q, io, simt=simt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = entry(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+                   _ptr(y), _ptr(fin), Bt, L, H, P, N, G, Q, io, _ptr(workspace),
+                   workspace.numel(), _stream(dev))
+    _check(rc, "ssd_chunk_scan_fwd_simt" if simt else "ssd_chunk_scan_fwd")
+    return y, fin
+
+
+def chunk_scan_fwd(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
+                   workspace=None, out=None, final_out=None):
+    """Chunked forward scan.  x [B,L,H,P], dt [B,L,H] f32, A [H] f32, B/C [B,L,G,N],
+    D [H] f32 or None, init_state [B,H,P,N] f32 or None.  Returns (y, final_state)."""
+    return _scan(load().ssd_chunk_scan_fwd, False, x, dt, A, B, C, D, chunk, init_state,
+                 want_final, workspace, out, final_out)
+
+
+def chunk_scan_fwd_simt(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
+                        workspace=None, out=None, final_out=None):
+    """The same operation on the float32 SIMT kernels (second GPU reference)."""
+    return _scan(load().ssd_chunk_scan_fwd_simt, True, x, dt, A, B, C, D, chunk, init_state,
+                 want_final, workspace, out, final_out)
+
+
+def step(state, x, dt, A, B, C, D, out=None):
+    """One decode step; updates ``state`` [B,H,P,N] f32 in place and returns y [B,H,P]."""
+    lib = load()
+    _need(state, "state", torch.float32)
+    dev = state.device
+    Bt, H, P, N = state.shape
+    io = _io(x)
+    _need(x, "x", x.dtype, (Bt, H, P), dev)
+    G = B.shape[1]
+    _need(B, "B", x.dtype, (Bt, G, N), dev)
+    _need(C, "C", x.dtype, (Bt, G, N), dev)
+    _need(dt, "dt", torch.float32, (Bt, H), dev)
+    _need(A, "A", torch.float32, (H,), dev)
+    if D is not None:
+        _need(D, "D", torch.float32, (H,), dev)
+    y = out if out is not None else torch.empty_like(x)
+    _need(y, "out", x.dtype, x.shape, dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_step(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                          _ptr(y), Bt, H, P, N, G, io, _stream(dev))
+    _check(rc, "ssd_step")
+    return y
+
+
+def device_status(device=None):
+    """Synchronise the current stream and read/clear the kernels' device status word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return load().ssd_get_device_status(_stream(dev))
+
+
+def version():
+    return load().ssd_version().decode()

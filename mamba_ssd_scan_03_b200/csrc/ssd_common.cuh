@@ -1,0 +1,67 @@
+// ssd_common.cuh -- small helpers shared by the SSD kernels (one translation unit: ssd_lib.cu).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ssd.h"
+
+namespace ssd {
+
+// log2(e): decays are evaluated as exp2(a * log2 e) on the MUFU ex2 unit.
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Device status word latched by kernels whose bounded waits expire (0 = OK).  Bits:
+// low byte = ssd_status code, upper bits = site id of the wait that gave up.
+__device__ unsigned int g_status;
+
+__device__ __forceinline__ void latch_status(unsigned code, unsigned site) {
+  atomicCAS(&g_status, 0u, code | (site << 8));
+}
+
+// Hardware 2^x (MUFU ex2, approximate, flush-to-zero): a PTX instruction, not a library call.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <typename T> struct io_traits;
+template <> struct io_traits<float> {
+  static __device__ __forceinline__ float load(const float* p, int64_t i) { return p[i]; }
+  static __device__ __forceinline__ void store(float* p, int64_t i, float v) { p[i] = v; }
+};
+template <> struct io_traits<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16* p, int64_t i) {
+    return __bfloat162float(p[i]);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, int64_t i, float v) {
+    p[i] = __float2bfloat16_rn(v);
+  }
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_inclusive_scan(float v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    float u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+// bf16 helpers on raw 16-bit patterns (round to nearest even via the CUDA intrinsic).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+}  // namespace ssd

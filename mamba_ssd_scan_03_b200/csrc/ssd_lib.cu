@@ -1,0 +1,416 @@
+// ssd_lib.cu -- the C ABI of libssd.so (declared in include/ssd.h): argument validation, path
+// selection, workspace carving, TMA descriptor set-up and the stream-ordered launches.
+// Single translation unit: the kernels live in the headers included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "simt_kernels.cuh"
+#include "ssd_common.cuh"
+#include "step_kernels.cuh"
+#include "tc_kernels.cuh"
+
+namespace {
+
+using ssd::tc::Seg;
+
+constexpr int kUnitsTarget = 8 * 148;  // tensor-core grids: ~8 CTAs per SM of a B200
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool is_device_ptr(const void* p) {
+  if (!p) return false;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || !na || !nb) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Shape {
+  int64_t batch, seqlen;
+  int nheads, headdim, dstate, ngroups, chunk;
+  ssd_dtype io;
+};
+
+ssd_status check_shape(const Shape& s) {
+  if (s.batch <= 0 || s.seqlen <= 0 || s.nheads <= 0 || s.headdim <= 0 || s.dstate <= 0 ||
+      s.ngroups <= 0)
+    return SSD_ERR_INVALID_ARG;
+  if (s.nheads % s.ngroups != 0) return SSD_ERR_INVALID_ARG;
+  if (s.chunk != 64 && s.chunk != 128 && s.chunk != 256) return SSD_ERR_INVALID_ARG;
+  if (s.io != SSD_F32 && s.io != SSD_BF16) return SSD_ERR_INVALID_ARG;
+  return SSD_OK;
+}
+
+bool simt_supported(const Shape& s) {
+  return s.headdim <= 256 && s.dstate <= 2048 && s.batch * s.nheads <= 65535 &&
+         (s.seqlen + s.chunk - 1) / s.chunk <= (int64_t(1) << 30);
+}
+
+bool tc_shape_ok(const Shape& s) {
+  const int hpg = s.nheads / s.ngroups;
+  return s.io == SSD_BF16 && s.headdim == 64 && s.dstate == 128 && (hpg % 2) == 0 &&
+         s.seqlen <= (int64_t(1) << 30) && s.batch <= (int64_t(1) << 20);
+}
+
+Seg tc_segments(const Shape& s) {
+  Seg sg;
+  sg.nblk = int((s.seqlen + ssd::tc::kBlk - 1) / ssd::tc::kBlk);
+  const int64_t pairs = s.batch * (s.nheads / 2);
+  int nseg = int(std::min<int64_t>(sg.nblk, std::max<int64_t>(1, (kUnitsTarget + pairs - 1) / pairs)));
+  sg.seg_blks = (sg.nblk + nseg - 1) / nseg;
+  sg.nseg = (sg.nblk + sg.seg_blks - 1) / sg.seg_blks;
+  return sg;
+}
+
+size_t tc_workspace(const Shape& s) {
+  const Seg sg = tc_segments(s);
+  const size_t states = size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float);
+  const size_t decay = size_t(s.batch) * sg.nseg * s.nheads * sizeof(float);
+  return align256(states) + align256(decay);
+}
+
+size_t simt_workspace(const Shape& s) {
+  const int64_t nchunks = (s.seqlen + s.chunk - 1) / s.chunk;
+  const size_t cs = size_t(s.batch) * s.nheads * nchunks * s.chunk * sizeof(float);
+  const size_t states =
+      size_t(s.batch) * nchunks * s.nheads * size_t(s.headdim) * s.dstate * sizeof(float);
+  return align256(cs) + align256(states);
+}
+
+// ---- TMA descriptor encoding through the driver entry point (no link-time libcuda) ---------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 3-D bf16 view [outer][mid][inner] with a {64, 128, 1} box and 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kTcSmem = ssd::tc::kSmemTiles + 1024;
+template <int HQ>
+constexpr size_t seg_state_smem() { return 2 * (2 + HQ) * size_t(ssd::tc::kTile) + 1024; }
+
+ssd_status set_smem_attrs() {
+  static ssd_status st = SSD_ERR_CUDA;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
+          cudaSuccess;
+    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<4>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(seg_state_smem<4>())) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(seg_state_smem<2>())) == cudaSuccess;
+    for (auto f : {(const void*)ssd::simt::chunk_out_kernel<float>,
+                   (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16>,
+                   (const void*)ssd::simt::chunk_state_kernel<float>,
+                   (const void*)ssd::simt::chunk_state_kernel<__nv_bfloat16>})
+      ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
+            cudaSuccess;
+    st = ok ? SSD_OK : SSD_ERR_CUDA;
+    if (!ok) cudaGetLastError();
+  });
+  return st;
+}
+
+ssd_status launched() {
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+struct ScanArgs {
+  const void *x, *B, *C;
+  const float *dt, *A, *D, *init;
+  void* y;
+  float* fin;
+  void* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+};
+
+ssd_status validate_scan(const Shape& s, const ScanArgs& a, size_t need) {
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  for (const void* p : {a.x, (const void*)a.dt, (const void*)a.A, a.B, a.C, (const void*)a.y})
+    if (!is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)a.D, (const void*)a.init, (const void*)a.fin})
+    if (p && !is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  const size_t es = s.io == SSD_BF16 ? 2 : 4;
+  const size_t nx = size_t(s.batch) * s.seqlen * s.nheads * s.headdim * es;
+  const size_t nbc = size_t(s.batch) * s.seqlen * s.ngroups * s.dstate * es;
+  const size_t ndt = size_t(s.batch) * s.seqlen * s.nheads * 4;
+  const size_t nst = size_t(s.batch) * s.nheads * s.headdim * s.dstate * 4;
+  if (overlaps(a.y, nx, a.x, nx) || overlaps(a.y, nx, a.B, nbc) || overlaps(a.y, nx, a.C, nbc) ||
+      overlaps(a.y, nx, a.dt, ndt) || overlaps(a.y, nx, a.init, nst) ||
+      overlaps(a.y, nx, a.fin, nst))
+    return SSD_ERR_INVALID_ARG;
+  if (a.fin && a.fin != a.init &&
+      (overlaps(a.fin, nst, a.init, nst) || overlaps(a.fin, nst, a.x, nx) ||
+       overlaps(a.fin, nst, a.B, nbc) || overlaps(a.fin, nst, a.C, nbc)))
+    return SSD_ERR_INVALID_ARG;
+  if (need > 0) {
+    if (!a.ws || a.ws_bytes < need || (reinterpret_cast<uintptr_t>(a.ws) & 255u) ||
+        !is_device_ptr(a.ws))
+      return SSD_ERR_WORKSPACE;
+    if (overlaps(a.ws, need, a.y, nx) || overlaps(a.ws, need, a.x, nx) ||
+        overlaps(a.ws, need, a.init, nst) || overlaps(a.ws, need, a.fin, nst))
+      return SSD_ERR_INVALID_ARG;
+  }
+  return SSD_OK;
+}
+
+template <typename T>
+ssd_status run_simt(const Shape& s, const ScanArgs& a) {
+  const int64_t nchunks = (s.seqlen + s.chunk - 1) / s.chunk;
+  float* cs = static_cast<float*>(a.ws);
+  float* states = reinterpret_cast<float*>(
+      static_cast<char*>(a.ws) +
+      align256(size_t(s.batch) * s.nheads * nchunks * s.chunk * sizeof(float)));
+  const dim3 grid(unsigned(nchunks), unsigned(s.batch * s.nheads));
+  ssd::simt::cumsum_kernel<<<grid, s.chunk, 0, a.stream>>>(a.dt, a.A, cs, s.seqlen, s.nheads,
+                                                           s.chunk, int(nchunks));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const size_t sm_state = 16 * size_t(s.headdim + s.dstate) * sizeof(float);
+  ssd::simt::chunk_state_kernel<T><<<grid, 256, sm_state, a.stream>>>(
+      static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), cs, states, s.seqlen,
+      s.nheads, s.headdim, s.dstate, s.ngroups, s.chunk, int(nchunks));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const int64_t nel = s.batch * s.nheads * int64_t(s.headdim) * s.dstate;
+  ssd::simt::state_pass_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
+      states, cs, a.init, a.fin, s.batch, s.nheads, s.headdim, s.dstate, s.chunk, int(nchunks));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const size_t sm_out = (3072 + 64 * size_t(s.headdim)) * sizeof(float);
+  ssd::simt::chunk_out_kernel<T><<<grid, 256, sm_out, a.stream>>>(
+      static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), static_cast<const T*>(a.C),
+      a.D, cs, states, static_cast<T*>(a.y), s.seqlen, s.nheads, s.headdim, s.dstate,
+      s.ngroups, s.chunk, int(nchunks));
+  return launched();
+}
+
+ssd_status run_tc(const Shape& s, const ScanArgs& a) {
+  const Seg sg = tc_segments(s);
+  float* seg_states = static_cast<float*>(a.ws);
+  float* seg_decay = reinterpret_cast<float*>(
+      static_cast<char*>(a.ws) +
+      align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)));
+  CUtensorMap mx, mb, mc;
+  const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
+  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch) ||
+      !make_map(&mc, a.C, GN, s.seqlen, s.batch))
+    return SSD_ERR_CUDA;
+  const int hpg = s.nheads / s.ngroups;
+  if (hpg % 4 == 0) {
+    const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 4));
+    ssd::tc::seg_state_kernel<4><<<grid, 128, seg_state_smem<4>(), a.stream>>>(
+        mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
+  } else {
+    const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
+    ssd::tc::seg_state_kernel<2><<<grid, 128, seg_state_smem<2>(), a.stream>>>(
+        mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
+  }
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;
+  ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
+      seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
+  ssd::tc::chunk_out_kernel<<<grid, 128, kTcSmem, a.stream>>>(
+      mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<__nv_bfloat16*>(a.y), s.seqlen,
+      s.nheads, hpg, sg);
+  return launched();
+}
+
+bool tc_pointers_ok(const ScanArgs& a) {
+  return aligned16(a.x) && aligned16(a.B) && aligned16(a.C) && aligned16(a.y);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_chunk_scan_workspace_size(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                     int dstate, int ngroups, int chunk, ssd_dtype io) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  if (check_shape(s) != SSD_OK) return 0;
+  if (tc_shape_ok(s)) return tc_workspace(s);
+  return simt_supported(s) ? simt_workspace(s) : 0;
+}
+
+ssd_path ssd_chunk_scan_path(int64_t batch, int64_t seqlen, int nheads, int headdim, int dstate,
+                             int ngroups, int chunk, ssd_dtype io) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  return (check_shape(s) == SSD_OK && tc_shape_ok(s)) ? SSD_PATH_TCGEN05 : SSD_PATH_SIMT;
+}
+
+size_t ssd_chunk_scan_simt_workspace_size(int64_t batch, int64_t seqlen, int nheads,
+                                          int headdim, int dstate, int ngroups, int chunk,
+                                          ssd_dtype io) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  if (check_shape(s) != SSD_OK || !simt_supported(s)) return 0;
+  return simt_workspace(s);
+}
+
+ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
+                              const void* C, const float* D, const float* init_state, void* y,
+                              float* final_state, int64_t batch, int64_t seqlen, int nheads,
+                              int headdim, int dstate, int ngroups, int chunk, ssd_dtype io,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  const ScanArgs a{x, B, C, dt, A, D, init_state, y, final_state, workspace, workspace_bytes,
+                   stream};
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  const bool tc = tc_shape_ok(s);
+  if (!tc && !simt_supported(s)) return SSD_ERR_UNSUPPORTED;
+  st = validate_scan(s, a, tc ? tc_workspace(s) : simt_workspace(s));
+  if (st != SSD_OK) return st;
+  if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
+  if (tc) {
+    if (!tc_pointers_ok(a)) return SSD_ERR_UNSUPPORTED;
+    return run_tc(s, a);
+  }
+  return io == SSD_BF16 ? run_simt<__nv_bfloat16>(s, a) : run_simt<float>(s, a);
+}
+
+ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* A,
+                                   const void* B, const void* C, const float* D,
+                                   const float* init_state, void* y, float* final_state,
+                                   int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                   int dstate, int ngroups, int chunk, ssd_dtype io,
+                                   void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  const ScanArgs a{x, B, C, dt, A, D, init_state, y, final_state, workspace, workspace_bytes,
+                   stream};
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  if (!simt_supported(s)) return SSD_ERR_UNSUPPORTED;
+  st = validate_scan(s, a, simt_workspace(s));
+  if (st != SSD_OK) return st;
+  if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
+  return io == SSD_BF16 ? run_simt<__nv_bfloat16>(s, a) : run_simt<float>(s, a);
+}
+
+ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A,
+                    const void* B, const void* C, const float* D, void* y, int64_t batch,
+                    int nheads, int headdim, int dstate, int ngroups, ssd_dtype io,
+                    cudaStream_t stream) {
+  if (batch <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+      nheads % ngroups != 0 || (io != SSD_F32 && io != SSD_BF16))
+    return SSD_ERR_INVALID_ARG;
+  if (batch * nheads > (int64_t(1) << 31) - 1) return SSD_ERR_UNSUPPORTED;
+  for (const void* p : {(const void*)state, x, (const void*)dt, (const void*)A, B, C,
+                        (const void*)y})
+    if (!is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  if (D && !is_device_ptr(D)) return SSD_ERR_INVALID_ARG;
+  const size_t es = io == SSD_BF16 ? 2 : 4;
+  const size_t nst = size_t(batch) * nheads * headdim * dstate * 4;
+  const size_t nx = size_t(batch) * nheads * headdim * es;
+  const size_t nbc = size_t(batch) * ngroups * dstate * es;
+  if (overlaps(y, nx, state, nst) || overlaps(y, nx, x, nx) || overlaps(y, nx, B, nbc) ||
+      overlaps(y, nx, C, nbc) || overlaps(state, nst, x, nx) || overlaps(state, nst, B, nbc) ||
+      overlaps(state, nst, C, nbc))
+    return SSD_ERR_INVALID_ARG;
+  const int hpg = nheads / ngroups;
+  const unsigned grid = unsigned(batch * nheads);
+  const bool fast = dstate == 128 && headdim % 8 == 0 && aligned16(state) &&
+                    (headdim / 8 == 1 || headdim / 8 == 2 || headdim / 8 == 4 ||
+                     headdim / 8 == 8 || headdim / 8 == 16);
+#define SSD_STEP_FAST(T, RPW)                                                              \
+  ssd::step_n128_kernel<T, RPW><<<grid, 256, 0, stream>>>(                                 \
+      state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B),                    \
+      static_cast<const T*>(C), D, static_cast<T*>(y), nheads, hpg, ngroups)
+#define SSD_STEP_DISPATCH(T)                          \
+  switch (headdim / 8) {                              \
+    case 1: SSD_STEP_FAST(T, 1); break;               \
+    case 2: SSD_STEP_FAST(T, 2); break;               \
+    case 4: SSD_STEP_FAST(T, 4); break;               \
+    case 8: SSD_STEP_FAST(T, 8); break;               \
+    default: SSD_STEP_FAST(T, 16); break;             \
+  }
+  if (fast) {
+    if (io == SSD_BF16) { SSD_STEP_DISPATCH(__nv_bfloat16) } else { SSD_STEP_DISPATCH(float) }
+  } else if (io == SSD_BF16) {
+    ssd::step_generic_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        state, static_cast<const __nv_bfloat16*>(x), dt, A,
+        static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
+        static_cast<__nv_bfloat16*>(y), nheads, headdim, dstate, hpg, ngroups);
+  } else {
+    ssd::step_generic_kernel<float><<<grid, 256, 0, stream>>>(
+        state, static_cast<const float*>(x), dt, A, static_cast<const float*>(B),
+        static_cast<const float*>(C), D, static_cast<float*>(y), nheads, headdim, dstate, hpg,
+        ngroups);
+  }
+#undef SSD_STEP_DISPATCH
+#undef SSD_STEP_FAST
+  return launched();
+}
+
+const char* ssd_status_string(ssd_status s) {
+  switch (s) {
+    case SSD_OK: return "SSD_OK";
+    case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument";
+    case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape or alignment not supported";
+    case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing or too small";
+    case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA launch or runtime failure";
+    case SSD_ERR_DEVICE_TIMEOUT: return "SSD_ERR_DEVICE_TIMEOUT: a kernel's bounded wait expired";
+  }
+  return "unknown ssd_status";
+}
+
+ssd_status ssd_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SSD_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, ssd::g_status, sizeof v) != cudaSuccess) return SSD_ERR_CUDA;
+  if (v == 0) return SSD_OK;
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(ssd::g_status, &zero, sizeof zero) != cudaSuccess) return SSD_ERR_CUDA;
+  return static_cast<ssd_status>(v & 0xffu);
+}
+
+const char* ssd_version(void) { return "ssd-b200 0.1 sm_100a"; }
+
+}  // extern "C"

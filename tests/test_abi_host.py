@@ -1,0 +1,99 @@
+"""Host-only checks of the C ABI (no GPU needed): the library builds and loads, exports every
+function include/ssd.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mamba_ssd_scan_03_b200 as ssd
+from mamba_ssd_scan_03_b200 import build as ssd_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssd_build.build()
+    return ssd.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(ssd.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", ssd.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ssd_[a-z_0-9]+)\b", out))
+    for name in declared_functions():
+        assert name in exported, name
+        getattr(lib, name)  # resolvable through ctypes
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.ssd_status_string(code).decode().startswith(ssd.STATUS[code])
+    assert ssd.version().startswith("ssd-b200")
+
+
+def test_path_selection(lib):
+    # bf16, headdim 64, dstate 128, even heads per group -> tensor cores
+    assert ssd.path(4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16) == ssd.SSD_PATH_TCGEN05
+    assert ssd.path(1, 1 << 20, 24, 64, 128, 1, 256, ssd.SSD_BF16) == ssd.SSD_PATH_TCGEN05
+    assert ssd.path(1, 256, 4, 16, 16, 1, 64, ssd.SSD_F32) == ssd.SSD_PATH_SIMT
+    assert ssd.path(4, 8192, 80, 64, 128, 1, 256, ssd.SSD_F32) == ssd.SSD_PATH_SIMT
+    assert ssd.path(2, 512, 4, 64, 128, 4, 256, ssd.SSD_BF16) == ssd.SSD_PATH_SIMT  # 1 head/group
+    assert ssd.path(2, 512, 4, 64, 128, 2, 256, ssd.SSD_BF16) == ssd.SSD_PATH_TCGEN05
+
+
+def test_workspace_sizes(lib):
+    # tensor-core path: one float32 state per (batch, segment, head) plus a decay per segment
+    ws = ssd.workspace_size(4, 8192, 80, 64, 128, 1, 256)
+    assert ws > 0 and ws % 256 == 0
+    assert ws >= 4 * 80 * 64 * 128 * 4
+    # SIMT path: cumsums + one state per chunk
+    ws0 = ssd.workspace_size(1, 256, 4, 16, 16, 1, 64, ssd.SSD_F32)
+    assert ws0 >= (4 * 4 * 64 + 4 * 4 * 16 * 16) * 4
+    # invalid shapes report 0
+    assert ssd.workspace_size(1, 256, 4, 16, 16, 1, 100, ssd.SSD_F32) == 0
+    assert ssd.workspace_size(1, 256, 3, 16, 16, 2, 64, ssd.SSD_F32) == 0
+
+
+def _scan_call(lib, **kw):
+    args = dict(x=None, dt=None, A=None, B=None, C=None, D=None, init=None, y=None, fin=None,
+                batch=1, seqlen=256, nheads=4, headdim=16, dstate=16, ngroups=1, chunk=64,
+                io=ssd.SSD_F32, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    return lib.ssd_chunk_scan_fwd(*args.values())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(chunk=100), dict(chunk=0), dict(batch=0), dict(seqlen=0), dict(nheads=3, ngroups=2),
+    dict(headdim=0), dict(dstate=-1), dict(io=7),
+    dict(),  # all pointers NULL
+])
+def test_scan_rejects_bad_arguments_on_host(lib, bad):
+    assert _scan_call(lib, **bad) == 1  # SSD_ERR_INVALID_ARG
+
+
+def test_step_rejects_bad_arguments_on_host(lib):
+    assert lib.ssd_step(*([None] * 8), 0, 4, 16, 16, 1, 1, None) == 1
+    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 3, 1, None) == 1
+    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 1, 1, None) == 1  # NULL pointers
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.chunk_scan_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 128),
+                           torch.zeros(1, 4, 1, 128), None, 256)

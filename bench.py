@@ -39,16 +39,18 @@ SCAN_CFG = 2
 DECODE_CFG = 4
 
 
-def scan_bytes(c):
-    """Algorithmic bytes of one scan: every input read once, y written once, init/final state."""
+def scan_bytes(c, y_bytes=4):
+    """Algorithmic bytes of one scan: every input read once, y (float32) written once,
+    init/final state."""
     tok = c["batch"] * c["seqlen"]
     es = 2 if c["io"] == "bf16" else 4
     x = tok * c["nheads"] * c["headdim"] * es
+    y = tok * c["nheads"] * c["headdim"] * y_bytes
     bc = 2 * tok * c["ngroups"] * c["dstate"] * es
     dt = tok * c["nheads"] * 4
     st = c["batch"] * c["nheads"] * c["headdim"] * c["dstate"] * 4
     init = st if c["init"] != "zeros" else 0
-    return 2 * x + bc + dt + 2 * c["nheads"] * 4 + init + st
+    return x + y + bc + dt + 2 * c["nheads"] * 4 + init + st
 
 
 def scan_flops(c):
@@ -57,12 +59,13 @@ def scan_flops(c):
     return c["batch"] * c["seqlen"] * (G * (Q + 1) * N + H * ((Q + 1) * P + 4 * N * P))
 
 
-def step_bytes(c):
+def step_bytes(c, y_bytes=4):
     es = 2
     st = c["batch"] * c["nheads"] * c["headdim"] * c["dstate"] * 4
     x = c["batch"] * c["nheads"] * c["headdim"] * es
+    y = c["batch"] * c["nheads"] * c["headdim"] * y_bytes
     bc = 2 * c["batch"] * c["ngroups"] * c["dstate"] * es
-    return 2 * st + 2 * x + bc + c["batch"] * c["nheads"] * 4 + 2 * c["nheads"] * 4
+    return 2 * st + x + y + bc + c["batch"] * c["nheads"] * 4 + 2 * c["nheads"] * 4
 
 
 def peaks():
@@ -186,7 +189,7 @@ def run_ours(args):
     c = inp["cfg"]
     names = ("x", "dt", "A", "B", "C", "D", "init")
     t = {k: to_dev(inp[k], k in ("x", "B", "C"), dev) for k in names}
-    y = torch.empty_like(t["x"])
+    y = torch.empty(t["x"].shape, dtype=torch.float32, device=dev)  # y in float32
     fin = torch.empty_like(t["init"])
     ws = torch.empty(ssd.workspace_size(c["batch"], c["seqlen"], c["nheads"], c["headdim"],
                                         c["dstate"], c["ngroups"], c["chunk"]),
@@ -268,7 +271,7 @@ def run_ours(args):
     for k in range(n_dec_inputs):  # distinct per-step inputs, cycled
         s = ssd_inputs.decode_step_inputs(dec, k)
         steps_in.append({n: to_dev(s[n], n != "dt", dev) for n in ("x", "dt", "B", "C")})
-    ydec = torch.empty_like(steps_in[0]["x"])
+    ydec = torch.empty(steps_in[0]["x"].shape, dtype=torch.float32, device=dev)
 
     def dec_once(k):
         s = steps_in[k % n_dec_inputs]

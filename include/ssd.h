@@ -20,14 +20,18 @@
  *    memory; anything else is rejected with SSD_ERR_INVALID_ARG before any launch).  The
  *    library never allocates device memory; scratch comes from the caller's workspace.
  *  - Layouts are dense row-major (contiguous):
- *        x, y         [batch, seqlen, nheads, headdim]   io dtype
+ *        x            [batch, seqlen, nheads, headdim]   io dtype
+ *        y            [batch, seqlen, nheads, headdim]   y dtype
  *        dt           [batch, seqlen, nheads]            float32 (used as given, > 0)
  *        A, D         [nheads]                           float32 (A < 0; D may be NULL = 0)
  *        B, C         [batch, seqlen, ngroups, dstate]   io dtype
  *        states       [batch, nheads, headdim, dstate]   float32; element [b,h,p,n] is h[n,p]
  *    Head h reads group g = h / (nheads / ngroups).
- *  - io dtype (x, B, C, y): SSD_F32 or SSD_BF16.  Arithmetic is float32 with float32
- *    accumulation; y is rounded to the io dtype (nearest even).
+ *  - io dtype (x, B, C): SSD_F32 or SSD_BF16.  y dtype: SSD_F32 or equal to the io dtype.
+ *    Arithmetic is float32 with float32 accumulation (tensor-core operands are bf16, split
+ *    into a high and a low bf16 part where a single bf16 would cost accuracy); y is written in
+ *    its dtype, rounded to nearest even.  A bf16 y carries up to half a bf16 ulp of rounding
+ *    (2^-9 relative), so a float32 y is the default of the Python binding.
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument errors are
  *    reported synchronously and nothing is launched.  A launch failure returns
  *    SSD_ERR_CUDA.  Errors found by the kernels themselves (a bounded wait that expired)
@@ -83,8 +87,8 @@ ssd_path ssd_chunk_scan_path(int64_t batch, int64_t seqlen, int nheads, int head
  *   x, dt, A, B, C, D : inputs as above (D may be NULL).
  *   init_state        : [batch, nheads, headdim, dstate] float32, the state before token 0
  *                       (token 0 decays it once); NULL means zeros.
- *   y                 : output [batch, seqlen, nheads, headdim], io dtype; must not overlap
- *                       any input.
+ *   y                 : output [batch, seqlen, nheads, headdim] in y_dtype (SSD_F32 or the io
+ *                       dtype); must not overlap any input.
  *   final_state       : output state after token seqlen-1, float32; NULL = not written.
  *                       May equal init_state (in-place streaming prefill).
  *   chunk             : 64, 128 or 256.  The SIMT path uses it as its block length; the
@@ -102,7 +106,8 @@ ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, co
                               const void* C, const float* D, const float* init_state, void* y,
                               float* final_state, int64_t batch, int64_t seqlen, int nheads,
                               int headdim, int dstate, int ngroups, int chunk, ssd_dtype io,
-                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                              ssd_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
 
 /* The same operation forced onto the float32 SIMT kernels (any supported shape), with its
  * own workspace query.  Used as a second GPU reference and for float32 io. */
@@ -114,7 +119,7 @@ ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* 
                                    const float* init_state, void* y, float* final_state,
                                    int64_t batch, int64_t seqlen, int nheads, int headdim,
                                    int dstate, int ngroups, int chunk, ssd_dtype io,
-                                   void* workspace, size_t workspace_bytes,
+                                   ssd_dtype y_dtype, void* workspace, size_t workspace_bytes,
                                    cudaStream_t stream);
 
 /*
@@ -124,14 +129,15 @@ ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* 
  * "State Space Models (SSM)" (ultralytics.com glossary), section "Come funzionano gli SSM":
  * the recurrent form used during generation, constant memory per token.
  *   state [batch, nheads, headdim, dstate] float32 (read and written once per call);
- *   x, y [batch, nheads, headdim] io dtype; dt [batch, nheads] float32;
+ *   x [batch, nheads, headdim] io dtype; y the same shape in y_dtype (SSD_F32 or io);
+ *   dt [batch, nheads] float32;
  *   B, C [batch, ngroups, dstate] io dtype; A, D [nheads] float32 (D may be NULL).
  *   y must not overlap state or any input.  No workspace, no allocation.
  */
 ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A,
                     const void* B, const void* C, const float* D, void* y, int64_t batch,
                     int nheads, int headdim, int dstate, int ngroups, ssd_dtype io,
-                    cudaStream_t stream);
+                    ssd_dtype y_dtype, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* ssd_status_string(ssd_status s);

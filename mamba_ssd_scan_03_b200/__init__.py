@@ -37,7 +37,7 @@ _lib = None
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 _SHAPE = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32]  # batch .. chunk, io
-_SCAN = [_vp] * 9 + [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
+_SCAN = [_vp] * 9 + [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
 
 
 def load():
@@ -59,7 +59,7 @@ def load():
         fn.restype = _i32
         fn.argtypes = _SCAN
     lib.ssd_step.restype = _i32
-    lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp]
+    lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_status_string.argtypes = [_i32]
     lib.ssd_get_device_status.restype = _i32
@@ -82,11 +82,15 @@ def _check(code, what):
 
 
 def _io(t):
-    if t.dtype == torch.bfloat16:
+    return _code(t.dtype)
+
+
+def _code(dtype):
+    if dtype == torch.bfloat16:
         return SSD_BF16
-    if t.dtype == torch.float32:
+    if dtype == torch.float32:
         return SSD_F32
-    raise TypeError(f"x/B/C must be bfloat16 or float32, got {t.dtype}")
+    raise TypeError(f"tensor dtype must be bfloat16 or float32, got {dtype}")
 
 
 def _ptr(t):
@@ -130,7 +134,7 @@ def path(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io=SSD_BF16):
 
 
 def _scan(entry, simt, x, dt, A, B, C, D, chunk, init_state, want_final, workspace, out,
-          final_out):
+          final_out, y_dtype):
     lib = load()
     _need(x, "x")
     dev = x.device
@@ -143,8 +147,9 @@ def _scan(entry, simt, x, dt, A, B, C, D, chunk, init_state, want_final, workspa
         _need(D, "D", torch.float32, (H,), dev)
     if init_state is not None:
         _need(init_state, "init_state", torch.float32, (Bt, H, P, N), dev)
-    y = out if out is not None else torch.empty_like(x)
-    _need(y, "out", x.dtype, x.shape, dev)
+    y_dtype = out.dtype if out is not None else y_dtype
+    y = out if out is not None else torch.empty(x.shape, dtype=y_dtype, device=dev)
+    _need(y, "out", y_dtype, x.shape, dev)
     fin = None
     if want_final:
         fin = final_out if final_out is not None else torch.empty(
@@ -156,29 +161,31 @@ def _scan(entry, simt, x, dt, A, B, C, D, chunk, init_state, want_final, workspa
     _need(workspace, "workspace", torch.uint8, device=dev)
     with torch.cuda.device(dev):
         rc = entry(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
-                   _ptr(y), _ptr(fin), Bt, L, H, P, N, G, Q, io, _ptr(workspace),
+                   _ptr(y), _ptr(fin), Bt, L, H, P, N, G, Q, io, _code(y_dtype), _ptr(workspace),
                    workspace.numel(), _stream(dev))
     _check(rc, "ssd_chunk_scan_fwd_simt" if simt else "ssd_chunk_scan_fwd")
     return y, fin
 
 
 def chunk_scan_fwd(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
-                   workspace=None, out=None, final_out=None):
+                   workspace=None, out=None, final_out=None, y_dtype=torch.float32):
     """Chunked forward scan.  x [B,L,H,P], dt [B,L,H] f32, A [H] f32, B/C [B,L,G,N],
-    D [H] f32 or None, init_state [B,H,P,N] f32 or None.  Returns (y, final_state)."""
+    D [H] f32 or None, init_state [B,H,P,N] f32 or None.  y is float32 by default (or the io
+    dtype).  Returns (y, final_state)."""
     return _scan(load().ssd_chunk_scan_fwd, False, x, dt, A, B, C, D, chunk, init_state,
-                 want_final, workspace, out, final_out)
+                 want_final, workspace, out, final_out, y_dtype)
 
 
 def chunk_scan_fwd_simt(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
-                        workspace=None, out=None, final_out=None):
+                        workspace=None, out=None, final_out=None, y_dtype=torch.float32):
     """The same operation on the float32 SIMT kernels (second GPU reference)."""
     return _scan(load().ssd_chunk_scan_fwd_simt, True, x, dt, A, B, C, D, chunk, init_state,
-                 want_final, workspace, out, final_out)
+                 want_final, workspace, out, final_out, y_dtype)
 
 
-def step(state, x, dt, A, B, C, D, out=None):
-    """One decode step; updates ``state`` [B,H,P,N] f32 in place and returns y [B,H,P]."""
+def step(state, x, dt, A, B, C, D, out=None, y_dtype=torch.float32):
+    """One decode step; updates ``state`` [B,H,P,N] f32 in place and returns y [B,H,P]
+    (float32 by default, or the io dtype)."""
     lib = load()
     _need(state, "state", torch.float32)
     dev = state.device
@@ -192,11 +199,12 @@ def step(state, x, dt, A, B, C, D, out=None):
     _need(A, "A", torch.float32, (H,), dev)
     if D is not None:
         _need(D, "D", torch.float32, (H,), dev)
-    y = out if out is not None else torch.empty_like(x)
-    _need(y, "out", x.dtype, x.shape, dev)
+    y_dtype = out.dtype if out is not None else y_dtype
+    y = out if out is not None else torch.empty(x.shape, dtype=y_dtype, device=dev)
+    _need(y, "out", y_dtype, x.shape, dev)
     with torch.cuda.device(dev):
         rc = lib.ssd_step(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                          _ptr(y), Bt, H, P, N, G, io, _stream(dev))
+                          _ptr(y), Bt, H, P, N, G, io, _code(y_dtype), _stream(dev))
     _check(rc, "ssd_step")
     return y
 

@@ -127,11 +127,11 @@ __global__ void state_pass_kernel(float* __restrict__ states, const float* __res
 }
 
 // ---- 4. outputs: grid (nchunks, batch*nheads), block 256 -------------------------------------
-template <typename T>
+template <typename T, typename TY>
 __global__ void __launch_bounds__(256) chunk_out_kernel(
     const T* __restrict__ x, const float* __restrict__ dt, const T* __restrict__ Bm,
     const T* __restrict__ Cm, const float* __restrict__ D, const float* __restrict__ cs,
-    const float* __restrict__ states, T* __restrict__ y, int64_t seqlen, int nheads,
+    const float* __restrict__ states, TY* __restrict__ y, int64_t seqlen, int nheads,
     int headdim, int dstate, int ngroups, int chunk, int nchunks) {
   constexpr int TT = 32;  // token tile (rows t and columns s)
   constexpr int NC = 32;  // state slice
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(256) chunk_out_kernel(
         const int64_t tok = c0 + tt + r;
         if (tok < seqlen) {
           const int64_t xi = ((b * seqlen + tok) * nheads + h) * headdim + p;
-          io_traits<T>::store(y, xi, acc[i] + dh * io_traits<T>::load(x, xi));
+          io_traits<TY>::store(y, xi, acc[i] + dh * io_traits<T>::load(x, xi));
         }
       }
     }

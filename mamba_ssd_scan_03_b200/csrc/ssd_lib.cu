@@ -128,25 +128,25 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, ui
 }
 
 constexpr size_t kTcSmem = ssd::tc::kSmemTiles + 1024;
-template <int HQ>
-constexpr size_t seg_state_smem() { return 2 * (2 + HQ) * size_t(ssd::tc::kTile) + 1024; }
+constexpr size_t kSegSmem = 2 * size_t(ssd::tc::kSegStage) + 1024;
 
 ssd_status set_smem_attrs() {
   static ssd_status st = SSD_ERR_CUDA;
   static std::once_flag once;
   std::call_once(once, [] {
     bool ok = true;
-    ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel,
+    ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<float>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
           cudaSuccess;
-    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<4>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(seg_state_smem<4>())) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(seg_state_smem<2>())) == cudaSuccess;
-    for (auto f : {(const void*)ssd::simt::chunk_out_kernel<float>,
-                   (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16>,
+    ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
+          cudaSuccess;
+    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem)) ==
+          cudaSuccess;
+    for (auto f : {(const void*)ssd::simt::chunk_out_kernel<float, float>,
+                   (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16, float>,
+                   (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16, __nv_bfloat16>,
                    (const void*)ssd::simt::chunk_state_kernel<float>,
                    (const void*)ssd::simt::chunk_state_kernel<__nv_bfloat16>})
       ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
@@ -162,6 +162,7 @@ ssd_status launched() {
 }
 
 struct ScanArgs {
+  ssd_dtype ydt;
   const void *x, *B, *C;
   const float *dt, *A, *D, *init;
   void* y;
@@ -178,14 +179,17 @@ ssd_status validate_scan(const Shape& s, const ScanArgs& a, size_t need) {
     if (!is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
   for (const void* p : {(const void*)a.D, (const void*)a.init, (const void*)a.fin})
     if (p && !is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  if (a.ydt != SSD_F32 && a.ydt != s.io) return SSD_ERR_INVALID_ARG;
   const size_t es = s.io == SSD_BF16 ? 2 : 4;
+  const size_t ey = a.ydt == SSD_BF16 ? 2 : 4;
   const size_t nx = size_t(s.batch) * s.seqlen * s.nheads * s.headdim * es;
+  const size_t ny = size_t(s.batch) * s.seqlen * s.nheads * s.headdim * ey;
   const size_t nbc = size_t(s.batch) * s.seqlen * s.ngroups * s.dstate * es;
   const size_t ndt = size_t(s.batch) * s.seqlen * s.nheads * 4;
   const size_t nst = size_t(s.batch) * s.nheads * s.headdim * s.dstate * 4;
-  if (overlaps(a.y, nx, a.x, nx) || overlaps(a.y, nx, a.B, nbc) || overlaps(a.y, nx, a.C, nbc) ||
-      overlaps(a.y, nx, a.dt, ndt) || overlaps(a.y, nx, a.init, nst) ||
-      overlaps(a.y, nx, a.fin, nst))
+  if (overlaps(a.y, ny, a.x, nx) || overlaps(a.y, ny, a.B, nbc) || overlaps(a.y, ny, a.C, nbc) ||
+      overlaps(a.y, ny, a.dt, ndt) || overlaps(a.y, ny, a.init, nst) ||
+      overlaps(a.y, ny, a.fin, nst))
     return SSD_ERR_INVALID_ARG;
   if (a.fin && a.fin != a.init &&
       (overlaps(a.fin, nst, a.init, nst) || overlaps(a.fin, nst, a.x, nx) ||
@@ -195,14 +199,14 @@ ssd_status validate_scan(const Shape& s, const ScanArgs& a, size_t need) {
     if (!a.ws || a.ws_bytes < need || (reinterpret_cast<uintptr_t>(a.ws) & 255u) ||
         !is_device_ptr(a.ws))
       return SSD_ERR_WORKSPACE;
-    if (overlaps(a.ws, need, a.y, nx) || overlaps(a.ws, need, a.x, nx) ||
+    if (overlaps(a.ws, need, a.y, ny) || overlaps(a.ws, need, a.x, nx) ||
         overlaps(a.ws, need, a.init, nst) || overlaps(a.ws, need, a.fin, nst))
       return SSD_ERR_INVALID_ARG;
   }
   return SSD_OK;
 }
 
-template <typename T>
+template <typename T, typename TY>
 ssd_status run_simt(const Shape& s, const ScanArgs& a) {
   const int64_t nchunks = (s.seqlen + s.chunk - 1) / s.chunk;
   float* cs = static_cast<float*>(a.ws);
@@ -223,9 +227,9 @@ ssd_status run_simt(const Shape& s, const ScanArgs& a) {
       states, cs, a.init, a.fin, s.batch, s.nheads, s.headdim, s.dstate, s.chunk, int(nchunks));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   const size_t sm_out = (3072 + 64 * size_t(s.headdim)) * sizeof(float);
-  ssd::simt::chunk_out_kernel<T><<<grid, 256, sm_out, a.stream>>>(
+  ssd::simt::chunk_out_kernel<T, TY><<<grid, 256, sm_out, a.stream>>>(
       static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), static_cast<const T*>(a.C),
-      a.D, cs, states, static_cast<T*>(a.y), s.seqlen, s.nheads, s.headdim, s.dstate,
+      a.D, cs, states, static_cast<TY*>(a.y), s.seqlen, s.nheads, s.headdim, s.dstate,
       s.ngroups, s.chunk, int(nchunks));
   return launched();
 }
@@ -242,25 +246,29 @@ ssd_status run_tc(const Shape& s, const ScanArgs& a) {
       !make_map(&mc, a.C, GN, s.seqlen, s.batch))
     return SSD_ERR_CUDA;
   const int hpg = s.nheads / s.ngroups;
-  if (hpg % 4 == 0) {
-    const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 4));
-    ssd::tc::seg_state_kernel<4><<<grid, 128, seg_state_smem<4>(), a.stream>>>(
-        mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
-  } else {
-    const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-    ssd::tc::seg_state_kernel<2><<<grid, 128, seg_state_smem<2>(), a.stream>>>(
-        mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
-  }
+  const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
+  ssd::tc::seg_state_kernel<<<grid, 256, kSegSmem, a.stream>>>(
+      mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;
   ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
       seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-  ssd::tc::chunk_out_kernel<<<grid, 128, kTcSmem, a.stream>>>(
-      mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<__nv_bfloat16*>(a.y), s.seqlen,
-      s.nheads, hpg, sg);
+  if (a.ydt == SSD_F32)
+    ssd::tc::chunk_out_kernel<float><<<grid, 256, kTcSmem, a.stream>>>(
+        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<float*>(a.y), s.seqlen, s.nheads,
+        hpg, sg);
+  else
+    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, 256, kTcSmem, a.stream>>>(
+        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<__nv_bfloat16*>(a.y), s.seqlen,
+        s.nheads, hpg, sg);
   return launched();
+}
+
+ssd_status run_simt_any(const Shape& s, const ScanArgs& a) {
+  if (s.io == SSD_F32) return run_simt<float, float>(s, a);
+  if (a.ydt == SSD_F32) return run_simt<__nv_bfloat16, float>(s, a);
+  return run_simt<__nv_bfloat16, __nv_bfloat16>(s, a);
 }
 
 bool tc_pointers_ok(const ScanArgs& a) {
@@ -297,10 +305,11 @@ ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, co
                               const void* C, const float* D, const float* init_state, void* y,
                               float* final_state, int64_t batch, int64_t seqlen, int nheads,
                               int headdim, int dstate, int ngroups, int chunk, ssd_dtype io,
-                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                              ssd_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
   const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
-  const ScanArgs a{x, B, C, dt, A, D, init_state, y, final_state, workspace, workspace_bytes,
-                   stream};
+  const ScanArgs a{y_dtype, x, B, C, dt, A, D, init_state, y, final_state, workspace,
+                   workspace_bytes, stream};
   ssd_status st = check_shape(s);
   if (st != SSD_OK) return st;
   const bool tc = tc_shape_ok(s);
@@ -312,7 +321,7 @@ ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, co
     if (!tc_pointers_ok(a)) return SSD_ERR_UNSUPPORTED;
     return run_tc(s, a);
   }
-  return io == SSD_BF16 ? run_simt<__nv_bfloat16>(s, a) : run_simt<float>(s, a);
+  return run_simt_any(s, a);
 }
 
 ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* A,
@@ -320,26 +329,27 @@ ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* 
                                    const float* init_state, void* y, float* final_state,
                                    int64_t batch, int64_t seqlen, int nheads, int headdim,
                                    int dstate, int ngroups, int chunk, ssd_dtype io,
-                                   void* workspace, size_t workspace_bytes,
+                                   ssd_dtype y_dtype, void* workspace, size_t workspace_bytes,
                                    cudaStream_t stream) {
   const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
-  const ScanArgs a{x, B, C, dt, A, D, init_state, y, final_state, workspace, workspace_bytes,
-                   stream};
+  const ScanArgs a{y_dtype, x, B, C, dt, A, D, init_state, y, final_state, workspace,
+                   workspace_bytes, stream};
   ssd_status st = check_shape(s);
   if (st != SSD_OK) return st;
   if (!simt_supported(s)) return SSD_ERR_UNSUPPORTED;
   st = validate_scan(s, a, simt_workspace(s));
   if (st != SSD_OK) return st;
   if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
-  return io == SSD_BF16 ? run_simt<__nv_bfloat16>(s, a) : run_simt<float>(s, a);
+  return run_simt_any(s, a);
 }
 
 ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A,
                     const void* B, const void* C, const float* D, void* y, int64_t batch,
                     int nheads, int headdim, int dstate, int ngroups, ssd_dtype io,
-                    cudaStream_t stream) {
+                    ssd_dtype y_dtype, cudaStream_t stream) {
   if (batch <= 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
-      nheads % ngroups != 0 || (io != SSD_F32 && io != SSD_BF16))
+      nheads % ngroups != 0 || (io != SSD_F32 && io != SSD_BF16) ||
+      (y_dtype != SSD_F32 && y_dtype != io))
     return SSD_ERR_INVALID_ARG;
   if (batch * nheads > (int64_t(1) << 31) - 1) return SSD_ERR_UNSUPPORTED;
   for (const void* p : {(const void*)state, x, (const void*)dt, (const void*)A, B, C,
@@ -349,9 +359,10 @@ ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A
   const size_t es = io == SSD_BF16 ? 2 : 4;
   const size_t nst = size_t(batch) * nheads * headdim * dstate * 4;
   const size_t nx = size_t(batch) * nheads * headdim * es;
+  const size_t ny = size_t(batch) * nheads * headdim * (y_dtype == SSD_BF16 ? 2 : 4);
   const size_t nbc = size_t(batch) * ngroups * dstate * es;
-  if (overlaps(y, nx, state, nst) || overlaps(y, nx, x, nx) || overlaps(y, nx, B, nbc) ||
-      overlaps(y, nx, C, nbc) || overlaps(state, nst, x, nx) || overlaps(state, nst, B, nbc) ||
+  if (overlaps(y, ny, state, nst) || overlaps(y, ny, x, nx) || overlaps(y, ny, B, nbc) ||
+      overlaps(y, ny, C, nbc) || overlaps(state, nst, x, nx) || overlaps(state, nst, B, nbc) ||
       overlaps(state, nst, C, nbc))
     return SSD_ERR_INVALID_ARG;
   const int hpg = nheads / ngroups;
@@ -359,31 +370,32 @@ ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A
   const bool fast = dstate == 128 && headdim % 8 == 0 && aligned16(state) &&
                     (headdim / 8 == 1 || headdim / 8 == 2 || headdim / 8 == 4 ||
                      headdim / 8 == 8 || headdim / 8 == 16);
-#define SSD_STEP_FAST(T, RPW)                                                              \
-  ssd::step_n128_kernel<T, RPW><<<grid, 256, 0, stream>>>(                                 \
+#define SSD_STEP_FAST(T, TY, RPW)                                                          \
+  ssd::step_n128_kernel<T, TY, RPW><<<grid, 256, 0, stream>>>(                             \
       state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B),                    \
-      static_cast<const T*>(C), D, static_cast<T*>(y), nheads, hpg, ngroups)
-#define SSD_STEP_DISPATCH(T)                          \
+      static_cast<const T*>(C), D, static_cast<TY*>(y), nheads, hpg, ngroups)
+#define SSD_STEP_DISPATCH(T, TY)                      \
   switch (headdim / 8) {                              \
-    case 1: SSD_STEP_FAST(T, 1); break;               \
-    case 2: SSD_STEP_FAST(T, 2); break;               \
-    case 4: SSD_STEP_FAST(T, 4); break;               \
-    case 8: SSD_STEP_FAST(T, 8); break;               \
-    default: SSD_STEP_FAST(T, 16); break;             \
+    case 1: SSD_STEP_FAST(T, TY, 1); break;           \
+    case 2: SSD_STEP_FAST(T, TY, 2); break;           \
+    case 4: SSD_STEP_FAST(T, TY, 4); break;           \
+    case 8: SSD_STEP_FAST(T, TY, 8); break;           \
+    default: SSD_STEP_FAST(T, TY, 16); break;         \
   }
+#define SSD_STEP_GENERIC(T, TY)                                                            \
+  ssd::step_generic_kernel<T, TY><<<grid, 256, 0, stream>>>(                               \
+      state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B),                    \
+      static_cast<const T*>(C), D, static_cast<TY*>(y), nheads, headdim, dstate, hpg, ngroups)
   if (fast) {
-    if (io == SSD_BF16) { SSD_STEP_DISPATCH(__nv_bfloat16) } else { SSD_STEP_DISPATCH(float) }
-  } else if (io == SSD_BF16) {
-    ssd::step_generic_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        state, static_cast<const __nv_bfloat16*>(x), dt, A,
-        static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
-        static_cast<__nv_bfloat16*>(y), nheads, headdim, dstate, hpg, ngroups);
+    if (io == SSD_F32) { SSD_STEP_DISPATCH(float, float) }
+    else if (y_dtype == SSD_F32) { SSD_STEP_DISPATCH(__nv_bfloat16, float) }
+    else { SSD_STEP_DISPATCH(__nv_bfloat16, __nv_bfloat16) }
   } else {
-    ssd::step_generic_kernel<float><<<grid, 256, 0, stream>>>(
-        state, static_cast<const float*>(x), dt, A, static_cast<const float*>(B),
-        static_cast<const float*>(C), D, static_cast<float*>(y), nheads, headdim, dstate, hpg,
-        ngroups);
+    if (io == SSD_F32) { SSD_STEP_GENERIC(float, float); }
+    else if (y_dtype == SSD_F32) { SSD_STEP_GENERIC(__nv_bfloat16, float); }
+    else { SSD_STEP_GENERIC(__nv_bfloat16, __nv_bfloat16); }
   }
+#undef SSD_STEP_GENERIC
 #undef SSD_STEP_DISPATCH
 #undef SSD_STEP_FAST
   return launched();

@@ -14,11 +14,11 @@ namespace ssd {
 
 // Fast path: dstate == 128 (one float4 of the row per lane, a warp per row), block of 8 warps
 // per (b, h), RPW rows per warp issued back to back so each lane has RPW 16-byte loads in flight.
-template <typename T, int RPW>
+template <typename T, typename TY, int RPW>
 __global__ void __launch_bounds__(256) step_n128_kernel(
     float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
-    const float* __restrict__ D, T* __restrict__ y, int nheads, int heads_per_group,
+    const float* __restrict__ D, TY* __restrict__ y, int nheads, int heads_per_group,
     int ngroups) {
   constexpr int N = 128;
   constexpr int P = 8 * RPW;
@@ -65,16 +65,16 @@ __global__ void __launch_bounds__(256) step_n128_kernel(
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
       if (lane == r) { out = acc[r]; xo = xv[r]; }
-    io_traits<T>::store(y, bh * P + p0 + lane, out + dh * xo);
+    io_traits<TY>::store(y, bh * P + p0 + lane, out + dh * xo);
   }
 }
 
 // General shapes: a warp per (p) row, lanes stride over dstate.
-template <typename T>
+template <typename T, typename TY>
 __global__ void __launch_bounds__(256) step_generic_kernel(
     float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
-    const float* __restrict__ D, T* __restrict__ y, int nheads, int headdim, int dstate,
+    const float* __restrict__ D, TY* __restrict__ y, int nheads, int headdim, int dstate,
     int heads_per_group, int ngroups) {
   const int64_t bh = blockIdx.x;
   const int h = int(bh % nheads);
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(256) step_generic_kernel(
       acc += io_traits<T>::load(Cm, bc + n) * sv;
     }
     acc = warp_sum(acc);
-    if (lane == 0) io_traits<T>::store(y, bh * headdim + p, acc + dh * xv);
+    if (lane == 0) io_traits<TY>::store(y, bh * headdim + p, acc + dh * xv);
   }
 }
 

@@ -41,17 +41,20 @@ struct Seg {
   int nseg;      // segments per sequence
 };
 
-// 128-thread inclusive scan; returns the prefix and writes the block total to *total.
-__device__ __forceinline__ float block_scan128(float v, float* scratch4, float* total) {
+// Inclusive scan over the 128 threads of one half of a 256-thread CTA (warps 0-3 form half 0,
+// warps 4-7 half 1).  Returns the prefix and writes the half's total to *total.  Every thread
+// of the CTA must call it (it synchronises the CTA).
+__device__ __forceinline__ float half_scan128(float v, float* scratch8, float* total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   v = warp_inclusive_scan(v);
-  if (lane == 31) scratch4[warp] = v;
+  if (lane == 31) scratch8[warp] = v;
   __syncthreads();
+  const int w0 = warp & ~3;
   float off = 0.f, tot = 0.f;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
-    const float s = scratch4[w];
-    off += (w < warp) ? s : 0.f;
+    const float s = scratch8[w0 + w];
+    off += (w0 + w < warp) ? s : 0.f;
     tot += s;
   }
   __syncthreads();
@@ -59,8 +62,8 @@ __device__ __forceinline__ float block_scan128(float v, float* scratch4, float* 
   return v + off;
 }
 
-// Wait until every outstanding async op a CTA started has finished (bounded, used only on
-// the abort path so that no copy or MMA is still writing when the CTA leaves).
+// Wait (bounded) for a phase of an mbarrier; used only on the abort path so that no copy or
+// MMA is still writing shared memory or TMEM when the CTA leaves.
 __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (!mbar_test(bar, parity)) {
@@ -68,33 +71,42 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Split a float pair into bf16 high parts and the bf16 rounding of the remainders.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  lo = pack_bf16x2(a - bf16lo(hi), b - bf16hi(hi));
+}
+
 // =============================================================================================
-// seg_state: grid = batch * nseg * (nheads / HQ), block = 128 threads.
-// Shared memory per stage: B tile (2 x 16 KB, n halves), x tiles (HQ x 16 KB) -- two stages.
-// TMEM: 64*HQ columns, lane n / column (h, p) = S_seg[n, (h, p)].
+// seg_state: grid = batch * nseg * (nheads / 2), block = 256 threads: thread (row = tid % 128,
+// head j = tid / 128) owns token row `row` of head j's x tile.  Per stage (two stages):
+//   B tile (2 x 16 KB, n halves) | X'hi (2 heads x 16 KB) | X'lo (2 heads x 16 KB)
+// X' = w * x is split into a bf16 high part (written over x) and a bf16 low part, and both go
+// through the tensor core, so the segment state carries ~16 significant bits of X'.
+// TMEM: 128 columns, lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
-template <int HQ>
-__global__ void __launch_bounds__(128, 1) seg_state_kernel(
+constexpr uint32_t kSegStage = 6 * kTile;
+
+__global__ void __launch_bounds__(256, 1) seg_state_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const float* __restrict__ dt, const float* __restrict__ A, float* __restrict__ seg_states,
     float* __restrict__ seg_decay, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
-  constexpr uint32_t kStage = 2 * kTile + HQ * kTile;
-  constexpr uint32_t kCols = (64 * HQ < 32) ? 32 : 64 * HQ;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   __shared__ uint64_t full_bar[2], mma_bar[2];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float scan_scratch[4];
+  __shared__ float scan_scratch[8];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
-  const int nq = nheads / HQ;
+  const int row = tid & 127, j = tid >> 7, warp = tid >> 5;
+  const int npair = nheads / 2;
   const int unit = blockIdx.x;
-  const int q = unit % nq;
-  const int seg = (unit / nq) % sg.nseg;
-  const int b = unit / (nq * sg.nseg);
-  const int h0 = q * HQ;
+  const int hp = unit % npair;
+  const int seg = (unit / npair) % sg.nseg;
+  const int b = unit / (npair * sg.nseg);
+  const int h0 = hp * 2;
   const int g = h0 / heads_per_group;
   const int blk0 = seg * sg.seg_blks;
   const int nb = min(sg.nblk, blk0 + sg.seg_blks) - blk0;
@@ -106,32 +118,27 @@ __global__ void __launch_bounds__(128, 1) seg_state_kernel(
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_b);
   }
-  if (tid < 32) tmem_alloc(&tmem_base_sh, kCols);
+  if (warp == 0) tmem_alloc(&tmem_base_sh, 128);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-
   volatile int* abort_v = &abort_flag;
   uint32_t n_loads[2] = {0, 0}, n_commits[2] = {0, 0};  // thread 0's issue counts per stage
-  auto issue_loads = [&](int i, int stage) {  // block i of the walk (reverse order)
+
+  auto issue_loads = [&](int i, int stage) {  // block i of the walk (last block first)
     const int blk = blk0 + nb - 1 - i;
-    uint8_t* st = smem + stage * kStage;
+    uint8_t* st = smem + stage * kSegStage;
     ++n_loads[stage];
-    mbar_arrive_expect_tx(&full_bar[stage], kStage);
+    mbar_arrive_expect_tx(&full_bar[stage], 4 * kTile);
     tma_load_3d(st, &tm_b, &full_bar[stage], g * kN, blk * kBlk, b);
     tma_load_3d(st + kTile, &tm_b, &full_bar[stage], g * kN + 64, blk * kBlk, b);
-    for (int j = 0; j < HQ; ++j)
-      tma_load_3d(st + (2 + j) * kTile, &tm_x, &full_bar[stage], (h0 + j) * kP, blk * kBlk, b);
+    tma_load_3d(st + 2 * kTile, &tm_x, &full_bar[stage], h0 * kP, blk * kBlk, b);
+    tma_load_3d(st + 3 * kTile, &tm_x, &full_bar[stage], (h0 + 1) * kP, blk * kBlk, b);
   };
 
-  float run[HQ];  // log2-decay of the blocks after the current one, within the segment
-#pragma unroll
-  for (int j = 0; j < HQ; ++j) run[j] = 0.f;
-  float Alog[HQ];
-#pragma unroll
-  for (int j = 0; j < HQ; ++j) Alog[j] = A[h0 + j] * kLog2e;
-
+  float run = 0.f;  // log2-decay of the blocks after the current one, within the segment
+  const float Alog = A[h0 + j] * kLog2e;
   if (tid == 0) issue_loads(0, 0);
   bool ok = true;
   for (int i = 0; i < nb; ++i) {
@@ -142,35 +149,28 @@ __global__ void __launch_bounds__(128, 1) seg_state_kernel(
       if (i >= 1) ok = mbar_wait(&mma_bar[stage ^ 1], ((i - 1) >> 1) & 1, abort_v, 11);
       if (ok) issue_loads(i + 1, stage ^ 1);
     }
-    // suffix sums within the block: w_t = exp(sum_{k>t, k in segment} a_k) * dt_t
-    const int64_t tok = int64_t(blk) * kBlk + tid;
-    float w[HQ];
-#pragma unroll
-    for (int j = 0; j < HQ; ++j) {
-      const float d = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0 + j] : 0.f;
-      const float a = d * Alog[j];
-      float tot;
-      const float incl = block_scan128(a, scan_scratch, &tot);
-      w[j] = ex2(tot - incl + run[j]) * d;  // tot - incl = sum over k > t in this block
-      run[j] += tot;
-    }
+    // w_t = exp(sum_{k > t, k in segment} a_k) * dt_t
+    const int64_t tok = int64_t(blk) * kBlk + row;
+    const float d = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0 + j] : 0.f;
+    float tot;
+    const float incl = half_scan128(d * Alog, scan_scratch, &tot);
+    const float w = ex2(tot - incl + run) * d;
+    run += tot;
     ok = ok && mbar_wait(&full_bar[stage], (i >> 1) & 1, abort_v, 12);
     if (ok) {
-      // scale row `tid` of each x tile in place: X' = w * x
-      uint8_t* st = smem + stage * kStage;
+      uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
+      uint8_t* lr = smem + stage * kSegStage + (4 + j) * kTile;
 #pragma unroll
-      for (int j = 0; j < HQ; ++j) {
-        uint8_t* row = st + (2 + j) * kTile;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4* pch = reinterpret_cast<uint4*>(row + swz(tid, c));
-          uint4 v = *pch;
-          v.x = pack_bf16x2(bf16lo(v.x) * w[j], bf16hi(v.x) * w[j]);
-          v.y = pack_bf16x2(bf16lo(v.y) * w[j], bf16hi(v.y) * w[j]);
-          v.z = pack_bf16x2(bf16lo(v.z) * w[j], bf16hi(v.z) * w[j]);
-          v.w = pack_bf16x2(bf16lo(v.w) * w[j], bf16hi(v.w) * w[j]);
-          *pch = v;
-        }
+      for (int c = 0; c < 8; ++c) {
+        uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
+        const uint4 v = *ph;
+        uint4 hi, lo;
+        split2(bf16lo(v.x) * w, bf16hi(v.x) * w, hi.x, lo.x);
+        split2(bf16lo(v.y) * w, bf16hi(v.y) * w, hi.y, lo.y);
+        split2(bf16lo(v.z) * w, bf16hi(v.z) * w, hi.z, lo.z);
+        split2(bf16lo(v.w) * w, bf16hi(v.w) * w, hi.w, lo.w);
+        *ph = hi;
+        *reinterpret_cast<uint4*>(lr + swz(row, c)) = lo;
       }
       fence_proxy_async_smem();
     }
@@ -178,13 +178,14 @@ __global__ void __launch_bounds__(128, 1) seg_state_kernel(
     if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t sb = smem_u32(smem + stage * kStage);
-      const uint32_t idesc = idesc_bf16(128, 64 * HQ, 1, 1);
+      const uint32_t sb = smem_u32(smem + stage * kSegStage);
+      const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
 #pragma unroll
       for (int k = 0; k < kBlk / 16; ++k) {
-        const uint64_t ad = sdesc(sb + k * 2048, kTile, 1024);          // B^T: M = n
-        const uint64_t bd = sdesc(sb + 2 * kTile + k * 2048, kTile, 1024);  // X': N = (h,p)
-        mma_ss(tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+        const uint64_t ad = sdesc(sb + k * 2048, kTile, 1024);               // B^T: M = n
+        mma_ss(tmem, ad, sdesc(sb + 2 * kTile + k * 2048, kTile, 1024), idesc,
+               (i > 0 || k > 0) ? 1u : 0u);                                   // X'hi
+        mma_ss(tmem, ad, sdesc(sb + 4 * kTile + k * 2048, kTile, 1024), idesc, 1u);  // X'lo
       }
       mma_commit(&mma_bar[stage]);
       ++n_commits[stage];
@@ -205,43 +206,36 @@ __global__ void __launch_bounds__(128, 1) seg_state_kernel(
     __syncthreads();
   } else {
     tc_fence_after();
-    // epilogue: lane n = tid, column (j, p)
-    const int n = tid;
-    const uint32_t lane_addr = tmem + (uint32_t(tid & ~31) << 16);
+    // epilogue: lane n = row, columns of head j
+    const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + j * 64;
+    float* out = seg_states + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP) * kN + row;
 #pragma unroll
-    for (int j = 0; j < HQ; ++j) {
-      float* out = seg_states +
-                   (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP) * kN + n;
+    for (int pc = 0; pc < 4; ++pc) {
+      uint32_t r[16];
+      tmem_ld16(lane_addr + pc * 16, r);
+      tmem_wait_ld();
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        uint32_t r[16];
-        tmem_ld16(lane_addr + j * 64 + pc * 16, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) out[(pc * 16 + e) * kN] = nb > 0 ? __uint_as_float(r[e]) : 0.f;
-      }
+      for (int e = 0; e < 16; ++e) out[(pc * 16 + e) * kN] = nb > 0 ? __uint_as_float(r[e]) : 0.f;
     }
-    if (tid < HQ) {
-      float v = 0.f;
-#pragma unroll
-      for (int j = 0; j < HQ; ++j) v = (tid == j) ? run[j] : v;
-      seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + tid] = v;
-    }
+    if (row == 0) seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + j] = run;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid < 32) tmem_free(tmem, kCols);
+  if (warp == 0) tmem_free(tmem, 128);
 }
 
 // =============================================================================================
 // seg_scan: one thread per state element; H_in(0) = init, H_in(s+1) = 2^decay(s) H_in(s) + S(s).
 // seg_states is overwritten in place with H_in; final_state receives the state after the last
 // segment (it may alias init_state: each element is read before it is written, by one thread).
+// Segments are processed eight at a time so that eight independent loads are in flight.
 // =============================================================================================
-__global__ void seg_scan_kernel(float* __restrict__ seg_states,
-                                const float* __restrict__ seg_decay, const float* init_state,
-                                float* final_state, int batch, int nheads, int nseg) {
+__global__ void __launch_bounds__(256) seg_scan_kernel(float* __restrict__ seg_states,
+                                                       const float* __restrict__ seg_decay,
+                                                       const float* init_state,
+                                                       float* final_state, int batch,
+                                                       int nheads, int nseg) {
   const int64_t per_bh = int64_t(kP) * kN;
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= int64_t(batch) * nheads * per_bh) return;
@@ -249,45 +243,83 @@ __global__ void seg_scan_kernel(float* __restrict__ seg_states,
   const int h = int(bh % nheads);
   const int64_t b = bh / nheads;
   float run = init_state ? init_state[e] : 0.f;
-  for (int s = 0; s < nseg; ++s) {
-    float* slot = seg_states + ((b * nseg + s) * nheads + h) * per_bh + pn;
-    const float v = *slot;
-    *slot = run;
-    run = fmaf(ex2(seg_decay[(b * nseg + s) * nheads + h]), run, v);
+  const int64_t stride = int64_t(nheads) * per_bh;
+  float* base = seg_states + (b * nseg * nheads + h) * per_bh + pn;
+  const float* dbase = seg_decay + b * nseg * nheads + h;
+  for (int s0 = 0; s0 < nseg; s0 += 8) {
+    float v[8], dcy[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (s0 + i < nseg) {
+        v[i] = base[(s0 + i) * stride];
+        dcy[i] = dbase[(s0 + i) * nheads];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (s0 + i < nseg) {
+        base[(s0 + i) * stride] = run;
+        run = fmaf(ex2(dcy[i]), run, v[i]);
+      }
+    }
   }
   if (final_state) final_state[e] = run;
 }
 
 // =============================================================================================
-// chunk_out: grid = batch * nseg * (nheads / 2), block = 128 threads (thread t <-> token row t
-// of a block, and <-> state row n for the state passes).  Shared memory (1024-aligned):
-//   sC  2 x 16 KB   C tile, K-major (rows t), n halves
-//   sB  2 x 16 KB   B tile, rows s, n halves: K-major for G = C B^T, MN-major for B^T X'
-//   sX  2 x 16 KB   x tiles of the two heads (rows t, 64 p): MN-major; scaled in place to X'
-//   sM  2 x 32 KB   masked tiles of the two heads, K-major (rows t, s halves)
-//   sH  2 x 16 KB   bf16 copy of the entering state of the two heads (rows n, 64 p): MN-major
+// chunk_out: grid = batch * nseg * (nheads / 2), block = 256 threads.  Thread (row = tid % 128,
+// half = tid / 128): token row `row` of a block (and state row n = row for the state passes);
+// `half` selects the head (state pass, epilogue) or the 64-column half of G (masks).
+// Shared memory (1024-aligned, 10 x 16 KB):
+//   sC   2 tiles  C, K-major (rows t), n halves
+//   sB   2 tiles  B, rows s, n halves: K-major for G = C B^T, MN-major for B^T X'
+//   sX   2 tiles  x of the two heads (rows t, 64 p), MN-major; scaled in place to X'
+//   sHh  2 tiles  bf16 high part of the entering state of the two heads (rows n, 64 p)
+//   sHl  2 tiles  bf16 low part (the state's rounding remainder), same layout
 // TMEM (512 columns): [0,128) running state H (head, p) | [128,256) diagonal accumulators |
-//                     [256,384) off-diagonal accumulators C H | [384,512) G = C B^T.
+//   [256,384) off-diagonal accumulators C H | [384,512) G = C B^T, overwritten in place, one
+//   head at a time, by that head's masked tile as bf16 high and low parts, which the diagonal
+//   MMAs read as their A operand.
 // =============================================================================================
-constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 4 * kTile, kOffM = 6 * kTile,
-                   kOffH = 10 * kTile, kSmemTiles = 12 * kTile;
+constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 4 * kTile, kOffHh = 6 * kTile,
+                   kOffHl = 8 * kTile, kSmemTiles = 10 * kTile;
 
-__global__ void __launch_bounds__(128, 1) chunk_out_kernel(
+template <typename TY> struct yout;
+template <> struct yout<float> {
+  static __device__ __forceinline__ void store16(float* p, const float (&v)[16]) {
+    float4* q = reinterpret_cast<float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+};
+template <> struct yout<__nv_bfloat16> {
+  static __device__ __forceinline__ void store16(__nv_bfloat16* p, const float (&v)[16]) {
+    uint4* q = reinterpret_cast<uint4*>(p);
+    q[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                      pack_bf16x2(v[6], v[7]));
+    q[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                      pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+  }
+};
+
+template <typename TY>
+__global__ void __launch_bounds__(256, 1) chunk_out_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ dt,
     const float* __restrict__ A, const float* __restrict__ D, const float* __restrict__ h_in,
-    __nv_bfloat16* __restrict__ y, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
+    TY* __restrict__ y, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   __shared__ uint64_t tma_bar, mma_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ float cs_sh[2][kBlk], dt_sh[2][kBlk], v_sh[2][kBlk];
-  __shared__ float scan_scratch[4];
+  __shared__ float scan_scratch[8];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int row = tid & 127, half = tid >> 7;
   const int npair = nheads / 2;
   const int unit = blockIdx.x;
   const int hp = unit % npair;
@@ -307,33 +339,30 @@ __global__ void __launch_bounds__(128, 1) chunk_out_kernel(
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_c);
   }
-  if (tid < 32) tmem_alloc(&tmem_base_sh, 512);
+  if (warp == 0) tmem_alloc(&tmem_base_sh, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const uint32_t tH = tmem, tD = tmem + 128, tO = tmem + 256, tG = tmem + 384;
-  const uint32_t lane_off = uint32_t(warp * 32) << 16;  // this warp's TMEM lane quarter
+  const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;  // this warp's TMEM lane quarter
   const uint32_t sbase = smem_u32(smem);
 
-  // entering state of the segment -> TMEM (lane n = tid, column (head, p))
+  // entering state of the segment -> TMEM (lane n = row, columns of head `half`)
   {
-    const int n = tid;
+    const float* src =
+        h_in + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + half) * kP) * kN + row;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float* src = h_in + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP) * kN + n;
+    for (int pc = 0; pc < 4; ++pc) {
+      uint32_t r[16];
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        uint32_t r[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(src[(pc * 16 + e) * kN]);
-        tmem_st16(tH + lane_off + j * 64 + pc * 16, r);
-      }
+      for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(src[(pc * 16 + e) * kN]);
+      tmem_st16(tH + lane_off + half * 64 + pc * 16, r);
     }
     tmem_wait_st();
   }
-  const float Alog0 = A[h0] * kLog2e, Alog1 = A[h0 + 1] * kLog2e;
-  const float Dh0 = D ? D[h0] : 0.f, Dh1 = D ? D[h0 + 1] : 0.f;
+  const float Alog = A[h0 + half] * kLog2e;
+  const float Dh = D ? D[h0 + half] : 0.f;
   uint32_t tma_phase = 0, mma_phase = 0;
   bool ok = true;
   volatile int* abort_v = &abort_flag;
@@ -352,20 +381,16 @@ __global__ void __launch_bounds__(128, 1) chunk_out_kernel(
       tma_load_3d(smem + kOffX, &tm_x, &tma_bar, h0 * kP, int(t0), b);
       tma_load_3d(smem + kOffX + kTile, &tm_x, &tma_bar, (h0 + 1) * kP, int(t0), b);
     }
-    // within-block log2 cumsums, per head; v_s = exp(cs_r(s) - cs_s) dt_s, r(s) = s | 15
-    const int64_t tok = t0 + tid;
+    // within-block log2 cumsums of head `half`; v_s = exp(cs_r(s) - cs_s) dt_s, r(s) = s | 15
+    const int64_t tok = t0 + row;
     {
-      const float d0 = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0] : 0.f;
-      const float d1 = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0 + 1] : 0.f;
+      const float d = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0 + half] : 0.f;
       float tot;
-      const float c0 = block_scan128(d0 * Alog0, scan_scratch, &tot);
-      const float c1 = block_scan128(d1 * Alog1, scan_scratch, &tot);
-      cs_sh[0][tid] = c0; cs_sh[1][tid] = c1;
-      dt_sh[0][tid] = d0; dt_sh[1][tid] = d1;
+      const float c = half_scan128(d * Alog, scan_scratch, &tot);
+      cs_sh[half][row] = c;
+      dt_sh[half][row] = d;
       __syncthreads();
-      const int r = tid | 15;
-      v_sh[0][tid] = ex2(cs_sh[0][r] - c0) * d0;
-      v_sh[1][tid] = ex2(cs_sh[1][r] - c1) * d1;
+      v_sh[half][row] = ex2(cs_sh[half][row | 15] - c) * d;
     }
     ok = mbar_wait(&tma_bar, tma_phase, abort_v, 21);
     tma_phase ^= 1;
@@ -384,165 +409,167 @@ __global__ void __launch_bounds__(128, 1) chunk_out_kernel(
       }
       mma_commit(&mma_bar);
     }
-    // ---- H pass: bf16 copy of H for C H, then H <- exp(cs_end) H (lane n = tid) ----
+    // ---- H pass (lane n = row, head = half): hi/lo bf16 copy of H for C H, then
+    //      H <- exp(cs_end) H in place ----
     {
       tc_fence_after();
-      const float al0 = ex2(cs_sh[0][kBlk - 1]), al1 = ex2(cs_sh[1][kBlk - 1]);
+      const float al = ex2(cs_sh[half][kBlk - 1]);
+      uint8_t* hh = smem + kOffHh + half * kTile;
+      uint8_t* hl = smem + kOffHl + half * kTile;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float al = j ? al1 : al0;
-        uint8_t* hrow = smem + kOffH + j * kTile;
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t r[16];
+        tmem_ld16(tH + lane_off + half * 64 + pc * 16, r);
+        tmem_wait_ld();
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-          uint32_t r[16];
-          tmem_ld16(tH + lane_off + j * 64 + pc * 16, r);
-          tmem_wait_ld();
-          uint4 lo, hi;
-          lo.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-          lo.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-          lo.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-          lo.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-          hi.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-          hi.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-          hi.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-          hi.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-          *reinterpret_cast<uint4*>(hrow + swz(tid, pc * 2)) = lo;
-          *reinterpret_cast<uint4*>(hrow + swz(tid, pc * 2 + 1)) = hi;
+        for (int e = 0; e < 8; ++e)
+          split2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), hi[e], lo[e]);
+        *reinterpret_cast<uint4*>(hh + swz(row, pc * 2)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(hh + swz(row, pc * 2 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        *reinterpret_cast<uint4*>(hl + swz(row, pc * 2)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(hl + swz(row, pc * 2 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * al);
-          tmem_st16(tH + lane_off + j * 64 + pc * 16, r);
-        }
+        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * al);
+        tmem_st16(tH + lane_off + half * 64 + pc * 16, r);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
-    // ---- Off = C H (M = t, N = (head, p), K = n) ----
+    // ---- Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n) ----
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < kN / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * kTile + (kk & 3) * 32;
-        mma_ss(tO, sdesc(sbase + kOffC + koff, 16, 1024),
-               sdesc(sbase + kOffH + kk * 2048, kTile, 1024), idesc, kk > 0 ? 1u : 0u);
+        const uint64_t ad = sdesc(sbase + kOffC + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
+        mma_ss(tO, ad, sdesc(sbase + kOffHh + kk * 2048, kTile, 1024), idesc, kk > 0 ? 1u : 0u);
+        mma_ss(tO, ad, sdesc(sbase + kOffHl + kk * 2048, kTile, 1024), idesc, 1u);
       }
     }
     ok = mbar_wait(&mma_bar, mma_phase, abort_v, 22);  // G complete
     mma_phase ^= 1;
     tc_fence_after();
-    // ---- masked tiles: M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s  (s <= t), row t = tid ----
-    if (ok) {
-      const int t = tid;
-      const int jmax = 2 * warp + 1;  // last 16-column block any row of this warp needs
-      const float cst0 = cs_sh[0][t], cst1 = cs_sh[1][t];
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t region = (j >> 2) * kTile, c0 = (j & 3) * 2;
-        uint4 m0lo = make_uint4(0, 0, 0, 0), m0hi = m0lo, m1lo = m0lo, m1hi = m0lo;
-        if (j <= jmax) {
-          uint32_t r[16];
-          tmem_ld16(tG + lane_off + j * 16, r);
-          tmem_wait_ld();
-          const int s0 = j * 16;
-          float f0[16], f1[16];
-          if (t >= s0 + 15) {  // whole sub-block at or before t: split at r = s0 + 15
-            const float u0 = ex2(cst0 - cs_sh[0][s0 + 15]);
-            const float u1 = ex2(cst1 - cs_sh[1][s0 + 15]);
+    // ---- masked tiles, one head at a time: M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for
+    //      s <= t.  Thread (row t, column half c) keeps G[t, 64c .. 64c+64) in registers and
+    //      writes head h's mask over those TMEM columns as a bf16 high part (columns
+    //      64c .. 64c+32) and the bf16 rounding of the remainder (64c+32 .. 64c+64); the
+    //      diagonal MMAs read both as their A operand, so the mask carries ~16 bits. ----
+    float gv[64];
+    const bool g_live = (warp & 3) * 32 + 31 >= half * 64;  // some row of the warp reaches 64c
+    if (ok && g_live) {
+      const uint32_t gaddr = tG + lane_off + half * 64;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float gv = __uint_as_float(r[e]);
-              f0[e] = gv * (u0 * v_sh[0][s0 + e]);
-              f1[e] = gv * (u1 * v_sh[1][s0 + e]);
-            }
-          } else {  // diagonal sub-block (or beyond): exact exps, zero above the diagonal
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[16];
+        tmem_ld16(gaddr + q * 16, r);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int s = s0 + e;
-              const float gv = __uint_as_float(r[e]);
-              f0[e] = s <= t ? gv * ex2(cst0 - cs_sh[0][s]) * dt_sh[0][s] : 0.f;
-              f1[e] = s <= t ? gv * ex2(cst1 - cs_sh[1][s]) * dt_sh[1][s] : 0.f;
-            }
-          }
-          m0lo = make_uint4(pack_bf16x2(f0[0], f0[1]), pack_bf16x2(f0[2], f0[3]),
-                            pack_bf16x2(f0[4], f0[5]), pack_bf16x2(f0[6], f0[7]));
-          m0hi = make_uint4(pack_bf16x2(f0[8], f0[9]), pack_bf16x2(f0[10], f0[11]),
-                            pack_bf16x2(f0[12], f0[13]), pack_bf16x2(f0[14], f0[15]));
-          m1lo = make_uint4(pack_bf16x2(f1[0], f1[1]), pack_bf16x2(f1[2], f1[3]),
-                            pack_bf16x2(f1[4], f1[5]), pack_bf16x2(f1[6], f1[7]));
-          m1hi = make_uint4(pack_bf16x2(f1[8], f1[9]), pack_bf16x2(f1[10], f1[11]),
-                            pack_bf16x2(f1[12], f1[13]), pack_bf16x2(f1[14], f1[15]));
-        }
-        uint8_t* m0 = smem + kOffM + region;
-        uint8_t* m1 = smem + kOffM + 2 * kTile + region;
-        *reinterpret_cast<uint4*>(m0 + swz(t, c0)) = m0lo;
-        *reinterpret_cast<uint4*>(m0 + swz(t, c0 + 1)) = m0hi;
-        *reinterpret_cast<uint4*>(m1 + swz(t, c0)) = m1lo;
-        *reinterpret_cast<uint4*>(m1 + swz(t, c0 + 1)) = m1hi;
+        for (int e = 0; e < 16; ++e) gv[q * 16 + e] = __uint_as_float(r[e]);
       }
-      fence_proxy_async_smem();
+      tmem_wait_ld();
+    }
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      if (ok) {
+        const int t = row, c = half;
+        const uint32_t gaddr = tG + lane_off + c * 64;
+        uint32_t hi[32], lo[32];
+        if (g_live) {
+          const float ct = cs_sh[h][t];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int s0 = c * 64 + q * 16;
+            float f[16];
+            if (t >= s0 + 15) {  // the whole 16-column sub-block is at or before t
+              const float u = ex2(ct - cs_sh[h][s0 + 15]);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) f[e] = gv[q * 16 + e] * (u * v_sh[h][s0 + e]);
+            } else if (t >= s0) {  // diagonal sub-block: exact exps, zero above the diagonal
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int s = s0 + e;
+                f[e] = s <= t ? gv[q * 16 + e] * ex2(ct - cs_sh[h][s]) * dt_sh[h][s] : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) f[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) split2(f[2 * e], f[2 * e + 1], hi[q * 8 + e], lo[q * 8 + e]);
+          }
+        } else {  // every row of this warp lies before column 64c: zero masks
+#pragma unroll
+          for (int e = 0; e < 32; ++e) { hi[e] = 0u; lo[e] = 0u; }
+        }
+        uint32_t r[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = hi[e];
+        tmem_st16(gaddr, r);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = hi[16 + e];
+        tmem_st16(gaddr + 16, r);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = lo[e];
+        tmem_st16(gaddr + 32, r);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = lo[16 + e];
+        tmem_st16(gaddr + 48, r);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
+      // ---- Diag_h = (Mhi_h + Mlo_h) X_h (M = t, N = p, K = s), A from TMEM ----
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          const uint32_t acol = tG + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint64_t bd = sdesc(sbase + kOffX + h * kTile + kk * 2048, kTile, 1024);
+          mma_ts(tD + h * 64, acol, bd, idesc, kk > 0 ? 1u : 0u);
+          mma_ts(tD + h * 64, acol + 32, bd, idesc, 1u);
+        }
+        mma_commit(&mma_bar);  // head 0: covers Off as well
+      }
+      ok = mbar_wait(&mma_bar, mma_phase, abort_v, 23);
+      mma_phase ^= 1;
+      tc_fence_after();
     }
     tc_fence_before();
     if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
-    // ---- Diag_h = M_h X_h (M = t, N = p, K = s) ----
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(128, 64, 0, 1);
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * kTile + (kk & 3) * 32;
-          mma_ss(tD + j * 64, sdesc(sbase + kOffM + j * 2 * kTile + koff, 16, 1024),
-                 sdesc(sbase + kOffX + j * kTile + kk * 2048, kTile, 1024), idesc,
-                 kk > 0 ? 1u : 0u);
-        }
-      }
-      mma_commit(&mma_bar);  // covers Off and both Diag
-    }
-    ok = mbar_wait(&mma_bar, mma_phase, abort_v, 23);
-    mma_phase ^= 1;
     tc_fence_after();
-    // ---- epilogue: y_t = Diag + exp(cs_t) Off + D x_t; then X' = w * x in place ----
+    // ---- epilogue (row t, head = half): y_t = Diag + exp(cs_t) Off + D x_t; then X' = w x ----
     if (ok) {
-      const int t = tid;
-      const float e0 = ex2(cs_sh[0][t]), e1 = ex2(cs_sh[1][t]);
-      const float w0 = ex2(cs_sh[0][kBlk - 1] - cs_sh[0][t]) * dt_sh[0][t];
-      const float w1 = ex2(cs_sh[1][kBlk - 1] - cs_sh[1][t]) * dt_sh[1][t];
+      const int t = row, j = half;
+      const float ej = ex2(cs_sh[j][t]);
+      const float wj = ex2(cs_sh[j][kBlk - 1] - cs_sh[j][t]) * dt_sh[j][t];
+      uint8_t* xrow = smem + kOffX + j * kTile;
+      TY* yrow = y + ((int64_t(b) * seqlen + tok) * nheads + h0 + j) * kP;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float ej = j ? e1 : e0, Dj = j ? Dh1 : Dh0, wj = j ? w1 : w0;
-        uint8_t* xrow = smem + kOffX + j * kTile;
-        __nv_bfloat16* yrow = y + ((int64_t(b) * seqlen + tok) * nheads + h0 + j) * kP;
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t rd[16], ro[16];
+        tmem_ld16(tD + lane_off + j * 64 + pc * 16, rd);
+        tmem_ld16(tO + lane_off + j * 64 + pc * 16, ro);
+        tmem_wait_ld();
+        uint4* x0p = reinterpret_cast<uint4*>(xrow + swz(t, pc * 2));
+        uint4* x1p = reinterpret_cast<uint4*>(xrow + swz(t, pc * 2 + 1));
+        const uint4 xa = *x0p, xb = *x1p;
+        const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        float yv[16];
+        uint32_t xs[8];
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-          uint32_t rd[16], ro[16];
-          tmem_ld16(tD + lane_off + j * 64 + pc * 16, rd);
-          tmem_ld16(tO + lane_off + j * 64 + pc * 16, ro);
-          tmem_wait_ld();
-          uint4* x0p = reinterpret_cast<uint4*>(xrow + swz(t, pc * 2));
-          uint4* x1p = reinterpret_cast<uint4*>(xrow + swz(t, pc * 2 + 1));
-          const uint4 xa = *x0p, xb = *x1p;
-          const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-          uint32_t yo[8], xs[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float xl = bf16lo(xw[e]), xh = bf16hi(xw[e]);
-            const float yl = __uint_as_float(rd[2 * e]) + ej * __uint_as_float(ro[2 * e]) + Dj * xl;
-            const float yh =
-                __uint_as_float(rd[2 * e + 1]) + ej * __uint_as_float(ro[2 * e + 1]) + Dj * xh;
-            yo[e] = pack_bf16x2(yl, yh);
-            xs[e] = pack_bf16x2(xl * wj, xh * wj);
-          }
-          if (tok < seqlen) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow + pc * 16);
-            dst[0] = make_uint4(yo[0], yo[1], yo[2], yo[3]);
-            dst[1] = make_uint4(yo[4], yo[5], yo[6], yo[7]);
-          }
-          *x0p = make_uint4(xs[0], xs[1], xs[2], xs[3]);
-          *x1p = make_uint4(xs[4], xs[5], xs[6], xs[7]);
+        for (int e = 0; e < 8; ++e) {
+          const float xl = bf16lo(xw[e]), xh = bf16hi(xw[e]);
+          yv[2 * e] = __uint_as_float(rd[2 * e]) + ej * __uint_as_float(ro[2 * e]) + Dh * xl;
+          yv[2 * e + 1] =
+              __uint_as_float(rd[2 * e + 1]) + ej * __uint_as_float(ro[2 * e + 1]) + Dh * xh;
+          xs[e] = pack_bf16x2(xl * wj, xh * wj);
         }
+        if (tok < seqlen) yout<TY>::store16(yrow + pc * 16, yv);
+        *x0p = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+        *x1p = make_uint4(xs[4], xs[5], xs[6], xs[7]);
       }
       fence_proxy_async_smem();
     }
@@ -573,7 +600,7 @@ __global__ void __launch_bounds__(128, 1) chunk_out_kernel(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid < 32) tmem_free(tmem, 512);
+  if (warp == 0) tmem_free(tmem, 512);
 }
 
 }  // namespace tc

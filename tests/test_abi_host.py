@@ -71,14 +71,14 @@ def test_workspace_sizes(lib):
 def _scan_call(lib, **kw):
     args = dict(x=None, dt=None, A=None, B=None, C=None, D=None, init=None, y=None, fin=None,
                 batch=1, seqlen=256, nheads=4, headdim=16, dstate=16, ngroups=1, chunk=64,
-                io=ssd.SSD_F32, ws=None, ws_bytes=0, stream=None)
+                io=ssd.SSD_F32, y_dtype=ssd.SSD_F32, ws=None, ws_bytes=0, stream=None)
     args.update(kw)
     return lib.ssd_chunk_scan_fwd(*args.values())
 
 
 @pytest.mark.parametrize("bad", [
     dict(chunk=100), dict(chunk=0), dict(batch=0), dict(seqlen=0), dict(nheads=3, ngroups=2),
-    dict(headdim=0), dict(dstate=-1), dict(io=7),
+    dict(headdim=0), dict(dstate=-1), dict(io=7), dict(y_dtype=5),
     dict(),  # all pointers NULL
 ])
 def test_scan_rejects_bad_arguments_on_host(lib, bad):
@@ -86,9 +86,10 @@ def test_scan_rejects_bad_arguments_on_host(lib, bad):
 
 
 def test_step_rejects_bad_arguments_on_host(lib):
-    assert lib.ssd_step(*([None] * 8), 0, 4, 16, 16, 1, 1, None) == 1
-    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 3, 1, None) == 1
-    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 1, 1, None) == 1  # NULL pointers
+    assert lib.ssd_step(*([None] * 8), 0, 4, 16, 16, 1, 1, 0, None) == 1
+    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 3, 1, 0, None) == 1
+    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 1, 0, 1, None) == 1  # f32 io, bf16 y
+    assert lib.ssd_step(*([None] * 8), 2, 4, 16, 16, 1, 1, 0, None) == 1  # NULL pointers
 
 
 def test_binding_refuses_cpu_tensors(lib):

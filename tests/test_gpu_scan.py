@@ -14,7 +14,8 @@ import torch
 import mamba_ssd_scan_03_b200 as ssd
 import oracle
 import ssd_inputs
-from gpu_util import TOL, dev_inputs, oracle_chains, rel_err, sample_chains, to_dev, to_np
+from gpu_util import (TOL, bf16_excess, dev_inputs, oracle_chains, rel_err, sample_chains,
+                      to_dev, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -182,7 +183,7 @@ def test_output_canaries():
     inp = small(seed=16, batch=2, seqlen=333, nheads=4)
     t = dev_inputs(inp)
     n = t["x"].numel()
-    ybuf = torch.full((n + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    ybuf = torch.full((n + 4096,), 7.0, dtype=torch.float32, device="cuda")
     fbuf = torch.full((2 * 4 * 64 * 128 + 1024,), -3.0, dtype=torch.float32, device="cuda")
     y = ybuf[1024:1024 + n].view(t["x"].shape)
     fin = fbuf[256:256 + 2 * 4 * 64 * 128].view(2, 4, 64, 128)
@@ -211,20 +212,20 @@ def test_device_argument_errors():
     inp = small(seed=18, batch=1, seqlen=256, nheads=2)
     t = dev_inputs(inp)
     lib = ssd.load()
-    y = torch.empty_like(t["x"])
+    y = torch.empty(t["x"].shape, dtype=torch.float32, device="cuda")
     need = ssd.workspace_size(1, 256, 2, 64, 128, 1, 256)
     small_ws = torch.empty(max(need // 2, 256), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
 
-    def call(x=t["x"], yv=y, ws=small_ws, wsb=None, B=t["B"]):
+    def call(x=t["x"], yv=y, ws=small_ws, wsb=None, B=t["B"], ydt=0):
         return lib.ssd_chunk_scan_fwd(x.data_ptr(), t["dt"].data_ptr(), t["A"].data_ptr(),
                                       B.data_ptr(), t["C"].data_ptr(), t["D"].data_ptr(), None,
-                                      yv.data_ptr(), None, 1, 256, 2, 64, 128, 1, 256, 1,
+                                      yv.data_ptr(), None, 1, 256, 2, 64, 128, 1, 256, 1, ydt,
                                       ws.data_ptr(), ws.numel() if wsb is None else wsb, stream)
     assert call() == 3                                    # workspace too small
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     assert call(ws=ws) == 0
-    assert call(ws=ws, yv=t["x"]) == 1                    # y aliases x
+    assert call(ws=ws, yv=t["x"], ydt=1) == 1             # y aliases x
     host = torch.empty_like(t["x"], device="cpu")
     assert call(ws=ws, x=host) == 1                       # host pointer
     xb = torch.empty(t["x"].numel() + 8, dtype=torch.bfloat16, device="cuda")
@@ -265,3 +266,16 @@ def test_million_token_context():
     fg = to_np(fin[torch.as_tensor(b), torch.as_tensor(h), torch.as_tensor(p)])
     assert rel_err(yg, yo) <= TOL["bf16"]
     assert rel_err(fg, fo) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("simt", [False, True])
+def test_bf16_output(simt):
+    """y in the io dtype (bf16): the error beyond the output's own rounding (half a bf16 ulp,
+    <= 2^-8 |y|) stays within the bf16 tolerance."""
+    inp = small(seed=19, batch=2, seqlen=700, nheads=4)
+    y, fin = run(inp, dev_inputs(inp), simt=simt, y_dtype=torch.bfloat16)
+    assert y.dtype == torch.bfloat16
+    yo, fo = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                         init=inp["init"])
+    assert bf16_excess(to_np(y), yo, TOL["bf16"]) <= TOL["bf16"]
+    assert rel_err(to_np(fin), fo) <= TOL["bf16"]

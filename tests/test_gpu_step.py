@@ -8,7 +8,7 @@ import torch
 import mamba_ssd_scan_03_b200 as ssd
 import oracle
 import ssd_inputs
-from gpu_util import TOL, dev_inputs, rel_err, sample_chains, to_dev, to_np
+from gpu_util import TOL, bf16_excess, dev_inputs, rel_err, sample_chains, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +48,7 @@ def test_decode_touches_only_state_and_y():
     st = buf[1024:1024 + n].view(dec["state"].shape)
     st.copy_(to_dev(dec["state"]))
     s, t = _step_dev(dec, 0)
-    ybuf = torch.full((t["x"].numel() + 512,), 9.0, dtype=torch.bfloat16, device="cuda")
+    ybuf = torch.full((t["x"].numel() + 512,), 9.0, dtype=torch.float32, device="cuda")
     y = ybuf[256:256 + t["x"].numel()].view(t["x"].shape)
     ssd.step(st, t["x"], t["dt"], A, t["B"], t["C"], D, out=y)
     torch.cuda.synchronize()
@@ -102,3 +102,16 @@ def test_decode_workload_1000_steps():
         if k + 1 in (1, 10, 100, 1000):
             assert rel_err(to_np(st[bi, hi, pi]), so) <= TOL["bf16"], k + 1
     assert ssd.device_status() == 0
+
+
+def test_decode_bf16_output():
+    dec = ssd_inputs.make_decode_inputs(4, batch=4, nheads=4)
+    A, D = to_dev(dec["A"]), to_dev(dec["D"])
+    st = to_dev(dec["state"])
+    so = dec["state"].astype(np.float64)
+    for k in range(10):
+        s, t = _step_dev(dec, k)
+        y = ssd.step(st, t["x"], t["dt"], A, t["B"], t["C"], D, y_dtype=torch.bfloat16)
+        assert y.dtype == torch.bfloat16
+        yo, so = oracle.step(so, s["x"], s["dt"], dec["A"], s["B"], s["C"], dec["D"])
+        assert bf16_excess(to_np(y), yo, TOL["bf16"]) <= TOL["bf16"], k

@@ -139,6 +139,37 @@ ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A
                     int nheads, int headdim, int dstate, int ngroups, ssd_dtype io,
                     ssd_dtype y_dtype, cudaStream_t stream);
 
+/*
+ * ssd_chunk_scan_fwd without a workspace argument, for callers that cannot allocate device
+ * memory: code running where cudaMalloc is unavailable or forbidden (inside an allocator-free
+ * serving loop, a plugin that owns no memory pool, a context whose allocator is locked), or
+ * that must not grow the process's device footprint per call.  The pages have no counterpart;
+ * this is a deployment convenience around the same tensor-core kernels.
+ *
+ * Scratch comes from one fixed array of SSD_NOALLOC_SCRATCH_BYTES (32 MiB) that the library
+ * holds in every GPU that loads it, until the process exits.  The call allocates nothing.
+ *   - Shapes: the tensor-core shapes only (io = SSD_BF16, headdim 64, dstate 128, an even
+ *     number of heads per group).  The sequence is cut into as many segments as the array can
+ *     hold states for (one float32 headdim x dstate state per batch row, segment and head);
+ *     when batch * nheads states (32 KiB each) do not fit even with one segment, the call
+ *     returns SSD_ERR_UNSUPPORTED before launching anything.  Other shapes also return
+ *     SSD_ERR_UNSUPPORTED.
+ *   - The first call on each device looks up the array's device address (and configures the
+ *     kernels) for that device; make that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Calls whose kernels overlap on the GPU
+ *     (different streams without ordering, or several host threads) race on it and give wrong
+ *     results: order them.  Nothing in the array needs to start at zero; each call writes every
+ *     scratch value before it reads it.
+ * Arguments, layouts and the result are exactly those of ssd_chunk_scan_fwd.
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (32u << 20)
+ssd_status ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, const float* A,
+                                      const void* B, const void* C, const float* D,
+                                      const float* init_state, void* y, float* final_state,
+                                      int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                      int dstate, int ngroups, int chunk, ssd_dtype io,
+                                      ssd_dtype y_dtype, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* ssd_status_string(ssd_status s);
 

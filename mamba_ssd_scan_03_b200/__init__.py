@@ -24,7 +24,11 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 # The symbols include/ssd.h declares (tests check that the library exports each one).
 EXPORTS = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path", "ssd_chunk_scan_fwd",
            "ssd_chunk_scan_simt_workspace_size", "ssd_chunk_scan_fwd_simt", "ssd_step",
-           "ssd_status_string", "ssd_get_device_status", "ssd_version")
+           "ssd_chunk_scan_fwd_noalloc", "ssd_status_string", "ssd_get_device_status",
+           "ssd_version")
+
+# Size of the fixed device array ssd_chunk_scan_fwd_noalloc uses instead of a workspace.
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class SSDError(RuntimeError):
@@ -58,6 +62,8 @@ def load():
     for fn in (lib.ssd_chunk_scan_fwd, lib.ssd_chunk_scan_fwd_simt):
         fn.restype = _i32
         fn.argtypes = _SCAN
+    lib.ssd_chunk_scan_fwd_noalloc.restype = _i32
+    lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 9 + [_i64, _i64] + [_i32] * 7 + [_vp]
     lib.ssd_step.restype = _i32
     lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
@@ -181,6 +187,42 @@ def chunk_scan_fwd_simt(x, dt, A, B, C, D, chunk, init_state=None, want_final=Tr
     """The same operation on the float32 SIMT kernels (second GPU reference)."""
     return _scan(load().ssd_chunk_scan_fwd_simt, True, x, dt, A, B, C, D, chunk, init_state,
                  want_final, workspace, out, final_out, y_dtype)
+
+
+def chunk_scan_fwd_noalloc(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
+                           out=None, final_out=None, y_dtype=torch.float32):
+    """The chunked scan for callers that cannot allocate device memory: the library's scratch
+    lives in a fixed 32 MiB device array (NOALLOC_SCRATCH_BYTES) instead of a workspace.
+    Tensor-core shapes only.  Calls that overlap on the GPU share that array and race, so
+    order them; the first call on a device sets the array up and should precede any stream
+    capture.  (This wrapper still allocates y and the final state with PyTorch unless `out`
+    and `final_out` are given.)"""
+    lib = load()
+    _need(x, "x")
+    dev = x.device
+    Bt, L, H, P, N, G, Q, io = _scan_shape(x, B, chunk)
+    _need(B, "B", x.dtype, (Bt, L, G, N), dev)
+    _need(C, "C", x.dtype, (Bt, L, G, N), dev)
+    _need(dt, "dt", torch.float32, (Bt, L, H), dev)
+    _need(A, "A", torch.float32, (H,), dev)
+    if D is not None:
+        _need(D, "D", torch.float32, (H,), dev)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (Bt, H, P, N), dev)
+    y_dtype = out.dtype if out is not None else y_dtype
+    y = out if out is not None else torch.empty(x.shape, dtype=y_dtype, device=dev)
+    _need(y, "out", y_dtype, x.shape, dev)
+    fin = None
+    if want_final:
+        fin = final_out if final_out is not None else torch.empty(
+            (Bt, H, P, N), dtype=torch.float32, device=dev)
+        _need(fin, "final_state", torch.float32, (Bt, H, P, N), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_chunk_scan_fwd_noalloc(
+            _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(y),
+            _ptr(fin), Bt, L, H, P, N, G, Q, io, _code(y_dtype), _stream(dev))
+    _check(rc, "ssd_chunk_scan_fwd_noalloc")
+    return y, fin
 
 
 def step(state, x, dt, A, B, C, D, out=None, y_dtype=torch.float32):

@@ -426,3 +426,126 @@ ssd_status ssd_get_device_status(cudaStream_t stream) {
 const char* ssd_version(void) { return "ssd-b200 0.1 sm_100a"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// ssd_chunk_scan_fwd_noalloc: the tensor-core scan with its scratch (the per-segment states and
+// decays) in a fixed device array instead of a caller workspace, for callers that cannot
+// allocate device memory.  The array lives in every GPU that loads this library until exit.
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SSD_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};  // device address of the array, per device
+
+// Once per device, with that device current: the array's device address (host code may not use
+// the symbol itself, which on the host is only a stand-in) and the kernels' shared-memory limits.
+ssd_status noalloc_setup(void** scratch) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SSD_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return SSD_ERR_CUDA;
+    }
+    const bool ok =
+        cudaFuncSetAttribute(ssd::tc::seg_state_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem)) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
+            cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return SSD_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *scratch = g_noalloc_addr[dev];
+  return SSD_OK;
+}
+
+size_t seg_scratch_bytes(const Shape& s, const Seg& sg) {
+  return align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)) +
+         align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float));
+}
+
+// The usual segmentation, with fewer (longer) segments when their states would not fit in
+// `cap` bytes.  Returns false when even one segment per sequence does not fit.
+bool segments_within(const Shape& s, size_t cap, Seg* out) {
+  Seg sg = tc_segments(s);
+  for (int nseg = sg.nseg; nseg >= 1; --nseg) {
+    Seg t;
+    t.nblk = sg.nblk;
+    t.seg_blks = (t.nblk + nseg - 1) / nseg;
+    t.nseg = (t.nblk + t.seg_blks - 1) / t.seg_blks;
+    if (seg_scratch_bytes(s, t) <= cap) {
+      *out = t;
+      return true;
+    }
+  }
+  return false;
+}
+
+ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, void* scratch) {
+  float* seg_states = static_cast<float*>(scratch);
+  float* seg_decay = reinterpret_cast<float*>(
+      static_cast<char*>(scratch) +
+      align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)));
+  CUtensorMap mx, mb, mc;
+  const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
+  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch) ||
+      !make_map(&mc, a.C, GN, s.seqlen, s.batch))
+    return SSD_ERR_CUDA;
+  const int hpg = s.nheads / s.ngroups;
+  const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
+  ssd::tc::seg_state_kernel<<<grid, 256, kSegSmem, a.stream>>>(
+      mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;
+  ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
+      seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  if (a.ydt == SSD_F32)
+    ssd::tc::chunk_out_kernel<float><<<grid, 256, kTcSmem, a.stream>>>(
+        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<float*>(a.y), s.seqlen, s.nheads,
+        hpg, sg);
+  else
+    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, 256, kTcSmem, a.stream>>>(
+        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<__nv_bfloat16*>(a.y), s.seqlen,
+        s.nheads, hpg, sg);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" ssd_status ssd_chunk_scan_fwd_noalloc(
+    const void* x, const float* dt, const float* A, const void* B, const void* C,
+    const float* D, const float* init_state, void* y, float* final_state, int64_t batch,
+    int64_t seqlen, int nheads, int headdim, int dstate, int ngroups, int chunk, ssd_dtype io,
+    ssd_dtype y_dtype, cudaStream_t stream) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  const ScanArgs a{y_dtype, x, B, C, dt, A, D, init_state, y, final_state, nullptr, 0, stream};
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  if (!tc_shape_ok(s)) return SSD_ERR_UNSUPPORTED;
+  Seg sg;
+  if (!segments_within(s, SSD_NOALLOC_SCRATCH_BYTES, &sg)) return SSD_ERR_UNSUPPORTED;
+  st = validate_scan(s, a, 0);
+  if (st != SSD_OK) return st;
+  if (!tc_pointers_ok(a)) return SSD_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  st = noalloc_setup(&scratch);
+  if (st != SSD_OK) return st;
+  return run_tc_segments(s, a, sg, scratch);
+}

@@ -114,17 +114,21 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 view [outer][mid][inner] with a {64, 128, 1} box and 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer) {
+// 3-D view [outer][mid][inner] with a {128 bytes of inner, 128, 1} box and 128-byte swizzle:
+// bf16 tiles of 64 elements, float32 tiles of 32.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+              bool f32 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[3] = {inner, mid, outer};
-  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint64_t strides[2] = {inner * es, inner * mid * es};
+  cuuint32_t box[3] = {f32 ? 32u : 64u, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 constexpr size_t kTcSmem = ssd::tc::kSmemTiles + 1024;
@@ -254,14 +258,14 @@ ssd_status run_tc(const Shape& s, const ScanArgs& a) {
   ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
       seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  CUtensorMap my;
+  if (!make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32)) return SSD_ERR_CUDA;
   if (a.ydt == SSD_F32)
-    ssd::tc::chunk_out_kernel<float><<<grid, 256, kTcSmem, a.stream>>>(
-        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<float*>(a.y), s.seqlen, s.nheads,
-        hpg, sg);
+    ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
+        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
   else
-    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, 256, kTcSmem, a.stream>>>(
-        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<__nv_bfloat16*>(a.y), s.seqlen,
-        s.nheads, hpg, sg);
+    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
+        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
   return launched();
 }
 
@@ -516,14 +520,14 @@ ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, voi
   ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
       seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  CUtensorMap my;
+  if (!make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32)) return SSD_ERR_CUDA;
   if (a.ydt == SSD_F32)
-    ssd::tc::chunk_out_kernel<float><<<grid, 256, kTcSmem, a.stream>>>(
-        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<float*>(a.y), s.seqlen, s.nheads,
-        hpg, sg);
+    ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
+        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
   else
-    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, 256, kTcSmem, a.stream>>>(
-        mx, mb, mc, a.dt, a.A, a.D, seg_states, static_cast<__nv_bfloat16*>(a.y), s.seqlen,
-        s.nheads, hpg, sg);
+    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
+        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
   return launched();
 }
 

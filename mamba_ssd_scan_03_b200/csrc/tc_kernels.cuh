@@ -267,59 +267,105 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(float* __restrict__ seg_s
 }
 
 // =============================================================================================
-// chunk_out: grid = batch * nseg * (nheads / 2), block = 256 threads.  Thread (row = tid % 128,
-// half = tid / 128): token row `row` of a block (and state row n = row for the state passes);
-// `half` selects the head (state pass, epilogue) or the 64-column half of G (masks).
-// Shared memory (1024-aligned, 10 x 16 KB):
+// chunk_out: grid = batch * nseg * (nheads / 2), block = 576 threads in three roles:
+//   warps 0-15  compute (512 threads).  Thread (row = tid % 128, q = tid / 128): token row
+//               `row` of a block (state row n = row in the state passes) and a quarter of the
+//               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and
+//               the epilogue; G columns [32 q, 32 q + 32) for the masks.  Four warps share each
+//               TMEM lane quarter, so every phase is spread over all 16 warps.
+//   warp 16     TMA producer (lane 0): C, x (single buffers), B (double buffer) per block.
+//   warp 17     MMA issuer (lane 0).
+// The roles hand blocks to each other through mbarriers, so the loads of the next block, the
+// tensor-core work and the CUDA-core work of different phases overlap.
+// Shared memory (1024-aligned, 12 x 16 KB):
 //   sC   2 tiles  C, K-major (rows t), n halves
-//   sB   2 tiles  B, rows s, n halves: K-major for G = C B^T, MN-major for B^T X'
-//   sX   2 tiles  x of the two heads (rows t, 64 p), MN-major; scaled in place to X'
+//   sB   4 tiles  B, rows s, n halves, two slots (blocks k % 2): K-major for G = C B^T,
+//                 MN-major for B^T X'
+//   sX   2 tiles  x of the two heads (rows t, 64 p), MN-major; scaled in place to X' = w x
+//                 once the diagonal MMAs have read it
 //   sHh  2 tiles  bf16 high part of the entering state of the two heads (rows n, 64 p)
 //   sHl  2 tiles  bf16 low part (the state's rounding remainder), same layout
+//   (sHh + sHl, free once C H has been computed, stage the block's y for the TMA stores)
 // TMEM (512 columns): [0,128) running state H (head, p) | [128,256) diagonal accumulators |
 //   [256,384) off-diagonal accumulators C H | [384,512) G = C B^T, overwritten in place, one
-//   head at a time, by that head's masked tile as bf16 high and low parts, which the diagonal
-//   MMAs read as their A operand.
+//   head at a time, by that head's masked tile: for each 16-column group kk, 8 columns of bf16
+//   high parts then 8 of low parts, which the diagonal MMAs read as their A operand.
 // =============================================================================================
-constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 4 * kTile, kOffHh = 6 * kTile,
-                   kOffHl = 8 * kTile, kSmemTiles = 10 * kTile;
+constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 6 * kTile, kOffHh = 8 * kTile,
+                   kOffHl = 10 * kTile, kSmemTiles = 12 * kTile;
+constexpr int kComputeThreads = 512;
+constexpr int kOutThreads = kComputeThreads + 64;
 
-template <typename TY> struct yout;
-template <> struct yout<float> {
-  static __device__ __forceinline__ void store16(float* p, const float (&v)[16]) {
-    float4* q = reinterpret_cast<float4*>(p);
+// y staging (in sHh/sHl) and its TMA stores.  Float32 y: 4 boxes {32 p, 128 t} (one per
+// thread quarter q: head q/2, p-half q%2), 128B-swizzled.  Bf16 y: 2 boxes {64 p, 128 t} (one
+// per head).
+template <typename TY> struct ystage;
+template <> struct ystage<float> {
+  static constexpr int kBoxes = 4;
+  // thread (t, q) writes its 32 values (16 per call, half = 0/1) into box q, row t
+  static __device__ __forceinline__ void put16(uint8_t* stage, int t, int q, int half,
+                                               const float (&v)[16]) {
+    uint8_t* box = stage + q * kTile;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(box + swz(t, half * 4 + i)) =
+          make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  static __device__ __forceinline__ void store(const CUtensorMap* map, const uint8_t* stage,
+                                               int h0, int t0, int b) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      tma_store_3d(map, stage + q * kTile, (h0 + q / 2) * kP + (q % 2) * 32, t0, b);
   }
 };
-template <> struct yout<__nv_bfloat16> {
-  static __device__ __forceinline__ void store16(__nv_bfloat16* p, const float (&v)[16]) {
-    uint4* q = reinterpret_cast<uint4*>(p);
-    q[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                      pack_bf16x2(v[6], v[7]));
-    q[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                      pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+template <> struct ystage<__nv_bfloat16> {
+  static constexpr int kBoxes = 2;
+  static __device__ __forceinline__ void put16(uint8_t* stage, int t, int q, int half,
+                                               const float (&v)[16]) {
+    uint8_t* box = stage + (q / 2) * kTile;
+    const int c0 = (q % 2) * 4 + half * 2;
+    *reinterpret_cast<uint4*>(box + swz(t, c0)) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                   pack_bf16x2(v[6], v[7]));
+    *reinterpret_cast<uint4*>(box + swz(t, c0 + 1)) =
+        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                   pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
   }
+  static __device__ __forceinline__ void store(const CUtensorMap* map, const uint8_t* stage,
+                                               int h0, int t0, int b) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) tma_store_3d(map, stage + j * kTile, (h0 + j) * kP, t0, b);
+  }
+};
+
+// mbarriers of chunk_out (all in shared memory)
+struct OutBars {
+  uint64_t c_full, b_full[2], x_full;      // TMA -> consumers
+  uint64_t c_empty, b_empty[2], x_empty;   // MMA completion -> producer
+  uint64_t g_done, d0_done, d1_done, st_done;  // MMA completion -> compute
+  uint64_t h_ready, m0_ready, m1_ready, xp_ready;  // compute -> MMA issuer
+  uint64_t drain;
 };
 
 template <typename TY>
-__global__ void __launch_bounds__(256, 1) chunk_out_kernel(
+__global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-    const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ dt,
-    const float* __restrict__ A, const float* __restrict__ D, const float* __restrict__ h_in,
-    TY* __restrict__ y, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
+    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+    const float* __restrict__ dt, const float* __restrict__ A, const float* __restrict__ D,
+    const float* __restrict__ h_in, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ uint64_t tma_bar, mma_bar;
+  __shared__ OutBars bars;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float cs_sh[2][kBlk], dt_sh[2][kBlk], v_sh[2][kBlk];
-  __shared__ float scan_scratch[8];
+  __shared__ __align__(16) float cs_sh[2][kBlk];
+  __shared__ __align__(16) float dt_sh[2][kBlk];
+  __shared__ __align__(16) float v_sh[2][kBlk];
+  __shared__ float scan_scratch[16];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int row = tid & 127, half = tid >> 7;
+  const int warp = tid >> 5, lane = tid & 31;
   const int npair = nheads / 2;
   const int unit = blockIdx.x;
   const int hp = unit % npair;
@@ -329,15 +375,18 @@ __global__ void __launch_bounds__(256, 1) chunk_out_kernel(
   const int g = h0 / heads_per_group;
   const int blk0 = seg * sg.seg_blks;
   const int nb = min(sg.nblk, blk0 + sg.seg_blks) - blk0;
+  volatile int* abort_v = &abort_flag;
+  uint32_t n_c = 0, n_x = 0, n_b[2] = {0, 0};  // the producer's loads issued per barrier
 
   if (tid == 0) {
     abort_flag = 0;
-    mbar_init(&tma_bar, 1);
-    mbar_init(&mma_bar, 1);
+    uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
+    for (int i = 0; i < int(sizeof(OutBars) / 8); ++i) mbar_init(all + i, 1);
+    mbar_init(&bars.h_ready, kComputeThreads);
+    mbar_init(&bars.m0_ready, kComputeThreads);
+    mbar_init(&bars.m1_ready, kComputeThreads);
+    mbar_init(&bars.xp_ready, kComputeThreads);
     fence_mbar_init();
-    prefetch_tmap(&tm_x);
-    prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_c);
   }
   if (warp == 0) tmem_alloc(&tmem_base_sh, 512);
   tc_fence_before();
@@ -345,257 +394,341 @@ __global__ void __launch_bounds__(256, 1) chunk_out_kernel(
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const uint32_t tH = tmem, tD = tmem + 128, tO = tmem + 256, tG = tmem + 384;
-  const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;  // this warp's TMEM lane quarter
   const uint32_t sbase = smem_u32(smem);
 
-  // entering state of the segment -> TMEM (lane n = row, columns of head `half`)
-  {
-    const float* src =
-        h_in + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + half) * kP) * kN + row;
-#pragma unroll
-    for (int pc = 0; pc < 4; ++pc) {
-      uint32_t r[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(src[(pc * 16 + e) * kN]);
-      tmem_st16(tH + lane_off + half * 64 + pc * 16, r);
-    }
-    tmem_wait_st();
-  }
-  const float Alog = A[h0 + half] * kLog2e;
-  const float Dh = D ? D[h0 + half] : 0.f;
-  uint32_t tma_phase = 0, mma_phase = 0;
-  bool ok = true;
-  volatile int* abort_v = &abort_flag;
-
-  for (int k = 0; k < nb; ++k) {
-    const int blk = blk0 + k;
-    const int64_t t0 = int64_t(blk) * kBlk;
-    tc_fence_before();
-    if (__syncthreads_or(*abort_v)) { ok = false; break; }
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&tma_bar, 6 * kTile);
-      tma_load_3d(smem + kOffC, &tm_c, &tma_bar, g * kN, int(t0), b);
-      tma_load_3d(smem + kOffC + kTile, &tm_c, &tma_bar, g * kN + 64, int(t0), b);
-      tma_load_3d(smem + kOffB, &tm_b, &tma_bar, g * kN, int(t0), b);
-      tma_load_3d(smem + kOffB + kTile, &tm_b, &tma_bar, g * kN + 64, int(t0), b);
-      tma_load_3d(smem + kOffX, &tm_x, &tma_bar, h0 * kP, int(t0), b);
-      tma_load_3d(smem + kOffX + kTile, &tm_x, &tma_bar, (h0 + 1) * kP, int(t0), b);
-    }
-    // within-block log2 cumsums of head `half`; v_s = exp(cs_r(s) - cs_s) dt_s, r(s) = s | 15
-    const int64_t tok = t0 + row;
-    {
-      const float d = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0 + half] : 0.f;
-      float tot;
-      const float c = half_scan128(d * Alog, scan_scratch, &tot);
-      cs_sh[half][row] = c;
-      dt_sh[half][row] = d;
-      __syncthreads();
-      v_sh[half][row] = ex2(cs_sh[half][row | 15] - c) * d;
-    }
-    ok = mbar_wait(&tma_bar, tma_phase, abort_v, 21);
-    tma_phase ^= 1;
-    tc_fence_before();
-    if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
-
-    // ---- G = C B^T (M = t, N = s, K = n) ----
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < kN / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * kTile + (kk & 3) * 32;
-        mma_ss(tG, sdesc(sbase + kOffC + koff, 16, 1024), sdesc(sbase + kOffB + koff, 16, 1024),
-               idesc, kk > 0 ? 1u : 0u);
+  if (warp == 16) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_b);
+      prefetch_tmap(&tm_c);
+      auto load_c = [&](int k) {
+        const int t0 = (blk0 + k) * kBlk;
+        ++n_c;
+        mbar_arrive_expect_tx(&bars.c_full, 2 * kTile);
+        tma_load_3d(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b);
+        tma_load_3d(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b);
+      };
+      auto load_b = [&](int k) {
+        const int t0 = (blk0 + k) * kBlk;
+        uint8_t* dst = smem + kOffB + (k & 1) * 2 * kTile;
+        ++n_b[k & 1];
+        mbar_arrive_expect_tx(&bars.b_full[k & 1], 2 * kTile);
+        tma_load_3d(dst, &tm_b, &bars.b_full[k & 1], g * kN, t0, b);
+        tma_load_3d(dst + kTile, &tm_b, &bars.b_full[k & 1], g * kN + 64, t0, b);
+      };
+      auto load_x = [&](int k) {
+        const int t0 = (blk0 + k) * kBlk;
+        ++n_x;
+        mbar_arrive_expect_tx(&bars.x_full, 2 * kTile);
+        tma_load_3d(smem + kOffX, &tm_x, &bars.x_full, h0 * kP, t0, b);
+        tma_load_3d(smem + kOffX + kTile, &tm_x, &bars.x_full, (h0 + 1) * kP, t0, b);
+      };
+      if (nb > 0) { load_c(0); load_b(0); load_x(0); }
+      if (nb > 1) load_b(1);
+      for (int k = 0; k + 1 < nb; ++k) {
+        if (!mbar_wait(&bars.c_empty, k & 1, abort_v, 31)) break;  // C H of block k done
+        load_c(k + 1);
+        if (!mbar_wait(&bars.x_empty, k & 1, abort_v, 32)) break;  // state MMA of block k done
+        load_x(k + 1);
+        if (k + 2 < nb) {
+          if (!mbar_wait(&bars.b_empty[k & 1], (k >> 1) & 1, abort_v, 33)) break;
+          load_b(k + 2);
+        }
       }
-      mma_commit(&mma_bar);
     }
-    // ---- H pass (lane n = row, head = half): hi/lo bf16 copy of H for C H, then
-    //      H <- exp(cs_end) H in place ----
+  } else if (warp == 17) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
+      const uint32_t id_off = idesc_bf16(128, 128, 0, 1);
+      const uint32_t id_diag = idesc_bf16(128, 64, 0, 1);
+      const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
+      for (int k = 0; k < nb; ++k) {
+        const uint32_t par = k & 1;
+        const uint32_t sx = sbase + kOffX;
+        const uint32_t sb = sbase + kOffB + (k & 1) * 2 * kTile;
+        if (k > 0 && !mbar_wait(&bars.d1_done, par ^ 1, abort_v, 41)) break;  // G region free
+        if (!mbar_wait(&bars.c_full, par, abort_v, 42)) break;
+        if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43)) break;
+        tc_fence_after();
+        // G = C B^T (M = t, N = s, K = n)
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * kTile + (kk & 3) * 32;
+          mma_ss(tG, sdesc(sbase + kOffC + koff, 16, 1024), sdesc(sb + koff, 16, 1024), id_g,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars.g_done);
+        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n)
+        if (!mbar_wait(&bars.h_ready, par, abort_v, 44)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          const uint64_t ad = sdesc(sbase + kOffC + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
+          mma_ss(tO, ad, sdesc(sbase + kOffHh + kk * 2048, kTile, 1024), id_off,
+                 kk > 0 ? 1u : 0u);
+          mma_ss(tO, ad, sdesc(sbase + kOffHl + kk * 2048, kTile, 1024), id_off, 1u);
+        }
+        mma_commit(&bars.c_empty);
+        // Diag_h = (Mhi_h + Mlo_h) X_h (M = t, N = p, K = s), A from TMEM
+        if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
+        bool fail = false;
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(h ? &bars.m1_ready : &bars.m0_ready, par, abort_v, 46)) {
+            fail = true;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk) {
+            const uint32_t acol = tG + kk * 16;
+            const uint64_t bd = sdesc(sx + h * kTile + kk * 2048, kTile, 1024);
+            mma_ts(tD + h * 64, acol, bd, id_diag, kk > 0 ? 1u : 0u);
+            mma_ts(tD + h * 64, acol + 8, bd, id_diag, 1u);
+          }
+          mma_commit(h ? &bars.d1_done : &bars.d0_done);
+        }
+        if (fail) break;
+        // H += B^T X' (M = n, N = (head, p), K = t)
+        if (!mbar_wait(&bars.xp_ready, par, abort_v, 47)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          mma_ss(tH, sdesc(sb + kk * 2048, kTile, 1024), sdesc(sx + kk * 2048, kTile, 1024),
+                 id_st, 1u);
+        mma_commit(&bars.st_done);
+        mma_commit(&bars.x_empty);
+        mma_commit(&bars.b_empty[k & 1]);
+      }
+    }
+  } else {
+    // ------------------------------ compute warps ------------------------------
+    const int row = tid & 127, q = tid >> 7;
+    const int j = q >> 1, p0 = (q & 1) * 32;        // head and p-range of the state/epilogue
+    const int wq = warp & 3;                        // TMEM lane quarter of this warp
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    // entering state of the segment -> TMEM (lane n = row, columns (j, p0 .. p0+32))
     {
-      tc_fence_after();
-      const float al = ex2(cs_sh[half][kBlk - 1]);
-      uint8_t* hh = smem + kOffHh + half * kTile;
-      uint8_t* hl = smem + kOffHl + half * kTile;
+      const float* src =
+          h_in + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP + p0) * kN + row;
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
+      for (int pc = 0; pc < 2; ++pc) {
         uint32_t r[16];
-        tmem_ld16(tH + lane_off + half * 64 + pc * 16, r);
-        tmem_wait_ld();
-        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          split2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), hi[e], lo[e]);
-        *reinterpret_cast<uint4*>(hh + swz(row, pc * 2)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(hh + swz(row, pc * 2 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-        *reinterpret_cast<uint4*>(hl + swz(row, pc * 2)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4*>(hl + swz(row, pc * 2 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * al);
-        tmem_st16(tH + lane_off + half * 64 + pc * 16, r);
+        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(src[(pc * 16 + e) * kN]);
+        tmem_st16(tH + lane_off + j * 64 + p0 + pc * 16, r);
       }
       tmem_wait_st();
-      fence_proxy_async_smem();
     }
-    tc_fence_before();
-    __syncthreads();
-    // ---- Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n) ----
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+    const bool scan_thread = (q & 1) == 0;          // q = 0 scans head 0, q = 2 head 1
+    const float Alog = A[h0 + j] * kLog2e;
+    const float Dh = D ? D[h0 + j] : 0.f;
+    const float* dtp = dt + int64_t(b) * seqlen * nheads + h0 + j;
+    auto dt_at = [&](int k) {
+      const int64_t tok = int64_t(blk0 + k) * kBlk + row;
+      return (scan_thread && k < nb && tok < seqlen) ? dtp[tok * nheads] : 0.f;
+    };
+    float d_next = dt_at(0);
+    bool ok = true;
+    uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
+    for (int k = 0; k < nb; ++k) {
+      const uint32_t par = k & 1;
+      const int t0 = (blk0 + k) * kBlk;
+      const float d = d_next;
+      d_next = dt_at(k + 1);  // prefetch the next block's step sizes
+      // the previous block's y stores must have read the staging buffer (sHh/sHl) before the
+      // state pass below overwrites it
+      if (tid == 0) bulk_wait_read();
+      // ---- within-block log2 cumsums (warps 0-3: head 0, warps 8-11: head 1);
+      //      v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15 ----
+      {
+        float v = warp_inclusive_scan(d * Alog);
+        if (lane == 31) scan_scratch[warp] = v;
+        named_sync(1, kComputeThreads);
+        if (scan_thread) {
+          const int w0 = warp & ~3;
+          float off = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < kN / 16; ++kk) {
-        const uint64_t ad = sdesc(sbase + kOffC + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
-        mma_ss(tO, ad, sdesc(sbase + kOffHh + kk * 2048, kTile, 1024), idesc, kk > 0 ? 1u : 0u);
-        mma_ss(tO, ad, sdesc(sbase + kOffHl + kk * 2048, kTile, 1024), idesc, 1u);
+          for (int w = 0; w < 4; ++w) off += (w0 + w < warp) ? scan_scratch[w0 + w] : 0.f;
+          cs_sh[j][row] = v + off;
+          dt_sh[j][row] = d;
+        }
+        named_sync(1, kComputeThreads);
+        if (scan_thread) v_sh[j][row] = ex2(cs_sh[j][row | 15] - cs_sh[j][row]) * d;
       }
-    }
-    ok = mbar_wait(&mma_bar, mma_phase, abort_v, 22);  // G complete
-    mma_phase ^= 1;
-    tc_fence_after();
-    // ---- masked tiles, one head at a time: M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for
-    //      s <= t.  Thread (row t, column half c) keeps G[t, 64c .. 64c+64) in registers and
-    //      writes head h's mask over those TMEM columns as a bf16 high part (columns
-    //      64c .. 64c+32) and the bf16 rounding of the remainder (64c+32 .. 64c+64); the
-    //      diagonal MMAs read both as their A operand, so the mask carries ~16 bits. ----
-    float gv[64];
-    const bool g_live = (warp & 3) * 32 + 31 >= half * 64;  // some row of the warp reaches 64c
-    if (ok && g_live) {
-      const uint32_t gaddr = tG + lane_off + half * 64;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[16];
-        tmem_ld16(gaddr + q * 16, r);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) gv[q * 16 + e] = __uint_as_float(r[e]);
-      }
-      tmem_wait_ld();
-    }
-#pragma unroll 1
-    for (int h = 0; h < 2; ++h) {
+      // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
+      //      C H, then H <- exp(cs_end) H in place; needs the previous block's state MMA ----
+      if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51);
+      named_sync(1, kComputeThreads);  // cs/v published; staging free
       if (ok) {
-        const int t = row, c = half;
-        const uint32_t gaddr = tG + lane_off + c * 64;
-        uint32_t hi[32], lo[32];
-        if (g_live) {
+        tc_fence_after();
+        const float al = ex2(cs_sh[j][kBlk - 1]);
+        uint8_t* hh = smem + kOffHh + j * kTile;
+        uint8_t* hl = smem + kOffHl + j * kTile;
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc) {
+          uint32_t r[16];
+          tmem_ld16(tH + lane_off + j * 64 + p0 + pc * 16, r);
+          tmem_wait_ld();
+          uint32_t hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            split2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), hi[e], lo[e]);
+          const int ch = (p0 >> 3) + pc * 2;
+          *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+          *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * al);
+          tmem_st16(tH + lane_off + j * 64 + p0 + pc * 16, r);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.h_ready);
+      // ---- masked tiles, one head at a time.  Thread (row t, q): G columns [32q, 32q+32),
+      //      i.e. the 16-column groups kk = 2q, 2q+1; M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s
+      //      for s <= t, written over the group's TMEM columns as 8 columns of bf16 high parts
+      //      followed by 8 of low parts ----
+      const int t = row;
+      const bool live = q <= wq;  // group 2q starts at column 32q <= the warp's last row
+      const uint32_t gaddr = tG + lane_off + q * 32;
+      float gv[32];
+      ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52);
+      if (ok && live) {
+        tc_fence_after();
+        uint32_t r0[16], r1[16];
+        tmem_ld16(gaddr, r0);
+        tmem_ld16(gaddr + 16, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) { gv[e] = __uint_as_float(r0[e]); gv[16 + e] = __uint_as_float(r1[e]); }
+      }
+      // one 16-column group of head h's mask into r (8 high + 8 low packed pairs)
+      auto mask_group = [&](int h, int gg, uint32_t (&r)[16]) {
+        const int s0 = q * 32 + gg * 16;
+        if (live && t >= s0 + 15) {  // the whole group lies at or before t
+          const float u = ex2(cs_sh[h][t] - cs_sh[h][s0 + 15]);
+          const float4* vp = reinterpret_cast<const float4*>(&v_sh[h][s0]);
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 vv = vp[e4];
+            split2(gv[gg * 16 + 4 * e4 + 0] * (u * vv.x), gv[gg * 16 + 4 * e4 + 1] * (u * vv.y),
+                   r[2 * e4], r[8 + 2 * e4]);
+            split2(gv[gg * 16 + 4 * e4 + 2] * (u * vv.z), gv[gg * 16 + 4 * e4 + 3] * (u * vv.w),
+                   r[2 * e4 + 1], r[8 + 2 * e4 + 1]);
+          }
+        } else if (live && t >= s0) {  // diagonal group: exact exps, zero above the diagonal
           const float ct = cs_sh[h][t];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int s0 = c * 64 + q * 16;
-            float f[16];
-            if (t >= s0 + 15) {  // the whole 16-column sub-block is at or before t
-              const float u = ex2(ct - cs_sh[h][s0 + 15]);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) f[e] = gv[q * 16 + e] * (u * v_sh[h][s0 + e]);
-            } else if (t >= s0) {  // diagonal sub-block: exact exps, zero above the diagonal
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int s = s0 + e;
-                f[e] = s <= t ? gv[q * 16 + e] * ex2(ct - cs_sh[h][s]) * dt_sh[h][s] : 0.f;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) f[e] = 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) split2(f[2 * e], f[2 * e + 1], hi[q * 8 + e], lo[q * 8 + e]);
+          for (int e = 0; e < 8; ++e) {
+            const int sa = s0 + 2 * e, sb2 = sa + 1;
+            const float fa = sa <= t ? gv[gg * 16 + 2 * e] * ex2(ct - cs_sh[h][sa]) * dt_sh[h][sa] : 0.f;
+            const float fb = sb2 <= t ? gv[gg * 16 + 2 * e + 1] * ex2(ct - cs_sh[h][sb2]) * dt_sh[h][sb2] : 0.f;
+            split2(fa, fb, r[e], r[8 + e]);
           }
-        } else {  // every row of this warp lies before column 64c: zero masks
+        } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) { hi[e] = 0u; lo[e] = 0u; }
+          for (int e = 0; e < 16; ++e) r[e] = 0u;
         }
-        uint32_t r[16];
+      };
+      // head 0: compute and store group by group
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = hi[e];
-        tmem_st16(gaddr, r);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = hi[16 + e];
-        tmem_st16(gaddr + 16, r);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = lo[e];
-        tmem_st16(gaddr + 32, r);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = lo[16 + e];
-        tmem_st16(gaddr + 48, r);
+        for (int gg = 0; gg < 2; ++gg) {
+          uint32_t r[16];
+          mask_group(0, gg, r);
+          tmem_st16(gaddr + gg * 16, r);
+        }
         tmem_wait_st();
       }
       tc_fence_before();
-      if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
-      // ---- Diag_h = (Mhi_h + Mlo_h) X_h (M = t, N = p, K = s), A from TMEM ----
-      if (tid == 0) {
+      mbar_arrive(&bars.m0_ready);
+      // head 1: computed while the first diagonal MMA runs; stored over head 0's mask once
+      // that MMA has read it
+      {
+        uint32_t r0[16], r1[16];
+        if (ok) {
+          mask_group(1, 0, r0);
+          mask_group(1, 1, r1);
+        }
+        ok = ok && mbar_wait(&bars.d0_done, par, abort_v, 53);
+        if (ok) {
+          tc_fence_after();
+          tmem_st16(gaddr, r0);
+          tmem_st16(gaddr + 16, r1);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(&bars.m1_ready);
+      }
+      // ---- once both diagonal MMAs (and C H) are done: X' = w x in place for the state MMA
+      //      (row t, head j, p in [p0, p0+32)), then y_t = Diag + exp(cs_t) Off + D x_t staged
+      //      in shared memory and written by TMA ----
+      ok = ok && mbar_wait(&bars.d1_done, par, abort_v, 54);
+      uint32_t xw[16];
+      if (ok) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64, 0, 1);
+        const float wj = ex2(cs_sh[j][kBlk - 1] - cs_sh[j][t]) * dt_sh[j][t];
+        uint8_t* xrow = smem + kOffX + j * kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          const uint32_t acol = tG + (kk >> 2) * 64 + (kk & 3) * 8;
-          const uint64_t bd = sdesc(sbase + kOffX + h * kTile + kk * 2048, kTile, 1024);
-          mma_ts(tD + h * 64, acol, bd, idesc, kk > 0 ? 1u : 0u);
-          mma_ts(tD + h * 64, acol + 32, bd, idesc, 1u);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint4* pch = reinterpret_cast<uint4*>(xrow + swz(t, (p0 >> 3) + cc));
+          const uint4 v = *pch;
+          xw[cc * 4 + 0] = v.x; xw[cc * 4 + 1] = v.y; xw[cc * 4 + 2] = v.z; xw[cc * 4 + 3] = v.w;
+          *pch = make_uint4(pack_bf16x2(bf16lo(v.x) * wj, bf16hi(v.x) * wj),
+                            pack_bf16x2(bf16lo(v.y) * wj, bf16hi(v.y) * wj),
+                            pack_bf16x2(bf16lo(v.z) * wj, bf16hi(v.z) * wj),
+                            pack_bf16x2(bf16lo(v.w) * wj, bf16hi(v.w) * wj));
         }
-        mma_commit(&mma_bar);  // head 0: covers Off as well
+        fence_proxy_async_smem();
       }
-      ok = mbar_wait(&mma_bar, mma_phase, abort_v, 23);
-      mma_phase ^= 1;
-      tc_fence_after();
-    }
-    tc_fence_before();
-    if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
-    tc_fence_after();
-    // ---- epilogue (row t, head = half): y_t = Diag + exp(cs_t) Off + D x_t; then X' = w x ----
-    if (ok) {
-      const int t = row, j = half;
-      const float ej = ex2(cs_sh[j][t]);
-      const float wj = ex2(cs_sh[j][kBlk - 1] - cs_sh[j][t]) * dt_sh[j][t];
-      uint8_t* xrow = smem + kOffX + j * kTile;
-      TY* yrow = y + ((int64_t(b) * seqlen + tok) * nheads + h0 + j) * kP;
+      mbar_arrive(&bars.xp_ready);
+      if (ok) {
+        const float ej = ex2(cs_sh[j][t]);
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        uint32_t rd[16], ro[16];
-        tmem_ld16(tD + lane_off + j * 64 + pc * 16, rd);
-        tmem_ld16(tO + lane_off + j * 64 + pc * 16, ro);
-        tmem_wait_ld();
-        uint4* x0p = reinterpret_cast<uint4*>(xrow + swz(t, pc * 2));
-        uint4* x1p = reinterpret_cast<uint4*>(xrow + swz(t, pc * 2 + 1));
-        const uint4 xa = *x0p, xb = *x1p;
-        const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        float yv[16];
-        uint32_t xs[8];
+        for (int pc = 0; pc < 2; ++pc) {
+          uint32_t rd[16], ro[16];
+          tmem_ld16(tD + lane_off + j * 64 + p0 + pc * 16, rd);
+          tmem_ld16(tO + lane_off + j * 64 + p0 + pc * 16, ro);
+          tmem_wait_ld();
+          float yv[16];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float xl = bf16lo(xw[e]), xh = bf16hi(xw[e]);
-          yv[2 * e] = __uint_as_float(rd[2 * e]) + ej * __uint_as_float(ro[2 * e]) + Dh * xl;
-          yv[2 * e + 1] =
-              __uint_as_float(rd[2 * e + 1]) + ej * __uint_as_float(ro[2 * e + 1]) + Dh * xh;
-          xs[e] = pack_bf16x2(xl * wj, xh * wj);
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t xv = xw[pc * 8 + e];
+            yv[2 * e] = __uint_as_float(rd[2 * e]) + ej * __uint_as_float(ro[2 * e]) + Dh * bf16lo(xv);
+            yv[2 * e + 1] =
+                __uint_as_float(rd[2 * e + 1]) + ej * __uint_as_float(ro[2 * e + 1]) + Dh * bf16hi(xv);
+          }
+          ystage<TY>::put16(stage, t, q, pc, yv);
         }
-        if (tok < seqlen) yout<TY>::store16(yrow + pc * 16, yv);
-        *x0p = make_uint4(xs[0], xs[1], xs[2], xs[3]);
-        *x1p = make_uint4(xs[4], xs[5], xs[6], xs[7]);
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      tc_fence_before();
+      // all compute threads are done with this block's cs/dt/v, TMEM reads and y staging
+      if (named_sync_or(1, kComputeThreads, !ok || *abort_v)) { ok = false; break; }
+      if (tid == 0) {
+        ystage<TY>::store(&tm_y, stage, h0, t0, b);
+        bulk_commit();
+      }
     }
-    tc_fence_before();
-    if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
-    // ---- H += B^T X' (M = n, N = (head, p), K = t) ----
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
-#pragma unroll
-      for (int kk = 0; kk < kBlk / 16; ++kk)
-        mma_ss(tH, sdesc(sbase + kOffB + kk * 2048, kTile, 1024),
-               sdesc(sbase + kOffX + kk * 2048, kTile, 1024), idesc, 1u);
-      mma_commit(&mma_bar);
-    }
-    ok = mbar_wait(&mma_bar, mma_phase, abort_v, 24);
-    mma_phase ^= 1;
-    tc_fence_after();
+    if (tid == 0) bulk_wait_all();
   }
-  if (__syncthreads_or(!ok || *abort_v)) {
-    if (tid == 0) {  // let an in-flight copy and every issued MMA land before leaving
-      drain(&tma_bar, tma_phase ^ 1);
-      mma_commit(&mma_bar);
-      drain(&mma_bar, mma_phase);
-    }
-    __syncthreads();
+  // ------------------------------ teardown ------------------------------
+  __syncthreads();
+  if (*abort_v && warp == 17 && lane == 0) {  // let every issued MMA land before leaving
+    mma_commit(&bars.drain);
+    drain(&bars.drain, 0);
+  }
+  if (*abort_v && warp == 16 && lane == 0) {  // and every issued copy
+    if (n_c) drain(&bars.c_full, (n_c - 1) & 1);
+    if (n_x) drain(&bars.x_full, (n_x - 1) & 1);
+    for (int i = 0; i < 2; ++i)
+      if (n_b[i]) drain(&bars.b_full[i], (n_b[i] - 1) & 1);
   }
   tc_fence_before();
   __syncthreads();

@@ -251,7 +251,7 @@ ssd_status run_tc(const Shape& s, const ScanArgs& a) {
     return SSD_ERR_CUDA;
   const int hpg = s.nheads / s.ngroups;
   const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-  ssd::tc::seg_state_kernel<<<grid, 256, kSegSmem, a.stream>>>(
+  ssd::tc::seg_state_kernel<<<grid, ssd::tc::kSegThreads, kSegSmem, a.stream>>>(
       mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;
@@ -513,7 +513,7 @@ ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, voi
     return SSD_ERR_CUDA;
   const int hpg = s.nheads / s.ngroups;
   const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-  ssd::tc::seg_state_kernel<<<grid, 256, kSegSmem, a.stream>>>(
+  ssd::tc::seg_state_kernel<<<grid, ssd::tc::kSegThreads, kSegSmem, a.stream>>>(
       mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;

@@ -78,29 +78,33 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 }
 
 // =============================================================================================
-// seg_state: grid = batch * nseg * (nheads / 2), block = 256 threads: thread (row = tid % 128,
-// head j = tid / 128) owns token row `row` of head j's x tile.  Per stage (two stages):
-//   B tile (2 x 16 KB, n halves) | X'hi (2 heads x 16 KB) | X'lo (2 heads x 16 KB)
-// X' = w * x is split into a bf16 high part (written over x) and a bf16 low part, and both go
-// through the tensor core, so the segment state carries ~16 significant bits of X'.
+// seg_state: grid = batch * nseg * (nheads / 2), block = 320 threads:
+//   warps 0-7  compute: thread (row = tid % 128, j = tid / 128) scales token row `row` of head
+//              j's x tile to X' = w x and splits it into a bf16 high part (over x) and low part.
+//   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0).
+// Per stage (two stages):  B tile (2 x 16 KB, n halves) | X'hi (2 heads) | X'lo (2 heads).
+// Blocks are walked last to first so that the suffix sums of the log-decays are running totals;
+// both X' parts go through the tensor core, so the segment state carries ~16 bits of X'.
 // TMEM: 128 columns, lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
 constexpr uint32_t kSegStage = 6 * kTile;
+constexpr int kSegThreads = 320;
 
-__global__ void __launch_bounds__(256, 1) seg_state_kernel(
+__global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const float* __restrict__ dt, const float* __restrict__ A, float* __restrict__ seg_states,
     float* __restrict__ seg_decay, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ uint64_t full_bar[2], mma_bar[2];
+  __shared__ uint64_t full_bar[2], ready_bar[2], empty_bar[2], done_bar, drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ float scan_scratch[8];
+  __shared__ float dt_stage[2][2][kBlk];  // [walk block % 2][head][row], filled by cp.async
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
-  const int row = tid & 127, j = tid >> 7, warp = tid >> 5;
+  const int warp = tid >> 5, lane = tid & 31;
   const int npair = nheads / 2;
   const int unit = blockIdx.x;
   const int hp = unit % npair;
@@ -110,114 +114,164 @@ __global__ void __launch_bounds__(256, 1) seg_state_kernel(
   const int g = h0 / heads_per_group;
   const int blk0 = seg * sg.seg_blks;
   const int nb = min(sg.nblk, blk0 + sg.seg_blks) - blk0;
+  volatile int* abort_v = &abort_flag;
+  uint32_t n_loads[2] = {0, 0};  // the producer's loads per stage
 
   if (tid == 0) {
     abort_flag = 0;
-    for (int i = 0; i < 2; ++i) { mbar_init(&full_bar[i], 1); mbar_init(&mma_bar[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&ready_bar[i], 256);
+      mbar_init(&empty_bar[i], 1);
+    }
+    mbar_init(&done_bar, 1);
+    mbar_init(&drain_bar, 1);
     fence_mbar_init();
-    prefetch_tmap(&tm_x);
-    prefetch_tmap(&tm_b);
   }
   if (warp == 0) tmem_alloc(&tmem_base_sh, 128);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  volatile int* abort_v = &abort_flag;
-  uint32_t n_loads[2] = {0, 0}, n_commits[2] = {0, 0};  // thread 0's issue counts per stage
 
-  auto issue_loads = [&](int i, int stage) {  // block i of the walk (last block first)
-    const int blk = blk0 + nb - 1 - i;
-    uint8_t* st = smem + stage * kSegStage;
-    ++n_loads[stage];
-    mbar_arrive_expect_tx(&full_bar[stage], 4 * kTile);
-    tma_load_3d(st, &tm_b, &full_bar[stage], g * kN, blk * kBlk, b);
-    tma_load_3d(st + kTile, &tm_b, &full_bar[stage], g * kN + 64, blk * kBlk, b);
-    tma_load_3d(st + 2 * kTile, &tm_x, &full_bar[stage], h0 * kP, blk * kBlk, b);
-    tma_load_3d(st + 3 * kTile, &tm_x, &full_bar[stage], (h0 + 1) * kP, blk * kBlk, b);
-  };
-
-  float run = 0.f;  // log2-decay of the blocks after the current one, within the segment
-  const float Alog = A[h0 + j] * kLog2e;
-  if (tid == 0) issue_loads(0, 0);
-  bool ok = true;
-  for (int i = 0; i < nb; ++i) {
-    const int stage = i & 1;
-    const int blk = blk0 + nb - 1 - i;
-    if (tid == 0 && i + 1 < nb) {
-      // the other stage is free once the MMAs of block i-1 have read it
-      if (i >= 1) ok = mbar_wait(&mma_bar[stage ^ 1], ((i - 1) >> 1) & 1, abort_v, 11);
-      if (ok) issue_loads(i + 1, stage ^ 1);
-    }
-    // w_t = exp(sum_{k > t, k in segment} a_k) * dt_t
-    const int64_t tok = int64_t(blk) * kBlk + row;
-    const float d = tok < seqlen ? dt[(int64_t(b) * seqlen + tok) * nheads + h0 + j] : 0.f;
-    float tot;
-    const float incl = half_scan128(d * Alog, scan_scratch, &tot);
-    const float w = ex2(tot - incl + run) * d;
-    run += tot;
-    ok = ok && mbar_wait(&full_bar[stage], (i >> 1) & 1, abort_v, 12);
-    if (ok) {
-      uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
-      uint8_t* lr = smem + stage * kSegStage + (4 + j) * kTile;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
-        const uint4 v = *ph;
-        uint4 hi, lo;
-        split2(bf16lo(v.x) * w, bf16hi(v.x) * w, hi.x, lo.x);
-        split2(bf16lo(v.y) * w, bf16hi(v.y) * w, hi.y, lo.y);
-        split2(bf16lo(v.z) * w, bf16hi(v.z) * w, hi.z, lo.z);
-        split2(bf16lo(v.w) * w, bf16hi(v.w) * w, hi.w, lo.w);
-        *ph = hi;
-        *reinterpret_cast<uint4*>(lr + swz(row, c)) = lo;
+  if (warp == 8) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_b);
+      for (int i = 0; i < nb; ++i) {  // block i of the walk = block blk0 + nb - 1 - i
+        const int stage = i & 1;
+        if (i >= 2 && !mbar_wait(&empty_bar[stage], ((i - 2) >> 1) & 1, abort_v, 11)) break;
+        const int t0 = (blk0 + nb - 1 - i) * kBlk;
+        uint8_t* st = smem + stage * kSegStage;
+        ++n_loads[stage];
+        mbar_arrive_expect_tx(&full_bar[stage], 4 * kTile);
+        tma_load_3d(st, &tm_b, &full_bar[stage], g * kN, t0, b);
+        tma_load_3d(st + kTile, &tm_b, &full_bar[stage], g * kN + 64, t0, b);
+        tma_load_3d(st + 2 * kTile, &tm_x, &full_bar[stage], h0 * kP, t0, b);
+        tma_load_3d(st + 3 * kTile, &tm_x, &full_bar[stage], (h0 + 1) * kP, t0, b);
       }
-      fence_proxy_async_smem();
     }
-    tc_fence_before();
-    if (__syncthreads_or(!ok || *abort_v)) { ok = false; break; }
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sb = smem_u32(smem + stage * kSegStage);
+  } else if (warp == 9) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+      for (int i = 0; i < nb; ++i) {
+        const int stage = i & 1;
+        if (!mbar_wait(&ready_bar[stage], (i >> 1) & 1, abort_v, 12)) break;
+        tc_fence_after();
+        const uint32_t sb = smem_u32(smem + stage * kSegStage);
 #pragma unroll
-      for (int k = 0; k < kBlk / 16; ++k) {
-        const uint64_t ad = sdesc(sb + k * 2048, kTile, 1024);               // B^T: M = n
-        mma_ss(tmem, ad, sdesc(sb + 2 * kTile + k * 2048, kTile, 1024), idesc,
-               (i > 0 || k > 0) ? 1u : 0u);                                   // X'hi
-        mma_ss(tmem, ad, sdesc(sb + 4 * kTile + k * 2048, kTile, 1024), idesc, 1u);  // X'lo
-      }
-      mma_commit(&mma_bar[stage]);
-      ++n_commits[stage];
-    }
-  }
-  if (ok && nb > 0) {
-    const int last = nb - 1;
-    ok = mbar_wait(&mma_bar[last & 1], (last >> 1) & 1, abort_v, 13);
-  }
-  if (__syncthreads_or(!ok || *abort_v)) {
-    if (tid == 0) {  // let in-flight copies and MMAs land before the CTA leaves
-      for (int i = 0; i < 2; ++i) {
-        if (n_loads[i]) drain(&full_bar[i], (n_loads[i] - 1) & 1);
-        mma_commit(&mma_bar[i]);  // arrives once every earlier MMA is done
-        drain(&mma_bar[i], n_commits[i] & 1);
+        for (int k = 0; k < kBlk / 16; ++k) {
+          const uint64_t ad = sdesc(sb + k * 2048, kTile, 1024);               // B^T: M = n
+          mma_ss(tmem, ad, sdesc(sb + 2 * kTile + k * 2048, kTile, 1024), idesc,
+                 (i > 0 || k > 0) ? 1u : 0u);                                   // X' (high)
+          if (i == 0)
+            mma_ss(tmem, ad, sdesc(sb + 4 * kTile + k * 2048, kTile, 1024), idesc, 1u);  // low
+        }
+        mma_commit(&empty_bar[stage]);
+        if (i == nb - 1) mma_commit(&done_bar);
       }
     }
-    __syncthreads();
   } else {
-    tc_fence_after();
-    // epilogue: lane n = row, columns of head j
-    const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + j * 64;
-    float* out = seg_states + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP) * kN + row;
+    // ------------------------------ compute warps ------------------------------
+    const int row = tid & 127, j = tid >> 7;
+    const float Alog = A[h0 + j] * kLog2e;
+    const float* dtp = dt + int64_t(b) * seqlen * nheads + h0 + j;
+    // step sizes of walk block i -> dt_stage[i % 2], one block ahead
+    auto fetch_dt = [&](int i) {
+      const int64_t tok = int64_t(blk0 + nb - 1 - i) * kBlk + row;
+      const bool valid = i < nb && tok < seqlen;
+      cp_async4(&dt_stage[i & 1][j][row], valid ? dtp + tok * nheads : dtp, valid);
+      cp_async_commit();
+    };
+    float run = 0.f;  // log2-decay of the blocks after the current one, within the segment
+    fetch_dt(0);
+    bool ok = true;
+    for (int i = 0; i < nb; ++i) {
+      const int stage = i & 1;
+      fetch_dt(i + 1);
+      cp_async_wait_prev();  // this thread's element of block i has landed
+      const float d = dt_stage[i & 1][j][row];
+      // w_t = exp(sum_{k > t, k in segment} a_k) * dt_t
+      const float a = d * Alog;
+      float v = warp_inclusive_scan(a);
+      if (lane == 31) scan_scratch[warp] = v;
+      named_sync(1, 256);
+      const int w0 = warp & ~3;
+      float off = 0.f, tot = 0.f;
 #pragma unroll
-    for (int pc = 0; pc < 4; ++pc) {
-      uint32_t r[16];
-      tmem_ld16(lane_addr + pc * 16, r);
-      tmem_wait_ld();
+      for (int w = 0; w < 4; ++w) {
+        const float sw = scan_scratch[w0 + w];
+        off += (w0 + w < warp) ? sw : 0.f;
+        tot += sw;
+      }
+      named_sync(1, 256);  // scratch read by everyone before the next block overwrites it
+      const float incl = v + off;
+      const float wt = ex2(tot - incl + run) * d;  // tot - incl = sum over k > t in this block
+      run += tot;
+      ok = ok && mbar_wait(&full_bar[stage], (i >> 1) & 1, abort_v, 13);
+      if (ok) {
+        uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
+        uint8_t* lr = smem + stage * kSegStage + (4 + j) * kTile;
+        if (i == 0) {  // the segment's last block: bf16 high part in place, low part beside it
 #pragma unroll
-      for (int e = 0; e < 16; ++e) out[(pc * 16 + e) * kN] = nb > 0 ? __uint_as_float(r[e]) : 0.f;
+          for (int c = 0; c < 8; ++c) {
+            uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
+            const uint4 xv = *ph;
+            uint4 hi, lo;
+            split2(bf16lo(xv.x) * wt, bf16hi(xv.x) * wt, hi.x, lo.x);
+            split2(bf16lo(xv.y) * wt, bf16hi(xv.y) * wt, hi.y, lo.y);
+            split2(bf16lo(xv.z) * wt, bf16hi(xv.z) * wt, hi.z, lo.z);
+            split2(bf16lo(xv.w) * wt, bf16hi(xv.w) * wt, hi.w, lo.w);
+            *ph = hi;
+            *reinterpret_cast<uint4*>(lr + swz(row, c)) = lo;
+          }
+        } else {  // earlier blocks: bf16 X' in place
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
+            const uint4 xv = *ph;
+            *ph = make_uint4(pack_bf16x2(bf16lo(xv.x) * wt, bf16hi(xv.x) * wt),
+                             pack_bf16x2(bf16lo(xv.y) * wt, bf16hi(xv.y) * wt),
+                             pack_bf16x2(bf16lo(xv.z) * wt, bf16hi(xv.z) * wt),
+                             pack_bf16x2(bf16lo(xv.w) * wt, bf16hi(xv.w) * wt));
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(&ready_bar[stage]);
+      if (named_sync_or(1, 256, !ok || *abort_v)) { ok = false; break; }
     }
-    if (row == 0) seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + j] = run;
+    cp_async_wait_all();  // the copy issued past the last block
+    // epilogue: lane n = row, columns of head j
+    if (ok && nb > 0) ok = mbar_wait(&done_bar, 0, abort_v, 14);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + j * 64;
+      float* out =
+          seg_states + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP) * kN + row;
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t r[16];
+        tmem_ld16(lane_addr + pc * 16, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          out[(pc * 16 + e) * kN] = nb > 0 ? __uint_as_float(r[e]) : 0.f;
+      }
+      if (row == 0) seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + j] = run;
+    }
+  }
+  // ------------------------------ teardown ------------------------------
+  __syncthreads();
+  if (*abort_v && warp == 9 && lane == 0) {  // let every issued MMA land before leaving
+    mma_commit(&drain_bar);
+    drain(&drain_bar, 0);
+  }
+  if (*abort_v && warp == 8 && lane == 0) {  // and every issued copy
+    for (int i = 0; i < 2; ++i)
+      if (n_loads[i]) drain(&full_bar[i], (n_loads[i] - 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -275,6 +329,7 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(float* __restrict__ seg_s
 //               TMEM lane quarter, so every phase is spread over all 16 warps.
 //   warp 16     TMA producer (lane 0): C, x (single buffers), B (double buffer) per block.
 //   warp 17     MMA issuer (lane 0).
+//   warp 18     y writer (lane 0): TMA stores of each block's staged y, off the compute path.
 // The roles hand blocks to each other through mbarriers, so the loads of the next block, the
 // tensor-core work and the CUDA-core work of different phases overlap.
 // Shared memory (1024-aligned, 12 x 16 KB):
@@ -288,13 +343,13 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(float* __restrict__ seg_s
 //   (sHh + sHl, free once C H has been computed, stage the block's y for the TMA stores)
 // TMEM (512 columns): [0,128) running state H (head, p) | [128,256) diagonal accumulators |
 //   [256,384) off-diagonal accumulators C H | [384,512) G = C B^T, overwritten in place, one
-//   head at a time, by that head's masked tile: for each 16-column group kk, 8 columns of bf16
-//   high parts then 8 of low parts, which the diagonal MMAs read as their A operand.
+//   head at a time, by that head's bf16 masked tile (16-column group kk -> its first 8
+//   columns), which the diagonal MMAs read as their A operand.
 // =============================================================================================
 constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 6 * kTile, kOffHh = 8 * kTile,
                    kOffHl = 10 * kTile, kSmemTiles = 12 * kTile;
 constexpr int kComputeThreads = 512;
-constexpr int kOutThreads = kComputeThreads + 64;
+constexpr int kOutThreads = kComputeThreads + 96;
 
 // y staging (in sHh/sHl) and its TMA stores.  Float32 y: 4 boxes {32 p, 128 t} (one per
 // thread quarter q: head q/2, p-half q%2), 128B-swizzled.  Bf16 y: 2 boxes {64 p, 128 t} (one
@@ -344,6 +399,7 @@ struct OutBars {
   uint64_t c_empty, b_empty[2], x_empty;   // MMA completion -> producer
   uint64_t g_done, d0_done, d1_done, st_done;  // MMA completion -> compute
   uint64_t h_ready, m0_ready, m1_ready, xp_ready;  // compute -> MMA issuer
+  uint64_t y_staged, stage_free;  // compute <-> y writer
   uint64_t drain;
 };
 
@@ -359,8 +415,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
   __shared__ OutBars bars;
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(16) float cs_sh[2][kBlk];
-  __shared__ __align__(16) float dt_sh[2][kBlk];
+  __shared__ __align__(16) float cl_sh[2][kBlk];  // cs_s - log2(dt_s) (+inf where dt = 0)
   __shared__ __align__(16) float v_sh[2][kBlk];
+  __shared__ float dt_stage[2][2][kBlk];  // [block % 2][head][row], filled by cp.async
   __shared__ float scan_scratch[16];
   __shared__ int abort_flag;
 
@@ -386,6 +443,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     mbar_init(&bars.m0_ready, kComputeThreads);
     mbar_init(&bars.m1_ready, kComputeThreads);
     mbar_init(&bars.xp_ready, kComputeThreads);
+    mbar_init(&bars.y_staged, kComputeThreads);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&tmem_base_sh, 512);
@@ -460,6 +518,19 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars.g_done);
+        // Diag_h = (Mhi_h + Mlo_h) X_h (M = t, N = p, K = s), A from TMEM; head 0 first, then
+        // C H while head 1's mask is being written, then head 1
+        if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
+        auto diag = [&](int h) {
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk)
+            mma_ts(tD + h * 64, tG + kk * 16,
+                   sdesc(sx + h * kTile + kk * 2048, kTile, 1024), id_diag, kk > 0 ? 1u : 0u);
+        };
+        if (!mbar_wait(&bars.m0_ready, par, abort_v, 46)) break;
+        tc_fence_after();
+        diag(0);
+        mma_commit(&bars.d0_done);
         // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n)
         if (!mbar_wait(&bars.h_ready, par, abort_v, 44)) break;
         tc_fence_after();
@@ -471,25 +542,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
           mma_ss(tO, ad, sdesc(sbase + kOffHl + kk * 2048, kTile, 1024), id_off, 1u);
         }
         mma_commit(&bars.c_empty);
-        // Diag_h = (Mhi_h + Mlo_h) X_h (M = t, N = p, K = s), A from TMEM
-        if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
-        bool fail = false;
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(h ? &bars.m1_ready : &bars.m0_ready, par, abort_v, 46)) {
-            fail = true;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {
-            const uint32_t acol = tG + kk * 16;
-            const uint64_t bd = sdesc(sx + h * kTile + kk * 2048, kTile, 1024);
-            mma_ts(tD + h * 64, acol, bd, id_diag, kk > 0 ? 1u : 0u);
-            mma_ts(tD + h * 64, acol + 8, bd, id_diag, 1u);
-          }
-          mma_commit(h ? &bars.d1_done : &bars.d0_done);
-        }
-        if (fail) break;
+        if (!mbar_wait(&bars.m1_ready, par, abort_v, 48)) break;
+        tc_fence_after();
+        diag(1);
+        mma_commit(&bars.d1_done);  // covers C H as well
         // H += B^T X' (M = n, N = (head, p), K = t)
         if (!mbar_wait(&bars.xp_ready, par, abort_v, 47)) break;
         tc_fence_after();
@@ -501,6 +557,20 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         mma_commit(&bars.x_empty);
         mma_commit(&bars.b_empty[k & 1]);
       }
+    }
+  } else if (warp == 18) {
+    // ------------------------------ y writer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tm_y);
+      const uint8_t* stage = smem + kOffHh;
+      for (int k = 0; k < nb; ++k) {
+        if (!mbar_wait(&bars.y_staged, k & 1, abort_v, 61)) break;
+        ystage<TY>::store(&tm_y, stage, h0, (blk0 + k) * kBlk, b);
+        bulk_commit();
+        bulk_wait_read();  // the staging buffer may be reused once the stores have read it
+        mbar_arrive(&bars.stage_free);
+      }
+      bulk_wait_all();
     }
   } else {
     // ------------------------------ compute warps ------------------------------
@@ -525,21 +595,26 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     const float Alog = A[h0 + j] * kLog2e;
     const float Dh = D ? D[h0 + j] : 0.f;
     const float* dtp = dt + int64_t(b) * seqlen * nheads + h0 + j;
-    auto dt_at = [&](int k) {
-      const int64_t tok = int64_t(blk0 + k) * kBlk + row;
-      return (scan_thread && k < nb && tok < seqlen) ? dtp[tok * nheads] : 0.f;
+    // step sizes of block k -> dt_stage[k % 2] (scan threads only), one block ahead
+    auto fetch_dt = [&](int k) {
+      if (scan_thread) {
+        const int64_t tok = int64_t(blk0 + k) * kBlk + row;
+        const bool valid = k < nb && tok < seqlen;
+        cp_async4(&dt_stage[k & 1][j][row], valid ? dtp + tok * nheads : dtp, valid);
+        cp_async_commit();
+      }
     };
-    float d_next = dt_at(0);
+    fetch_dt(0);
     bool ok = true;
     uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
     for (int k = 0; k < nb; ++k) {
       const uint32_t par = k & 1;
-      const int t0 = (blk0 + k) * kBlk;
-      const float d = d_next;
-      d_next = dt_at(k + 1);  // prefetch the next block's step sizes
-      // the previous block's y stores must have read the staging buffer (sHh/sHl) before the
-      // state pass below overwrites it
-      if (tid == 0) bulk_wait_read();
+      fetch_dt(k + 1);
+      float d = 0.f;
+      if (scan_thread) {
+        cp_async_wait_prev();  // block k's copy has landed (this thread's own element)
+        d = dt_stage[k & 1][j][row];
+      }
       // ---- within-block log2 cumsums (warps 0-3: head 0, warps 8-11: head 1);
       //      v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15 ----
       {
@@ -552,98 +627,107 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
 #pragma unroll
           for (int w = 0; w < 4; ++w) off += (w0 + w < warp) ? scan_scratch[w0 + w] : 0.f;
           cs_sh[j][row] = v + off;
-          dt_sh[j][row] = d;
+          cl_sh[j][row] = d > 0.f ? v + off - __log2f(d) : __int_as_float(0x7f800000);
         }
         named_sync(1, kComputeThreads);
-        if (scan_thread) v_sh[j][row] = ex2(cs_sh[j][row | 15] - cs_sh[j][row]) * d;
+        if (scan_thread) v_sh[j][row] = ex2(cs_sh[j][row | 15] - cl_sh[j][row]);
       }
       // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
-      //      C H, then H <- exp(cs_end) H in place; needs the previous block's state MMA ----
+      //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA, and
+      //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
       if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51);
-      named_sync(1, kComputeThreads);  // cs/v published; staging free
+      if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55);
+      named_sync(1, kComputeThreads);  // cs/v published
       if (ok) {
         tc_fence_after();
         const float al = ex2(cs_sh[j][kBlk - 1]);
         uint8_t* hh = smem + kOffHh + j * kTile;
         uint8_t* hl = smem + kOffHl + j * kTile;
-#pragma unroll
-        for (int pc = 0; pc < 2; ++pc) {
-          uint32_t r[16];
-          tmem_ld16(tH + lane_off + j * 64 + p0 + pc * 16, r);
-          tmem_wait_ld();
-          uint32_t hi[8], lo[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            split2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), hi[e], lo[e]);
-          const int ch = (p0 >> 3) + pc * 2;
-          *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-          *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-          *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * al);
-          tmem_st16(tH + lane_off + j * 64 + p0 + pc * 16, r);
-        }
+        uint32_t ra[16], rb[16];
+        tmem_ld16(tH + lane_off + j * 64 + p0, ra);
+        tmem_wait_ld();
+#define SSD_HPASS(R, PC)                                                                      \
+  {                                                                                           \
+    uint32_t hi[8], lo[8];                                                                    \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
+        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
+    const int ch = (p0 >> 3) + (PC) * 2;                                                      \
+    *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);    \
+    *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
+    *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
+    *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
+    _Pragma("unroll") for (int e = 0; e < 16; ++e) R[e] = __float_as_uint(__uint_as_float(R[e]) * al); \
+    tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
+  }
+        SSD_HPASS(ra, 0)
+        tmem_ld16(tH + lane_off + j * 64 + p0 + 16, rb);
+        tmem_wait_ld();
+        SSD_HPASS(rb, 1)
+#undef SSD_HPASS
         tmem_wait_st();
         fence_proxy_async_smem();
       }
       tc_fence_before();
       mbar_arrive(&bars.h_ready);
-      // ---- masked tiles, one head at a time.  Thread (row t, q): G columns [32q, 32q+32),
-      //      i.e. the 16-column groups kk = 2q, 2q+1; M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s
-      //      for s <= t, written over the group's TMEM columns as 8 columns of bf16 high parts
-      //      followed by 8 of low parts ----
+      // ---- masked tiles, one head at a time.  Thread (row t, q) owns the 16-column groups
+      //      q and q + 4 of G (columns [16q, 16q+16) and [16q+64, 16q+80)), which spreads the
+      //      rows' diagonal groups over all warps.  M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for
+      //      s <= t, written in bf16 over the first 8 TMEM columns of the group ----
       const int t = row;
-      const bool live = q <= wq;  // group 2q starts at column 32q <= the warp's last row
-      const uint32_t gaddr = tG + lane_off + q * 32;
+      const int wlast = wq * 32 + 31;                     // last row of this warp
+      const bool live0 = q * 16 <= wlast, live1 = (q + 4) * 16 <= wlast;
+      const uint32_t gaddr0 = tG + lane_off + q * 16, gaddr1 = gaddr0 + 64;
       float gv[32];
       ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52);
-      if (ok && live) {
+      if (ok && live0) {
         tc_fence_after();
         uint32_t r0[16], r1[16];
-        tmem_ld16(gaddr, r0);
-        tmem_ld16(gaddr + 16, r1);
+        tmem_ld16(gaddr0, r0);
+        if (live1) tmem_ld16(gaddr1, r1);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) { gv[e] = __uint_as_float(r0[e]); gv[16 + e] = __uint_as_float(r1[e]); }
       }
-      // one 16-column group of head h's mask into r (8 high + 8 low packed pairs)
-      auto mask_group = [&](int h, int gg, uint32_t (&r)[16]) {
-        const int s0 = q * 32 + gg * 16;
-        if (live && t >= s0 + 15) {  // the whole group lies at or before t
-          const float u = ex2(cs_sh[h][t] - cs_sh[h][s0 + 15]);
-          const float4* vp = reinterpret_cast<const float4*>(&v_sh[h][s0]);
-#pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 vv = vp[e4];
-            split2(gv[gg * 16 + 4 * e4 + 0] * (u * vv.x), gv[gg * 16 + 4 * e4 + 1] * (u * vv.y),
-                   r[2 * e4], r[8 + 2 * e4]);
-            split2(gv[gg * 16 + 4 * e4 + 2] * (u * vv.z), gv[gg * 16 + 4 * e4 + 3] * (u * vv.w),
-                   r[2 * e4 + 1], r[8 + 2 * e4 + 1]);
-          }
-        } else if (live && t >= s0) {  // diagonal group: exact exps, zero above the diagonal
-          const float ct = cs_sh[h][t];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int sa = s0 + 2 * e, sb2 = sa + 1;
-            const float fa = sa <= t ? gv[gg * 16 + 2 * e] * ex2(ct - cs_sh[h][sa]) * dt_sh[h][sa] : 0.f;
-            const float fb = sb2 <= t ? gv[gg * 16 + 2 * e + 1] * ex2(ct - cs_sh[h][sb2]) * dt_sh[h][sb2] : 0.f;
-            split2(fa, fb, r[e], r[8 + e]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = 0u;
-        }
-      };
-      // head 0: compute and store group by group
+      // one 16-column group (gg = 0: group q, gg = 1: group q + 4) of head h's mask, packed
+#define SSD_MASK_GROUP(H, GG, R)                                                               \
+  {                                                                                            \
+    const int s0 = (q + 4 * (GG)) * 16;                                                        \
+    const bool live = (GG) ? live1 : live0;                                                    \
+    if (live && t >= s0 + 15) {                                                                \
+      const float u = ex2(cs_sh[H][t] - cs_sh[H][s0 + 15]);                                    \
+      const float4* vp = reinterpret_cast<const float4*>(&v_sh[H][s0]);                        \
+      _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
+        const float4 vv = vp[e4];                                                              \
+        R[2 * e4] = pack_bf16x2(gv[(GG) * 16 + 4 * e4] * (u * vv.x),                           \
+                                gv[(GG) * 16 + 4 * e4 + 1] * (u * vv.y));                      \
+        R[2 * e4 + 1] = pack_bf16x2(gv[(GG) * 16 + 4 * e4 + 2] * (u * vv.z),                   \
+                                    gv[(GG) * 16 + 4 * e4 + 3] * (u * vv.w));                  \
+      }                                                                                        \
+    } else if (live && t >= s0) {                                                              \
+      const float ct = cs_sh[H][t];                                                            \
+      const float4* cp = reinterpret_cast<const float4*>(&cl_sh[H][s0]);                       \
+      _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
+        const float4 cl = cp[e4];                                                              \
+        const int s = s0 + 4 * e4;                                                             \
+        const float f0 = s + 0 <= t ? gv[(GG) * 16 + 4 * e4 + 0] * ex2(ct - cl.x) : 0.f;       \
+        const float f1 = s + 1 <= t ? gv[(GG) * 16 + 4 * e4 + 1] * ex2(ct - cl.y) : 0.f;       \
+        const float f2 = s + 2 <= t ? gv[(GG) * 16 + 4 * e4 + 2] * ex2(ct - cl.z) : 0.f;       \
+        const float f3 = s + 3 <= t ? gv[(GG) * 16 + 4 * e4 + 3] * ex2(ct - cl.w) : 0.f;       \
+        R[2 * e4] = pack_bf16x2(f0, f1);                                                       \
+        R[2 * e4 + 1] = pack_bf16x2(f2, f3);                                                   \
+      }                                                                                        \
+    } else {                                                                                   \
+      _Pragma("unroll") for (int e = 0; e < 8; ++e) R[e] = 0u;                                \
+    }                                                                                          \
+  }
+      // head 0
       if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-          uint32_t r[16];
-          mask_group(0, gg, r);
-          tmem_st16(gaddr + gg * 16, r);
-        }
+        uint32_t r[8];
+        SSD_MASK_GROUP(0, 0, r)
+        tmem_st8(gaddr0, r);
+        SSD_MASK_GROUP(0, 1, r)
+        tmem_st8(gaddr1, r);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -651,21 +735,22 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       // head 1: computed while the first diagonal MMA runs; stored over head 0's mask once
       // that MMA has read it
       {
-        uint32_t r0[16], r1[16];
+        uint32_t r0[8], r1[8];
         if (ok) {
-          mask_group(1, 0, r0);
-          mask_group(1, 1, r1);
+          SSD_MASK_GROUP(1, 0, r0)
+          SSD_MASK_GROUP(1, 1, r1)
         }
         ok = ok && mbar_wait(&bars.d0_done, par, abort_v, 53);
         if (ok) {
           tc_fence_after();
-          tmem_st16(gaddr, r0);
-          tmem_st16(gaddr + 16, r1);
+          tmem_st8(gaddr0, r0);
+          tmem_st8(gaddr1, r1);
           tmem_wait_st();
         }
         tc_fence_before();
         mbar_arrive(&bars.m1_ready);
       }
+#undef SSD_MASK_GROUP
       // ---- once both diagonal MMAs (and C H) are done: X' = w x in place for the state MMA
       //      (row t, head j, p in [p0, p0+32)), then y_t = Diag + exp(cs_t) Off + D x_t staged
       //      in shared memory and written by TMA ----
@@ -673,7 +758,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       uint32_t xw[16];
       if (ok) {
         tc_fence_after();
-        const float wj = ex2(cs_sh[j][kBlk - 1] - cs_sh[j][t]) * dt_sh[j][t];
+        const float wj = ex2(cs_sh[j][kBlk - 1] - cl_sh[j][t]);
         uint8_t* xrow = smem + kOffX + j * kTile;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -708,15 +793,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         }
         fence_proxy_async_smem();
       }
+      mbar_arrive(&bars.y_staged);
       tc_fence_before();
       // all compute threads are done with this block's cs/dt/v, TMEM reads and y staging
       if (named_sync_or(1, kComputeThreads, !ok || *abort_v)) { ok = false; break; }
-      if (tid == 0) {
-        ystage<TY>::store(&tm_y, stage, h0, t0, b);
-        bulk_commit();
-      }
     }
-    if (tid == 0) bulk_wait_all();
+    cp_async_wait_all();  // the step-size copy issued past the last block
   }
   // ------------------------------ teardown ------------------------------
   __syncthreads();

@@ -77,12 +77,29 @@ Seg tc_segments(const Shape& s) {
   return sg;
 }
 
-size_t tc_workspace(const Shape& s) {
-  const Seg sg = tc_segments(s);
-  const size_t states = size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float);
-  const size_t decay = size_t(s.batch) * sg.nseg * s.nheads * sizeof(float);
-  return align256(states) + align256(decay);
+// Tensor-core path scratch: segment states [b, seg, h, 64, 128] f32 | segment log2-decays
+// [b, seg, h] f32 | per (b, head pair) completion counts (zeroed by the call itself).
+struct SegScratch {
+  float* states;
+  float* decay;
+  unsigned* count;
+};
+size_t seg_scratch_bytes(const Shape& s, const Seg& sg) {
+  return align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)) +
+         align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float)) +
+         align256(size_t(s.batch) * (s.nheads / 2) * sizeof(unsigned));
 }
+SegScratch seg_scratch(const Shape& s, const Seg& sg, void* base) {
+  char* p = static_cast<char*>(base);
+  SegScratch r;
+  r.states = reinterpret_cast<float*>(p);
+  p += align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float));
+  r.decay = reinterpret_cast<float*>(p);
+  p += align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float));
+  r.count = reinterpret_cast<unsigned*>(p);
+  return r;
+}
+size_t tc_workspace(const Shape& s) { return seg_scratch_bytes(s, tc_segments(s)); }
 
 size_t simt_workspace(const Shape& s) {
   const int64_t nchunks = (s.seqlen + s.chunk - 1) / s.chunk;
@@ -238,35 +255,34 @@ ssd_status run_simt(const Shape& s, const ScanArgs& a) {
   return launched();
 }
 
-ssd_status run_tc(const Shape& s, const ScanArgs& a) {
-  const Seg sg = tc_segments(s);
-  float* seg_states = static_cast<float*>(a.ws);
-  float* seg_decay = reinterpret_cast<float*>(
-      static_cast<char*>(a.ws) +
-      align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)));
-  CUtensorMap mx, mb, mc;
+ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, void* scratch) {
+  const SegScratch w = seg_scratch(s, sg, scratch);
+  CUtensorMap mx, mb, mc, my;
   const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
   if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch) ||
-      !make_map(&mc, a.C, GN, s.seqlen, s.batch))
+      !make_map(&mc, a.C, GN, s.seqlen, s.batch) ||
+      !make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32))
     return SSD_ERR_CUDA;
   const int hpg = s.nheads / s.ngroups;
   const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
+  if (cudaMemsetAsync(w.count, 0, size_t(s.batch) * (s.nheads / 2) * sizeof(unsigned),
+                      a.stream) != cudaSuccess)
+    return SSD_ERR_CUDA;
   ssd::tc::seg_state_kernel<<<grid, ssd::tc::kSegThreads, kSegSmem, a.stream>>>(
-      mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
+      mx, mb, a.dt, a.A, w.states, w.decay, w.count, a.init, a.fin, s.seqlen, s.nheads, hpg,
+      sg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;
-  ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
-      seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
-  if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  CUtensorMap my;
-  if (!make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32)) return SSD_ERR_CUDA;
   if (a.ydt == SSD_F32)
     ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
-        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
+        mx, mb, mc, my, a.dt, a.A, a.D, w.states, s.seqlen, s.nheads, hpg, sg);
   else
     ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
-        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
+        mx, mb, mc, my, a.dt, a.A, a.D, w.states, s.seqlen, s.nheads, hpg, sg);
   return launched();
+}
+
+ssd_status run_tc(const Shape& s, const ScanArgs& a) {
+  return run_tc_segments(s, a, tc_segments(s), a.ws);
 }
 
 ssd_status run_simt_any(const Shape& s, const ScanArgs& a) {
@@ -479,10 +495,7 @@ ssd_status noalloc_setup(void** scratch) {
   return SSD_OK;
 }
 
-size_t seg_scratch_bytes(const Shape& s, const Seg& sg) {
-  return align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)) +
-         align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float));
-}
+
 
 // The usual segmentation, with fewer (longer) segments when their states would not fit in
 // `cap` bytes.  Returns false when even one segment per sequence does not fit.
@@ -499,36 +512,6 @@ bool segments_within(const Shape& s, size_t cap, Seg* out) {
     }
   }
   return false;
-}
-
-ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, void* scratch) {
-  float* seg_states = static_cast<float*>(scratch);
-  float* seg_decay = reinterpret_cast<float*>(
-      static_cast<char*>(scratch) +
-      align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)));
-  CUtensorMap mx, mb, mc;
-  const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
-  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch) ||
-      !make_map(&mc, a.C, GN, s.seqlen, s.batch))
-    return SSD_ERR_CUDA;
-  const int hpg = s.nheads / s.ngroups;
-  const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-  ssd::tc::seg_state_kernel<<<grid, ssd::tc::kSegThreads, kSegSmem, a.stream>>>(
-      mx, mb, a.dt, a.A, seg_states, seg_decay, s.seqlen, s.nheads, hpg, sg);
-  if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  const int64_t nel = s.batch * s.nheads * int64_t(64) * 128;
-  ssd::tc::seg_scan_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
-      seg_states, seg_decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
-  if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  CUtensorMap my;
-  if (!make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32)) return SSD_ERR_CUDA;
-  if (a.ydt == SSD_F32)
-    ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
-        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
-  else
-    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
-        mx, mb, mc, my, a.dt, a.A, a.D, seg_states, s.seqlen, s.nheads, hpg, sg);
-  return launched();
 }
 
 }  // namespace

@@ -1,13 +1,13 @@
 // tc_kernels.cuh -- the chunked scan on sm_100a tensor cores (bf16 io, headdim 64, dstate 128).
 //
 // The sequence of each (batch row, head) is cut into 128-token blocks (the tcgen05 M=128 tile)
-// and the blocks into segments of consecutive blocks.  Three kernels, in stream order:
+// and the blocks into segments of consecutive blocks.  Two kernels, in stream order:
 //
-//  seg_state   per (b, segment, head quad): S_seg = sum_{t in seg} exp(sum_{k>t in seg} a_k)
+//  seg_state   per (b, segment, head pair): S_seg = sum_{t in seg} exp(sum_{k>t in seg} a_k)
 //              dt_t B_t x_t^T, one long-K GEMM on the tensor cores (A = B^T, B = w*x, K =
-//              tokens), plus the segment's total log-decay.  Reads x and B once.
-//  seg_scan    per state element: H_in(seg) = state entering each segment (the linear state
-//              passing between blocks, here at segment granularity), and final_state.
+//              tokens), plus the segment's total log-decay.  Reads x and B once.  The last CTA
+//              of each (b, head pair) to finish then passes the state along the segments:
+//              H_in(seg) = state entering each segment, and final_state.
 //  chunk_out   per (b, segment, head pair): walks the segment's blocks in order with the
 //              running state resident in TMEM.  Per block: G = C B^T (once for both heads),
 //              masked diagonal tile (L o G o dt) X, off-diagonal C H, skip term D x, y store,
@@ -83,8 +83,12 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 //              j's x tile to X' = w x and splits it into a bf16 high part (over x) and low part.
 //   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0).
 // Per stage (two stages):  B tile (2 x 16 KB, n halves) | X'hi (2 heads) | X'lo (2 heads).
-// Blocks are walked last to first so that the suffix sums of the log-decays are running totals;
-// both X' parts go through the tensor core, so the segment state carries ~16 bits of X'.
+// Blocks are walked last to first so that the suffix sums of the log-decays are running totals.
+// The segment's last block (first of the walk) sends both X' parts through the tensor core, so
+// the tokens that dominate a fast-decaying state carry ~16 bits of X'; earlier blocks, whose
+// terms reach the state through at least one block's decay, send the bf16 high part only.
+// The CTA that completes a (sequence, head pair) last then runs the state passing over the
+// segments (counted in seg_count, which must be zero at launch).
 // TMEM: 128 columns, lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
 constexpr uint32_t kSegStage = 6 * kTile;
@@ -92,8 +96,9 @@ constexpr int kSegThreads = 320;
 
 __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-    const float* __restrict__ dt, const float* __restrict__ A, float* __restrict__ seg_states,
-    float* __restrict__ seg_decay, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
+    const float* __restrict__ dt, const float* __restrict__ A, float* seg_states,
+    float* seg_decay, unsigned* seg_count, const float* init_state, float* final_state,
+    int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   __shared__ uint32_t tmem_base_sh;
   __shared__ float scan_scratch[8];
   __shared__ float dt_stage[2][2][kBlk];  // [walk block % 2][head][row], filled by cp.async
-  __shared__ int abort_flag;
+  __shared__ int abort_flag, last_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -190,8 +195,7 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const int stage = i & 1;
-      fetch_dt(i + 1);
-      cp_async_wait_prev();  // this thread's element of block i has landed
+      cp_async_wait_all();  // this thread's element of block i has landed
       const float d = dt_stage[i & 1][j][row];
       // w_t = exp(sum_{k > t, k in segment} a_k) * dt_t
       const float a = d * Alog;
@@ -207,6 +211,7 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
         tot += sw;
       }
       named_sync(1, 256);  // scratch read by everyone before the next block overwrites it
+      fetch_dt(i + 1);     // after the scan, so that no shared-memory read of it queues behind
       const float incl = v + off;
       const float wt = ex2(tot - incl + run) * d;  // tot - incl = sum over k > t in this block
       run += tot;
@@ -277,47 +282,47 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_free(tmem, 128);
-}
-
-// =============================================================================================
-// seg_scan: one thread per state element; H_in(0) = init, H_in(s+1) = 2^decay(s) H_in(s) + S(s).
-// seg_states is overwritten in place with H_in; final_state receives the state after the last
-// segment (it may alias init_state: each element is read before it is written, by one thread).
-// Segments are processed eight at a time so that eight independent loads are in flight.
-// =============================================================================================
-__global__ void __launch_bounds__(256) seg_scan_kernel(float* __restrict__ seg_states,
-                                                       const float* __restrict__ seg_decay,
-                                                       const float* init_state,
-                                                       float* final_state, int batch,
-                                                       int nheads, int nseg) {
-  const int64_t per_bh = int64_t(kP) * kN;
-  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= int64_t(batch) * nheads * per_bh) return;
-  const int64_t bh = e / per_bh, pn = e % per_bh;
-  const int h = int(bh % nheads);
-  const int64_t b = bh / nheads;
-  float run = init_state ? init_state[e] : 0.f;
-  const int64_t stride = int64_t(nheads) * per_bh;
-  float* base = seg_states + (b * nseg * nheads + h) * per_bh + pn;
-  const float* dbase = seg_decay + b * nseg * nheads + h;
-  for (int s0 = 0; s0 < nseg; s0 += 8) {
-    float v[8], dcy[8];
+  // ---- the last CTA of this (sequence, head pair) to finish passes the state along its
+  //      segments: H_in(0) = init, H_in(s + 1) = 2^decay(s) H_in(s) + S(s).  seg_states is
+  //      overwritten in place with H_in; final_state receives the state after the last segment
+  //      (it may alias init_state: each element is read before it is written, by one thread) --
+  __threadfence();  // this CTA's states and decays, before the count that publishes them
+  __syncthreads();
+  if (tid == 0) last_flag = atomicAdd(&seg_count[int64_t(b) * npair + hp], 1u) ==
+                            unsigned(sg.nseg - 1);
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+  constexpr int kPN = kP * kN;
+  const int64_t seg_stride = int64_t(nheads) * kPN;
+  for (int e = tid; e < 2 * kPN / 4; e += kSegThreads) {
+    const int h = h0 + e / (kPN / 4);
+    const int off = (e % (kPN / 4)) * 4;
+    const int64_t bh = (int64_t(b) * nheads + h) * kPN + off;
+    float4 run = init_state ? *reinterpret_cast<const float4*>(init_state + bh)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    float* base = seg_states + (int64_t(b) * sg.nseg * nheads + h) * kPN + off;
+    const float* dbase = seg_decay + int64_t(b) * sg.nseg * nheads + h;
+    for (int s0 = 0; s0 < sg.nseg; s0 += 4) {
+      float4 v[4];
+      float dc[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (s0 + i < nseg) {
-        v[i] = base[(s0 + i) * stride];
-        dcy[i] = dbase[(s0 + i) * nheads];
-      }
-    }
+      for (int i = 0; i < 4; ++i)
+        if (s0 + i < sg.nseg) {
+          v[i] = __ldcg(reinterpret_cast<const float4*>(base + (s0 + i) * seg_stride));
+          dc[i] = __ldcg(dbase + (s0 + i) * nheads);
+        }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (s0 + i < nseg) {
-        base[(s0 + i) * stride] = run;
-        run = fmaf(ex2(dcy[i]), run, v[i]);
-      }
+      for (int i = 0; i < 4; ++i)
+        if (s0 + i < sg.nseg) {
+          *reinterpret_cast<float4*>(base + (s0 + i) * seg_stride) = run;
+          const float a = ex2(dc[i]);
+          run = make_float4(fmaf(a, run.x, v[i].x), fmaf(a, run.y, v[i].y),
+                            fmaf(a, run.z, v[i].z), fmaf(a, run.w, v[i].w));
+        }
     }
+    if (final_state) *reinterpret_cast<float4*>(final_state + bh) = run;
   }
-  if (final_state) final_state[e] = run;
 }
 
 // =============================================================================================
@@ -342,9 +347,9 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(float* __restrict__ seg_s
 //   sHl  2 tiles  bf16 low part (the state's rounding remainder), same layout
 //   (sHh + sHl, free once C H has been computed, stage the block's y for the TMA stores)
 // TMEM (512 columns): [0,128) running state H (head, p) | [128,256) diagonal accumulators |
-//   [256,384) off-diagonal accumulators C H | [384,512) G = C B^T, overwritten in place, one
-//   head at a time, by that head's bf16 masked tile (16-column group kk -> its first 8
-//   columns), which the diagonal MMAs read as their A operand.
+//   [256,384) off-diagonal accumulators C H | [384,512) G = C B^T, overwritten in place by
+//   the two heads' bf16 masked tiles (16-column group kk -> columns 8h .. 8h+7 for head h),
+//   which the diagonal MMAs read as their A operand.
 // =============================================================================================
 constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 6 * kTile, kOffHh = 8 * kTile,
                    kOffHl = 10 * kTile, kSmemTiles = 12 * kTile;
@@ -397,9 +402,10 @@ template <> struct ystage<__nv_bfloat16> {
 struct OutBars {
   uint64_t c_full, b_full[2], x_full;      // TMA -> consumers
   uint64_t c_empty, b_empty[2], x_empty;   // MMA completion -> producer
-  uint64_t g_done, d0_done, d1_done, st_done;  // MMA completion -> compute
+  uint64_t g_done, d_done, st_done;  // MMA completion -> compute
   uint64_t h_ready, m0_ready, m1_ready, xp_ready;  // compute -> MMA issuer
   uint64_t y_staged, stage_free;  // compute <-> y writer
+  uint64_t cs_full[2], cs_empty[2];  // scan warps <-> compute (per cumsum buffer)
   uint64_t drain;
 };
 
@@ -414,11 +420,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
                                              ~uintptr_t(1023));
   __shared__ OutBars bars;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ __align__(16) float cs_sh[2][kBlk];
-  __shared__ __align__(16) float cl_sh[2][kBlk];  // cs_s - log2(dt_s) (+inf where dt = 0)
-  __shared__ __align__(16) float v_sh[2][kBlk];
-  __shared__ float dt_stage[2][2][kBlk];  // [block % 2][head][row], filled by cp.async
-  __shared__ float scan_scratch[16];
+  // per block (two buffers, block k in buffer k % 2) and head: log2 cumsums cs, cl = cs -
+  // log2(dt) (+inf where dt = 0), v_s = exp(cs_{s|15} - cs_s) dt_s
+  __shared__ __align__(16) float cs_sh[2][2][kBlk];
+  __shared__ __align__(16) float cl_sh[2][2][kBlk];
+  __shared__ __align__(16) float v_sh[2][2][kBlk];
+  __shared__ __align__(16) float dt_stage[2][2][kBlk];  // [block % 2][head][row], cp.async
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
@@ -444,6 +451,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     mbar_init(&bars.m1_ready, kComputeThreads);
     mbar_init(&bars.xp_ready, kComputeThreads);
     mbar_init(&bars.y_staged, kComputeThreads);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.cs_full[i], 64);
+      mbar_init(&bars.cs_empty[i], kComputeThreads);
+    }
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&tmem_base_sh, 512);
@@ -506,7 +517,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         const uint32_t par = k & 1;
         const uint32_t sx = sbase + kOffX;
         const uint32_t sb = sbase + kOffB + (k & 1) * 2 * kTile;
-        if (k > 0 && !mbar_wait(&bars.d1_done, par ^ 1, abort_v, 41)) break;  // G region free
+        if (k > 0 && !mbar_wait(&bars.d_done, par ^ 1, abort_v, 41)) break;  // G region free
         if (!mbar_wait(&bars.c_full, par, abort_v, 42)) break;
         if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43)) break;
         tc_fence_after();
@@ -518,20 +529,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars.g_done);
-        // Diag_h = (Mhi_h + Mlo_h) X_h (M = t, N = p, K = s), A from TMEM; head 0 first, then
-        // C H while head 1's mask is being written, then head 1
-        if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
-        auto diag = [&](int h) {
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk)
-            mma_ts(tD + h * 64, tG + kk * 16,
-                   sdesc(sx + h * kTile + kk * 2048, kTile, 1024), id_diag, kk > 0 ? 1u : 0u);
-        };
-        if (!mbar_wait(&bars.m0_ready, par, abort_v, 46)) break;
-        tc_fence_after();
-        diag(0);
-        mma_commit(&bars.d0_done);
-        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n)
+        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n), while the masks are being written
         if (!mbar_wait(&bars.h_ready, par, abort_v, 44)) break;
         tc_fence_after();
 #pragma unroll
@@ -542,10 +540,22 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
           mma_ss(tO, ad, sdesc(sbase + kOffHl + kk * 2048, kTile, 1024), id_off, 1u);
         }
         mma_commit(&bars.c_empty);
+        // Diag_h = M_h X_h (M = t, N = p, K = s), A = head h's bf16 mask in TMEM (columns
+        // 8h .. 8h+7 of each 16-column group); head 0 while head 1's mask is being written
+        if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
+        auto diag = [&](int h) {
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk)
+            mma_ts(tD + h * 64, tG + kk * 16 + h * 8,
+                   sdesc(sx + h * kTile + kk * 2048, kTile, 1024), id_diag, kk > 0 ? 1u : 0u);
+        };
+        if (!mbar_wait(&bars.m0_ready, par, abort_v, 46)) break;
+        tc_fence_after();
+        diag(0);
         if (!mbar_wait(&bars.m1_ready, par, abort_v, 48)) break;
         tc_fence_after();
         diag(1);
-        mma_commit(&bars.d1_done);  // covers C H as well
+        mma_commit(&bars.d_done);  // covers C H as well
         // H += B^T X' (M = n, N = (head, p), K = t)
         if (!mbar_wait(&bars.xp_ready, par, abort_v, 47)) break;
         tc_fence_after();
@@ -591,56 +601,67 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       }
       tmem_wait_st();
     }
-    const bool scan_thread = (q & 1) == 0;          // q = 0 scans head 0, q = 2 head 1
-    const float Alog = A[h0 + j] * kLog2e;
     const float Dh = D ? D[h0 + j] : 0.f;
-    const float* dtp = dt + int64_t(b) * seqlen * nheads + h0 + j;
-    // step sizes of block k -> dt_stage[k % 2] (scan threads only), one block ahead
-    auto fetch_dt = [&](int k) {
-      if (scan_thread) {
-        const int64_t tok = int64_t(blk0 + k) * kBlk + row;
-        const bool valid = k < nb && tok < seqlen;
-        cp_async4(&dt_stage[k & 1][j][row], valid ? dtp + tok * nheads : dtp, valid);
-        cp_async_commit();
+    // ---- within-block log2 cumsums, one warp per head (warp 0: head 0, warp 1: head 1; lane
+    //      owns rows 4 lane .. 4 lane + 3).  Block k + 1's are computed during block k's
+    //      diagonal MMAs, into the other buffer ----
+    const bool scan_warp = warp < 2;
+    const int hs = warp & 1;
+    const float Alog_s = A[h0 + hs] * kLog2e;
+    const float* dts = dt + int64_t(b) * seqlen * nheads + h0 + hs;
+    auto fetch_dt = [&](int kb) {  // step sizes of block kb -> dt_stage[kb % 2][hs]
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t tok = int64_t(blk0 + kb) * kBlk + 4 * lane + i;
+        const bool valid = kb < nb && tok < seqlen;
+        cp_async4(&dt_stage[kb & 1][hs][4 * lane + i], valid ? dts + tok * nheads : dts, valid);
       }
+      cp_async_commit();
     };
-    fetch_dt(0);
+    auto scan_block = [&](int kb) {
+      const int bf = kb & 1;
+      cp_async_wait_all();  // this lane's step sizes of block kb have landed
+      const float4 dv = *reinterpret_cast<const float4*>(&dt_stage[bf][hs][4 * lane]);
+      float c0 = dv.x * Alog_s;
+      float c1 = fmaf(dv.y, Alog_s, c0);
+      float c2 = fmaf(dv.z, Alog_s, c1);
+      float c3 = fmaf(dv.w, Alog_s, c2);
+      const float off = warp_inclusive_scan(c3) - c3;
+      c0 += off;
+      c1 += off;
+      c2 += off;
+      c3 += off;
+      const float inf = __int_as_float(0x7f800000);
+      const float l0 = dv.x > 0.f ? c0 - __log2f(dv.x) : inf;
+      const float l1 = dv.y > 0.f ? c1 - __log2f(dv.y) : inf;
+      const float l2 = dv.z > 0.f ? c2 - __log2f(dv.z) : inf;
+      const float l3 = dv.w > 0.f ? c3 - __log2f(dv.w) : inf;
+      const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
+      *reinterpret_cast<float4*>(&cs_sh[bf][hs][4 * lane]) = make_float4(c0, c1, c2, c3);
+      *reinterpret_cast<float4*>(&cl_sh[bf][hs][4 * lane]) = make_float4(l0, l1, l2, l3);
+      *reinterpret_cast<float4*>(&v_sh[bf][hs][4 * lane]) =
+          make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
+    };
+    if (scan_warp) {
+      fetch_dt(0);
+      scan_block(0);
+      fetch_dt(1);
+      mbar_arrive(&bars.cs_full[0]);
+    }
     bool ok = true;
     uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
     for (int k = 0; k < nb; ++k) {
       const uint32_t par = k & 1;
-      fetch_dt(k + 1);
-      float d = 0.f;
-      if (scan_thread) {
-        cp_async_wait_prev();  // block k's copy has landed (this thread's own element)
-        d = dt_stage[k & 1][j][row];
-      }
-      // ---- within-block log2 cumsums (warps 0-3: head 0, warps 8-11: head 1);
-      //      v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15 ----
-      {
-        float v = warp_inclusive_scan(d * Alog);
-        if (lane == 31) scan_scratch[warp] = v;
-        named_sync(1, kComputeThreads);
-        if (scan_thread) {
-          const int w0 = warp & ~3;
-          float off = 0.f;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) off += (w0 + w < warp) ? scan_scratch[w0 + w] : 0.f;
-          cs_sh[j][row] = v + off;
-          cl_sh[j][row] = d > 0.f ? v + off - __log2f(d) : __int_as_float(0x7f800000);
-        }
-        named_sync(1, kComputeThreads);
-        if (scan_thread) v_sh[j][row] = ex2(cs_sh[j][row | 15] - cl_sh[j][row]);
-      }
+      const int bf = k & 1;
+      ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 50);
       // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
       //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA, and
       //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
       if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51);
       if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55);
-      named_sync(1, kComputeThreads);  // cs/v published
       if (ok) {
         tc_fence_after();
-        const float al = ex2(cs_sh[j][kBlk - 1]);
+        const float al = ex2(cs_sh[bf][j][kBlk - 1]);
         uint8_t* hh = smem + kOffHh + j * kTile;
         uint8_t* hl = smem + kOffHl + j * kTile;
         uint32_t ra[16], rb[16];
@@ -669,10 +690,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       }
       tc_fence_before();
       mbar_arrive(&bars.h_ready);
-      // ---- masked tiles, one head at a time.  Thread (row t, q) owns the 16-column groups
-      //      q and q + 4 of G (columns [16q, 16q+16) and [16q+64, 16q+80)), which spreads the
-      //      rows' diagonal groups over all warps.  M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for
-      //      s <= t, written in bf16 over the first 8 TMEM columns of the group ----
+      // ---- masked tiles.  Thread (row t, q) owns the 16-column groups q and q + 4 of G
+      //      (columns [16q, 16q+16) and [16q+64, 16q+80)), which spreads the rows' diagonal
+      //      groups over all warps.  M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for s <= t, in
+      //      bf16, written over TMEM columns 8h .. 8h+7 of the group.  Each warp takes one
+      //      branch per group: the factorized product where all its rows are past the group,
+      //      the exact exponent where some row meets it, zeros where none reaches it ----
       const int t = row;
       const int wlast = wq * 32 + 31;                     // last row of this warp
       const bool live0 = q * 16 <= wlast, live1 = (q + 4) * 16 <= wlast;
@@ -693,9 +716,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
   {                                                                                            \
     const int s0 = (q + 4 * (GG)) * 16;                                                        \
     const bool live = (GG) ? live1 : live0;                                                    \
-    if (live && t >= s0 + 15) {                                                                \
-      const float u = ex2(cs_sh[H][t] - cs_sh[H][s0 + 15]);                                    \
-      const float4* vp = reinterpret_cast<const float4*>(&v_sh[H][s0]);                        \
+    if (wq * 32 >= s0 + 15) {                                                                  \
+      const float u = ex2(cs_sh[bf][H][t] - cs_sh[bf][H][s0 + 15]);                            \
+      const float4* vp = reinterpret_cast<const float4*>(&v_sh[bf][H][s0]);                    \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 vv = vp[e4];                                                              \
         R[2 * e4] = pack_bf16x2(gv[(GG) * 16 + 4 * e4] * (u * vv.x),                           \
@@ -703,9 +726,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         R[2 * e4 + 1] = pack_bf16x2(gv[(GG) * 16 + 4 * e4 + 2] * (u * vv.z),                   \
                                     gv[(GG) * 16 + 4 * e4 + 3] * (u * vv.w));                  \
       }                                                                                        \
-    } else if (live && t >= s0) {                                                              \
-      const float ct = cs_sh[H][t];                                                            \
-      const float4* cp = reinterpret_cast<const float4*>(&cl_sh[H][s0]);                       \
+    } else if (live) {                                                                         \
+      const float ct = cs_sh[bf][H][t];                                                        \
+      const float4* cp = reinterpret_cast<const float4*>(&cl_sh[bf][H][s0]);                   \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 cl = cp[e4];                                                              \
         const int s = s0 + 4 * e4;                                                             \
@@ -720,45 +743,42 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       _Pragma("unroll") for (int e = 0; e < 8; ++e) R[e] = 0u;                                \
     }                                                                                          \
   }
-      // head 0
-      if (ok) {
-        tc_fence_after();
-        uint32_t r[8];
-        SSD_MASK_GROUP(0, 0, r)
-        tmem_st8(gaddr0, r);
-        SSD_MASK_GROUP(0, 1, r)
-        tmem_st8(gaddr1, r);
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      mbar_arrive(&bars.m0_ready);
-      // head 1: computed while the first diagonal MMA runs; stored over head 0's mask once
-      // that MMA has read it
-      {
-        uint32_t r0[8], r1[8];
+      // head 0, then head 1 (its own TMEM columns, so no wait for the first diagonal MMA)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
         if (ok) {
-          SSD_MASK_GROUP(1, 0, r0)
-          SSD_MASK_GROUP(1, 1, r1)
-        }
-        ok = ok && mbar_wait(&bars.d0_done, par, abort_v, 53);
-        if (ok) {
-          tc_fence_after();
-          tmem_st8(gaddr0, r0);
-          tmem_st8(gaddr1, r1);
+          uint32_t r0[8], r1[8];
+          if (hh == 0) {
+            SSD_MASK_GROUP(0, 0, r0)
+            SSD_MASK_GROUP(0, 1, r1)
+          } else {
+            SSD_MASK_GROUP(1, 0, r0)
+            SSD_MASK_GROUP(1, 1, r1)
+          }
+          tmem_st8(gaddr0 + hh * 8, r0);
+          tmem_st8(gaddr1 + hh * 8, r1);
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(&bars.m1_ready);
+        mbar_arrive(hh == 0 ? &bars.m0_ready : &bars.m1_ready);
       }
 #undef SSD_MASK_GROUP
+      // ---- the next block's cumsums (scan warps), once every thread is done with the buffer
+      //      block k - 1 used ----
+      if (scan_warp && k + 1 < nb) {
+        if (k >= 1) ok = ok && mbar_wait(&bars.cs_empty[bf ^ 1], ((k - 1) >> 1) & 1, abort_v, 56);
+        if (ok) scan_block(k + 1);
+        fetch_dt(k + 2);
+        mbar_arrive(&bars.cs_full[bf ^ 1]);
+      }
       // ---- once both diagonal MMAs (and C H) are done: X' = w x in place for the state MMA
       //      (row t, head j, p in [p0, p0+32)), then y_t = Diag + exp(cs_t) Off + D x_t staged
       //      in shared memory and written by TMA ----
-      ok = ok && mbar_wait(&bars.d1_done, par, abort_v, 54);
+      ok = ok && mbar_wait(&bars.d_done, par, abort_v, 54);
       uint32_t xw[16];
       if (ok) {
         tc_fence_after();
-        const float wj = ex2(cs_sh[j][kBlk - 1] - cl_sh[j][t]);
+        const float wj = ex2(cs_sh[bf][j][kBlk - 1] - cl_sh[bf][j][t]);
         uint8_t* xrow = smem + kOffX + j * kTile;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -774,7 +794,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       }
       mbar_arrive(&bars.xp_ready);
       if (ok) {
-        const float ej = ex2(cs_sh[j][t]);
+        const float ej = ex2(cs_sh[bf][j][t]);
 #pragma unroll
         for (int pc = 0; pc < 2; ++pc) {
           uint32_t rd[16], ro[16];
@@ -795,10 +815,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       }
       mbar_arrive(&bars.y_staged);
       tc_fence_before();
-      // all compute threads are done with this block's cs/dt/v, TMEM reads and y staging
-      if (named_sync_or(1, kComputeThreads, !ok || *abort_v)) { ok = false; break; }
+      mbar_arrive(&bars.cs_empty[bf]);  // done with block k's cumsums
+      if (!ok || *abort_v) break;
     }
-    cp_async_wait_all();  // the step-size copy issued past the last block
+    if (scan_warp) cp_async_wait_all();  // step-size copies issued past the last block
   }
   // ------------------------------ teardown ------------------------------
   __syncthreads();

@@ -81,7 +81,8 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // seg_state: grid = batch * nseg * (nheads / 2), block = 320 threads:
 //   warps 0-7  compute: thread (row = tid % 128, j = tid / 128) scales token row `row` of head
 //              j's x tile to X' = w x and splits it into a bf16 high part (over x) and low part.
-//   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0).
+//   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0);  warp 10  step-size
+//              loader (dt of the two heads into shared memory, up to two blocks ahead).
 // Per stage (two stages):  B tile (2 x 16 KB, n halves) | X'hi (2 heads) | X'lo (2 heads).
 // Blocks are walked last to first so that the suffix sums of the log-decays are running totals.
 // The segment's last block (first of the walk) sends both X' parts through the tensor core, so
@@ -92,7 +93,7 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // TMEM: 128 columns, lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
 constexpr uint32_t kSegStage = 6 * kTile;
-constexpr int kSegThreads = 320;
+constexpr int kSegThreads = 352;
 
 __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -103,9 +104,10 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   __shared__ uint64_t full_bar[2], ready_bar[2], empty_bar[2], done_bar, drain_bar;
+  __shared__ uint64_t dt_full[2], dt_empty[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ float scan_scratch[8];
-  __shared__ float dt_stage[2][2][kBlk];  // [walk block % 2][head][row], filled by cp.async
+  __shared__ __align__(16) float dt_stage[2][2][kBlk];  // [walk block % 2][head][row]
   __shared__ int abort_flag, last_flag;
 
   const int tid = threadIdx.x;
@@ -128,6 +130,8 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       mbar_init(&full_bar[i], 1);
       mbar_init(&ready_bar[i], 256);
       mbar_init(&empty_bar[i], 1);
+      mbar_init(&dt_full[i], 32);
+      mbar_init(&dt_empty[i], 256);
     }
     mbar_init(&done_bar, 1);
     mbar_init(&drain_bar, 1);
@@ -161,42 +165,54 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+      // descriptors are built once; a K step or a tile offset adds (bytes >> 4) to the start
+      // address field (every address stays below 256 KB, so the field cannot carry)
+      const uint64_t d0 = sdesc(smem_u32(smem), kTile, 1024);
       for (int i = 0; i < nb; ++i) {
         const int stage = i & 1;
         if (!mbar_wait(&ready_bar[stage], (i >> 1) & 1, abort_v, 12)) break;
         tc_fence_after();
-        const uint32_t sb = smem_u32(smem + stage * kSegStage);
+        const uint64_t ds = d0 + (stage ? (kSegStage >> 4) : 0u);
 #pragma unroll
         for (int k = 0; k < kBlk / 16; ++k) {
-          const uint64_t ad = sdesc(sb + k * 2048, kTile, 1024);               // B^T: M = n
-          mma_ss(tmem, ad, sdesc(sb + 2 * kTile + k * 2048, kTile, 1024), idesc,
-                 (i > 0 || k > 0) ? 1u : 0u);                                   // X' (high)
-          if (i == 0)
-            mma_ss(tmem, ad, sdesc(sb + 4 * kTile + k * 2048, kTile, 1024), idesc, 1u);  // low
+          const uint64_t ad = ds + k * 128;                                     // B^T: M = n
+          mma_ss(tmem, ad, ad + ((2 * kTile) >> 4), idesc, (i > 0 || k > 0) ? 1u : 0u);  // X'
+          if (i == 0) mma_ss(tmem, ad, ad + ((4 * kTile) >> 4), idesc, 1u);   // X' low part
         }
         mma_commit(&empty_bar[stage]);
         if (i == nb - 1) mma_commit(&done_bar);
       }
     }
+  } else if (warp == 10) {
+    // ------------------------------ step-size loader ------------------------------
+    // lane l: rows 4l .. 4l+3 of both heads of walk block i (8 independent loads)
+    const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
+    for (int i = 0; i < nb; ++i) {
+      const int bf = i & 1;
+      if (i >= 2 && !mbar_wait(&dt_empty[bf], ((i - 2) >> 1) & 1, abort_v, 15)) break;
+      float v[8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int64_t tok = int64_t(blk0 + nb - 1 - i) * kBlk + 4 * lane + r;
+        const bool in = tok < seqlen;
+        v[2 * r] = in ? dtb[tok * nheads] : 0.f;
+        v[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
+      }
+      *reinterpret_cast<float4*>(&dt_stage[bf][0][4 * lane]) = make_float4(v[0], v[2], v[4], v[6]);
+      *reinterpret_cast<float4*>(&dt_stage[bf][1][4 * lane]) = make_float4(v[1], v[3], v[5], v[7]);
+      mbar_arrive_warp(&dt_full[bf]);
+    }
   } else {
     // ------------------------------ compute warps ------------------------------
     const int row = tid & 127, j = tid >> 7;
     const float Alog = A[h0 + j] * kLog2e;
-    const float* dtp = dt + int64_t(b) * seqlen * nheads + h0 + j;
-    // step sizes of walk block i -> dt_stage[i % 2], one block ahead
-    auto fetch_dt = [&](int i) {
-      const int64_t tok = int64_t(blk0 + nb - 1 - i) * kBlk + row;
-      const bool valid = i < nb && tok < seqlen;
-      cp_async4(&dt_stage[i & 1][j][row], valid ? dtp + tok * nheads : dtp, valid);
-      cp_async_commit();
-    };
     float run = 0.f;  // log2-decay of the blocks after the current one, within the segment
-    fetch_dt(0);
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const int stage = i & 1;
-      cp_async_wait_all();  // this thread's element of block i has landed
+      ok = ok && mbar_wait(&dt_full[i & 1], (i >> 1) & 1, abort_v, 16);
       const float d = dt_stage[i & 1][j][row];
+      mbar_arrive_warp(&dt_empty[i & 1]);
       // w_t = exp(sum_{k > t, k in segment} a_k) * dt_t
       const float a = d * Alog;
       float v = warp_inclusive_scan(a);
@@ -211,7 +227,6 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
         tot += sw;
       }
       named_sync(1, 256);  // scratch read by everyone before the next block overwrites it
-      fetch_dt(i + 1);     // after the scan, so that no shared-memory read of it queues behind
       const float incl = v + off;
       const float wt = ex2(tot - incl + run) * d;  // tot - incl = sum over k > t in this block
       run += tot;
@@ -248,7 +263,6 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       mbar_arrive(&ready_bar[stage]);
       if (named_sync_or(1, 256, !ok || *abort_v)) { ok = false; break; }
     }
-    cp_async_wait_all();  // the copy issued past the last block
     // epilogue: lane n = row, columns of head j
     if (ok && nb > 0) ok = mbar_wait(&done_bar, 0, abort_v, 14);
     if (ok) {
@@ -293,50 +307,72 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   __syncthreads();
   if (!last_flag) return;
   __threadfence();
+  // Thread tid carries the running states of float4 elements e = tid + i * kSegThreads of
+  // the pair's two 64 x 128 states in registers and walks the segments in order, so each step
+  // issues all its loads at once.
   constexpr int kPN = kP * kN;
+  constexpr int kVec = 2 * kPN / 4;
+  constexpr int kPer = (kVec + kSegThreads - 1) / kSegThreads;
   const int64_t seg_stride = int64_t(nheads) * kPN;
-  for (int e = tid; e < 2 * kPN / 4; e += kSegThreads) {
-    const int h = h0 + e / (kPN / 4);
-    const int off = (e % (kPN / 4)) * 4;
-    const int64_t bh = (int64_t(b) * nheads + h) * kPN + off;
-    float4 run = init_state ? *reinterpret_cast<const float4*>(init_state + bh)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-    float* base = seg_states + (int64_t(b) * sg.nseg * nheads + h) * kPN + off;
-    const float* dbase = seg_decay + int64_t(b) * sg.nseg * nheads + h;
-    for (int s0 = 0; s0 < sg.nseg; s0 += 4) {
-      float4 v[4];
-      float dc[4];
+  float* sbase = seg_states + int64_t(b) * sg.nseg * seg_stride + int64_t(h0) * kPN;
+  const float* dbase = seg_decay + int64_t(b) * sg.nseg * nheads + h0;
+  const int64_t ibase = (int64_t(b) * nheads + h0) * kPN;
+  float4 run[kPer];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (s0 + i < sg.nseg) {
-          v[i] = __ldcg(reinterpret_cast<const float4*>(base + (s0 + i) * seg_stride));
-          dc[i] = __ldcg(dbase + (s0 + i) * nheads);
-        }
+  for (int i = 0; i < kPer; ++i) {
+    const int e = tid + i * kSegThreads;
+    run[i] = (init_state && e < kVec) ? *reinterpret_cast<const float4*>(init_state + ibase + 4 * e)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int sgi = 0; sgi < sg.nseg; ++sgi) {
+    float* st = sbase + sgi * seg_stride;  // heads h0, h0 + 1 of segment sgi, contiguous
+    const float a0 = ex2(__ldcg(dbase + int64_t(sgi) * nheads));
+    const float a1 = ex2(__ldcg(dbase + int64_t(sgi) * nheads + 1));
+    float4 v[kPer];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (s0 + i < sg.nseg) {
-          *reinterpret_cast<float4*>(base + (s0 + i) * seg_stride) = run;
-          const float a = ex2(dc[i]);
-          run = make_float4(fmaf(a, run.x, v[i].x), fmaf(a, run.y, v[i].y),
-                            fmaf(a, run.z, v[i].z), fmaf(a, run.w, v[i].w));
-        }
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + i * kSegThreads;
+      if (e < kVec) v[i] = __ldcg(reinterpret_cast<const float4*>(st + 4 * e));
     }
-    if (final_state) *reinterpret_cast<float4*>(final_state + bh) = run;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + i * kSegThreads;
+      if (e < kVec) {
+        *reinterpret_cast<float4*>(st + 4 * e) = run[i];
+        const float a = e < kVec / 2 ? a0 : a1;
+        run[i] = make_float4(fmaf(a, run[i].x, v[i].x), fmaf(a, run[i].y, v[i].y),
+                             fmaf(a, run[i].z, v[i].z), fmaf(a, run[i].w, v[i].w));
+      }
+    }
+  }
+  if (final_state) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + i * kSegThreads;
+      if (e < kVec) *reinterpret_cast<float4*>(final_state + ibase + 4 * e) = run[i];
+    }
   }
 }
 
 // =============================================================================================
-// chunk_out: grid = batch * nseg * (nheads / 2), block = 576 threads in three roles:
+// chunk_out: grid = batch * nseg * (nheads / 2), block = 608 threads in four roles:
 //   warps 0-15  compute (512 threads).  Thread (row = tid % 128, q = tid / 128): token row
 //               `row` of a block (state row n = row in the state passes) and a quarter of the
 //               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and
-//               the epilogue; G columns [32 q, 32 q + 32) for the masks.  Four warps share each
-//               TMEM lane quarter, so every phase is spread over all 16 warps.
+//               the epilogue; G column groups q and q + 4 for the masks.  Four warps share
+//               each TMEM lane quarter, so every phase is spread over all 16 warps.  Warps 0
+//               and 1 also compute the next block's cumsums (one head each).
 //   warp 16     TMA producer (lane 0): C, x (single buffers), B (double buffer) per block.
 //   warp 17     MMA issuer (lane 0).
-//   warp 18     y writer (lane 0): TMA stores of each block's staged y, off the compute path.
-// The roles hand blocks to each other through mbarriers, so the loads of the next block, the
-// tensor-core work and the CUDA-core work of different phases overlap.
+//   warp 18     y writer (lane 0): TMA stores of each block's staged y.
+//   warp 19     step-size loader: each block's dt of the two heads into shared memory, up to
+//               two blocks ahead (plain loads, off the compute warps).
+// Per block k the compute warps write the masks (MMA: diagonal tiles), then the state pass
+// (MMA: C H), then X' (MMA: state update) and the epilogue.  The masks come first so that the
+// previous block's y stores, which read the staging buffer the state pass overwrites, drain
+// while they are computed.  Roles hand blocks to each other through mbarriers only; a thread
+// is never more than one phase of a barrier ahead of the slowest, because every barrier it
+// waits on next needs an arrival that the slowest makes after its own previous wait.
 // Shared memory (1024-aligned, 12 x 16 KB):
 //   sC   2 tiles  C, K-major (rows t), n halves
 //   sB   4 tiles  B, rows s, n halves, two slots (blocks k % 2): K-major for G = C B^T,
@@ -354,14 +390,13 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
 constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 6 * kTile, kOffHh = 8 * kTile,
                    kOffHl = 10 * kTile, kSmemTiles = 12 * kTile;
 constexpr int kComputeThreads = 512;
-constexpr int kOutThreads = kComputeThreads + 96;
+constexpr int kOutThreads = kComputeThreads + 128;
 
 // y staging (in sHh/sHl) and its TMA stores.  Float32 y: 4 boxes {32 p, 128 t} (one per
 // thread quarter q: head q/2, p-half q%2), 128B-swizzled.  Bf16 y: 2 boxes {64 p, 128 t} (one
 // per head).
 template <typename TY> struct ystage;
 template <> struct ystage<float> {
-  static constexpr int kBoxes = 4;
   // thread (t, q) writes its 32 values (16 per call, half = 0/1) into box q, row t
   static __device__ __forceinline__ void put16(uint8_t* stage, int t, int q, int half,
                                                const float (&v)[16]) {
@@ -379,7 +414,6 @@ template <> struct ystage<float> {
   }
 };
 template <> struct ystage<__nv_bfloat16> {
-  static constexpr int kBoxes = 2;
   static __device__ __forceinline__ void put16(uint8_t* stage, int t, int q, int half,
                                                const float (&v)[16]) {
     uint8_t* box = stage + (q / 2) * kTile;
@@ -400,12 +434,13 @@ template <> struct ystage<__nv_bfloat16> {
 
 // mbarriers of chunk_out (all in shared memory)
 struct OutBars {
-  uint64_t c_full, b_full[2], x_full;      // TMA -> consumers
-  uint64_t c_empty, b_empty[2], x_empty;   // MMA completion -> producer
-  uint64_t g_done, d_done, st_done;  // MMA completion -> compute
-  uint64_t h_ready, m0_ready, m1_ready, xp_ready;  // compute -> MMA issuer
-  uint64_t y_staged, stage_free;  // compute <-> y writer
-  uint64_t cs_full[2], cs_empty[2];  // scan warps <-> compute (per cumsum buffer)
+  uint64_t c_full, b_full[2], x_full;        // TMA -> consumers
+  uint64_t c_empty, b_empty[2], x_empty;     // MMA completion -> producer
+  uint64_t g_done, d_done, o_done, st_done;  // MMA completion -> compute
+  uint64_t m0_ready, m1_ready, h_ready, xp_ready;  // compute -> MMA issuer
+  uint64_t y_staged, stage_free;             // compute <-> y writer
+  uint64_t cs_full[2], cs_empty[2];          // scan warps <-> compute (per cumsum buffer)
+  uint64_t dt_full[2], dt_empty[2];          // step-size loader <-> scan warps
   uint64_t drain;
 };
 
@@ -425,7 +460,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
   __shared__ __align__(16) float cs_sh[2][2][kBlk];
   __shared__ __align__(16) float cl_sh[2][2][kBlk];
   __shared__ __align__(16) float v_sh[2][2][kBlk];
-  __shared__ __align__(16) float dt_stage[2][2][kBlk];  // [block % 2][head][row], cp.async
+  __shared__ __align__(16) float dt_stage[2][2][kBlk];  // [block % 2][head][row]
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
@@ -446,14 +481,16 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     abort_flag = 0;
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
     for (int i = 0; i < int(sizeof(OutBars) / 8); ++i) mbar_init(all + i, 1);
-    mbar_init(&bars.h_ready, kComputeThreads);
     mbar_init(&bars.m0_ready, kComputeThreads);
     mbar_init(&bars.m1_ready, kComputeThreads);
+    mbar_init(&bars.h_ready, kComputeThreads);
     mbar_init(&bars.xp_ready, kComputeThreads);
     mbar_init(&bars.y_staged, kComputeThreads);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.cs_full[i], 64);
       mbar_init(&bars.cs_empty[i], kComputeThreads);
+      mbar_init(&bars.dt_full[i], 32);
+      mbar_init(&bars.dt_empty[i], 64);
     }
     fence_mbar_init();
   }
@@ -513,41 +550,35 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       const uint32_t id_off = idesc_bf16(128, 128, 0, 1);
       const uint32_t id_diag = idesc_bf16(128, 64, 0, 1);
       const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
+      // descriptors are built once; a K step or a tile offset adds (bytes >> 4) to the start
+      // address field (every address stays below 256 KB, so the field cannot carry)
+      const uint64_t dC = sdesc(sbase + kOffC, 16, 1024);       // K-major (rows t or s)
+      const uint64_t dBk = sdesc(sbase + kOffB, 16, 1024);
+      const uint64_t dBm = sdesc(sbase + kOffB, kTile, 1024);   // MN-major
+      const uint64_t dX = sdesc(sbase + kOffX, kTile, 1024);
+      const uint64_t dHh = sdesc(sbase + kOffHh, kTile, 1024);
+      const uint64_t dHl = sdesc(sbase + kOffHl, kTile, 1024);
+      auto kmaj = [](int kk) { return uint64_t(((kk >> 2) * kTile + (kk & 3) * 32) >> 4); };
       for (int k = 0; k < nb; ++k) {
         const uint32_t par = k & 1;
-        const uint32_t sx = sbase + kOffX;
-        const uint32_t sb = sbase + kOffB + (k & 1) * 2 * kTile;
+        const uint64_t bslot = (k & 1) ? uint64_t((2 * kTile) >> 4) : 0u;
         if (k > 0 && !mbar_wait(&bars.d_done, par ^ 1, abort_v, 41)) break;  // G region free
         if (!mbar_wait(&bars.c_full, par, abort_v, 42)) break;
         if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43)) break;
         tc_fence_after();
         // G = C B^T (M = t, N = s, K = n)
 #pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * kTile + (kk & 3) * 32;
-          mma_ss(tG, sdesc(sbase + kOffC + koff, 16, 1024), sdesc(sb + koff, 16, 1024), id_g,
-                 kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kN / 16; ++kk)
+          mma_ss(tG, dC + kmaj(kk), dBk + bslot + kmaj(kk), id_g, kk > 0 ? 1u : 0u);
         mma_commit(&bars.g_done);
-        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n), while the masks are being written
-        if (!mbar_wait(&bars.h_ready, par, abort_v, 44)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
-          const uint64_t ad = sdesc(sbase + kOffC + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
-          mma_ss(tO, ad, sdesc(sbase + kOffHh + kk * 2048, kTile, 1024), id_off,
-                 kk > 0 ? 1u : 0u);
-          mma_ss(tO, ad, sdesc(sbase + kOffHl + kk * 2048, kTile, 1024), id_off, 1u);
-        }
-        mma_commit(&bars.c_empty);
         // Diag_h = M_h X_h (M = t, N = p, K = s), A = head h's bf16 mask in TMEM (columns
         // 8h .. 8h+7 of each 16-column group); head 0 while head 1's mask is being written
         if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
         auto diag = [&](int h) {
 #pragma unroll
           for (int kk = 0; kk < kBlk / 16; ++kk)
-            mma_ts(tD + h * 64, tG + kk * 16 + h * 8,
-                   sdesc(sx + h * kTile + kk * 2048, kTile, 1024), id_diag, kk > 0 ? 1u : 0u);
+            mma_ts(tD + h * 64, tG + kk * 16 + h * 8, dX + h * (kTile >> 4) + kk * 128, id_diag,
+                   kk > 0 ? 1u : 0u);
         };
         if (!mbar_wait(&bars.m0_ready, par, abort_v, 46)) break;
         tc_fence_after();
@@ -555,14 +586,23 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         if (!mbar_wait(&bars.m1_ready, par, abort_v, 48)) break;
         tc_fence_after();
         diag(1);
-        mma_commit(&bars.d_done);  // covers C H as well
+        mma_commit(&bars.d_done);
+        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n)
+        if (!mbar_wait(&bars.h_ready, par, abort_v, 44)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          mma_ss(tO, dC + kmaj(kk), dHh + kk * 128, id_off, kk > 0 ? 1u : 0u);
+          mma_ss(tO, dC + kmaj(kk), dHl + kk * 128, id_off, 1u);
+        }
+        mma_commit(&bars.o_done);
+        mma_commit(&bars.c_empty);
         // H += B^T X' (M = n, N = (head, p), K = t)
         if (!mbar_wait(&bars.xp_ready, par, abort_v, 47)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ss(tH, sdesc(sb + kk * 2048, kTile, 1024), sdesc(sx + kk * 2048, kTile, 1024),
-                 id_st, 1u);
+          mma_ss(tH, dBm + bslot + kk * 128, dX + kk * 128, id_st, 1u);
         mma_commit(&bars.st_done);
         mma_commit(&bars.x_empty);
         mma_commit(&bars.b_empty[k & 1]);
@@ -581,6 +621,25 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         mbar_arrive(&bars.stage_free);
       }
       bulk_wait_all();
+    }
+  } else if (warp == 19) {
+    // ------------------------------ step-size loader ------------------------------
+    // lane l: rows 4l .. 4l+3 of both heads (8 independent loads per block)
+    const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
+    for (int kb = 0; kb < nb; ++kb) {
+      const int bf = kb & 1;
+      if (kb >= 2 && !mbar_wait(&bars.dt_empty[bf], ((kb - 2) >> 1) & 1, abort_v, 71)) break;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t tok = int64_t(blk0 + kb) * kBlk + 4 * lane + i;
+        const bool in = tok < seqlen;
+        v[2 * i] = in ? dtb[tok * nheads] : 0.f;
+        v[2 * i + 1] = in ? dtb[tok * nheads + 1] : 0.f;
+      }
+      *reinterpret_cast<float4*>(&dt_stage[bf][0][4 * lane]) = make_float4(v[0], v[2], v[4], v[6]);
+      *reinterpret_cast<float4*>(&dt_stage[bf][1][4 * lane]) = make_float4(v[1], v[3], v[5], v[7]);
+      mbar_arrive_warp(&bars.dt_full[bf]);
     }
   } else {
     // ------------------------------ compute warps ------------------------------
@@ -603,25 +662,18 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     }
     const float Dh = D ? D[h0 + j] : 0.f;
     // ---- within-block log2 cumsums, one warp per head (warp 0: head 0, warp 1: head 1; lane
-    //      owns rows 4 lane .. 4 lane + 3).  Block k + 1's are computed during block k's
-    //      diagonal MMAs, into the other buffer ----
+    //      owns rows 4 lane .. 4 lane + 3).  Block k + 1's are computed during block k, into
+    //      the other buffer ----
     const bool scan_warp = warp < 2;
     const int hs = warp & 1;
     const float Alog_s = A[h0 + hs] * kLog2e;
-    const float* dts = dt + int64_t(b) * seqlen * nheads + h0 + hs;
-    auto fetch_dt = [&](int kb) {  // step sizes of block kb -> dt_stage[kb % 2][hs]
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t tok = int64_t(blk0 + kb) * kBlk + 4 * lane + i;
-        const bool valid = kb < nb && tok < seqlen;
-        cp_async4(&dt_stage[kb & 1][hs][4 * lane + i], valid ? dts + tok * nheads : dts, valid);
-      }
-      cp_async_commit();
-    };
+    // the cumsums of block kb (false if a wait gave up)
     auto scan_block = [&](int kb) {
       const int bf = kb & 1;
-      cp_async_wait_all();  // this lane's step sizes of block kb have landed
+      const bool got = mbar_wait(&bars.dt_full[bf], (kb >> 1) & 1, abort_v, 58);
       const float4 dv = *reinterpret_cast<const float4*>(&dt_stage[bf][hs][4 * lane]);
+      mbar_arrive_warp(&bars.dt_empty[bf]);
+      if (!__all_sync(0xffffffffu, got)) return false;
       float c0 = dv.x * Alog_s;
       float c1 = fmaf(dv.y, Alog_s, c0);
       float c2 = fmaf(dv.z, Alog_s, c1);
@@ -641,65 +693,28 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       *reinterpret_cast<float4*>(&cl_sh[bf][hs][4 * lane]) = make_float4(l0, l1, l2, l3);
       *reinterpret_cast<float4*>(&v_sh[bf][hs][4 * lane]) =
           make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
+      return true;
     };
-    if (scan_warp) {
-      fetch_dt(0);
-      scan_block(0);
-      fetch_dt(1);
-      mbar_arrive(&bars.cs_full[0]);
-    }
     bool ok = true;
+    if (scan_warp) {
+      if (nb > 0) ok = scan_block(0);
+      mbar_arrive_warp(&bars.cs_full[0]);
+    }
     uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
+    const int t = row;
+    const int wlast = wq * 32 + 31;                 // last row of this warp
+    const bool live0 = q * 16 <= wlast, live1 = (q + 4) * 16 <= wlast;
+    const uint32_t gaddr0 = tG + lane_off + q * 16, gaddr1 = gaddr0 + 64;
     for (int k = 0; k < nb; ++k) {
       const uint32_t par = k & 1;
       const int bf = k & 1;
       ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 50);
-      // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
-      //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA, and
-      //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
-      if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51);
-      if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55);
-      if (ok) {
-        tc_fence_after();
-        const float al = ex2(cs_sh[bf][j][kBlk - 1]);
-        uint8_t* hh = smem + kOffHh + j * kTile;
-        uint8_t* hl = smem + kOffHl + j * kTile;
-        uint32_t ra[16], rb[16];
-        tmem_ld16(tH + lane_off + j * 64 + p0, ra);
-        tmem_wait_ld();
-#define SSD_HPASS(R, PC)                                                                      \
-  {                                                                                           \
-    uint32_t hi[8], lo[8];                                                                    \
-    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
-        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
-    const int ch = (p0 >> 3) + (PC) * 2;                                                      \
-    *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);    \
-    *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
-    *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
-    *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
-    _Pragma("unroll") for (int e = 0; e < 16; ++e) R[e] = __float_as_uint(__uint_as_float(R[e]) * al); \
-    tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
-  }
-        SSD_HPASS(ra, 0)
-        tmem_ld16(tH + lane_off + j * 64 + p0 + 16, rb);
-        tmem_wait_ld();
-        SSD_HPASS(rb, 1)
-#undef SSD_HPASS
-        tmem_wait_st();
-        fence_proxy_async_smem();
-      }
-      tc_fence_before();
-      mbar_arrive(&bars.h_ready);
       // ---- masked tiles.  Thread (row t, q) owns the 16-column groups q and q + 4 of G
       //      (columns [16q, 16q+16) and [16q+64, 16q+80)), which spreads the rows' diagonal
       //      groups over all warps.  M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for s <= t, in
       //      bf16, written over TMEM columns 8h .. 8h+7 of the group.  Each warp takes one
       //      branch per group: the factorized product where all its rows are past the group,
       //      the exact exponent where some row meets it, zeros where none reaches it ----
-      const int t = row;
-      const int wlast = wq * 32 + 31;                     // last row of this warp
-      const bool live0 = q * 16 <= wlast, live1 = (q + 4) * 16 <= wlast;
-      const uint32_t gaddr0 = tG + lane_off + q * 16, gaddr1 = gaddr0 + 64;
       float gv[32];
       ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52);
       if (ok && live0) {
@@ -760,20 +775,55 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(hh == 0 ? &bars.m0_ready : &bars.m1_ready);
+        mbar_arrive_warp(hh == 0 ? &bars.m0_ready : &bars.m1_ready);
       }
 #undef SSD_MASK_GROUP
+      // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
+      //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA and
+      //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
+      if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51);
+      if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55);
+      if (ok) {
+        tc_fence_after();
+        const float al = ex2(cs_sh[bf][j][kBlk - 1]);
+        uint8_t* hh = smem + kOffHh + j * kTile;
+        uint8_t* hl = smem + kOffHl + j * kTile;
+        uint32_t ra[16], rb[16];
+        tmem_ld16(tH + lane_off + j * 64 + p0, ra);
+        tmem_wait_ld();
+#define SSD_HPASS(R, PC)                                                                      \
+  {                                                                                           \
+    uint32_t hi[8], lo[8];                                                                    \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
+        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
+    const int ch = (p0 >> 3) + (PC) * 2;                                                      \
+    *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);    \
+    *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
+    *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
+    *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
+    _Pragma("unroll") for (int e = 0; e < 16; ++e) R[e] = __float_as_uint(__uint_as_float(R[e]) * al); \
+    tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
+  }
+        SSD_HPASS(ra, 0)
+        tmem_ld16(tH + lane_off + j * 64 + p0 + 16, rb);
+        tmem_wait_ld();
+        SSD_HPASS(rb, 1)
+#undef SSD_HPASS
+        tmem_wait_st();
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive_warp(&bars.h_ready);
       // ---- the next block's cumsums (scan warps), once every thread is done with the buffer
       //      block k - 1 used ----
       if (scan_warp && k + 1 < nb) {
         if (k >= 1) ok = ok && mbar_wait(&bars.cs_empty[bf ^ 1], ((k - 1) >> 1) & 1, abort_v, 56);
-        if (ok) scan_block(k + 1);
-        fetch_dt(k + 2);
-        mbar_arrive(&bars.cs_full[bf ^ 1]);
+        if (__all_sync(0xffffffffu, ok)) ok = scan_block(k + 1);
+        mbar_arrive_warp(&bars.cs_full[bf ^ 1]);
       }
-      // ---- once both diagonal MMAs (and C H) are done: X' = w x in place for the state MMA
-      //      (row t, head j, p in [p0, p0+32)), then y_t = Diag + exp(cs_t) Off + D x_t staged
-      //      in shared memory and written by TMA ----
+      // ---- once the diagonal MMAs are done: X' = w x in place for the state MMA (row t,
+      //      head j, p in [p0, p0+32)); then, once C H is done too, y_t = Diag + exp(cs_t) Off
+      //      + D x_t staged in shared memory and written by TMA ----
       ok = ok && mbar_wait(&bars.d_done, par, abort_v, 54);
       uint32_t xw[16];
       if (ok) {
@@ -792,8 +842,10 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         }
         fence_proxy_async_smem();
       }
-      mbar_arrive(&bars.xp_ready);
+      mbar_arrive_warp(&bars.xp_ready);
+      ok = ok && mbar_wait(&bars.o_done, par, abort_v, 57);
       if (ok) {
+        tc_fence_after();
         const float ej = ex2(cs_sh[bf][j][t]);
 #pragma unroll
         for (int pc = 0; pc < 2; ++pc) {
@@ -813,12 +865,11 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         }
         fence_proxy_async_smem();
       }
-      mbar_arrive(&bars.y_staged);
       tc_fence_before();
-      mbar_arrive(&bars.cs_empty[bf]);  // done with block k's cumsums
-      if (!ok || *abort_v) break;
+      mbar_arrive_warp(&bars.y_staged);
+      mbar_arrive_warp(&bars.cs_empty[bf]);  // done with block k's cumsums and TMEM reads
+      if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
     }
-    if (scan_warp) cp_async_wait_all();  // step-size copies issued past the last block
   }
   // ------------------------------ teardown ------------------------------
   __syncthreads();

@@ -149,7 +149,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, ui
 }
 
 constexpr size_t kTcSmem = ssd::tc::kSmemTiles + 1024;
-constexpr size_t kSegSmem = 2 * size_t(ssd::tc::kSegStage) + 1024;
+constexpr size_t kSegSmem = ssd::tc::kSegStages * size_t(ssd::tc::kSegStage) + 1024;
 
 ssd_status set_smem_attrs() {
   static ssd_status st = SSD_ERR_CUDA;

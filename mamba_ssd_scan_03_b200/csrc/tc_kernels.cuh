@@ -81,9 +81,12 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // seg_state: grid = batch * nseg * (nheads / 2), block = 320 threads:
 //   warps 0-7  compute: thread (row = tid % 128, j = tid / 128) scales token row `row` of head
 //              j's x tile to X' = w x and splits it into a bf16 high part (over x) and low part.
-//   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0);  warp 10  step-size
-//              loader (dt of the two heads into shared memory, up to two blocks ahead).
-// Per stage (two stages):  B tile (2 x 16 KB, n halves) | X'hi (2 heads) | X'lo (2 heads).
+//   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0);  warp 10  weights: loads
+//              each block's dt of the two heads (four blocks of loads in flight) and writes
+//              w_t into a four-slot ring in shared memory (lane l: rows 4l .. 4l+3).
+// Per stage (three stages):  B tile (2 x 16 KB, n halves) | x, scaled in place to X' (2 heads).
+// The low part of the segment's last block goes to stage 2's x area, which the producer fills
+// only once that block's MMAs are done.
 // Blocks are walked last to first so that the suffix sums of the log-decays are running totals.
 // The segment's last block (first of the walk) sends both X' parts through the tensor core, so
 // the tokens that dominate a fast-decaying state carry ~16 bits of X'; earlier blocks, whose
@@ -92,7 +95,9 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // segments (counted in seg_count, which must be zero at launch).
 // TMEM: 128 columns, lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
-constexpr uint32_t kSegStage = 6 * kTile;
+constexpr uint32_t kSegStage = 4 * kTile;
+constexpr int kSegStages = 3;
+constexpr int kWtSlots = 4;
 constexpr int kSegThreads = 352;
 
 __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
@@ -103,11 +108,11 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ uint64_t full_bar[2], ready_bar[2], empty_bar[2], done_bar, drain_bar;
-  __shared__ uint64_t dt_full[2], dt_empty[2];
+  __shared__ uint64_t full_bar[kSegStages], ready_bar[kSegStages], empty_bar[kSegStages];
+  __shared__ uint64_t done_bar, drain_bar;
+  __shared__ uint64_t wt_full[kWtSlots], wt_empty[kWtSlots];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float scan_scratch[8];
-  __shared__ __align__(16) float dt_stage[2][2][kBlk];  // [walk block % 2][head][row]
+  __shared__ __align__(16) float wt_stage[kWtSlots][2][kBlk];  // [walk block % 4][head][row]
   __shared__ int abort_flag, last_flag;
 
   const int tid = threadIdx.x;
@@ -122,16 +127,18 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   const int blk0 = seg * sg.seg_blks;
   const int nb = min(sg.nblk, blk0 + sg.seg_blks) - blk0;
   volatile int* abort_v = &abort_flag;
-  uint32_t n_loads[2] = {0, 0};  // the producer's loads per stage
+  uint32_t n_loads[kSegStages] = {0, 0, 0};  // the producer's loads per stage
 
   if (tid == 0) {
     abort_flag = 0;
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSegStages; ++i) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&ready_bar[i], 256);
       mbar_init(&empty_bar[i], 1);
-      mbar_init(&dt_full[i], 32);
-      mbar_init(&dt_empty[i], 256);
+    }
+    for (int i = 0; i < kWtSlots; ++i) {
+      mbar_init(&wt_full[i], 32);
+      mbar_init(&wt_empty[i], 256);
     }
     mbar_init(&done_bar, 1);
     mbar_init(&drain_bar, 1);
@@ -149,8 +156,12 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
       for (int i = 0; i < nb; ++i) {  // block i of the walk = block blk0 + nb - 1 - i
-        const int stage = i & 1;
-        if (i >= 2 && !mbar_wait(&empty_bar[stage], ((i - 2) >> 1) & 1, abort_v, 11)) break;
+        const int stage = i % kSegStages;
+        // stage reuse; block 2 also waits for block 0's MMAs (its low part is in stage 2)
+        const int after = i >= kSegStages ? i - kSegStages : (i == 2 ? 0 : -1);
+        if (after >= 0 && !mbar_wait(&empty_bar[after % kSegStages],
+                                     (after / kSegStages) & 1, abort_v, 11))
+          break;
         const int t0 = (blk0 + nb - 1 - i) * kBlk;
         uint8_t* st = smem + stage * kSegStage;
         ++n_loads[stage];
@@ -169,71 +180,88 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       // address field (every address stays below 256 KB, so the field cannot carry)
       const uint64_t d0 = sdesc(smem_u32(smem), kTile, 1024);
       for (int i = 0; i < nb; ++i) {
-        const int stage = i & 1;
-        if (!mbar_wait(&ready_bar[stage], (i >> 1) & 1, abort_v, 12)) break;
+        const int stage = i % kSegStages;
+        if (!mbar_wait(&ready_bar[stage], (i / kSegStages) & 1, abort_v, 12)) break;
         tc_fence_after();
-        const uint64_t ds = d0 + (stage ? (kSegStage >> 4) : 0u);
+        const uint64_t ds = d0 + uint64_t(stage) * (kSegStage >> 4);
+        const uint64_t dlo = d0 + ((2 * kSegStage + 2 * kTile) >> 4);  // stage 2's x area
 #pragma unroll
         for (int k = 0; k < kBlk / 16; ++k) {
           const uint64_t ad = ds + k * 128;                                     // B^T: M = n
           mma_ss(tmem, ad, ad + ((2 * kTile) >> 4), idesc, (i > 0 || k > 0) ? 1u : 0u);  // X'
-          if (i == 0) mma_ss(tmem, ad, ad + ((4 * kTile) >> 4), idesc, 1u);   // X' low part
+          if (i == 0) mma_ss(tmem, ad, dlo + k * 128, idesc, 1u);             // X' low part
         }
         mma_commit(&empty_bar[stage]);
         if (i == nb - 1) mma_commit(&done_bar);
       }
     }
   } else if (warp == 10) {
-    // ------------------------------ step-size loader ------------------------------
-    // lane l: rows 4l .. 4l+3 of both heads of walk block i (8 independent loads)
+    // ------------------------------ weights ------------------------------
+    // w_t = exp(sum_{k > t, k in segment} a_k) dt_t, a_k = dt_k A log2(e) (log2 units); the
+    // walk goes from the segment's last block to its first, so `run` (the blocks after the
+    // current one) is a running total.
     const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
-    for (int i = 0; i < nb; ++i) {
-      const int bf = i & 1;
-      if (i >= 2 && !mbar_wait(&dt_empty[bf], ((i - 2) >> 1) & 1, abort_v, 15)) break;
-      float v[8];
+    const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
+    float run[2] = {0.f, 0.f};
+    float v[kWtSlots][8];  // dt of walk block i in v[i % 4]: rows 4 lane + r, head h at [2r + h]
+    auto load = [&](int i, float (&w)[8]) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int64_t tok = int64_t(blk0 + nb - 1 - i) * kBlk + 4 * lane + r;
-        const bool in = tok < seqlen;
-        v[2 * r] = in ? dtb[tok * nheads] : 0.f;
-        v[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
+        const bool in = i < nb && tok < seqlen;
+        w[2 * r] = in ? dtb[tok * nheads] : 0.f;
+        w[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
       }
-      *reinterpret_cast<float4*>(&dt_stage[bf][0][4 * lane]) = make_float4(v[0], v[2], v[4], v[6]);
-      *reinterpret_cast<float4*>(&dt_stage[bf][1][4 * lane]) = make_float4(v[1], v[3], v[5], v[7]);
-      mbar_arrive_warp(&dt_full[bf]);
+    };
+#pragma unroll
+    for (int u = 0; u < kWtSlots; ++u) load(u, v[u]);
+    bool wok = true;
+    for (int i0 = 0; i0 < nb && wok; i0 += kWtSlots) {
+#pragma unroll
+      for (int u = 0; u < kWtSlots; ++u) {
+        const int i = i0 + u;
+        if (i < nb && wok) {
+          // (warp-uniform decisions: every lane reaches the same __syncwarp)
+          if (i >= kWtSlots &&
+              !__all_sync(0xffffffffu,
+                          mbar_wait(&wt_empty[u], ((i / kWtSlots) - 1) & 1, abort_v, 15))) {
+            wok = false;
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float c0 = v[u][h] * al[h];
+              const float c1 = fmaf(v[u][2 + h], al[h], c0);
+              const float c2 = fmaf(v[u][4 + h], al[h], c1);
+              const float c3 = fmaf(v[u][6 + h], al[h], c2);
+              const float incl = warp_inclusive_scan(c3);
+              const float off = incl - c3;
+              const float tot = __shfl_sync(0xffffffffu, incl, 31);
+              const float rest = tot - off + run[h];  // minus the prefix through row 4 lane - 1
+              *reinterpret_cast<float4*>(&wt_stage[u][h][4 * lane]) =
+                  make_float4(ex2(rest - c0) * v[u][h], ex2(rest - c1) * v[u][2 + h],
+                              ex2(rest - c2) * v[u][4 + h], ex2(rest - c3) * v[u][6 + h]);
+              run[h] += tot;
+            }
+            mbar_arrive_warp(&wt_full[u]);
+            load(i + kWtSlots, v[u]);  // in flight while the next blocks are processed
+          }
+        }
+      }
     }
+    if (lane < 2) seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + lane] = run[lane];
   } else {
     // ------------------------------ compute warps ------------------------------
     const int row = tid & 127, j = tid >> 7;
-    const float Alog = A[h0 + j] * kLog2e;
-    float run = 0.f;  // log2-decay of the blocks after the current one, within the segment
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
-      const int stage = i & 1;
-      ok = ok && mbar_wait(&dt_full[i & 1], (i >> 1) & 1, abort_v, 16);
-      const float d = dt_stage[i & 1][j][row];
-      mbar_arrive_warp(&dt_empty[i & 1]);
-      // w_t = exp(sum_{k > t, k in segment} a_k) * dt_t
-      const float a = d * Alog;
-      float v = warp_inclusive_scan(a);
-      if (lane == 31) scan_scratch[warp] = v;
-      named_sync(1, 256);
-      const int w0 = warp & ~3;
-      float off = 0.f, tot = 0.f;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float sw = scan_scratch[w0 + w];
-        off += (w0 + w < warp) ? sw : 0.f;
-        tot += sw;
-      }
-      named_sync(1, 256);  // scratch read by everyone before the next block overwrites it
-      const float incl = v + off;
-      const float wt = ex2(tot - incl + run) * d;  // tot - incl = sum over k > t in this block
-      run += tot;
-      ok = ok && mbar_wait(&full_bar[stage], (i >> 1) & 1, abort_v, 13);
+      const int stage = i % kSegStages;
+      ok = ok && mbar_wait(&wt_full[i % kWtSlots], (i / kWtSlots) & 1, abort_v, 16);
+      const float wt = wt_stage[i % kWtSlots][j][row];
+      mbar_arrive_warp(&wt_empty[i % kWtSlots]);
+      ok = ok && mbar_wait(&full_bar[stage], (i / kSegStages) & 1, abort_v, 13);
       if (ok) {
         uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
-        uint8_t* lr = smem + stage * kSegStage + (4 + j) * kTile;
+        uint8_t* lr = smem + 2 * kSegStage + (2 + j) * kTile;
         if (i == 0) {  // the segment's last block: bf16 high part in place, low part beside it
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -260,8 +288,8 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
         }
         fence_proxy_async_smem();
       }
-      mbar_arrive(&ready_bar[stage]);
-      if (named_sync_or(1, 256, !ok || *abort_v)) { ok = false; break; }
+      mbar_arrive_warp(&ready_bar[stage]);
+      if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
     }
     // epilogue: lane n = row, columns of head j
     if (ok && nb > 0) ok = mbar_wait(&done_bar, 0, abort_v, 14);
@@ -279,7 +307,6 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
         for (int e = 0; e < 16; ++e)
           out[(pc * 16 + e) * kN] = nb > 0 ? __uint_as_float(r[e]) : 0.f;
       }
-      if (row == 0) seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + j] = run;
     }
   }
   // ------------------------------ teardown ------------------------------
@@ -289,7 +316,7 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     drain(&drain_bar, 0);
   }
   if (*abort_v && warp == 8 && lane == 0) {  // and every issued copy
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kSegStages; ++i)
       if (n_loads[i]) drain(&full_bar[i], (n_loads[i] - 1) & 1);
   }
   tc_fence_before();
@@ -360,13 +387,12 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
 //               `row` of a block (state row n = row in the state passes) and a quarter of the
 //               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and
 //               the epilogue; G column groups q and q + 4 for the masks.  Four warps share
-//               each TMEM lane quarter, so every phase is spread over all 16 warps.  Warps 0
-//               and 1 also compute the next block's cumsums (one head each).
+//               each TMEM lane quarter, so every phase is spread over all 16 warps.
 //   warp 16     TMA producer (lane 0): C, x (single buffers), B (double buffer) per block.
 //   warp 17     MMA issuer (lane 0).
 //   warp 18     y writer (lane 0): TMA stores of each block's staged y.
-//   warp 19     step-size loader: each block's dt of the two heads into shared memory, up to
-//               two blocks ahead (plain loads, off the compute warps).
+//   warp 19     cumsums: loads each block's dt of the two heads and writes its log2 cumsums
+//               to shared memory, up to two blocks ahead (lane l: rows 4l .. 4l+3).
 // Per block k the compute warps write the masks (MMA: diagonal tiles), then the state pass
 // (MMA: C H), then X' (MMA: state update) and the epilogue.  The masks come first so that the
 // previous block's y stores, which read the staging buffer the state pass overwrites, drain
@@ -439,8 +465,7 @@ struct OutBars {
   uint64_t g_done, d_done, o_done, st_done;  // MMA completion -> compute
   uint64_t m0_ready, m1_ready, h_ready, xp_ready;  // compute -> MMA issuer
   uint64_t y_staged, stage_free;             // compute <-> y writer
-  uint64_t cs_full[2], cs_empty[2];          // scan warps <-> compute (per cumsum buffer)
-  uint64_t dt_full[2], dt_empty[2];          // step-size loader <-> scan warps
+  uint64_t cs_full[2], cs_empty[2];          // cumsum warp <-> compute (per cumsum buffer)
   uint64_t drain;
 };
 
@@ -460,7 +485,6 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
   __shared__ __align__(16) float cs_sh[2][2][kBlk];
   __shared__ __align__(16) float cl_sh[2][2][kBlk];
   __shared__ __align__(16) float v_sh[2][2][kBlk];
-  __shared__ __align__(16) float dt_stage[2][2][kBlk];  // [block % 2][head][row]
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
@@ -487,10 +511,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     mbar_init(&bars.xp_ready, kComputeThreads);
     mbar_init(&bars.y_staged, kComputeThreads);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.cs_full[i], 64);
+      mbar_init(&bars.cs_full[i], 32);
       mbar_init(&bars.cs_empty[i], kComputeThreads);
-      mbar_init(&bars.dt_full[i], 32);
-      mbar_init(&bars.dt_empty[i], 64);
     }
     fence_mbar_init();
   }
@@ -623,23 +645,52 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       bulk_wait_all();
     }
   } else if (warp == 19) {
-    // ------------------------------ step-size loader ------------------------------
-    // lane l: rows 4l .. 4l+3 of both heads (8 independent loads per block)
+    // ------------------------------ cumsums ------------------------------
+    // Per block and head: cs_t = inclusive log2 cumsum of dt A (within the block), cl_t =
+    // cs_t - log2(dt_t) (+inf where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15.
     const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
+    const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
+    float v[8];  // dt of rows 4 lane + r, head h at v[2r + h]
+    auto load = [&](int kb) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int64_t tok = int64_t(blk0 + kb) * kBlk + 4 * lane + r;
+        const bool in = tok < seqlen;
+        v[2 * r] = in ? dtb[tok * nheads] : 0.f;
+        v[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
+      }
+    };
+    load(0);
+    const float inf = __int_as_float(0x7f800000);
     for (int kb = 0; kb < nb; ++kb) {
       const int bf = kb & 1;
-      if (kb >= 2 && !mbar_wait(&bars.dt_empty[bf], ((kb - 2) >> 1) & 1, abort_v, 71)) break;
-      float v[8];
+      if (kb >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars.cs_empty[bf], ((kb - 2) >> 1) & 1,
+                                                        abort_v, 58)))
+        break;  // warp-uniform, so every lane reaches the same __syncwarp
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t tok = int64_t(blk0 + kb) * kBlk + 4 * lane + i;
-        const bool in = tok < seqlen;
-        v[2 * i] = in ? dtb[tok * nheads] : 0.f;
-        v[2 * i + 1] = in ? dtb[tok * nheads + 1] : 0.f;
+      for (int h = 0; h < 2; ++h) {
+        const float d0 = v[h], d1 = v[2 + h], d2 = v[4 + h], d3 = v[6 + h];
+        float c0 = d0 * al[h];
+        float c1 = fmaf(d1, al[h], c0);
+        float c2 = fmaf(d2, al[h], c1);
+        float c3 = fmaf(d3, al[h], c2);
+        const float off = warp_inclusive_scan(c3) - c3;
+        c0 += off;
+        c1 += off;
+        c2 += off;
+        c3 += off;
+        const float l0 = d0 > 0.f ? c0 - __log2f(d0) : inf;
+        const float l1 = d1 > 0.f ? c1 - __log2f(d1) : inf;
+        const float l2 = d2 > 0.f ? c2 - __log2f(d2) : inf;
+        const float l3 = d3 > 0.f ? c3 - __log2f(d3) : inf;
+        const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
+        *reinterpret_cast<float4*>(&cs_sh[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
+        *reinterpret_cast<float4*>(&cl_sh[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
+        *reinterpret_cast<float4*>(&v_sh[bf][h][4 * lane]) =
+            make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
       }
-      *reinterpret_cast<float4*>(&dt_stage[bf][0][4 * lane]) = make_float4(v[0], v[2], v[4], v[6]);
-      *reinterpret_cast<float4*>(&dt_stage[bf][1][4 * lane]) = make_float4(v[1], v[3], v[5], v[7]);
-      mbar_arrive_warp(&bars.dt_full[bf]);
+      mbar_arrive_warp(&bars.cs_full[bf]);
+      if (kb + 1 < nb) load(kb + 1);
     }
   } else {
     // ------------------------------ compute warps ------------------------------
@@ -661,45 +712,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       tmem_wait_st();
     }
     const float Dh = D ? D[h0 + j] : 0.f;
-    // ---- within-block log2 cumsums, one warp per head (warp 0: head 0, warp 1: head 1; lane
-    //      owns rows 4 lane .. 4 lane + 3).  Block k + 1's are computed during block k, into
-    //      the other buffer ----
-    const bool scan_warp = warp < 2;
-    const int hs = warp & 1;
-    const float Alog_s = A[h0 + hs] * kLog2e;
-    // the cumsums of block kb (false if a wait gave up)
-    auto scan_block = [&](int kb) {
-      const int bf = kb & 1;
-      const bool got = mbar_wait(&bars.dt_full[bf], (kb >> 1) & 1, abort_v, 58);
-      const float4 dv = *reinterpret_cast<const float4*>(&dt_stage[bf][hs][4 * lane]);
-      mbar_arrive_warp(&bars.dt_empty[bf]);
-      if (!__all_sync(0xffffffffu, got)) return false;
-      float c0 = dv.x * Alog_s;
-      float c1 = fmaf(dv.y, Alog_s, c0);
-      float c2 = fmaf(dv.z, Alog_s, c1);
-      float c3 = fmaf(dv.w, Alog_s, c2);
-      const float off = warp_inclusive_scan(c3) - c3;
-      c0 += off;
-      c1 += off;
-      c2 += off;
-      c3 += off;
-      const float inf = __int_as_float(0x7f800000);
-      const float l0 = dv.x > 0.f ? c0 - __log2f(dv.x) : inf;
-      const float l1 = dv.y > 0.f ? c1 - __log2f(dv.y) : inf;
-      const float l2 = dv.z > 0.f ? c2 - __log2f(dv.z) : inf;
-      const float l3 = dv.w > 0.f ? c3 - __log2f(dv.w) : inf;
-      const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
-      *reinterpret_cast<float4*>(&cs_sh[bf][hs][4 * lane]) = make_float4(c0, c1, c2, c3);
-      *reinterpret_cast<float4*>(&cl_sh[bf][hs][4 * lane]) = make_float4(l0, l1, l2, l3);
-      *reinterpret_cast<float4*>(&v_sh[bf][hs][4 * lane]) =
-          make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
-      return true;
-    };
     bool ok = true;
-    if (scan_warp) {
-      if (nb > 0) ok = scan_block(0);
-      mbar_arrive_warp(&bars.cs_full[0]);
-    }
     uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
     const int t = row;
     const int wlast = wq * 32 + 31;                 // last row of this warp
@@ -814,13 +827,6 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       }
       tc_fence_before();
       mbar_arrive_warp(&bars.h_ready);
-      // ---- the next block's cumsums (scan warps), once every thread is done with the buffer
-      //      block k - 1 used ----
-      if (scan_warp && k + 1 < nb) {
-        if (k >= 1) ok = ok && mbar_wait(&bars.cs_empty[bf ^ 1], ((k - 1) >> 1) & 1, abort_v, 56);
-        if (__all_sync(0xffffffffu, ok)) ok = scan_block(k + 1);
-        mbar_arrive_warp(&bars.cs_full[bf ^ 1]);
-      }
       // ---- once the diagonal MMAs are done: X' = w x in place for the state MMA (row t,
       //      head j, p in [p0, p0+32)); then, once C H is done too, y_t = Diag + exp(cs_t) Off
       //      + D x_t staged in shared memory and written by TMA ----

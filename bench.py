@@ -17,6 +17,9 @@ the data path; times are the max over ranks.
 --impl reference runs the float64 CPU oracle (the plain sequential recurrence) on the host
 cores, each step a bounded sample of the same workload (batch row 0: 80 heads x 64 channels
 x 8192 tokens), and reports the same metric.
+
+--profile scan|decode runs only W + K calls of that workload and prints nothing else: the
+command the launch lists and ncu captures under profiles/ were taken with.
 """
 import argparse
 import json
@@ -223,7 +226,7 @@ def run_ours(args):
     achieved = nbytes / (statistics.mean(per) / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "traffic": args.traffic,
-            "kernel": "ssd_chunk_scan_fwd (seg_state + seg_scan + chunk_out, one call)",
+            "kernel": "ssd_chunk_scan_fwd (one call: seg_state + chunk_out)",
             "algorithmic_bytes": nbytes, "flops": scan_flops(c),
             "peak_source": peak_src,
             "flop_frac": round(scan_flops(c) / (statistics.mean(per) / 1e3) / 1e12 / tflops, 4)}
@@ -316,9 +319,11 @@ def run_ours(args):
                       "nheads": c["nheads"], "headdim": c["headdim"], "dstate": c["dstate"],
                       "ngroups": c["ngroups"], "chunk": c["chunk"], "init_state": c["init"],
                       "parallelism": f"replicas{world}" if world > 1 else "single",
-                      "l2": "inputs larger than L2 (719 MB per step > 126 MB), no flush"},
+                      "y_dtype": "f32",
+                      "l2": "inputs and outputs larger than L2 (1055 MB per step > 126 MB), "
+                            "no flush"},
            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
-           "gpu_launches": 3 * args.steps, "decode": decode, "device_status": status,
+           "gpu_launches": 2 * args.steps, "decode": decode, "device_status": status,
            "path": "tcgen05" if ssd.path(c["batch"], c["seqlen"], c["nheads"], c["headdim"],
                                         c["dstate"], c["ngroups"], c["chunk"]) == 1 else "simt"}
     if rank == 0:
@@ -374,6 +379,31 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_profile(args):
+    """W + K calls of one workload and nothing else (for ncu launch lists and captures)."""
+    import torch
+    import mamba_ssd_scan_03_b200 as ssd
+    dev = torch.device("cuda", 0)
+    if args.profile == "scan":
+        inp = ssd_inputs.make_scan_inputs(SCAN_CFG, seqlen=args.seqlen)
+        c = inp["cfg"]
+        t = {k: to_dev(inp[k], k in ("x", "B", "C"), dev)
+             for k in ("x", "dt", "A", "B", "C", "D", "init")}
+        for _ in range(args.warmup + args.steps):
+            ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], c["chunk"],
+                               init_state=t["init"])
+    else:
+        dec = ssd_inputs.make_decode_inputs(DECODE_CFG)
+        st = to_dev(dec["state"], False, dev)
+        A4, D4 = to_dev(dec["A"], False, dev), to_dev(dec["D"], False, dev)
+        s = ssd_inputs.decode_step_inputs(dec, 0)
+        t = {n: to_dev(s[n], n != "dt", dev) for n in ("x", "dt", "B", "C")}
+        for _ in range(args.warmup + args.steps):
+            ssd.step(st, t["x"], t["dt"], A4, t["B"], t["C"], D4)
+    torch.cuda.synchronize()
+    assert ssd.device_status() == 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -385,10 +415,15 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per scan call (null when not measured)")
     ap.add_argument("--decode-traffic", type=float, default=None)
+    ap.add_argument("--profile", choices=["scan", "decode"], default=None)
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="with --profile scan: a shorter sequence (smaller capture)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

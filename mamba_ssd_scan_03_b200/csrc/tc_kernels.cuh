@@ -74,7 +74,13 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
 // Split a float pair into bf16 high parts and the bf16 rounding of the remainders.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16x2(a, b);
-  lo = pack_bf16x2(a - bf16lo(hi), b - bf16hi(hi));
+  const float2 r = sub2(make_float2(a, b), make_float2(bf16lo(hi), bf16hi(hi)));
+  lo = pack_bf16x2(r.x, r.y);
+}
+// a bf16 pair scaled by w, rounded back to a bf16 pair
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float2 ww) {
+  const float2 r = mul2(make_float2(bf16lo(v), bf16hi(v)), ww);
+  return pack_bf16x2(r.x, r.y);
 }
 
 // =============================================================================================
@@ -280,10 +286,9 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
           for (int c = 0; c < 8; ++c) {
             uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
             const uint4 xv = *ph;
-            *ph = make_uint4(pack_bf16x2(bf16lo(xv.x) * wt, bf16hi(xv.x) * wt),
-                             pack_bf16x2(bf16lo(xv.y) * wt, bf16hi(xv.y) * wt),
-                             pack_bf16x2(bf16lo(xv.z) * wt, bf16hi(xv.z) * wt),
-                             pack_bf16x2(bf16lo(xv.w) * wt, bf16hi(xv.w) * wt));
+            const float2 ww = make_float2(wt, wt);
+            *ph = make_uint4(scale_bf16x2(xv.x, ww), scale_bf16x2(xv.y, ww),
+                             scale_bf16x2(xv.z, ww), scale_bf16x2(xv.w, ww));
           }
         }
         fence_proxy_async_smem();
@@ -746,26 +751,30 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     const bool live = (GG) ? live1 : live0;                                                    \
     if (wq * 32 >= s0 + 15) {                                                                  \
       const float u = ex2(cs_sh[bf][H][t] - cs_sh[bf][H][s0 + 15]);                            \
+      const float2 uu = make_float2(u, u);                                                     \
       const float4* vp = reinterpret_cast<const float4*>(&v_sh[bf][H][s0]);                    \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 vv = vp[e4];                                                              \
-        R[2 * e4] = pack_bf16x2(gv[(GG) * 16 + 4 * e4] * (u * vv.x),                           \
-                                gv[(GG) * 16 + 4 * e4 + 1] * (u * vv.y));                      \
-        R[2 * e4 + 1] = pack_bf16x2(gv[(GG) * 16 + 4 * e4 + 2] * (u * vv.z),                   \
-                                    gv[(GG) * 16 + 4 * e4 + 3] * (u * vv.w));                  \
+        const float* gq = &gv[(GG) * 16 + 4 * e4];                                             \
+        const float2 a = mul2(make_float2(gq[0], gq[1]), mul2(uu, make_float2(vv.x, vv.y)));   \
+        const float2 c = mul2(make_float2(gq[2], gq[3]), mul2(uu, make_float2(vv.z, vv.w)));   \
+        R[2 * e4] = pack_bf16x2(a.x, a.y);                                                     \
+        R[2 * e4 + 1] = pack_bf16x2(c.x, c.y);                                                 \
       }                                                                                        \
     } else if (live) {                                                                         \
       const float ct = cs_sh[bf][H][t];                                                        \
+      const float2 cc = make_float2(ct, ct);                                                   \
       const float4* cp = reinterpret_cast<const float4*>(&cl_sh[bf][H][s0]);                   \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 cl = cp[e4];                                                              \
         const int s = s0 + 4 * e4;                                                             \
-        const float f0 = s + 0 <= t ? gv[(GG) * 16 + 4 * e4 + 0] * ex2(ct - cl.x) : 0.f;       \
-        const float f1 = s + 1 <= t ? gv[(GG) * 16 + 4 * e4 + 1] * ex2(ct - cl.y) : 0.f;       \
-        const float f2 = s + 2 <= t ? gv[(GG) * 16 + 4 * e4 + 2] * ex2(ct - cl.z) : 0.f;       \
-        const float f3 = s + 3 <= t ? gv[(GG) * 16 + 4 * e4 + 3] * ex2(ct - cl.w) : 0.f;       \
-        R[2 * e4] = pack_bf16x2(f0, f1);                                                       \
-        R[2 * e4 + 1] = pack_bf16x2(f2, f3);                                                   \
+        const float* gq = &gv[(GG) * 16 + 4 * e4];                                             \
+        const float2 d01 = sub2(cc, make_float2(cl.x, cl.y));                                  \
+        const float2 d23 = sub2(cc, make_float2(cl.z, cl.w));                                  \
+        const float2 a = mul2(make_float2(gq[0], gq[1]), make_float2(ex2(d01.x), ex2(d01.y))); \
+        const float2 c = mul2(make_float2(gq[2], gq[3]), make_float2(ex2(d23.x), ex2(d23.y))); \
+        R[2 * e4] = pack_bf16x2(s + 0 <= t ? a.x : 0.f, s + 1 <= t ? a.y : 0.f);              \
+        R[2 * e4 + 1] = pack_bf16x2(s + 2 <= t ? c.x : 0.f, s + 3 <= t ? c.y : 0.f);          \
       }                                                                                        \
     } else {                                                                                   \
       _Pragma("unroll") for (int e = 0; e < 8; ++e) R[e] = 0u;                                \
@@ -814,7 +823,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
     *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
     *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
     *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
-    _Pragma("unroll") for (int e = 0; e < 16; ++e) R[e] = __float_as_uint(__uint_as_float(R[e]) * al); \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e) {                                          \
+      const float2 sc = mul2(make_float2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1])), \
+                             make_float2(al, al));                                            \
+      R[2 * e] = __float_as_uint(sc.x);                                                       \
+      R[2 * e + 1] = __float_as_uint(sc.y);                                                   \
+    }                                                                                         \
     tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
   }
         SSD_HPASS(ra, 0)
@@ -841,10 +855,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
           uint4* pch = reinterpret_cast<uint4*>(xrow + swz(t, (p0 >> 3) + cc));
           const uint4 v = *pch;
           xw[cc * 4 + 0] = v.x; xw[cc * 4 + 1] = v.y; xw[cc * 4 + 2] = v.z; xw[cc * 4 + 3] = v.w;
-          *pch = make_uint4(pack_bf16x2(bf16lo(v.x) * wj, bf16hi(v.x) * wj),
-                            pack_bf16x2(bf16lo(v.y) * wj, bf16hi(v.y) * wj),
-                            pack_bf16x2(bf16lo(v.z) * wj, bf16hi(v.z) * wj),
-                            pack_bf16x2(bf16lo(v.w) * wj, bf16hi(v.w) * wj));
+          const float2 ww = make_float2(wj, wj);
+          *pch = make_uint4(scale_bf16x2(v.x, ww), scale_bf16x2(v.y, ww), scale_bf16x2(v.z, ww),
+                            scale_bf16x2(v.w, ww));
         }
         fence_proxy_async_smem();
       }
@@ -863,9 +876,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t xv = xw[pc * 8 + e];
-            yv[2 * e] = __uint_as_float(rd[2 * e]) + ej * __uint_as_float(ro[2 * e]) + Dh * bf16lo(xv);
-            yv[2 * e + 1] =
-                __uint_as_float(rd[2 * e + 1]) + ej * __uint_as_float(ro[2 * e + 1]) + Dh * bf16hi(xv);
+            const float2 dd = fma2(make_float2(ej, ej),
+                                   make_float2(__uint_as_float(ro[2 * e]), __uint_as_float(ro[2 * e + 1])),
+                                   make_float2(__uint_as_float(rd[2 * e]), __uint_as_float(rd[2 * e + 1])));
+            const float2 yy = fma2(make_float2(Dh, Dh), make_float2(bf16lo(xv), bf16hi(xv)), dd);
+            yv[2 * e] = yy.x;
+            yv[2 * e + 1] = yy.y;
           }
           ystage<TY>::put16(stage, t, q, pc, yv);
         }

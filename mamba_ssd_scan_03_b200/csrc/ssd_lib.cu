@@ -78,16 +78,14 @@ Seg tc_segments(const Shape& s) {
 }
 
 // Tensor-core path scratch: segment states [b, seg, h, 64, 128] f32 | segment log2-decays
-// [b, seg, h] f32 | per (b, head pair) completion counts (zeroed by the call itself).
+// [b, seg, h] f32.
 struct SegScratch {
   float* states;
   float* decay;
-  unsigned* count;
 };
 size_t seg_scratch_bytes(const Shape& s, const Seg& sg) {
   return align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float)) +
-         align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float)) +
-         align256(size_t(s.batch) * (s.nheads / 2) * sizeof(unsigned));
+         align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float));
 }
 SegScratch seg_scratch(const Shape& s, const Seg& sg, void* base) {
   char* p = static_cast<char*>(base);
@@ -95,8 +93,6 @@ SegScratch seg_scratch(const Shape& s, const Seg& sg, void* base) {
   r.states = reinterpret_cast<float*>(p);
   p += align256(size_t(s.batch) * sg.nseg * s.nheads * 64 * 128 * sizeof(float));
   r.decay = reinterpret_cast<float*>(p);
-  p += align256(size_t(s.batch) * sg.nseg * s.nheads * sizeof(float));
-  r.count = reinterpret_cast<unsigned*>(p);
   return r;
 }
 size_t tc_workspace(const Shape& s) { return seg_scratch_bytes(s, tc_segments(s)); }
@@ -265,12 +261,18 @@ ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, voi
     return SSD_ERR_CUDA;
   const int hpg = s.nheads / s.ngroups;
   const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-  if (cudaMemsetAsync(w.count, 0, size_t(s.batch) * (s.nheads / 2) * sizeof(unsigned),
-                      a.stream) != cudaSuccess)
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return SSD_ERR_CUDA;
-  ssd::tc::seg_state_kernel<<<grid, ssd::tc::kSegThreads, kSegSmem, a.stream>>>(
-      mx, mb, a.dt, a.A, w.states, w.decay, w.count, a.init, a.fin, s.seqlen, s.nheads, hpg,
-      sg);
+  ssd::tc::seg_state_kernel<<<std::min<unsigned>(grid, unsigned(nsm)), ssd::tc::kSegThreads,
+                              kSegSmem, a.stream>>>(mx, mb, a.dt, a.A, w.states, w.decay,
+                                                    s.seqlen, s.nheads, hpg, sg, int(grid));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const int64_t nvec = s.batch * s.nheads * int64_t(64) * 128 / 4;
+  ssd::tc::seg_pass_kernel<<<unsigned((nvec + ssd::tc::kPassThreads - 1) / ssd::tc::kPassThreads),
+                             ssd::tc::kPassThreads, 0, a.stream>>>(
+      w.states, w.decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   if (a.ydt == SSD_F32)
     ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(

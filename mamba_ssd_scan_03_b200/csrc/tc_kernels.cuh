@@ -1,13 +1,13 @@
 // tc_kernels.cuh -- the chunked scan on sm_100a tensor cores (bf16 io, headdim 64, dstate 128).
 //
 // The sequence of each (batch row, head) is cut into 128-token blocks (the tcgen05 M=128 tile)
-// and the blocks into segments of consecutive blocks.  Two kernels, in stream order:
+// and the blocks into segments of consecutive blocks.  Three kernels, in stream order:
 //
 //  seg_state   per (b, segment, head pair): S_seg = sum_{t in seg} exp(sum_{k>t in seg} a_k)
 //              dt_t B_t x_t^T, one long-K GEMM on the tensor cores (A = B^T, B = w*x, K =
-//              tokens), plus the segment's total log-decay.  Reads x and B once.  The last CTA
-//              of each (b, head pair) to finish then passes the state along the segments:
-//              H_in(seg) = state entering each segment, and final_state.
+//              tokens), plus the segment's total log-decay.  Reads x and B once.  Persistent.
+//  seg_pass    per state element: passes the state along the segments: H_in(seg) = state
+//              entering each segment, and final_state.
 //  chunk_out   per (b, segment, head pair): walks the segment's blocks in order with the
 //              running state resident in TMEM.  Per block: G = C B^T (once for both heads),
 //              masked diagonal tile (L o G o dt) X, off-diagonal C H, skip term D x, y store,
@@ -84,54 +84,62 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float2 ww) {
 }
 
 // =============================================================================================
-// seg_state: grid = batch * nseg * (nheads / 2), block = 320 threads:
+// seg_state (persistent): grid = min(units, SMs), units = batch * nseg * (nheads / 2) taken in
+// turn (u = blockIdx.x, + gridDim.x, ...).  The rings below run across units, so the next unit's
+// loads and MMAs start while the current unit's state is read out.  352 threads:
 //   warps 0-7  compute: thread (row = tid % 128, j = tid / 128) scales token row `row` of head
-//              j's x tile to X' = w x and splits it into a bf16 high part (over x) and low part.
+//              j's x tile to X' = w x (for a unit's first walk block also the bf16 remainder),
+//              and at a unit's end writes the state from TMEM to the workspace.
 //   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0);  warp 10  weights: loads
-//              each block's dt of the two heads (four blocks of loads in flight) and writes
-//              w_t into a four-slot ring in shared memory (lane l: rows 4l .. 4l+3).
-// Per stage (three stages):  B tile (2 x 16 KB, n halves) | x, scaled in place to X' (2 heads).
-// The low part of the segment's last block goes to stage 2's x area, which the producer fills
-// only once that block's MMAs are done.
-// Blocks are walked last to first so that the suffix sums of the log-decays are running totals.
-// The segment's last block (first of the walk) sends both X' parts through the tensor core, so
-// the tokens that dominate a fast-decaying state carry ~16 bits of X'; earlier blocks, whose
-// terms reach the state through at least one block's decay, send the bf16 high part only.
-// The CTA that completes a (sequence, head pair) last then runs the state passing over the
-// segments (counted in seg_count, which must be zero at launch).
-// TMEM: 128 columns, lane n / column (j, p) = S_seg[n, (j, p)].
+//              each block's dt of the two heads (four blocks of loads in flight), writes w_t
+//              into a four-slot ring, and each unit's total log2-decay to the workspace.
+// Stage ring (three stages of 64 KB):  B tile (2 x 16 KB, n halves) | x, scaled in place to X'
+// (2 heads).  Blocks are numbered g = 0, 1, ... over the CTA's units, stage g % 3.  Within a
+// unit blocks are walked last to first so that the suffix sums of the log-decays are running
+// totals.  A unit's first walk block (the segment's last block, which dominates a fast-decaying
+// state) sends both X' parts through the tensor core, so those tokens carry ~16 bits of X';
+// earlier blocks reach the state through at least one block's decay and send the high part only.
+// Its low part goes to stage (g + 2) % 3's x area: written once block g - 1's MMAs (the previous
+// occupant) are done, and block g + 2 is loaded there only after block g's MMAs.
+// TMEM: 2 x 128 columns (unit n in buffer n % 2), lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
 constexpr uint32_t kSegStage = 4 * kTile;
 constexpr int kSegStages = 3;
 constexpr int kWtSlots = 4;
 constexpr int kSegThreads = 352;
 
+// unit u -> (b, seg, head pair)
+struct SegUnit {
+  int b, seg, hp, blk0, nb;
+};
+__device__ __forceinline__ SegUnit seg_unit(int u, int npair, const Seg& sg) {
+  SegUnit r;
+  r.hp = u % npair;
+  r.seg = (u / npair) % sg.nseg;
+  r.b = u / (npair * sg.nseg);
+  r.blk0 = r.seg * sg.seg_blks;
+  r.nb = min(sg.nblk, r.blk0 + sg.seg_blks) - r.blk0;
+  return r;
+}
+
 __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-    const float* __restrict__ dt, const float* __restrict__ A, float* seg_states,
-    float* seg_decay, unsigned* seg_count, const float* init_state, float* final_state,
-    int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
+    const float* __restrict__ dt, const float* __restrict__ A, float* __restrict__ seg_states,
+    float* __restrict__ seg_decay, int64_t seqlen, int nheads, int heads_per_group, Seg sg,
+    int units) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   __shared__ uint64_t full_bar[kSegStages], ready_bar[kSegStages], empty_bar[kSegStages];
-  __shared__ uint64_t done_bar, drain_bar;
   __shared__ uint64_t wt_full[kWtSlots], wt_empty[kWtSlots];
+  __shared__ uint64_t acc_full[2], acc_empty[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ __align__(16) float wt_stage[kWtSlots][2][kBlk];  // [walk block % 4][head][row]
-  __shared__ int abort_flag, last_flag;
+  __shared__ __align__(16) float wt_stage[kWtSlots][2][kBlk];  // [block % 4][head][row]
+  __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int npair = nheads / 2;
-  const int unit = blockIdx.x;
-  const int hp = unit % npair;
-  const int seg = (unit / npair) % sg.nseg;
-  const int b = unit / (npair * sg.nseg);
-  const int h0 = hp * 2;
-  const int g = h0 / heads_per_group;
-  const int blk0 = seg * sg.seg_blks;
-  const int nb = min(sg.nblk, blk0 + sg.seg_blks) - blk0;
   volatile int* abort_v = &abort_flag;
   uint32_t n_loads[kSegStages] = {0, 0, 0};  // the producer's loads per stage
 
@@ -146,11 +154,14 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       mbar_init(&wt_full[i], 32);
       mbar_init(&wt_empty[i], 256);
     }
-    mbar_init(&done_bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 256);
+    }
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_base_sh, 128);
+  if (warp == 0) tmem_alloc(&tmem_base_sh, 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -161,21 +172,40 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
-      for (int i = 0; i < nb; ++i) {  // block i of the walk = block blk0 + nb - 1 - i
-        const int stage = i % kSegStages;
-        // stage reuse; block 2 also waits for block 0's MMAs (its low part is in stage 2)
-        const int after = i >= kSegStages ? i - kSegStages : (i == 2 ? 0 : -1);
-        if (after >= 0 && !mbar_wait(&empty_bar[after % kSegStages],
-                                     (after / kSegStages) & 1, abort_v, 11))
-          break;
-        const int t0 = (blk0 + nb - 1 - i) * kBlk;
-        uint8_t* st = smem + stage * kSegStage;
-        ++n_loads[stage];
-        mbar_arrive_expect_tx(&full_bar[stage], 4 * kTile);
-        tma_load_3d(st, &tm_b, &full_bar[stage], g * kN, t0, b);
-        tma_load_3d(st + kTile, &tm_b, &full_bar[stage], g * kN + 64, t0, b);
-        tma_load_3d(st + 2 * kTile, &tm_x, &full_bar[stage], h0 * kP, t0, b);
-        tma_load_3d(st + 3 * kTile, &tm_x, &full_bar[stage], (h0 + 1) * kP, t0, b);
+      int g = 0;
+      int g_first = -1;  // block number of the current unit's first walk block
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const SegUnit su = seg_unit(u, npair, sg);
+        const int gh = (su.hp * 2) / heads_per_group;
+        for (int i = 0; i < su.nb; ++i, ++g) {  // walk block i = block blk0 + nb - 1 - i
+          const int stage = g % kSegStages;
+          if (i == 0) g_first = g;
+          if (g >= kSegStages &&
+              !mbar_wait(&empty_bar[stage], ((g - kSegStages) / kSegStages) & 1, abort_v, 11)) {
+            ok = false;
+            break;
+          }
+          // this stage's x area held the low part of block g - 2 when that block was a first
+          if (g - 2 == g_first && i >= 2 &&
+              !mbar_wait(&empty_bar[(g - 2) % kSegStages], ((g - 2) / kSegStages) & 1, abort_v, 17)) {
+            ok = false;
+            break;
+          }
+          const int t0 = (su.blk0 + su.nb - 1 - i) * kBlk;
+          uint8_t* st = smem + stage * kSegStage;
+          ++n_loads[stage];
+          mbar_arrive_expect_tx(&full_bar[stage], 4 * kTile);
+          tma_load_3d(st, &tm_b, &full_bar[stage], gh * kN, t0, su.b);
+          tma_load_3d(st + kTile, &tm_b, &full_bar[stage], gh * kN + 64, t0, su.b);
+          tma_load_3d(st + 2 * kTile, &tm_x, &full_bar[stage], su.hp * 2 * kP, t0, su.b);
+          tma_load_3d(st + 3 * kTile, &tm_x, &full_bar[stage], (su.hp * 2 + 1) * kP, t0, su.b);
+        }
+        // a unit shorter than three blocks: the next unit's block g_first + 2 is not in this
+        // unit, so wait for the low part's MMA before any later load reuses its stage
+        if (ok && su.nb < 3 && g_first >= 0 &&
+            !mbar_wait(&empty_bar[g_first % kSegStages], (g_first / kSegStages) & 1, abort_v, 18))
+          ok = false;
       }
     }
   } else if (warp == 9) {
@@ -185,133 +215,177 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       // descriptors are built once; a K step or a tile offset adds (bytes >> 4) to the start
       // address field (every address stays below 256 KB, so the field cannot carry)
       const uint64_t d0 = sdesc(smem_u32(smem), kTile, 1024);
-      for (int i = 0; i < nb; ++i) {
-        const int stage = i % kSegStages;
-        if (!mbar_wait(&ready_bar[stage], (i / kSegStages) & 1, abort_v, 12)) break;
-        tc_fence_after();
-        const uint64_t ds = d0 + uint64_t(stage) * (kSegStage >> 4);
-        const uint64_t dlo = d0 + ((2 * kSegStage + 2 * kTile) >> 4);  // stage 2's x area
+      int g = 0, n = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++n) {
+        const SegUnit su = seg_unit(u, npair, sg);
+        const int ab = n & 1;
+        const uint32_t acc = tmem + ab * 128;
+        if (n >= 2 && !mbar_wait(&acc_empty[ab], ((n - 2) >> 1) & 1, abort_v, 19)) break;
+        for (int i = 0; i < su.nb; ++i, ++g) {
+          const int stage = g % kSegStages;
+          if (!mbar_wait(&ready_bar[stage], (g / kSegStages) & 1, abort_v, 12)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ds = d0 + uint64_t(stage) * (kSegStage >> 4);
+          // low part of a first walk block: stage (g + 2) % 3's x area
+          const uint64_t dlo = d0 + uint64_t((g + 2) % kSegStages) * (kSegStage >> 4) +
+                               ((2 * kTile) >> 4);
 #pragma unroll
-        for (int k = 0; k < kBlk / 16; ++k) {
-          const uint64_t ad = ds + k * 128;                                     // B^T: M = n
-          mma_ss(tmem, ad, ad + ((2 * kTile) >> 4), idesc, (i > 0 || k > 0) ? 1u : 0u);  // X'
-          if (i == 0) mma_ss(tmem, ad, dlo + k * 128, idesc, 1u);             // X' low part
+          for (int k = 0; k < kBlk / 16; ++k) {
+            const uint64_t ad = ds + k * 128;                                   // B^T: M = n
+            mma_ss(acc, ad, ad + ((2 * kTile) >> 4), idesc, (i > 0 || k > 0) ? 1u : 0u);  // X'
+            if (i == 0) mma_ss(acc, ad, dlo + k * 128, idesc, 1u);            // X' low part
+          }
+          mma_commit(&empty_bar[stage]);
+          if (i == su.nb - 1) mma_commit(&acc_full[ab]);
         }
-        mma_commit(&empty_bar[stage]);
-        if (i == nb - 1) mma_commit(&done_bar);
       }
     }
   } else if (warp == 10) {
     // ------------------------------ weights ------------------------------
     // w_t = exp(sum_{k > t, k in segment} a_k) dt_t, a_k = dt_k A log2(e) (log2 units); the
     // walk goes from the segment's last block to its first, so `run` (the blocks after the
-    // current one) is a running total.
-    const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
-    const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
-    float run[2] = {0.f, 0.f};
-    float v[kWtSlots][8];  // dt of walk block i in v[i % 4]: rows 4 lane + r, head h at [2r + h]
-    auto load = [&](int i, float (&w)[8]) {
+    // current one) is a running total.  Blocks are numbered across units like the stages.
+    float v[kWtSlots][8];  // dt of block g in v[g % 4]: rows 4 lane + r, head h at [2r + h]
+    // the (unit, walk block) of block number g, for the four-ahead loads
+    int lu = blockIdx.x, li = 0;
+    auto load_next = [&](float (&w)[8]) {
+      bool valid = lu < units;
+      SegUnit su;
+      if (valid) su = seg_unit(lu, npair, sg);
+      const float* dtb = dt + (valid ? (int64_t(su.b) * seqlen * nheads + su.hp * 2) : 0);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const int64_t tok = int64_t(blk0 + nb - 1 - i) * kBlk + 4 * lane + r;
-        const bool in = i < nb && tok < seqlen;
+        const int64_t tok = valid ? int64_t(su.blk0 + su.nb - 1 - li) * kBlk + 4 * lane + r : 0;
+        const bool in = valid && tok < seqlen;
         w[2 * r] = in ? dtb[tok * nheads] : 0.f;
         w[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
       }
+      if (valid && ++li == su.nb) {
+        li = 0;
+        lu += gridDim.x;
+      }
     };
 #pragma unroll
-    for (int u = 0; u < kWtSlots; ++u) load(u, v[u]);
+    for (int s = 0; s < kWtSlots; ++s) load_next(v[s]);
+    int g = 0;
     bool wok = true;
-    for (int i0 = 0; i0 < nb && wok; i0 += kWtSlots) {
-#pragma unroll
-      for (int u = 0; u < kWtSlots; ++u) {
-        const int i = i0 + u;
-        if (i < nb && wok) {
-          // (warp-uniform decisions: every lane reaches the same __syncwarp)
-          if (i >= kWtSlots &&
-              !__all_sync(0xffffffffu,
-                          mbar_wait(&wt_empty[u], ((i / kWtSlots) - 1) & 1, abort_v, 15))) {
-            wok = false;
-          } else {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float c0 = v[u][h] * al[h];
-              const float c1 = fmaf(v[u][2 + h], al[h], c0);
-              const float c2 = fmaf(v[u][4 + h], al[h], c1);
-              const float c3 = fmaf(v[u][6 + h], al[h], c2);
-              const float incl = warp_inclusive_scan(c3);
-              const float off = incl - c3;
-              const float tot = __shfl_sync(0xffffffffu, incl, 31);
-              const float rest = tot - off + run[h];  // minus the prefix through row 4 lane - 1
-              *reinterpret_cast<float4*>(&wt_stage[u][h][4 * lane]) =
-                  make_float4(ex2(rest - c0) * v[u][h], ex2(rest - c1) * v[u][2 + h],
-                              ex2(rest - c2) * v[u][4 + h], ex2(rest - c3) * v[u][6 + h]);
-              run[h] += tot;
-            }
-            mbar_arrive_warp(&wt_full[u]);
-            load(i + kWtSlots, v[u]);  // in flight while the next blocks are processed
-          }
+    for (int u = blockIdx.x; u < units && wok; u += gridDim.x) {
+      const SegUnit su = seg_unit(u, npair, sg);
+      const int h0 = su.hp * 2;
+      const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
+      float run[2] = {0.f, 0.f};
+      for (int i = 0; i < su.nb && wok; ++i, ++g) {
+        const int slot = g % kWtSlots;
+        // (warp-uniform decisions: every lane reaches the same __syncwarp)
+        if (g >= kWtSlots &&
+            !__all_sync(0xffffffffu,
+                        mbar_wait(&wt_empty[slot], ((g / kWtSlots) - 1) & 1, abort_v, 15))) {
+          wok = false;
+          break;
         }
+        float d[8];
+#pragma unroll
+        for (int s = 0; s < kWtSlots; ++s)
+          if (s == slot) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d[e] = v[s][e];
+          }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float c0 = d[h] * al[h];
+          const float c1 = fmaf(d[2 + h], al[h], c0);
+          const float c2 = fmaf(d[4 + h], al[h], c1);
+          const float c3 = fmaf(d[6 + h], al[h], c2);
+          const float incl = warp_inclusive_scan(c3);
+          const float off = incl - c3;
+          const float tot = __shfl_sync(0xffffffffu, incl, 31);
+          const float rest = tot - off + run[h];  // minus the prefix through row 4 lane - 1
+          *reinterpret_cast<float4*>(&wt_stage[slot][h][4 * lane]) =
+              make_float4(ex2(rest - c0) * d[h], ex2(rest - c1) * d[2 + h],
+                          ex2(rest - c2) * d[4 + h], ex2(rest - c3) * d[6 + h]);
+          run[h] += tot;
+        }
+        mbar_arrive_warp(&wt_full[slot]);
+#pragma unroll
+        for (int s = 0; s < kWtSlots; ++s)
+          if (s == slot) load_next(v[s]);  // in flight while the next blocks are processed
       }
+      if (wok && lane < 2)
+        seg_decay[(int64_t(su.b) * sg.nseg + su.seg) * nheads + h0 + lane] = run[lane];
     }
-    if (lane < 2) seg_decay[(int64_t(b) * sg.nseg + seg) * nheads + h0 + lane] = run[lane];
   } else {
     // ------------------------------ compute warps ------------------------------
     const int row = tid & 127, j = tid >> 7;
     bool ok = true;
-    for (int i = 0; i < nb; ++i) {
-      const int stage = i % kSegStages;
-      ok = ok && mbar_wait(&wt_full[i % kWtSlots], (i / kWtSlots) & 1, abort_v, 16);
-      const float wt = wt_stage[i % kWtSlots][j][row];
-      mbar_arrive_warp(&wt_empty[i % kWtSlots]);
-      ok = ok && mbar_wait(&full_bar[stage], (i / kSegStages) & 1, abort_v, 13);
-      if (ok) {
-        uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
-        uint8_t* lr = smem + 2 * kSegStage + (2 + j) * kTile;
-        if (i == 0) {  // the segment's last block: bf16 high part in place, low part beside it
+    int g = 0, n = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
+      const SegUnit su = seg_unit(u, npair, sg);
+      for (int i = 0; i < su.nb; ++i, ++g) {
+        const int stage = g % kSegStages;
+        const int slot = g % kWtSlots;
+        ok = ok && mbar_wait(&wt_full[slot], (g / kWtSlots) & 1, abort_v, 16);
+        const float wt = wt_stage[slot][j][row];
+        mbar_arrive_warp(&wt_empty[slot]);
+        ok = ok && mbar_wait(&full_bar[stage], (g / kSegStages) & 1, abort_v, 13);
+        // a first walk block's low part overwrites stage (g + 2) % 3's x area, whose previous
+        // occupant is block g - 1: wait for its MMAs
+        if (i == 0 && g >= 1)
+          ok = ok && mbar_wait(&empty_bar[(g - 1) % kSegStages], ((g - 1) / kSegStages) & 1,
+                               abort_v, 20);
+        if (ok) {
+          uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
+          uint8_t* lr = smem + ((g + 2) % kSegStages) * kSegStage + (2 + j) * kTile;
+          if (i == 0) {  // bf16 high part in place, low part in the other stage
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
-            const uint4 xv = *ph;
-            uint4 hi, lo;
-            split2(bf16lo(xv.x) * wt, bf16hi(xv.x) * wt, hi.x, lo.x);
-            split2(bf16lo(xv.y) * wt, bf16hi(xv.y) * wt, hi.y, lo.y);
-            split2(bf16lo(xv.z) * wt, bf16hi(xv.z) * wt, hi.z, lo.z);
-            split2(bf16lo(xv.w) * wt, bf16hi(xv.w) * wt, hi.w, lo.w);
-            *ph = hi;
-            *reinterpret_cast<uint4*>(lr + swz(row, c)) = lo;
-          }
-        } else {  // earlier blocks: bf16 X' in place
+            for (int c = 0; c < 8; ++c) {
+              uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
+              const uint4 xv = *ph;
+              uint4 hi, lo;
+              split2(bf16lo(xv.x) * wt, bf16hi(xv.x) * wt, hi.x, lo.x);
+              split2(bf16lo(xv.y) * wt, bf16hi(xv.y) * wt, hi.y, lo.y);
+              split2(bf16lo(xv.z) * wt, bf16hi(xv.z) * wt, hi.z, lo.z);
+              split2(bf16lo(xv.w) * wt, bf16hi(xv.w) * wt, hi.w, lo.w);
+              *ph = hi;
+              *reinterpret_cast<uint4*>(lr + swz(row, c)) = lo;
+            }
+          } else {  // bf16 X' in place
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
-            const uint4 xv = *ph;
-            const float2 ww = make_float2(wt, wt);
-            *ph = make_uint4(scale_bf16x2(xv.x, ww), scale_bf16x2(xv.y, ww),
-                             scale_bf16x2(xv.z, ww), scale_bf16x2(xv.w, ww));
+            for (int c = 0; c < 8; ++c) {
+              uint4* ph = reinterpret_cast<uint4*>(xr + swz(row, c));
+              const uint4 xv = *ph;
+              const float2 ww = make_float2(wt, wt);
+              *ph = make_uint4(scale_bf16x2(xv.x, ww), scale_bf16x2(xv.y, ww),
+                               scale_bf16x2(xv.z, ww), scale_bf16x2(xv.w, ww));
+            }
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        mbar_arrive_warp(&ready_bar[stage]);
       }
-      mbar_arrive_warp(&ready_bar[stage]);
+      // the unit's state: lane n = row, columns of head j
+      const int ab = n & 1;
+      ok = ok && mbar_wait(&acc_full[ab], (n >> 1) & 1, abort_v, 14);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t lane_addr = tmem + ab * 128 + (uint32_t((warp & 3) * 32) << 16) + j * 64;
+        float* out = seg_states +
+                     (((int64_t(su.b) * sg.nseg + su.seg) * nheads + su.hp * 2 + j) * kP) * kN + row;
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          uint32_t r[16];
+          tmem_ld16(lane_addr + pc * 16, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) out[(pc * 16 + e) * kN] = __uint_as_float(r[e]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_warp(&acc_empty[ab]);
       if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
-    }
-    // epilogue: lane n = row, columns of head j
-    if (ok && nb > 0) ok = mbar_wait(&done_bar, 0, abort_v, 14);
-    if (ok) {
-      tc_fence_after();
-      const uint32_t lane_addr = tmem + (uint32_t((warp & 3) * 32) << 16) + j * 64;
-      float* out =
-          seg_states + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP) * kN + row;
-#pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        uint32_t r[16];
-        tmem_ld16(lane_addr + pc * 16, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          out[(pc * 16 + e) * kN] = nb > 0 ? __uint_as_float(r[e]) : 0.f;
-      }
     }
   }
   // ------------------------------ teardown ------------------------------
@@ -327,63 +401,50 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_free(tmem, 128);
-  // ---- the last CTA of this (sequence, head pair) to finish passes the state along its
-  //      segments: H_in(0) = init, H_in(s + 1) = 2^decay(s) H_in(s) + S(s).  seg_states is
-  //      overwritten in place with H_in; final_state receives the state after the last segment
-  //      (it may alias init_state: each element is read before it is written, by one thread) --
-  __threadfence();  // this CTA's states and decays, before the count that publishes them
-  __syncthreads();
-  if (tid == 0) last_flag = atomicAdd(&seg_count[int64_t(b) * npair + hp], 1u) ==
-                            unsigned(sg.nseg - 1);
-  __syncthreads();
-  if (!last_flag) return;
-  __threadfence();
-  // Thread tid carries the running states of float4 elements e = tid + i * kSegThreads of
-  // the pair's two 64 x 128 states in registers and walks the segments in order, so each step
-  // issues all its loads at once.
-  constexpr int kPN = kP * kN;
-  constexpr int kVec = 2 * kPN / 4;
-  constexpr int kPer = (kVec + kSegThreads - 1) / kSegThreads;
-  const int64_t seg_stride = int64_t(nheads) * kPN;
-  float* sbase = seg_states + int64_t(b) * sg.nseg * seg_stride + int64_t(h0) * kPN;
-  const float* dbase = seg_decay + int64_t(b) * sg.nseg * nheads + h0;
-  const int64_t ibase = (int64_t(b) * nheads + h0) * kPN;
-  float4 run[kPer];
+  if (warp == 0) tmem_free(tmem, 256);
+}
+
+// =============================================================================================
+// seg_pass: the state passing between segments.  One thread per float4 of a (batch, head)
+// state, all segments: H_in(0) = init, H_in(s + 1) = 2^decay(s) H_in(s) + S(s).  seg_states
+// is overwritten in place with H_in; final_state receives the state after the last segment
+// (it may alias init_state: each element is read before it is written, by one thread).
+// Segments are taken eight at a time so that eight loads are in flight per thread.
+// =============================================================================================
+constexpr int kPassThreads = 256;
+__global__ void __launch_bounds__(kPassThreads) seg_pass_kernel(
+    float* __restrict__ seg_states, const float* __restrict__ seg_decay,
+    const float* init_state, float* final_state, int batch, int nheads, int nseg) {
+  constexpr int kVec = kP * kN / 4;  // float4 per (batch, head) state
+  const int64_t e = int64_t(blockIdx.x) * kPassThreads + threadIdx.x;
+  if (e >= int64_t(batch) * nheads * kVec) return;
+  const int64_t bh = e / kVec;
+  const int h = int(bh % nheads);
+  const int64_t b = bh / nheads;
+  const int64_t off = (e % kVec) * 4;
+  float4 run = init_state ? *reinterpret_cast<const float4*>(init_state + bh * kVec * 4 + off)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int64_t stride = int64_t(nheads) * kP * kN;
+  float* base = seg_states + (b * nseg * nheads + h) * int64_t(kP) * kN + off;
+  const float* dbase = seg_decay + b * nseg * nheads + h;
+  for (int s0 = 0; s0 < nseg; s0 += 8) {
+    float4 v[8];
+    float a[8];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = tid + i * kSegThreads;
-    run[i] = (init_state && e < kVec) ? *reinterpret_cast<const float4*>(init_state + ibase + 4 * e)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int sgi = 0; sgi < sg.nseg; ++sgi) {
-    float* st = sbase + sgi * seg_stride;  // heads h0, h0 + 1 of segment sgi, contiguous
-    const float a0 = ex2(__ldcg(dbase + int64_t(sgi) * nheads));
-    const float a1 = ex2(__ldcg(dbase + int64_t(sgi) * nheads + 1));
-    float4 v[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = tid + i * kSegThreads;
-      if (e < kVec) v[i] = __ldcg(reinterpret_cast<const float4*>(st + 4 * e));
-    }
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = tid + i * kSegThreads;
-      if (e < kVec) {
-        *reinterpret_cast<float4*>(st + 4 * e) = run[i];
-        const float a = e < kVec / 2 ? a0 : a1;
-        run[i] = make_float4(fmaf(a, run[i].x, v[i].x), fmaf(a, run[i].y, v[i].y),
-                             fmaf(a, run[i].z, v[i].z), fmaf(a, run[i].w, v[i].w));
+    for (int i = 0; i < 8; ++i)
+      if (s0 + i < nseg) {
+        v[i] = *reinterpret_cast<const float4*>(base + (s0 + i) * stride);
+        a[i] = ex2(dbase[int64_t(s0 + i) * nheads]);
       }
-    }
-  }
-  if (final_state) {
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = tid + i * kSegThreads;
-      if (e < kVec) *reinterpret_cast<float4*>(final_state + ibase + 4 * e) = run[i];
-    }
+    for (int i = 0; i < 8; ++i)
+      if (s0 + i < nseg) {
+        *reinterpret_cast<float4*>(base + (s0 + i) * stride) = run;
+        run = make_float4(fmaf(a[i], run.x, v[i].x), fmaf(a[i], run.y, v[i].y),
+                          fmaf(a[i], run.z, v[i].z), fmaf(a[i], run.w, v[i].w));
+      }
   }
+  if (final_state) *reinterpret_cast<float4*>(final_state + bh * kVec * 4 + off) = run;
 }
 
 // =============================================================================================

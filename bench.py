@@ -71,6 +71,29 @@ def step_bytes(c, y_bytes=4):
     return 2 * st + x + y + bc + c["batch"] * c["nheads"] * 4 + 2 * c["nheads"] * 4
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per scan call (sum over its kernels)
+# and per decode step, from one ncu capture of `python bench.py --profile ...` (profiles/), with
+# the hash of the kernel sources they were taken on: reported only while the sources match.
+MEASURED_TRAFFIC = {"scan": (1630156032, "76f342ec2d159186"),
+                    "decode": (1291559680, "76f342ec2d159186")}
+
+
+def kernel_source_hash():
+    import hashlib
+    d = os.path.join(ROOT, "mamba_ssd_scan_03_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kind):
+    nbytes, src = MEASURED_TRAFFIC[kind]
+    return nbytes if nbytes is not None and src == kernel_source_hash() else None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -225,7 +248,8 @@ def run_ours(args):
     nbytes = scan_bytes(c)
     achieved = nbytes / (statistics.mean(per) / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(achieved / hbm, 4), "traffic": args.traffic,
+            "frac": round(achieved / hbm, 4),
+            "traffic": args.traffic if args.traffic is not None else measured_traffic("scan"),
             "kernel": "ssd_chunk_scan_fwd (one call: seg_state + chunk_out)",
             "algorithmic_bytes": nbytes, "flops": scan_flops(c),
             "peak_source": peak_src,
@@ -302,7 +326,9 @@ def run_ours(args):
                          "headdim": dc["headdim"], "dstate": dc["dstate"]},
               "roofline": {"bound": "hbm", "achieved": round(dec_ach, 1), "peak": hbm,
                            "unit": "GB/s", "frac": round(dec_ach / hbm, 4),
-                           "traffic": args.decode_traffic, "kernel": "step_n128_kernel",
+                           "traffic": (args.decode_traffic if args.decode_traffic is not None
+                                       else measured_traffic("decode")),
+                           "kernel": "step_n128_kernel",
                            "algorithmic_bytes": sb, "peak_source": peak_src},
               "clocks": clk_dec.summary(), "gpu_launches": n_dec}
 

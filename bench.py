@@ -250,7 +250,7 @@ def run_ours(args):
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4),
             "traffic": args.traffic if args.traffic is not None else measured_traffic("scan"),
-            "kernel": "ssd_chunk_scan_fwd (one call: seg_state + chunk_out)",
+            "kernel": "ssd_chunk_scan_fwd (one call: seg_state + seg_pass + chunk_out)",
             "algorithmic_bytes": nbytes, "flops": scan_flops(c),
             "peak_source": peak_src,
             "flop_frac": round(scan_flops(c) / (statistics.mean(per) / 1e3) / 1e12 / tflops, 4)}
@@ -349,7 +349,7 @@ def run_ours(args):
                       "l2": "inputs and outputs larger than L2 (1055 MB per step > 126 MB), "
                             "no flush"},
            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
-           "gpu_launches": 2 * args.steps, "decode": decode, "device_status": status,
+           "gpu_launches": 3 * args.steps, "decode": decode, "device_status": status,
            "path": "tcgen05" if ssd.path(c["batch"], c["seqlen"], c["nheads"], c["headdim"],
                                         c["dstate"], c["ngroups"], c["chunk"]) == 1 else "simt"}
     if rank == 0:

@@ -145,7 +145,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, ui
 }
 
 constexpr size_t kTcSmem = ssd::tc::kSmemTiles + 1024;
-constexpr size_t kSegSmem = ssd::tc::kSegStages * size_t(ssd::tc::kSegStage) + 1024;
+template <int HU>
+constexpr size_t kSegSmem = ssd::tc::SegCfg<HU>::kSmem;
+
+// dt [B, L, H] float32 as TMA boxes {4 heads, 128 tokens}: needs H % 4 == 0 (16-byte rows) and
+// a 16-byte aligned base; otherwise seg_state loads dt with plain loads.
+bool make_dt_map(CUtensorMap* m, const float* dt, int64_t batch, int64_t seqlen, int nheads) {
+  if (nheads % 4 != 0 || (reinterpret_cast<uintptr_t>(dt) & 15) != 0) return false;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {uint64_t(nheads), uint64_t(seqlen), uint64_t(batch)};
+  cuuint64_t strides[2] = {uint64_t(nheads) * 4, uint64_t(nheads) * uint64_t(seqlen) * 4};
+  cuuint32_t box[3] = {4, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(dt), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 ssd_status set_smem_attrs() {
   static ssd_status st = SSD_ERR_CUDA;
@@ -158,8 +174,8 @@ ssd_status set_smem_attrs() {
     ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
           cudaSuccess;
-    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem)) ==
+    ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem<2>)) ==
           cudaSuccess;
     for (auto f : {(const void*)ssd::simt::chunk_out_kernel<float, float>,
                    (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16, float>,
@@ -265,9 +281,15 @@ ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, voi
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return SSD_ERR_CUDA;
-  ssd::tc::seg_state_kernel<<<std::min<unsigned>(grid, unsigned(nsm)), ssd::tc::kSegThreads,
-                              kSegSmem, a.stream>>>(mx, mb, a.dt, a.A, w.states, w.decay,
-                                                    s.seqlen, s.nheads, hpg, sg, int(grid));
+  CUtensorMap mdt;
+  std::memset(&mdt, 0, sizeof mdt);
+  const int dt_tma = make_dt_map(&mdt, a.dt, s.batch, s.seqlen, s.nheads) ? 1 : 0;
+  // two heads per unit: four (one B tile for four heads) measured slower at the 2.7B shape
+  // (two 96 KB stages instead of three of 64 KB, and half as many units to balance over SMs)
+  ssd::tc::seg_state_kernel<2><<<std::min<unsigned>(grid, unsigned(nsm)),
+                                 ssd::tc::SegCfg<2>::kThreads, kSegSmem<2>, a.stream>>>(
+      mx, mb, mdt, dt_tma, a.dt, a.A, w.states, w.decay, s.seqlen, s.nheads, hpg, sg,
+      int(grid));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   const int64_t nvec = s.batch * s.nheads * int64_t(64) * 128 / 4;
   ssd::tc::seg_pass_kernel<<<unsigned((nvec + ssd::tc::kPassThreads - 1) / ssd::tc::kPassThreads),
@@ -478,8 +500,8 @@ ssd_status noalloc_setup(void** scratch) {
       return SSD_ERR_CUDA;
     }
     const bool ok =
-        cudaFuncSetAttribute(ssd::tc::seg_state_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem)) ==
+        cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem<2>)) ==
             cudaSuccess &&
         cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<float>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==

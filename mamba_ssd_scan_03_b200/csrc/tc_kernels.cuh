@@ -84,155 +84,179 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float2 ww) {
 }
 
 // =============================================================================================
-// seg_state (persistent): grid = min(units, SMs), units = batch * nseg * (nheads / 2) taken in
-// turn (u = blockIdx.x, + gridDim.x, ...).  The rings below run across units, so the next unit's
-// loads and MMAs start while the current unit's state is read out.  352 threads:
-//   warps 0-7  compute: thread (row = tid % 128, j = tid / 128) scales token row `row` of head
-//              j's x tile to X' = w x (for a unit's first walk block also the bf16 remainder),
-//              and at a unit's end writes the state from TMEM to the workspace.
-//   warp 8     TMA producer (lane 0);  warp 9  MMA issuer (lane 0);  warp 10  weights: loads
-//              each block's dt of the two heads (four blocks of loads in flight), writes w_t
-//              into a four-slot ring, and each unit's total log2-decay to the workspace.
-// Stage ring (three stages of 64 KB):  B tile (2 x 16 KB, n halves) | x, scaled in place to X'
-// (2 heads).  Blocks are numbered g = 0, 1, ... over the CTA's units, stage g % 3.  Within a
-// unit blocks are walked last to first so that the suffix sums of the log-decays are running
-// totals.  A unit's first walk block (the segment's last block, which dominates a fast-decaying
-// state) sends both X' parts through the tensor core, so those tokens carry ~16 bits of X';
-// earlier blocks reach the state through at least one block's decay and send the high part only.
-// Its low part goes to stage (g + 2) % 3's x area: written once block g - 1's MMAs (the previous
-// occupant) are done, and block g + 2 is loaded there only after block g's MMAs.
-// TMEM: 2 x 128 columns (unit n in buffer n % 2), lane n / column (j, p) = S_seg[n, (j, p)].
+// seg_state (persistent): grid = min(units, SMs), units = batch * nseg * (nheads / HU) taken in
+// turn (u = blockIdx.x, + gridDim.x, ...), HU heads per unit (the library launches HU = 2; HU = 4,
+// one B tile for four heads, measured slower at the 2.7B shape).  The rings below run across
+// units, so the next unit's loads and MMAs start while the current unit's state is read out.
+// HU * 128 + 96 threads:
+//   compute    warps 0 .. 4 HU - 1: thread (row = tid % 128, j = tid / 128) scales token row
+//              `row` of head j's x tile to X' = w x (for a unit's first walk block also the bf16
+//              remainder), and at a unit's end writes the state from TMEM to the workspace.
+//   then       TMA producer (lane 0);  MMA issuer (lane 0);  weights: takes each block's dt,
+//              writes w_t into a four-slot ring, and each unit's total log2-decay to the
+//              workspace.  When nheads % 4 == 0 (and dt is 16-byte aligned) dt arrives with the
+//              stage as a TMA box {4 heads, 128 tokens}; otherwise (HU = 2 only) the warp loads
+//              it itself, four blocks ahead.
+// Stage ring (3 stages of 64 KB for HU = 2, 2 stages of 96 KB for HU = 4):  B tile (2 x 16 KB,
+// n halves) | x of the HU heads, scaled in place to X'.  Blocks are numbered g = 0, 1, ... over
+// the CTA's units, stage g % S.  Within a unit blocks are walked last to first so that the
+// suffix sums of the log-decays are running totals.  A unit's first walk block (the segment's
+// last block, which dominates a fast-decaying state) sends both X' parts through the tensor
+// core, so those tokens carry ~16 bits of X'; earlier blocks reach the state through at least
+// one block's decay and send the high part only.  Its low part goes to the x area of stage
+// (g + S - 1) % S: written once block g - 1's MMAs (the previous occupant) are done, and block
+// g + S - 1 is loaded there only after block g's MMAs.
+// TMEM: 2 x HU*64 columns (unit n in buffer n % 2), lane n / column (j, p) = S_seg[n, (j, p)].
 // =============================================================================================
-constexpr uint32_t kSegStage = 4 * kTile;
-constexpr int kSegStages = 3;
-constexpr int kWtSlots = 4;
-constexpr int kSegThreads = 352;
-
-// unit u -> (b, seg, head pair)
-struct SegUnit {
-  int b, seg, hp, blk0, nb;
+template <int HU>
+struct SegCfg {
+  static constexpr int kStages = HU == 2 ? 3 : 2;
+  static constexpr uint32_t kStage = (2 + HU) * kTile;
+  static constexpr uint32_t kDtOff = kStages * kStage;  // dt boxes: [stage][128 tokens][4 heads]
+  static constexpr uint32_t kDtBox = kBlk * 4 * 4;
+  static constexpr uint32_t kSmem = kStages * (kStage + kDtBox) + 1024;
+  static constexpr int kCompute = HU * 128;
+  static constexpr int kThreads = kCompute + 96;
+  static constexpr uint32_t kAccCols = HU * 64;
 };
-__device__ __forceinline__ SegUnit seg_unit(int u, int npair, const Seg& sg) {
+constexpr int kWtSlots = 4;
+
+// unit u -> (b, seg, head group of HU heads)
+struct SegUnit {
+  int b, seg, hq, blk0, nb;
+};
+__device__ __forceinline__ SegUnit seg_unit(int u, int nq, const Seg& sg) {
   SegUnit r;
-  r.hp = u % npair;
-  r.seg = (u / npair) % sg.nseg;
-  r.b = u / (npair * sg.nseg);
+  r.hq = u % nq;
+  r.seg = (u / nq) % sg.nseg;
+  r.b = u / (nq * sg.nseg);
   r.blk0 = r.seg * sg.seg_blks;
   r.nb = min(sg.nblk, r.blk0 + sg.seg_blks) - r.blk0;
   return r;
 }
 
-__global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
+template <int HU>
+__global__ void __launch_bounds__(SegCfg<HU>::kThreads, 1) seg_state_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-    const float* __restrict__ dt, const float* __restrict__ A, float* __restrict__ seg_states,
-    float* __restrict__ seg_decay, int64_t seqlen, int nheads, int heads_per_group, Seg sg,
-    int units) {
+    const __grid_constant__ CUtensorMap tm_dt, int dt_tma, const float* __restrict__ dt,
+    const float* __restrict__ A, float* __restrict__ seg_states, float* __restrict__ seg_decay,
+    int64_t seqlen, int nheads, int heads_per_group, Seg sg, int units) {
+  using Cfg = SegCfg<HU>;
+  constexpr int S = Cfg::kStages;
+  constexpr int kProd = Cfg::kCompute / 32, kMma = kProd + 1, kWts = kProd + 2;  // warp roles
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ uint64_t full_bar[kSegStages], ready_bar[kSegStages], empty_bar[kSegStages];
+  __shared__ uint64_t full_bar[S], ready_bar[S], empty_bar[S];
   __shared__ uint64_t wt_full[kWtSlots], wt_empty[kWtSlots];
   __shared__ uint64_t acc_full[2], acc_empty[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ __align__(16) float wt_stage[kWtSlots][2][kBlk];  // [block % 4][head][row]
+  __shared__ __align__(16) float wt_stage[kWtSlots][HU][kBlk];  // [block % 4][head][row]
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int npair = nheads / 2;
+  const int nq = nheads / HU;
   volatile int* abort_v = &abort_flag;
-  uint32_t n_loads[kSegStages] = {0, 0, 0};  // the producer's loads per stage
+  uint32_t n_loads[S];  // the producer's loads per stage
+#pragma unroll
+  for (int i = 0; i < S; ++i) n_loads[i] = 0;
 
   if (tid == 0) {
     abort_flag = 0;
-    for (int i = 0; i < kSegStages; ++i) {
+    for (int i = 0; i < S; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&ready_bar[i], 256);
+      mbar_init(&ready_bar[i], Cfg::kCompute);
       mbar_init(&empty_bar[i], 1);
     }
     for (int i = 0; i < kWtSlots; ++i) {
       mbar_init(&wt_full[i], 32);
-      mbar_init(&wt_empty[i], 256);
+      mbar_init(&wt_empty[i], Cfg::kCompute);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 256);
+      mbar_init(&acc_empty[i], Cfg::kCompute);
     }
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_base_sh, 256);
+  if (warp == 0) tmem_alloc(&tmem_base_sh, 2 * Cfg::kAccCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 8) {
+  if (warp == kProd) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
+      if (dt_tma) prefetch_tmap(&tm_dt);
       int g = 0;
       int g_first = -1;  // block number of the current unit's first walk block
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const SegUnit su = seg_unit(u, npair, sg);
-        const int gh = (su.hp * 2) / heads_per_group;
+        const SegUnit su = seg_unit(u, nq, sg);
+        const int h0 = su.hq * HU;
+        const int gh = h0 / heads_per_group;
         for (int i = 0; i < su.nb; ++i, ++g) {  // walk block i = block blk0 + nb - 1 - i
-          const int stage = g % kSegStages;
+          const int stage = g % S;
           if (i == 0) g_first = g;
-          if (g >= kSegStages &&
-              !mbar_wait(&empty_bar[stage], ((g - kSegStages) / kSegStages) & 1, abort_v, 11)) {
+          if (g >= S && !mbar_wait(&empty_bar[stage], ((g - S) / S) & 1, abort_v, 11)) {
             ok = false;
             break;
           }
-          // this stage's x area held the low part of block g - 2 when that block was a first
-          if (g - 2 == g_first && i >= 2 &&
-              !mbar_wait(&empty_bar[(g - 2) % kSegStages], ((g - 2) / kSegStages) & 1, abort_v, 17)) {
+          // this stage's x area held the low part of block g - (S - 1) when that was a first
+          if (g - (S - 1) == g_first && i >= S - 1 &&
+              !mbar_wait(&empty_bar[(g - (S - 1)) % S], ((g - (S - 1)) / S) & 1, abort_v, 17)) {
             ok = false;
             break;
           }
           const int t0 = (su.blk0 + su.nb - 1 - i) * kBlk;
-          uint8_t* st = smem + stage * kSegStage;
+          uint8_t* st = smem + stage * Cfg::kStage;
           ++n_loads[stage];
-          mbar_arrive_expect_tx(&full_bar[stage], 4 * kTile);
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStage + (dt_tma ? Cfg::kDtBox : 0u));
+          if (dt_tma)
+            tma_load_3d(smem + Cfg::kDtOff + stage * Cfg::kDtBox, &tm_dt, &full_bar[stage],
+                        h0 & ~3, t0, su.b);
           tma_load_3d(st, &tm_b, &full_bar[stage], gh * kN, t0, su.b);
           tma_load_3d(st + kTile, &tm_b, &full_bar[stage], gh * kN + 64, t0, su.b);
-          tma_load_3d(st + 2 * kTile, &tm_x, &full_bar[stage], su.hp * 2 * kP, t0, su.b);
-          tma_load_3d(st + 3 * kTile, &tm_x, &full_bar[stage], (su.hp * 2 + 1) * kP, t0, su.b);
+#pragma unroll
+          for (int hh = 0; hh < HU; ++hh)
+            tma_load_3d(st + (2 + hh) * kTile, &tm_x, &full_bar[stage], (h0 + hh) * kP, t0, su.b);
         }
-        // a unit shorter than three blocks: the next unit's block g_first + 2 is not in this
-        // unit, so wait for the low part's MMA before any later load reuses its stage
-        if (ok && su.nb < 3 && g_first >= 0 &&
-            !mbar_wait(&empty_bar[g_first % kSegStages], (g_first / kSegStages) & 1, abort_v, 18))
+        // a unit shorter than S blocks: block g_first + S - 1 is not in this unit, so wait for
+        // the low part's MMA before any later load reuses its stage
+        if (ok && su.nb < S && g_first >= 0 &&
+            !mbar_wait(&empty_bar[g_first % S], (g_first / S) & 1, abort_v, 18))
           ok = false;
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMma) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+      const uint32_t idesc = idesc_bf16(128, HU * 64, 1, 1);
       // descriptors are built once; a K step or a tile offset adds (bytes >> 4) to the start
       // address field (every address stays below 256 KB, so the field cannot carry)
       const uint64_t d0 = sdesc(smem_u32(smem), kTile, 1024);
       int g = 0, n = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++n) {
-        const SegUnit su = seg_unit(u, npair, sg);
+        const SegUnit su = seg_unit(u, nq, sg);
         const int ab = n & 1;
-        const uint32_t acc = tmem + ab * 128;
+        const uint32_t acc = tmem + ab * Cfg::kAccCols;
         if (n >= 2 && !mbar_wait(&acc_empty[ab], ((n - 2) >> 1) & 1, abort_v, 19)) break;
         for (int i = 0; i < su.nb; ++i, ++g) {
-          const int stage = g % kSegStages;
-          if (!mbar_wait(&ready_bar[stage], (g / kSegStages) & 1, abort_v, 12)) {
+          const int stage = g % S;
+          if (!mbar_wait(&ready_bar[stage], (g / S) & 1, abort_v, 12)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ds = d0 + uint64_t(stage) * (kSegStage >> 4);
-          // low part of a first walk block: stage (g + 2) % 3's x area
-          const uint64_t dlo = d0 + uint64_t((g + 2) % kSegStages) * (kSegStage >> 4) +
-                               ((2 * kTile) >> 4);
+          const uint64_t ds = d0 + uint64_t(stage) * (Cfg::kStage >> 4);
+          // low part of a first walk block: stage (g + S - 1) % S's x area
+          const uint64_t dlo =
+              d0 + uint64_t((g + S - 1) % S) * (Cfg::kStage >> 4) + ((2 * kTile) >> 4);
 #pragma unroll
           for (int k = 0; k < kBlk / 16; ++k) {
             const uint64_t ad = ds + k * 128;                                   // B^T: M = n
@@ -244,19 +268,19 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
         }
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == kWts) {
     // ------------------------------ weights ------------------------------
     // w_t = exp(sum_{k > t, k in segment} a_k) dt_t, a_k = dt_k A log2(e) (log2 units); the
     // walk goes from the segment's last block to its first, so `run` (the blocks after the
     // current one) is a running total.  Blocks are numbered across units like the stages.
+    // Without the dt box (HU = 2 only) lane l loads its rows itself, four blocks ahead.
     float v[kWtSlots][8];  // dt of block g in v[g % 4]: rows 4 lane + r, head h at [2r + h]
-    // the (unit, walk block) of block number g, for the four-ahead loads
-    int lu = blockIdx.x, li = 0;
+    int lu = blockIdx.x, li = 0;  // the (unit, walk block) of the next load
     auto load_next = [&](float (&w)[8]) {
       bool valid = lu < units;
       SegUnit su;
-      if (valid) su = seg_unit(lu, npair, sg);
-      const float* dtb = dt + (valid ? (int64_t(su.b) * seqlen * nheads + su.hp * 2) : 0);
+      if (valid) su = seg_unit(lu, nq, sg);
+      const float* dtb = dt + (valid ? (int64_t(su.b) * seqlen * nheads + su.hq * HU) : 0);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int64_t tok = valid ? int64_t(su.blk0 + su.nb - 1 - li) * kBlk + 4 * lane + r : 0;
@@ -269,15 +293,21 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
         lu += gridDim.x;
       }
     };
+    if (!dt_tma) {
 #pragma unroll
-    for (int s = 0; s < kWtSlots; ++s) load_next(v[s]);
+      for (int s = 0; s < kWtSlots; ++s) load_next(v[s]);
+    }
     int g = 0;
     bool wok = true;
     for (int u = blockIdx.x; u < units && wok; u += gridDim.x) {
-      const SegUnit su = seg_unit(u, npair, sg);
-      const int h0 = su.hp * 2;
-      const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
-      float run[2] = {0.f, 0.f};
+      const SegUnit su = seg_unit(u, nq, sg);
+      const int h0 = su.hq * HU;
+      float al[HU], run[HU];
+#pragma unroll
+      for (int h = 0; h < HU; ++h) {
+        al[h] = A[h0 + h] * kLog2e;
+        run[h] = 0.f;
+      }
       for (int i = 0; i < su.nb && wok; ++i, ++g) {
         const int slot = g % kWtSlots;
         // (warp-uniform decisions: every lane reaches the same __syncwarp)
@@ -287,58 +317,87 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
           wok = false;
           break;
         }
-        float d[8];
-#pragma unroll
-        for (int s = 0; s < kWtSlots; ++s)
-          if (s == slot) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) d[e] = v[s][e];
+        float d[4][HU];  // rows 4 lane + r, heads h
+        if (dt_tma) {  // the stage's box: [128 tokens][4 heads from h0 & ~3]
+          const int stage = g % S;
+          if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[stage], (g / S) & 1, abort_v, 21))) {
+            wok = false;
+            break;
           }
+          const float* box =
+              reinterpret_cast<const float*>(smem + Cfg::kDtOff + stage * Cfg::kDtBox);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float c0 = d[h] * al[h];
-          const float c1 = fmaf(d[2 + h], al[h], c0);
-          const float c2 = fmaf(d[4 + h], al[h], c1);
-          const float c3 = fmaf(d[6 + h], al[h], c2);
+          for (int r = 0; r < 4; ++r) {
+            if (HU == 4) {
+              const float4 dd = *reinterpret_cast<const float4*>(box + (4 * lane + r) * 4);
+              d[r][0] = dd.x;
+              d[r][HU > 1 ? 1 : 0] = dd.y;
+              d[r][HU > 2 ? 2 : 0] = dd.z;
+              d[r][HU > 3 ? 3 : 0] = dd.w;
+            } else {
+              const float2 dd =
+                  *reinterpret_cast<const float2*>(box + (4 * lane + r) * 4 + (h0 & 3));
+              d[r][0] = dd.x;
+              d[r][HU > 1 ? 1 : 0] = dd.y;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int s = 0; s < kWtSlots; ++s)
+            if (s == slot) {
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                d[r][0] = v[s][2 * r];
+                d[r][HU > 1 ? 1 : 0] = v[s][2 * r + 1];
+              }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < HU; ++h) {
+          const float c0 = d[0][h] * al[h];
+          const float c1 = fmaf(d[1][h], al[h], c0);
+          const float c2 = fmaf(d[2][h], al[h], c1);
+          const float c3 = fmaf(d[3][h], al[h], c2);
           const float incl = warp_inclusive_scan(c3);
           const float off = incl - c3;
           const float tot = __shfl_sync(0xffffffffu, incl, 31);
           const float rest = tot - off + run[h];  // minus the prefix through row 4 lane - 1
           *reinterpret_cast<float4*>(&wt_stage[slot][h][4 * lane]) =
-              make_float4(ex2(rest - c0) * d[h], ex2(rest - c1) * d[2 + h],
-                          ex2(rest - c2) * d[4 + h], ex2(rest - c3) * d[6 + h]);
+              make_float4(ex2(rest - c0) * d[0][h], ex2(rest - c1) * d[1][h],
+                          ex2(rest - c2) * d[2][h], ex2(rest - c3) * d[3][h]);
           run[h] += tot;
         }
         mbar_arrive_warp(&wt_full[slot]);
+        if (!dt_tma) {
 #pragma unroll
-        for (int s = 0; s < kWtSlots; ++s)
-          if (s == slot) load_next(v[s]);  // in flight while the next blocks are processed
+          for (int s = 0; s < kWtSlots; ++s)
+            if (s == slot) load_next(v[s]);  // in flight while the next blocks are processed
+        }
       }
-      if (wok && lane < 2)
+      if (wok && lane < HU)
         seg_decay[(int64_t(su.b) * sg.nseg + su.seg) * nheads + h0 + lane] = run[lane];
     }
-  } else {
+  } else if (warp < kProd) {
     // ------------------------------ compute warps ------------------------------
     const int row = tid & 127, j = tid >> 7;
     bool ok = true;
     int g = 0, n = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
-      const SegUnit su = seg_unit(u, npair, sg);
+      const SegUnit su = seg_unit(u, nq, sg);
       for (int i = 0; i < su.nb; ++i, ++g) {
-        const int stage = g % kSegStages;
+        const int stage = g % S;
         const int slot = g % kWtSlots;
         ok = ok && mbar_wait(&wt_full[slot], (g / kWtSlots) & 1, abort_v, 16);
         const float wt = wt_stage[slot][j][row];
         mbar_arrive_warp(&wt_empty[slot]);
-        ok = ok && mbar_wait(&full_bar[stage], (g / kSegStages) & 1, abort_v, 13);
-        // a first walk block's low part overwrites stage (g + 2) % 3's x area, whose previous
-        // occupant is block g - 1: wait for its MMAs
+        ok = ok && mbar_wait(&full_bar[stage], (g / S) & 1, abort_v, 13);
+        // a first walk block's low part overwrites stage (g + S - 1) % S's x area, whose
+        // previous occupant is block g - 1: wait for its MMAs
         if (i == 0 && g >= 1)
-          ok = ok && mbar_wait(&empty_bar[(g - 1) % kSegStages], ((g - 1) / kSegStages) & 1,
-                               abort_v, 20);
+          ok = ok && mbar_wait(&empty_bar[(g - 1) % S], ((g - 1) / S) & 1, abort_v, 20);
         if (ok) {
-          uint8_t* xr = smem + stage * kSegStage + (2 + j) * kTile;
-          uint8_t* lr = smem + ((g + 2) % kSegStages) * kSegStage + (2 + j) * kTile;
+          uint8_t* xr = smem + stage * Cfg::kStage + (2 + j) * kTile;
+          uint8_t* lr = smem + ((g + S - 1) % S) * Cfg::kStage + (2 + j) * kTile;
           if (i == 0) {  // bf16 high part in place, low part in the other stage
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -371,9 +430,11 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
       ok = ok && mbar_wait(&acc_full[ab], (n >> 1) & 1, abort_v, 14);
       if (ok) {
         tc_fence_after();
-        const uint32_t lane_addr = tmem + ab * 128 + (uint32_t((warp & 3) * 32) << 16) + j * 64;
+        const uint32_t lane_addr =
+            tmem + ab * Cfg::kAccCols + (uint32_t((warp & 3) * 32) << 16) + j * 64;
         float* out = seg_states +
-                     (((int64_t(su.b) * sg.nseg + su.seg) * nheads + su.hp * 2 + j) * kP) * kN + row;
+                     (((int64_t(su.b) * sg.nseg + su.seg) * nheads + su.hq * HU + j) * kP) * kN +
+                     row;
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc) {
           uint32_t r[16];
@@ -390,18 +451,18 @@ __global__ void __launch_bounds__(kSegThreads, 1) seg_state_kernel(
   }
   // ------------------------------ teardown ------------------------------
   __syncthreads();
-  if (*abort_v && warp == 9 && lane == 0) {  // let every issued MMA land before leaving
+  if (*abort_v && warp == kMma && lane == 0) {  // let every issued MMA land before leaving
     mma_commit(&drain_bar);
     drain(&drain_bar, 0);
   }
-  if (*abort_v && warp == 8 && lane == 0) {  // and every issued copy
-    for (int i = 0; i < kSegStages; ++i)
+  if (*abort_v && warp == kProd && lane == 0) {  // and every issued copy
+    for (int i = 0; i < S; ++i)
       if (n_loads[i]) drain(&full_bar[i], (n_loads[i] - 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_free(tmem, 256);
+  if (warp == 0) tmem_free(tmem, 2 * Cfg::kAccCols);
 }
 
 // =============================================================================================

@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(kPassThreads) seg_pass_kernel(
 }
 
 // =============================================================================================
-// chunk_out: grid = batch * nseg * (nheads / 2), block = 608 threads in four roles:
+// chunk_out: grid = batch * nseg * (nheads / 2), block = 640 threads in five roles:
 //   warps 0-15  compute (512 threads).  Thread (row = tid % 128, q = tid / 128): token row
 //               `row` of a block (state row n = row in the state passes) and a quarter of the
 //               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and

@@ -163,10 +163,19 @@ bool make_dt_map(CUtensorMap* m, const float* dt, int64_t batch, int64_t seqlen,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dynamic shared-memory limits of the kernels, set once per device (the attribute applies to
+// the current device only).
 ssd_status set_smem_attrs() {
-  static ssd_status st = SSD_ERR_CUDA;
-  static std::once_flag once;
-  std::call_once(once, [] {
+  constexpr int kMaxDev = 256;
+  static std::mutex mu;
+  static signed char done[kMaxDev] = {};  // 0 not yet, 1 ok, -1 failed
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return SSD_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev] == 0) {
     bool ok = true;
     ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<float>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
@@ -184,10 +193,10 @@ ssd_status set_smem_attrs() {
                    (const void*)ssd::simt::chunk_state_kernel<__nv_bfloat16>})
       ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
             cudaSuccess;
-    st = ok ? SSD_OK : SSD_ERR_CUDA;
     if (!ok) cudaGetLastError();
-  });
-  return st;
+    done[dev] = ok ? 1 : -1;
+  }
+  return done[dev] == 1 ? SSD_OK : SSD_ERR_CUDA;
 }
 
 ssd_status launched() {

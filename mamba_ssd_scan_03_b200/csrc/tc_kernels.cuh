@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(SegCfg<HU>::kThreads, 1) seg_state_kernel(
 // Segments are taken eight at a time so that eight loads are in flight per thread.
 // =============================================================================================
 constexpr int kPassThreads = 256;
-__global__ void __launch_bounds__(kPassThreads) seg_pass_kernel(
+__global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
     float* __restrict__ seg_states, const float* __restrict__ seg_decay,
     const float* init_state, float* final_state, int batch, int nheads, int nseg) {
   constexpr int kVec = kP * kN / 4;  // float4 per (batch, head) state

@@ -174,6 +174,48 @@ ssd_status ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, const floa
 const char* ssd_status_string(ssd_status s);
 
 /*
+ * Summary of a slice of the sequence: the state after its last token and its total log-decay,
+ * without y.  Sequence-sliced (multi-GPU) long context: each rank summarises its own slice from
+ * a zero state, the summaries are exchanged, ssd_state_pass gives every slice its entering state,
+ * and each rank runs ssd_chunk_scan_fwd on its slice from that state.  A slice's steps compose
+ * like a single step, h_out = exp(total_decay) h_in + S ("State Space Model", "Un sistema che
+ * riassume il passato": steps fuse pairwise by associativity); only these boundary summaries
+ * cross between devices ("Architektury Mamba-2, State Space Models i liniowa atencja" of the
+ * tech.tersel.eu article, "Wyzwania uczenia rozproszonego").
+ *
+ *   x, dt, A, B       : as for ssd_chunk_scan_fwd (the slice's tokens).
+ *   init_state        : state before the slice's first token, NULL = zeros.
+ *   final_state       : output [batch, nheads, headdim, dstate] float32 (required); may equal
+ *                       init_state.
+ *   total_decay       : output [batch, nheads] float32, sum over the slice of dt[b,t,h]*A[h]
+ *                       (natural log; the slice decays a state by exp(total_decay)).
+ *   workspace         : ssd_chunk_scan_workspace_size() bytes for the same shape and chunk.
+ * Same shapes, paths, errors and asynchrony as ssd_chunk_scan_fwd.
+ */
+ssd_status ssd_chunk_state_fwd(const void* x, const float* dt, const float* A, const void* B,
+                               const float* init_state, float* final_state, float* total_decay,
+                               int64_t batch, int64_t seqlen, int nheads, int headdim,
+                               int dstate, int ngroups, int chunk, ssd_dtype io,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * The state passing between slices: an exclusive scan over slice summaries.
+ *   states            : [nslices, batch, nheads, headdim, dstate] float32, in place.  In: each
+ *                       slice's state from a zero start (ssd_chunk_state_fwd with init NULL).
+ *                       Out: the state entering each slice, H_in(0) = init_state,
+ *                       H_in(r+1) = exp(decay[r]) * H_in(r) + S(r).
+ *   decay             : [nslices, batch, nheads] float32, each slice's total_decay.
+ *   init_state        : [batch, nheads, headdim, dstate] float32 before slice 0, NULL = zeros.
+ *   final_state       : output, the state after the last slice (NULL = not written); may equal
+ *                       init_state, must not overlap `states`.
+ * Any headdim and dstate.  Asynchronous on `stream`; argument errors are returned before any
+ * launch.
+ */
+ssd_status ssd_state_pass(float* states, const float* decay, const float* init_state,
+                          float* final_state, int64_t nslices, int64_t batch, int nheads,
+                          int headdim, int dstate, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that kernels latch
  * when a bounded wait expires (for the current device).  Returns SSD_OK,
  * SSD_ERR_DEVICE_TIMEOUT, or SSD_ERR_CUDA if the synchronisation itself failed.

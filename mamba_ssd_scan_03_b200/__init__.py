@@ -24,8 +24,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 # The symbols include/ssd.h declares (tests check that the library exports each one).
 EXPORTS = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path", "ssd_chunk_scan_fwd",
            "ssd_chunk_scan_simt_workspace_size", "ssd_chunk_scan_fwd_simt", "ssd_step",
-           "ssd_chunk_scan_fwd_noalloc", "ssd_status_string", "ssd_get_device_status",
-           "ssd_version")
+           "ssd_chunk_scan_fwd_noalloc", "ssd_chunk_state_fwd", "ssd_state_pass",
+           "ssd_status_string", "ssd_get_device_status", "ssd_version")
 
 # Size of the fixed device array ssd_chunk_scan_fwd_noalloc uses instead of a workspace.
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -64,6 +64,10 @@ def load():
         fn.argtypes = _SCAN
     lib.ssd_chunk_scan_fwd_noalloc.restype = _i32
     lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 9 + [_i64, _i64] + [_i32] * 7 + [_vp]
+    lib.ssd_chunk_state_fwd.restype = _i32
+    lib.ssd_chunk_state_fwd.argtypes = [_vp] * 7 + [_i64, _i64] + [_i32] * 6 + [_vp, _sz, _vp]
+    lib.ssd_state_pass.restype = _i32
+    lib.ssd_state_pass.argtypes = [_vp] * 4 + [_i64, _i64, _i32, _i32, _i32, _vp]
     lib.ssd_step.restype = _i32
     lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
@@ -223,6 +227,55 @@ def chunk_scan_fwd_noalloc(x, dt, A, B, C, D, chunk, init_state=None, want_final
             _ptr(fin), Bt, L, H, P, N, G, Q, io, _code(y_dtype), _stream(dev))
     _check(rc, "ssd_chunk_scan_fwd_noalloc")
     return y, fin
+
+
+def chunk_state_fwd(x, dt, A, B, chunk, init_state=None, workspace=None, final_out=None):
+    """Summary of a slice of the sequence: (final_state [B,H,P,N] f32, total_decay [B,H] f32 =
+    sum_t dt*A) from init_state (None = zeros), without y."""
+    lib = load()
+    _need(x, "x")
+    dev = x.device
+    Bt, L, H, P, N, G, Q, io = _scan_shape(x, B, chunk)
+    _need(B, "B", x.dtype, (Bt, L, G, N), dev)
+    _need(dt, "dt", torch.float32, (Bt, L, H), dev)
+    _need(A, "A", torch.float32, (H,), dev)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (Bt, H, P, N), dev)
+    fin = final_out if final_out is not None else torch.empty(
+        (Bt, H, P, N), dtype=torch.float32, device=dev)
+    _need(fin, "final_state", torch.float32, (Bt, H, P, N), dev)
+    dec = torch.empty((Bt, H), dtype=torch.float32, device=dev)
+    need = workspace_size(Bt, L, H, P, N, G, Q, io)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_chunk_state_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init_state),
+                                     _ptr(fin), _ptr(dec), Bt, L, H, P, N, G, Q, io,
+                                     _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(rc, "ssd_chunk_state_fwd")
+    return fin, dec
+
+
+def state_pass(states, decay, init_state=None, final_out=None):
+    """Exclusive scan over slice summaries.  states [R,B,H,P,N] f32 (each slice's state from a
+    zero start) becomes, in place, the state entering each slice; decay [R,B,H] f32.  Returns
+    the state after the last slice."""
+    lib = load()
+    _need(states, "states", torch.float32)
+    dev = states.device
+    R, Bt, H, P, N = states.shape
+    _need(decay, "decay", torch.float32, (R, Bt, H), dev)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (Bt, H, P, N), dev)
+    fin = final_out if final_out is not None else torch.empty(
+        (Bt, H, P, N), dtype=torch.float32, device=dev)
+    _need(fin, "final_state", torch.float32, (Bt, H, P, N), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_state_pass(_ptr(states), _ptr(decay), _ptr(init_state), _ptr(fin), R, Bt,
+                                H, P, N, _stream(dev))
+    _check(rc, "ssd_state_pass")
+    return fin
 
 
 def step(state, x, dt, A, B, C, D, out=None, y_dtype=torch.float32):

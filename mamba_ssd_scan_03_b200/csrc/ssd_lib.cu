@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "pass_kernels.cuh"
 #include "simt_kernels.cuh"
 #include "ssd_common.cuh"
 #include "step_kernels.cuh"
@@ -249,7 +250,7 @@ ssd_status validate_scan(const Shape& s, const ScanArgs& a, size_t need) {
 }
 
 template <typename T, typename TY>
-ssd_status run_simt(const Shape& s, const ScanArgs& a) {
+ssd_status run_simt(const Shape& s, const ScanArgs& a, bool with_output = true) {
   const int64_t nchunks = (s.seqlen + s.chunk - 1) / s.chunk;
   float* cs = static_cast<float*>(a.ws);
   float* states = reinterpret_cast<float*>(
@@ -268,6 +269,7 @@ ssd_status run_simt(const Shape& s, const ScanArgs& a) {
   ssd::simt::state_pass_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
       states, cs, a.init, a.fin, s.batch, s.nheads, s.headdim, s.dstate, s.chunk, int(nchunks));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  if (!with_output) return SSD_OK;
   const size_t sm_out = (3072 + 64 * size_t(s.headdim)) * sizeof(float);
   ssd::simt::chunk_out_kernel<T, TY><<<grid, 256, sm_out, a.stream>>>(
       static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), static_cast<const T*>(a.C),
@@ -276,13 +278,16 @@ ssd_status run_simt(const Shape& s, const ScanArgs& a) {
   return launched();
 }
 
-ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, void* scratch) {
+// with_output = false: the states only (seg_state and seg_pass), for ssd_chunk_state_fwd
+ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, void* scratch,
+                           bool with_output = true) {
   const SegScratch w = seg_scratch(s, sg, scratch);
   CUtensorMap mx, mb, mc, my;
   const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
-  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch) ||
-      !make_map(&mc, a.C, GN, s.seqlen, s.batch) ||
-      !make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32))
+  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch))
+    return SSD_ERR_CUDA;
+  if (with_output && (!make_map(&mc, a.C, GN, s.seqlen, s.batch) ||
+                      !make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32)))
     return SSD_ERR_CUDA;
   const int hpg = s.nheads / s.ngroups;
   const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
@@ -305,6 +310,7 @@ ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, voi
                              ssd::tc::kPassThreads, 0, a.stream>>>(
       w.states, w.decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  if (!with_output) return SSD_OK;
   if (a.ydt == SSD_F32)
     ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
         mx, mb, mc, my, a.dt, a.A, a.D, w.states, s.seqlen, s.nheads, hpg, sg);
@@ -326,6 +332,34 @@ ssd_status run_simt_any(const Shape& s, const ScanArgs& a) {
 
 bool tc_pointers_ok(const ScanArgs& a) {
   return aligned16(a.x) && aligned16(a.B) && aligned16(a.C) && aligned16(a.y);
+}
+
+ssd_status validate_state(const Shape& s, const ScanArgs& a, float* total_decay, size_t need) {
+  for (const void* p : {a.x, (const void*)a.dt, (const void*)a.A, a.B, (const void*)a.fin,
+                        (const void*)total_decay})
+    if (!is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  if (a.init && !is_device_ptr(a.init)) return SSD_ERR_INVALID_ARG;
+  const size_t es = s.io == SSD_BF16 ? 2 : 4;
+  const size_t nx = size_t(s.batch) * s.seqlen * s.nheads * s.headdim * es;
+  const size_t nbc = size_t(s.batch) * s.seqlen * s.ngroups * s.dstate * es;
+  const size_t ndt = size_t(s.batch) * s.seqlen * s.nheads * 4;
+  const size_t nst = size_t(s.batch) * s.nheads * s.headdim * s.dstate * 4;
+  const size_t nd = size_t(s.batch) * s.nheads * 4;
+  if ((a.fin != a.init && overlaps(a.fin, nst, a.init, nst)) || overlaps(a.fin, nst, a.x, nx) ||
+      overlaps(a.fin, nst, a.B, nbc) || overlaps(a.fin, nst, a.dt, ndt) ||
+      overlaps(total_decay, nd, a.fin, nst) || overlaps(total_decay, nd, a.dt, ndt) ||
+      overlaps(total_decay, nd, a.x, nx) || overlaps(total_decay, nd, a.B, nbc) ||
+      overlaps(total_decay, nd, a.init, nst))
+    return SSD_ERR_INVALID_ARG;
+  if (need > 0) {
+    if (!a.ws || a.ws_bytes < need || (reinterpret_cast<uintptr_t>(a.ws) & 255u) ||
+        !is_device_ptr(a.ws))
+      return SSD_ERR_WORKSPACE;
+    if (overlaps(a.ws, need, a.x, nx) || overlaps(a.ws, need, a.init, nst) ||
+        overlaps(a.ws, need, a.fin, nst) || overlaps(a.ws, need, total_decay, nd))
+      return SSD_ERR_INVALID_ARG;
+  }
+  return SSD_OK;
 }
 
 }  // namespace
@@ -464,6 +498,54 @@ const char* ssd_status_string(ssd_status s) {
     case SSD_ERR_DEVICE_TIMEOUT: return "SSD_ERR_DEVICE_TIMEOUT: a kernel's bounded wait expired";
   }
   return "unknown ssd_status";
+}
+
+ssd_status ssd_chunk_state_fwd(const void* x, const float* dt, const float* A, const void* B,
+                               const float* init_state, float* final_state, float* total_decay,
+                               int64_t batch, int64_t seqlen, int nheads, int headdim,
+                               int dstate, int ngroups, int chunk, ssd_dtype io,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  const ScanArgs a{SSD_F32, x, B, nullptr, dt, A, nullptr, init_state, nullptr, final_state,
+                   workspace, workspace_bytes, stream};
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  const bool tc = tc_shape_ok(s);
+  if (!tc && !simt_supported(s)) return SSD_ERR_UNSUPPORTED;
+  st = validate_state(s, a, total_decay, tc ? tc_workspace(s) : simt_workspace(s));
+  if (st != SSD_OK) return st;
+  if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
+  if (tc) {
+    if (!aligned16(x) || !aligned16(B)) return SSD_ERR_UNSUPPORTED;
+    st = run_tc_segments(s, a, tc_segments(s), a.ws, false);
+  } else {
+    st = s.io == SSD_F32 ? run_simt<float, float>(s, a, false)
+                         : run_simt<__nv_bfloat16, float>(s, a, false);
+  }
+  if (st != SSD_OK) return st;
+  const dim3 grid(unsigned(batch), unsigned((nheads + 31) / 32));
+  ssd::pass::decay_sum_kernel<<<grid, 256, 0, stream>>>(dt, A, total_decay, seqlen, nheads);
+  return launched();
+}
+
+ssd_status ssd_state_pass(float* states, const float* decay, const float* init_state,
+                          float* final_state, int64_t nslices, int64_t batch, int nheads,
+                          int headdim, int dstate, cudaStream_t stream) {
+  if (nslices < 1 || batch < 1 || nheads < 1 || headdim < 1 || dstate < 1)
+    return SSD_ERR_INVALID_ARG;
+  if (!is_device_ptr(states) || !is_device_ptr(decay)) return SSD_ERR_INVALID_ARG;
+  if ((init_state && !is_device_ptr(init_state)) || (final_state && !is_device_ptr(final_state)))
+    return SSD_ERR_INVALID_ARG;
+  const int64_t nbh = batch * nheads, per_bh = int64_t(headdim) * dstate;
+  const size_t nst = size_t(nbh * per_bh) * 4;
+  if (overlaps(final_state, nst, states, nst * size_t(nslices)) ||
+      overlaps(decay, size_t(nslices * nbh) * 4, states, nst * size_t(nslices)) ||
+      (final_state != init_state && overlaps(final_state, nst, init_state, nst)))
+    return SSD_ERR_INVALID_ARG;
+  const int64_t n = nbh * per_bh;
+  ssd::pass::slice_pass_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(
+      states, decay, init_state, final_state, nslices, nbh, per_bh);
+  return launched();
 }
 
 ssd_status ssd_get_device_status(cudaStream_t stream) {

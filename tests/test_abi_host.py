@@ -98,3 +98,30 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises((ValueError, RuntimeError)):
         ssd.chunk_scan_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 128),
                            torch.zeros(1, 4, 1, 128), None, 256)
+
+
+def test_state_entry_points_reject_bad_arguments_on_host(lib):
+    # ssd_chunk_state_fwd(x, dt, A, B, init, final, total_decay, batch, seqlen, nheads, headdim,
+    #                     dstate, ngroups, chunk, io, workspace, bytes, stream)
+    shape = [2, 300, 4, 64, 128, 1, 256, 1]
+    assert lib.ssd_chunk_state_fwd(*([None] * 7), *shape, None, 0, None) == 1  # NULL pointers
+    bad = list(shape)
+    bad[6] = 100  # chunk
+    assert lib.ssd_chunk_state_fwd(*([None] * 7), *bad, None, 0, None) == 1
+    bad = list(shape)
+    bad[2], bad[5] = 3, 2  # 3 heads in 2 groups
+    assert lib.ssd_chunk_state_fwd(*([None] * 7), *bad, None, 0, None) == 1
+    # ssd_state_pass(states, decay, init, final, nslices, batch, nheads, headdim, dstate, stream)
+    assert lib.ssd_state_pass(None, None, None, None, 0, 2, 4, 64, 128, None) == 1
+    assert lib.ssd_state_pass(None, None, None, None, 3, 2, 4, 64, 128, None) == 1
+    assert lib.ssd_state_pass(None, None, None, None, 3, 2, 0, 64, 128, None) == 1
+
+
+def test_sliced_scan_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.chunk_state_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 128),
+                            256)
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.state_pass(torch.zeros(2, 1, 2, 64, 128), torch.zeros(2, 1, 2))

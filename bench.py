@@ -20,6 +20,10 @@ x 8192 tokens), and reports the same metric.
 
 --profile scan|decode runs only W + K calls of that workload and prints nothing else: the
 command the launch lists and ncu captures under profiles/ were taken with.
+
+--glue times the block steps around the layer at the 2.7B shape (short convolution + SiLU over
+the 5376 x/B/C channels, dt softplus, SiLU output gate over y) and prints one JSON line with
+each kernel's HBM bytes, time and bandwidth against the measured copy peak.
 """
 import argparse
 import json
@@ -430,6 +434,55 @@ def run_profile(args):
     assert ssd.device_status() == 0
 
 
+def run_glue(args):
+    """CUDA-event timing of the three block-step kernels (inputs seeded on the device)."""
+    import torch
+    import mamba_ssd_scan_03_b200 as ssd
+    dev = torch.device("cuda", 0)
+    c = ssd_inputs.resolve(SCAN_CFG)
+    Bt, L, H, P, G, N = (c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["ngroups"],
+                         c["dstate"])
+    cdim, K = H * P + 2 * G * N, 4
+    gen = torch.Generator(device=dev).manual_seed(2002)
+    rnd = lambda *shape, dtype=torch.float32: torch.randn(*shape, generator=gen, device=dev,
+                                                          dtype=dtype)
+    u = rnd(Bt, L, cdim, dtype=torch.bfloat16)
+    w, cb = rnd(cdim, K) / 2, rnd(cdim) / 10
+    conv_out = torch.empty_like(u)
+    raw, dtb = rnd(Bt, L, H), rnd(H) - 4
+    dt = torch.empty_like(raw)
+    y, z = rnd(Bt, L, H, P), rnd(Bt, L, H, P, dtype=torch.bfloat16)
+    gate_out = torch.empty_like(z)
+    ntok = Bt * L
+    cases = {
+        "conv_silu": (lambda: ssd.conv_silu(u, w, cb, out=conv_out), ntok * cdim * 4 + cdim * 20,
+                      f"[{Bt},{L},{cdim}] bf16, width {K}"),
+        "dt_softplus": (lambda: ssd.dt_softplus(raw, dtb, out=dt), ntok * H * 8 + H * 4,
+                        f"[{Bt},{L},{H}] f32"),
+        "gate_silu": (lambda: ssd.gate_silu(y, z, out=gate_out), ntok * H * P * 8,
+                      f"[{Bt},{L},{H},{P}] y f32, z and out bf16"),
+    }
+    hbm, _, src = peaks()
+    res = {}
+    for name, (fn, nbytes, shape) in cases.items():
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"shape": shape, "bytes": nbytes, "ms": round(ms, 5),
+                     "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4)}
+    assert ssd.device_status() == 0
+    print(json.dumps({"glue": res, "peak_hbm_gbs": hbm, "peak_src": src,
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,12 +495,15 @@ def main():
                     help="ncu dram bytes per scan call (null when not measured)")
     ap.add_argument("--decode-traffic", type=float, default=None)
     ap.add_argument("--profile", choices=["scan", "decode"], default=None)
+    ap.add_argument("--glue", action="store_true")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="with --profile scan: a shorter sequence (smaller capture)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.profile:
+    if args.glue:
+        run_glue(args)
+    elif args.profile:
         run_profile(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -216,6 +216,38 @@ ssd_status ssd_state_pass(float* states, const float* decay, const float* init_s
                           int headdim, int dstate, cudaStream_t stream);
 
 /*
+ * Steps either side of the layer inside a Mamba block ("Puntata 205 -- State Space Models e
+ * Mamba" (aiperbabbani.it), "Da S4 a Mamba": every Mamba block wraps the selective SSM with a
+ * short convolution and a SiLU gate).  silu(v) = v / (1 + exp(-v)).  Float32 arithmetic,
+ * outputs rounded to nearest even in their dtype; asynchronous on `stream`; argument errors are
+ * returned before any launch.
+ *
+ * ssd_conv_silu: the short causal depthwise convolution with SiLU, applied to the layer's
+ *   inputs (x, and B, C where they come from the same projection):
+ *     out[b,t,c] = silu(bias[c] + sum_{k<kwidth} w[c,k] * u[b, t-kwidth+1+k, c]),
+ *   u taken as 0 before t = 0 (no history).
+ *   u, out : [batch, seqlen, cdim] in `io` (SSD_BF16 or SSD_F32), must not overlap; w
+ *   [cdim, kwidth] float32, kwidth 1..8; bias [cdim] float32 or NULL.  cdim a multiple of 8
+ *   (bf16) or 4 (f32) and u, out 16-byte aligned, else SSD_ERR_UNSUPPORTED.
+ */
+ssd_status ssd_conv_silu(const void* u, const float* w, const float* bias, void* out,
+                         int64_t batch, int64_t seqlen, int cdim, int kwidth, ssd_dtype io,
+                         cudaStream_t stream);
+
+/* ssd_dt_softplus: the positive step size dt[b,t,h] = softplus(raw[b,t,h] + bias[h]),
+ *   softplus(v) = log(1 + exp(v)).  raw, dt [batch, seqlen, nheads] float32 (dt may equal raw);
+ *   bias [nheads] float32 or NULL. */
+ssd_status ssd_dt_softplus(const float* raw, const float* bias, float* dt, int64_t batch,
+                           int64_t seqlen, int nheads, cudaStream_t stream);
+
+/* ssd_gate_silu: the output gate out[i] = y[i] * silu(z[i]) over n elements (y as the layer
+ *   writes it, [batch, seqlen, nheads, headdim]).  y float32; z in z_dtype (SSD_BF16 or SSD_F32);
+ *   out in out_dtype (SSD_F32 or z_dtype; out may equal y when float32).  n a multiple of 8
+ *   (bf16 z) or 4 (f32 z) and all pointers 16-byte aligned, else SSD_ERR_UNSUPPORTED. */
+ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ssd_dtype z_dtype,
+                         ssd_dtype out_dtype, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that kernels latch
  * when a bounded wait expires (for the current device).  Returns SSD_OK,
  * SSD_ERR_DEVICE_TIMEOUT, or SSD_ERR_CUDA if the synchronisation itself failed.

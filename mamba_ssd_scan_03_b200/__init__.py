@@ -25,7 +25,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 EXPORTS = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path", "ssd_chunk_scan_fwd",
            "ssd_chunk_scan_simt_workspace_size", "ssd_chunk_scan_fwd_simt", "ssd_step",
            "ssd_chunk_scan_fwd_noalloc", "ssd_chunk_state_fwd", "ssd_state_pass",
-           "ssd_status_string", "ssd_get_device_status", "ssd_version")
+           "ssd_conv_silu", "ssd_dt_softplus", "ssd_gate_silu", "ssd_status_string",
+           "ssd_get_device_status", "ssd_version")
 
 # Size of the fixed device array ssd_chunk_scan_fwd_noalloc uses instead of a workspace.
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -68,6 +69,12 @@ def load():
     lib.ssd_chunk_state_fwd.argtypes = [_vp] * 7 + [_i64, _i64] + [_i32] * 6 + [_vp, _sz, _vp]
     lib.ssd_state_pass.restype = _i32
     lib.ssd_state_pass.argtypes = [_vp] * 4 + [_i64, _i64, _i32, _i32, _i32, _vp]
+    lib.ssd_conv_silu.restype = _i32
+    lib.ssd_conv_silu.argtypes = [_vp] * 4 + [_i64, _i64, _i32, _i32, _i32, _vp]
+    lib.ssd_dt_softplus.restype = _i32
+    lib.ssd_dt_softplus.argtypes = [_vp] * 3 + [_i64, _i64, _i32, _vp]
+    lib.ssd_gate_silu.restype = _i32
+    lib.ssd_gate_silu.argtypes = [_vp] * 3 + [_i64, _i32, _i32, _vp]
     lib.ssd_step.restype = _i32
     lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
@@ -276,6 +283,59 @@ def state_pass(states, decay, init_state=None, final_out=None):
                                 H, P, N, _stream(dev))
     _check(rc, "ssd_state_pass")
     return fin
+
+
+def conv_silu(u, w, bias=None, out=None):
+    """Short causal depthwise convolution + SiLU: u [B,L,C] (bf16 or f32), w [C,K] f32,
+    bias [C] f32 or None -> out [B,L,C] in u's dtype."""
+    lib = load()
+    _need(u, "u")
+    dev = u.device
+    Bt, L, Cd = u.shape
+    K = w.shape[1]
+    _need(w, "w", torch.float32, (Cd, K), dev)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (Cd,), dev)
+    out = torch.empty_like(u) if out is None else out
+    _need(out, "out", u.dtype, u.shape, dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_conv_silu(_ptr(u), _ptr(w), _ptr(bias), _ptr(out), Bt, L, Cd, K, _io(u),
+                               _stream(dev))
+    _check(rc, "ssd_conv_silu")
+    return out
+
+
+def dt_softplus(raw, bias=None, out=None):
+    """dt = softplus(raw + bias): raw [B,L,H] f32, bias [H] f32 or None -> dt [B,L,H] f32."""
+    lib = load()
+    _need(raw, "raw", torch.float32)
+    dev = raw.device
+    Bt, L, H = raw.shape
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (H,), dev)
+    out = torch.empty_like(raw) if out is None else out
+    _need(out, "out", torch.float32, raw.shape, dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_dt_softplus(_ptr(raw), _ptr(bias), _ptr(out), Bt, L, H, _stream(dev))
+    _check(rc, "ssd_dt_softplus")
+    return out
+
+
+def gate_silu(y, z, out=None, out_dtype=torch.float32):
+    """Output gate y * silu(z): y f32, z (bf16 or f32) of the same shape -> out (f32 or z's
+    dtype)."""
+    lib = load()
+    _need(y, "y", torch.float32)
+    dev = y.device
+    _need(z, "z", None, y.shape, dev)
+    out_dtype = out.dtype if out is not None else out_dtype
+    out = torch.empty(y.shape, dtype=out_dtype, device=dev) if out is None else out
+    _need(out, "out", out_dtype, y.shape, dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_gate_silu(_ptr(y), _ptr(z), _ptr(out), y.numel(), _io(z), _code(out_dtype),
+                               _stream(dev))
+    _check(rc, "ssd_gate_silu")
+    return out
 
 
 def step(state, x, dt, A, B, C, D, out=None, y_dtype=torch.float32):

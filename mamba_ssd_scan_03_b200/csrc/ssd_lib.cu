@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "glue_kernels.cuh"
 #include "pass_kernels.cuh"
 #include "simt_kernels.cuh"
 #include "ssd_common.cuh"
@@ -545,6 +546,79 @@ ssd_status ssd_state_pass(float* states, const float* decay, const float* init_s
   const int64_t n = nbh * per_bh;
   ssd::pass::slice_pass_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(
       states, decay, init_state, final_state, nslices, nbh, per_bh);
+  return launched();
+}
+
+ssd_status ssd_conv_silu(const void* u, const float* w, const float* bias, void* out,
+                         int64_t batch, int64_t seqlen, int cdim, int kwidth, ssd_dtype io,
+                         cudaStream_t stream) {
+  if (batch < 1 || seqlen < 1 || cdim < 1 || kwidth < 1 || kwidth > 8 ||
+      (io != SSD_F32 && io != SSD_BF16))
+    return SSD_ERR_INVALID_ARG;
+  if (!is_device_ptr(u) || !is_device_ptr(w) || !is_device_ptr(out) ||
+      (bias && !is_device_ptr(bias)))
+    return SSD_ERR_INVALID_ARG;
+  const size_t es = io == SSD_BF16 ? 2 : 4;
+  const int64_t ntok = batch * seqlen;
+  const size_t nb = size_t(ntok) * cdim * es;
+  if (overlaps(out, nb, u, nb) || overlaps(out, nb, w, size_t(cdim) * kwidth * 4) ||
+      overlaps(out, nb, bias, size_t(cdim) * 4))
+    return SSD_ERR_INVALID_ARG;
+  const int vw = io == SSD_BF16 ? 8 : 4;
+  if (cdim % vw != 0 || !aligned16(u) || !aligned16(out)) return SSD_ERR_UNSUPPORTED;
+  const int64_t nthr = ntok * (cdim / vw);
+  if ((nthr + 255) / 256 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+  const unsigned grid = unsigned((nthr + 255) / 256);
+  if (io == SSD_BF16)
+    ssd::glue::conv_silu_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(u), w, bias, static_cast<__nv_bfloat16*>(out), seqlen,
+        ntok, cdim, kwidth);
+  else
+    ssd::glue::conv_silu_kernel<float><<<grid, 256, 0, stream>>>(
+        static_cast<const float*>(u), w, bias, static_cast<float*>(out), seqlen, ntok, cdim,
+        kwidth);
+  return launched();
+}
+
+ssd_status ssd_dt_softplus(const float* raw, const float* bias, float* dt, int64_t batch,
+                           int64_t seqlen, int nheads, cudaStream_t stream) {
+  if (batch < 1 || seqlen < 1 || nheads < 1) return SSD_ERR_INVALID_ARG;
+  if (!is_device_ptr(raw) || !is_device_ptr(dt) || (bias && !is_device_ptr(bias)))
+    return SSD_ERR_INVALID_ARG;
+  const int64_t n = batch * seqlen * nheads;
+  if (dt != raw && overlaps(dt, size_t(n) * 4, raw, size_t(n) * 4)) return SSD_ERR_INVALID_ARG;
+  if (overlaps(dt, size_t(n) * 4, bias, size_t(nheads) * 4)) return SSD_ERR_INVALID_ARG;
+  if ((n + 255) / 256 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+  ssd::glue::dt_softplus_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(raw, bias, dt, n,
+                                                                               nheads);
+  return launched();
+}
+
+ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ssd_dtype z_dtype,
+                         ssd_dtype out_dtype, cudaStream_t stream) {
+  if (n < 1 || (z_dtype != SSD_F32 && z_dtype != SSD_BF16) ||
+      (out_dtype != SSD_F32 && out_dtype != z_dtype))
+    return SSD_ERR_INVALID_ARG;
+  if (!is_device_ptr(y) || !is_device_ptr(z) || !is_device_ptr(out)) return SSD_ERR_INVALID_ARG;
+  const size_t nz = size_t(n) * (z_dtype == SSD_BF16 ? 2 : 4);
+  const size_t no = size_t(n) * (out_dtype == SSD_BF16 ? 2 : 4);
+  if ((out != static_cast<const void*>(y) && overlaps(out, no, y, size_t(n) * 4)) ||
+      overlaps(out, no, z, nz))
+    return SSD_ERR_INVALID_ARG;
+  const int vw = z_dtype == SSD_BF16 ? 8 : 4;
+  if (n % vw != 0 || !aligned16(y) || !aligned16(z) || !aligned16(out) ||
+      (n / vw + 255) / 256 > INT32_MAX)
+    return SSD_ERR_UNSUPPORTED;
+  const unsigned grid = unsigned((n / vw + 255) / 256);
+  if (z_dtype == SSD_F32)
+    ssd::glue::gate_silu_kernel<float, float><<<grid, 256, 0, stream>>>(
+        y, static_cast<const float*>(z), static_cast<float*>(out), n);
+  else if (out_dtype == SSD_F32)
+    ssd::glue::gate_silu_kernel<__nv_bfloat16, float><<<grid, 256, 0, stream>>>(
+        y, static_cast<const __nv_bfloat16*>(z), static_cast<float*>(out), n);
+  else
+    ssd::glue::gate_silu_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, stream>>>(
+        y, static_cast<const __nv_bfloat16*>(z), static_cast<__nv_bfloat16*>(out), n);
   return launched();
 }
 

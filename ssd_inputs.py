@@ -143,3 +143,26 @@ def decode_step_inputs(dec, k):
     B = _store(gen.standard_normal((Bt, G, N)) / math.sqrt(N), io)
     C = _store(gen.standard_normal((Bt, G, N)) / math.sqrt(N), io)
     return dict(x=x, dt=dt, B=B, C=C)
+
+
+def make_glue_inputs(batch, seqlen, cdim, kwidth, nheads, headdim, io="bf16", seed=2000):
+    """Inputs of the block steps around the layer.
+
+      u ~ N(0, 1)                 [batch, seqlen, cdim]   (io dtype) convolution input
+      w ~ N(0, 1) / sqrt(kwidth)  [cdim, kwidth]          float32
+      conv_bias ~ N(0, 0.1)       [cdim]                  float32
+      raw ~ N(0, 1)               [batch, seqlen, nheads] float32 (dt projection output)
+      dt_bias ~ U(-6, -2)         [nheads]                float32
+      y ~ N(0, 1)                 [batch, seqlen, nheads, headdim] float32
+      z ~ N(0, 1)                 [batch, seqlen, nheads, headdim] (io dtype) gate branch
+    """
+    kids = np.random.SeedSequence(seed).spawn(7)
+    g = [np.random.Generator(np.random.PCG64(k)) for k in kids]
+    u = _normal_slabs(g[0], (batch, seqlen, cdim), io)
+    w = (g[1].standard_normal((cdim, kwidth)) / math.sqrt(kwidth)).astype(np.float32)
+    conv_bias = (0.1 * g[2].standard_normal(cdim)).astype(np.float32)
+    raw = _normal_slabs(g[3], (batch, seqlen, nheads), "f32")
+    dt_bias = g[4].uniform(-6.0, -2.0, size=nheads).astype(np.float32)
+    y = _normal_slabs(g[5], (batch, seqlen, nheads, headdim), "f32")
+    z = _normal_slabs(g[6], (batch, seqlen, nheads, headdim), io)
+    return dict(u=u, w=w, conv_bias=conv_bias, raw=raw, dt_bias=dt_bias, y=y, z=z, io=io)

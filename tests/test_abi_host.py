@@ -125,3 +125,26 @@ def test_sliced_scan_binding_refuses_cpu_tensors(lib):
                             256)
     with pytest.raises((ValueError, RuntimeError)):
         ssd.state_pass(torch.zeros(2, 1, 2, 64, 128), torch.zeros(2, 1, 2))
+
+
+def test_glue_entry_points_reject_bad_arguments_on_host(lib):
+    # ssd_conv_silu(u, w, bias, out, batch, seqlen, cdim, kwidth, io, stream)
+    assert lib.ssd_conv_silu(None, None, None, None, 1, 8, 64, 4, 1, None) == 1  # NULL pointers
+    assert lib.ssd_conv_silu(None, None, None, None, 1, 8, 64, 9, 1, None) == 1  # kwidth > 8
+    assert lib.ssd_conv_silu(None, None, None, None, 1, 8, 64, 4, 7, None) == 1  # dtype code
+    # ssd_dt_softplus(raw, bias, dt, batch, seqlen, nheads, stream)
+    assert lib.ssd_dt_softplus(None, None, None, 1, 8, 4, None) == 1
+    assert lib.ssd_dt_softplus(None, None, None, 1, 0, 4, None) == 1
+    # ssd_gate_silu(y, z, out, n, z_dtype, out_dtype, stream): bf16 out needs bf16 z
+    assert lib.ssd_gate_silu(None, None, None, 64, 0, 1, None) == 1
+    assert lib.ssd_gate_silu(None, None, None, 0, 1, 1, None) == 1
+
+
+def test_glue_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.conv_silu(torch.zeros(1, 4, 8, dtype=torch.bfloat16), torch.zeros(8, 4))
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.dt_softplus(torch.zeros(1, 4, 2))
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.gate_silu(torch.zeros(16), torch.zeros(16))

@@ -24,6 +24,11 @@ command the launch lists and ncu captures under profiles/ were taken with.
 --glue times the block steps around the layer at the 2.7B shape (short convolution + SiLU over
 the 5376 x/B/C channels, dt softplus, SiLU output gate over y) and prints one JSON line with
 each kernel's HBM bytes, time and bandwidth against the measured copy peak.
+
+--selective times the selective scan with a per-state transition (the first Mamba
+generation's layer) on the same x and y as the scan workload (batch 4, seqlen 8192, 5120
+channels) with 16 states per channel, and prints one JSON line: tokens/s, the ex2 rate against
+the SFU peak that bounds it, and its HBM bandwidth.
 """
 import argparse
 import json
@@ -483,6 +488,62 @@ def run_glue(args):
                       "steps": args.steps, "warmup": args.warmup}), flush=True)
 
 
+# The selective scan needs one exp per (token, channel, state) and is bound by the SFU (MUFU)
+# ex2 rate: 16 results per clock per SM (4 per SM sub-partition) x 148 SMs x the 1965 MHz
+# maximum SM clock.
+SFU_EX2_PER_CLK_SM = 16
+N_SM = 148
+SM_MAX_MHZ = 1965.0
+
+
+def run_selective(args):
+    import torch
+    import mamba_ssd_scan_03_b200 as ssd
+    dev = torch.device("cuda", 0)
+    inp = ssd_inputs.make_selective_inputs(1)
+    c = inp["cfg"]
+    Bt, L, dim, N, G = c["batch"], c["seqlen"], c["dim"], c["dstate"], c["ngroups"]
+    t = {k: to_dev(inp[k], k in ("x", "B", "C"), dev) for k in ("x", "dt", "A", "B", "C", "D")}
+    y = torch.empty((Bt, L, dim), dtype=torch.float32, device=dev)
+    fin = torch.empty((Bt, dim, N), dtype=torch.float32, device=dev)
+
+    def once():
+        ssd.selective_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], None, out=y,
+                               final_out=fin)
+
+    for _ in range(args.warmup):
+        once()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(0) as clk:
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            once()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    assert ssd.device_status() == 0
+    ntok = Bt * L
+    exps = ntok * dim * N
+    peak = SFU_EX2_PER_CLK_SM * N_SM * SM_MAX_MHZ * 1e6
+    nbytes = ntok * dim * (2 + 4 + 4) + 2 * ntok * G * N * 2 + Bt * dim * N * 4 + dim * N * 4
+    hbm, _, src = peaks()
+    out = {"metric": "selective scan tokens/s (16 states per channel)",
+           "value": round(ntok / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_call": round(ms, 4),
+           "steps": args.steps, "warmup": args.warmup, "dtype": "f32", "data": "synthetic",
+           "config": {"workload": c["name"], "batch": Bt, "seqlen": L, "dim": dim, "dstate": N,
+                      "ngroups": G, "io": c["io"], "y_dtype": "f32",
+                      "l2": "inputs larger than L2"},
+           "roofline": {"bound": "alu", "achieved": round(exps / (ms * 1e-3) / 1e12, 4),
+                        "peak": round(peak / 1e12, 4), "unit": "Tex2/s",
+                        "frac": round(exps / (ms * 1e-3) / peak, 4),
+                        "peak_src": "16 ex2/clk/SM x 148 SMs x 1965 MHz"},
+           "hbm": {"bytes": nbytes, "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                   "frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4), "peak_src": src},
+           "gpu_launches": args.steps, "clocks": clk.summary()}
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,6 +557,7 @@ def main():
     ap.add_argument("--decode-traffic", type=float, default=None)
     ap.add_argument("--profile", choices=["scan", "decode"], default=None)
     ap.add_argument("--glue", action="store_true")
+    ap.add_argument("--selective", action="store_true")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="with --profile scan: a shorter sequence (smaller capture)")
     args = ap.parse_args()
@@ -503,6 +565,8 @@ def main():
         args.warmup = 3
     if args.glue:
         run_glue(args)
+    elif args.selective:
+        run_selective(args)
     elif args.profile:
         run_profile(args)
     elif args.impl == "reference":

@@ -248,6 +248,33 @@ ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ss
                          ssd_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * ssd_selective_scan_fwd: the selective scan with a per-state (diagonal) transition -- the
+ * first Mamba generation's layer, which the SSD layer replaces ("Architektury Mamba-2, State
+ * Space Models i liniowa atencja" (tech.tersel.eu), section "Od S4 do Mamba-1: Wprowadzenie
+ * mechanizmu selektywnego": input-dependent B, C and dt, scanned on CUDA cores with the state on
+ * chip).  Per batch row b and channel d, with g = d / (dim / ngroups):
+ *     h_t[n] = exp(dt_t[d] A[d,n]) h_{t-1}[n] + dt_t[d] B_t[g,n] x_t[d]
+ *     y_t[d] = sum_n C_t[g,n] h_t[n] + D[d] x_t[d]          (h_{-1} = init_state or 0)
+ *   x            : [batch, seqlen, dim] in `io` (SSD_BF16 or SSD_F32)
+ *   dt           : [batch, seqlen, dim] float32, used as given
+ *   A            : [dim, dstate] float32 (one decay rate per channel and state)
+ *   B, C         : [batch, seqlen, ngroups, dstate] in `io`
+ *   D            : [dim] float32, or NULL for no skip term
+ *   init_state   : [batch, dim, dstate] float32, or NULL for zeros
+ *   y            : output [batch, seqlen, dim] in y_dtype (SSD_F32 or `io`)
+ *   final_state  : output [batch, dim, dstate] float32, or NULL; may equal init_state
+ * All pointers are device memory owned by the caller; y and final_state must not overlap the
+ * inputs.  Float32 arithmetic, hardware exp2 for the decays; asynchronous on `stream`.
+ * Supported: dstate == 16, dim and dim / ngroups multiples of 8, every pointer 16-byte aligned
+ * (else SSD_ERR_UNSUPPORTED).  Argument errors are returned before any launch.
+ */
+ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                  const void* C, const float* D, const float* init_state,
+                                  void* y, float* final_state, int64_t batch, int64_t seqlen,
+                                  int dim, int dstate, int ngroups, ssd_dtype io,
+                                  ssd_dtype y_dtype, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that kernels latch
  * when a bounded wait expires (for the current device).  Returns SSD_OK,
  * SSD_ERR_DEVICE_TIMEOUT, or SSD_ERR_CUDA if the synchronisation itself failed.

@@ -25,7 +25,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 EXPORTS = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path", "ssd_chunk_scan_fwd",
            "ssd_chunk_scan_simt_workspace_size", "ssd_chunk_scan_fwd_simt", "ssd_step",
            "ssd_chunk_scan_fwd_noalloc", "ssd_chunk_state_fwd", "ssd_state_pass",
-           "ssd_conv_silu", "ssd_dt_softplus", "ssd_gate_silu", "ssd_status_string",
+           "ssd_conv_silu", "ssd_dt_softplus", "ssd_gate_silu", "ssd_selective_scan_fwd",
+           "ssd_status_string",
            "ssd_get_device_status", "ssd_version")
 
 # Size of the fixed device array ssd_chunk_scan_fwd_noalloc uses instead of a workspace.
@@ -75,6 +76,9 @@ def load():
     lib.ssd_dt_softplus.argtypes = [_vp] * 3 + [_i64, _i64, _i32, _vp]
     lib.ssd_gate_silu.restype = _i32
     lib.ssd_gate_silu.argtypes = [_vp] * 3 + [_i64, _i32, _i32, _vp]
+    lib.ssd_selective_scan_fwd.restype = _i32
+    lib.ssd_selective_scan_fwd.argtypes = [_vp] * 9 + [_i64, _i64, _i32, _i32, _i32, _i32,
+                                                       _i32, _vp]
     lib.ssd_step.restype = _i32
     lib.ssd_step.argtypes = [_vp] * 8 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
@@ -336,6 +340,45 @@ def gate_silu(y, z, out=None, out_dtype=torch.float32):
                                _stream(dev))
     _check(rc, "ssd_gate_silu")
     return out
+
+
+def selective_scan_fwd(x, dt, A, B, C, D=None, init_state=None, want_final=True, out=None,
+                       y_dtype=torch.float32, final_out=None):
+    """Selective scan with a per-state transition: x [Bt,L,dim] (bf16 or f32), dt [Bt,L,dim]
+    f32, A [dim,N] f32, B, C [Bt,L,G,N] in x's dtype, D [dim] f32 or None, init_state
+    [Bt,dim,N] f32 or None -> (y [Bt,L,dim] in y_dtype, final state [Bt,dim,N] f32 or None)."""
+    lib = load()
+    _need(x, "x")
+    dev = x.device
+    Bt, L, dim = x.shape
+    _need(dt, "dt", torch.float32, (Bt, L, dim), dev)
+    _need(A, "A", torch.float32, None, dev)
+    if A.dim() != 2 or A.shape[0] != dim:
+        raise ValueError(f"A must be [dim, dstate] with dim {dim}, got {tuple(A.shape)}")
+    N = A.shape[1]
+    _need(B, "B", x.dtype, None, dev)
+    if B.dim() != 4 or tuple(B.shape[:2]) != (Bt, L) or B.shape[3] != N:
+        raise ValueError(f"B must be [{Bt},{L},G,{N}], got {tuple(B.shape)}")
+    G = B.shape[2]
+    _need(C, "C", x.dtype, B.shape, dev)
+    if D is not None:
+        _need(D, "D", torch.float32, (dim,), dev)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (Bt, dim, N), dev)
+    y_dtype = out.dtype if out is not None else y_dtype
+    y = torch.empty((Bt, L, dim), dtype=y_dtype, device=dev) if out is None else out
+    _need(y, "out", y_dtype, (Bt, L, dim), dev)
+    fin = None
+    if want_final:
+        fin = torch.empty((Bt, dim, N), dtype=torch.float32, device=dev) \
+            if final_out is None else final_out
+        _need(fin, "final_out", torch.float32, (Bt, dim, N), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_selective_scan_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                        _ptr(init_state), _ptr(y), _ptr(fin), Bt, L, dim, N, G,
+                                        _io(x), _code(y_dtype), _stream(dev))
+    _check(rc, "ssd_selective_scan_fwd")
+    return y, fin
 
 
 def step(state, x, dt, A, B, C, D, out=None, y_dtype=torch.float32):

@@ -8,9 +8,11 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "glue_kernels.cuh"
 #include "pass_kernels.cuh"
+#include "selective_kernels.cuh"
 #include "simt_kernels.cuh"
 #include "ssd_common.cuh"
 #include "step_kernels.cuh"
@@ -619,6 +621,55 @@ ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ss
   else
     ssd::glue::gate_silu_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, stream>>>(
         y, static_cast<const __nv_bfloat16*>(z), static_cast<__nv_bfloat16*>(out), n);
+  return launched();
+}
+
+ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                  const void* C, const float* D, const float* init_state,
+                                  void* y, float* final_state, int64_t batch, int64_t seqlen,
+                                  int dim, int dstate, int ngroups, ssd_dtype io,
+                                  ssd_dtype y_dtype, cudaStream_t stream) {
+  if (batch < 1 || seqlen < 1 || dim < 1 || dstate < 1 || ngroups < 1 || dim % ngroups != 0 ||
+      (io != SSD_F32 && io != SSD_BF16) || (y_dtype != SSD_F32 && y_dtype != io))
+    return SSD_ERR_INVALID_ARG;
+  for (const void* p : {x, (const void*)dt, (const void*)A, B, C, (const void*)y})
+    if (!is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)D, (const void*)init_state, (const void*)final_state})
+    if (p && !is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  const size_t es = io == SSD_BF16 ? 2 : 4;
+  const size_t ntok = size_t(batch) * size_t(seqlen);
+  const size_t nx = ntok * dim * es, ndt = ntok * dim * 4;
+  const size_t ny = ntok * dim * (y_dtype == SSD_BF16 ? 2 : 4);
+  const size_t nbc = ntok * ngroups * dstate * es;
+  const size_t nst = size_t(batch) * dim * dstate * 4;
+  for (const auto& in : {std::make_pair(x, nx), std::make_pair((const void*)dt, ndt),
+                         std::make_pair(B, nbc), std::make_pair(C, nbc),
+                         std::make_pair((const void*)init_state, nst)}) {
+    if (overlaps(y, ny, in.first, in.second)) return SSD_ERR_INVALID_ARG;
+    if (final_state && in.first != init_state && overlaps(final_state, nst, in.first, in.second))
+      return SSD_ERR_INVALID_ARG;
+  }
+  if (overlaps(y, ny, final_state, nst)) return SSD_ERR_INVALID_ARG;
+  if (final_state && init_state && final_state != init_state &&
+      overlaps(final_state, nst, init_state, nst))
+    return SSD_ERR_INVALID_ARG;
+  namespace sel = ssd::sel;
+  if (dstate != sel::kN || dim % sel::kCpw != 0 || (dim / ngroups) % sel::kCpw != 0)
+    return SSD_ERR_UNSUPPORTED;
+  for (const void* p : {x, (const void*)dt, (const void*)A, B, C, (const void*)y,
+                        (const void*)init_state, (const void*)final_state})
+    if (p && !aligned16(p)) return SSD_ERR_UNSUPPORTED;
+  const int64_t warps = batch * (dim / sel::kCpw);
+  if (warps > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+  const unsigned grid = unsigned(warps);
+#define SSD_SEL(T, TY)                                                                      \
+  sel::selective_scan_kernel<T, TY><<<grid, 32, 0, stream>>>(                               \
+      static_cast<const T*>(x), dt, A, static_cast<const T*>(B), static_cast<const T*>(C),  \
+      D, init_state, static_cast<TY*>(y), final_state, seqlen, dim, ngroups)
+  if (io == SSD_F32) SSD_SEL(float, float);
+  else if (y_dtype == SSD_F32) SSD_SEL(__nv_bfloat16, float);
+  else SSD_SEL(__nv_bfloat16, __nv_bfloat16);
+#undef SSD_SEL
   return launched();
 }
 

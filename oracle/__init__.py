@@ -15,8 +15,11 @@ Contents
 ``forms``       independent small-case forms used to pin ``scan``: the explicit masked
                 semiseparable (attention-like) matrix, brute-force products of decays,
                 the LTI convolution kernel, and closed forms of special cases.
+``glue``        float64 definitions of the block steps around the layer (short causal
+                convolution + SiLU, dt softplus, SiLU output gate).
 
-Every function is pinned by ``tests/test_oracle.py``; no function is "parity unpinned".
+Every function is pinned by ``tests/test_oracle.py`` (``glue`` by
+``tests/test_oracle_glue.py``); no function is "parity unpinned".
 """
 import ctypes
 import os

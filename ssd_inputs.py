@@ -166,3 +166,50 @@ def make_glue_inputs(batch, seqlen, cdim, kwidth, nheads, headdim, io="bf16", se
     y = _normal_slabs(g[5], (batch, seqlen, nheads, headdim), "f32")
     z = _normal_slabs(g[6], (batch, seqlen, nheads, headdim), io)
     return dict(u=u, w=w, conv_bias=conv_bias, raw=raw, dt_bias=dt_bias, y=y, z=z, io=io)
+
+
+# Selective scan with a per-state transition (the first Mamba generation): the same x and y
+# as the 2.7B-shape SSD workload (5120 = 80 x 64 channels), 16 states per channel.
+SELECTIVE_CONFIGS = [
+    dict(name="selective_small", batch=2, seqlen=300, dim=64, dstate=16, ngroups=1, io="bf16",
+         init="normal0.1"),
+    dict(name="selective_5120x16", batch=4, seqlen=8192, dim=5120, dstate=16, ngroups=1,
+         io="bf16", init="zeros"),
+]
+
+
+def make_selective_inputs(cfg, seed=None, **overrides):
+    """Inputs of one selective-scan workload (``cfg``: index into SELECTIVE_CONFIGS or a dict).
+
+      x ~ N(0, 1)                          [batch, seqlen, dim]            io dtype
+      dt = softplus(z), z ~ N(-2, 0.5)     [batch, seqlen, dim]            float32
+      A[d, n] = -exp(u), u ~ U(ln 1, ln 16), independent per (d, n)   [dim, dstate] float32
+      B, C ~ N(0, 1) / sqrt(dstate)        [batch, seqlen, ngroups, dstate] io dtype
+      D ~ N(0, 1)                          [dim]                           float32
+      init ~ N(0, 0.1) or zeros            [batch, dim, dstate]            float32
+    seed = 3000 + index unless given; SeedSequence(seed).spawn(7) children in that order.
+    """
+    idx = cfg if isinstance(cfg, int) else None
+    if isinstance(cfg, int):
+        cfg = SELECTIVE_CONFIGS[cfg]
+    cfg = dict(cfg)
+    cfg.update({k: v for k, v in overrides.items() if v is not None})
+    if seed is None:
+        seed = 3000 + (idx if idx is not None else 0)
+    g = [np.random.Generator(np.random.PCG64(k)) for k in np.random.SeedSequence(seed).spawn(7)]
+    Bt, L, dim, N, G, io = (cfg["batch"], cfg["seqlen"], cfg["dim"], cfg["dstate"],
+                            cfg["ngroups"], cfg["io"])
+    x = _normal_slabs(g[0], (Bt, L, dim), io)
+    dt = np.empty((Bt, L, dim), dtype=np.float32)
+    for b in range(Bt):
+        for t0 in range(0, L, SLAB_TOKENS):
+            t1 = min(L, t0 + SLAB_TOKENS)
+            dt[b, t0:t1] = _softplus(-2.0 + 0.5 * g[1].standard_normal((t1 - t0, dim)))
+    A = (-np.exp(g[2].uniform(0.0, math.log(16.0), size=(dim, N)))).astype(np.float32)
+    B = _normal_slabs(g[3], (Bt, L, G, N), io, scale=1.0 / math.sqrt(N))
+    C = _normal_slabs(g[4], (Bt, L, G, N), io, scale=1.0 / math.sqrt(N))
+    D = g[5].standard_normal(dim).astype(np.float32)
+    init = None
+    if cfg["init"] == "normal0.1":
+        init = (0.1 * g[6].standard_normal((Bt, dim, N))).astype(np.float32)
+    return dict(x=x, dt=dt, A=A, B=B, C=C, D=D, init=init, cfg=cfg)

@@ -148,3 +148,28 @@ def test_glue_binding_refuses_cpu_tensors(lib):
         ssd.dt_softplus(torch.zeros(1, 4, 2))
     with pytest.raises((ValueError, RuntimeError)):
         ssd.gate_silu(torch.zeros(16), torch.zeros(16))
+
+
+def test_selective_entry_point_rejects_bad_arguments_on_host(lib):
+    # ssd_selective_scan_fwd(x, dt, A, B, C, D, init, y, final, batch, seqlen, dim, dstate,
+    #                        ngroups, io, y_dtype, stream)
+    shape = [2, 64, 64, 16, 1, 1, 0]
+    assert lib.ssd_selective_scan_fwd(*([None] * 9), *shape, None) == 1  # NULL pointers
+    bad = list(shape)
+    bad[2], bad[4] = 64, 3  # 64 channels in 3 groups
+    assert lib.ssd_selective_scan_fwd(*([None] * 9), *bad, None) == 1
+    bad = list(shape)
+    bad[5], bad[6] = 0, 1  # bf16 y with f32 io
+    assert lib.ssd_selective_scan_fwd(*([None] * 9), *bad, None) == 1
+    bad = list(shape)
+    bad[1] = 0  # empty sequence
+    assert lib.ssd_selective_scan_fwd(*([None] * 9), *bad, None) == 1
+
+
+def test_selective_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 16, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.selective_scan_fwd(x, torch.zeros(1, 4, 16), torch.zeros(16, 16),
+                               torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16),
+                               torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16))

@@ -82,19 +82,20 @@ def step_bytes(c, y_bytes=4):
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per scan call (sum over its kernels)
 # and per decode step, from one ncu capture of `python bench.py --profile ...` (profiles/), with
-# the hash of the kernel sources they were taken on: reported only while the sources match.
-MEASURED_TRAFFIC = {"scan": (1621108736, "6c894c5e3a2f0ba9"),
-                    "decode": (1291106304, "6c894c5e3a2f0ba9")}
+# the hash of the device-code headers of those kernels (KERNEL_SOURCES) they were taken on:
+# reported only while those sources match.
+KERNEL_SOURCES = ("ssd_common.cuh", "tc_prims.cuh", "tc_kernels.cuh", "step_kernels.cuh")
+MEASURED_TRAFFIC = {"scan": (1633198592, "73cb014a6c26db98"),
+                    "decode": (1291061248, "73cb014a6c26db98")}
 
 
 def kernel_source_hash():
     import hashlib
     d = os.path.join(ROOT, "mamba_ssd_scan_03_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 

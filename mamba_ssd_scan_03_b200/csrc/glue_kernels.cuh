@@ -41,46 +41,106 @@ template <> struct vec<float> {
   }
 };
 
+// SiLU for the streaming kernels: the hardware exp2-based exponential and the approximate
+// divide (a few float32 ulps; v / (1 + inf) gives -0 for v below about -88).
+__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.f + __expf(-v)); }
+
 // out[b,t,c] = silu(bias[c] + sum_{k<K} w[c,k] u[b, t-K+1+k, c]), u = 0 before t = 0.
-// One thread per (b, t, group of VW channels); the K input rows it reads are shared with the
-// neighbouring tokens' threads through L1.
-template <typename T>
-__global__ void __launch_bounds__(256) conv_silu_kernel(const T* __restrict__ u,
+// One thread per (batch row, 16-byte group of channels, run of kConvTok tokens): its weights
+// and bias sit in registers, the last K-1 input rows in a register window, and each input row
+// is read once with a 16-byte load (a warp reads 32 neighbouring groups: 512 contiguous bytes).
+// The K-1 rows before the run are read again by the previous run's thread (K-1 of kConvTok).
+constexpr int kConvTok = 64;
+
+template <typename T, int K>
+__global__ void __launch_bounds__(128) conv_silu_kernel(const T* __restrict__ u,
                                                         const float* __restrict__ w,
                                                         const float* __restrict__ bias,
                                                         T* __restrict__ out, int64_t seqlen,
-                                                        int64_t ntok, int cdim, int K) {
+                                                        int cdim) {
   constexpr int VW = vec<T>::VW;
-  const int ng = cdim / VW;
-  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= ntok * ng) return;
-  const int64_t tok = i / ng;  // b * seqlen + t
-  const int c0 = int(i % ng) * VW;
-  const int64_t t = tok % seqlen;
-  float acc[VW];
+  const int cg = blockIdx.x * blockDim.x + threadIdx.x;
+  if (cg >= cdim / VW) return;
+  const int c0 = cg * VW;
+  const int64_t t0 = int64_t(blockIdx.y) * kConvTok;
+  const int64_t t1 = t0 + kConvTok < seqlen ? t0 + kConvTok : seqlen;
+  const T* ub = u + int64_t(blockIdx.z) * seqlen * cdim + c0;
+  T* ob = out + int64_t(blockIdx.z) * seqlen * cdim + c0;
+
+  float wr[VW][K], bv[VW];
+  {  // this thread's VW x K weights are contiguous: VW*K/4 float4 loads
+    const float4* w4 = reinterpret_cast<const float4*>(w + int64_t(c0) * K);
 #pragma unroll
-  for (int j = 0; j < VW; ++j) acc[j] = bias ? bias[c0 + j] : 0.f;
-  for (int k = 0; k < K; ++k) {
-    const int64_t ts = t - (K - 1) + k;
-    if (ts < 0) continue;
-    float v[VW];
-    vec<T>::load(u + (tok - (K - 1) + k) * cdim + c0, v);
+    for (int i = 0; i < VW * K / 4; ++i) {
+      const float4 v = __ldg(w4 + i);
+      const float f[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int j = 0; j < VW; ++j) acc[j] = fmaf(w[(c0 + j) * K + k], v[j], acc[j]);
+      for (int e = 0; e < 4; ++e) wr[(4 * i + e) / K][(4 * i + e) % K] = f[e];
+    }
   }
 #pragma unroll
-  for (int j = 0; j < VW; ++j) acc[j] = silu(acc[j]);
-  vec<T>::store(out + tok * cdim + c0, acc);
+  for (int j = 0; j < VW; ++j) bv[j] = bias ? bias[c0 + j] : 0.f;
+
+  float win[K][VW];  // win[k] = input row t-K+1+k; rows before t = 0 are zero
+#pragma unroll
+  for (int k = 0; k < K - 1; ++k) {
+    const int64_t ts = t0 - (K - 1) + k;
+    if (ts >= 0) vec<T>::load(ub + ts * cdim, win[k]);
+    else {
+#pragma unroll
+      for (int j = 0; j < VW; ++j) win[k][j] = 0.f;
+    }
+  }
+  for (int64_t t = t0; t < t1; ++t) {
+    vec<T>::load(ub + t * cdim, win[K - 1]);
+    float o[VW];
+#pragma unroll
+    for (int j = 0; j < VW; ++j) {
+      float acc = bv[j];
+#pragma unroll
+      for (int k = 0; k < K; ++k) acc = fmaf(wr[j][k], win[k][j], acc);
+      o[j] = silu_fast(acc);
+    }
+    vec<T>::store(ob + t * cdim, o);
+#pragma unroll
+    for (int k = 0; k < K - 1; ++k)
+#pragma unroll
+      for (int j = 0; j < VW; ++j) win[k][j] = win[k + 1][j];
+  }
 }
 
-// dt[b,t,h] = softplus(raw[b,t,h] + bias[h])
+// dt[b,t,h] = softplus(raw[b,t,h] + bias[h]); 8 consecutive elements per thread, read as two
+// 16-byte loads when the pointers allow it (enough bytes in flight to stream HBM).
 __global__ void __launch_bounds__(256) dt_softplus_kernel(const float* raw,
                                                           const float* __restrict__ bias,
-                                                          float* dt, int64_t n,
-                                                          int nheads) {
-  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  dt[i] = softplus(raw[i] + (bias ? bias[i % nheads] : 0.f));
+                                                          float* dt, int64_t n, int nheads,
+                                                          bool vec4) {
+  const int64_t i0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (i0 >= n) return;
+  int h = int(i0 % nheads);
+  float v[8];
+  if (vec4 && i0 + 8 <= n) {
+    const float4 a = *reinterpret_cast<const float4*>(raw + i0);
+    const float4 b = *reinterpret_cast<const float4*>(raw + i0 + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = i0 + j < n ? raw[i0 + j] : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[j] = softplus(v[j] + (bias ? bias[h] : 0.f));
+    h = h + 1 == nheads ? 0 : h + 1;
+  }
+  if (vec4 && i0 + 8 <= n) {
+    *reinterpret_cast<float4*>(dt + i0) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(dt + i0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (i0 + j < n) dt[i0 + j] = v[j];
+  }
 }
 
 // out[i] = y[i] * silu(z[i]); VW elements per thread (the element count is a multiple of VW)

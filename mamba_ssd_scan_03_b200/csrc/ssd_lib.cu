@@ -567,18 +567,29 @@ ssd_status ssd_conv_silu(const void* u, const float* w, const float* bias, void*
       overlaps(out, nb, bias, size_t(cdim) * 4))
     return SSD_ERR_INVALID_ARG;
   const int vw = io == SSD_BF16 ? 8 : 4;
-  if (cdim % vw != 0 || !aligned16(u) || !aligned16(out)) return SSD_ERR_UNSUPPORTED;
-  const int64_t nthr = ntok * (cdim / vw);
-  if ((nthr + 255) / 256 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
-  const unsigned grid = unsigned((nthr + 255) / 256);
-  if (io == SSD_BF16)
-    ssd::glue::conv_silu_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(u), w, bias, static_cast<__nv_bfloat16*>(out), seqlen,
-        ntok, cdim, kwidth);
-  else
-    ssd::glue::conv_silu_kernel<float><<<grid, 256, 0, stream>>>(
-        static_cast<const float*>(u), w, bias, static_cast<float*>(out), seqlen, ntok, cdim,
-        kwidth);
+  if (cdim % vw != 0 || !aligned16(u) || !aligned16(out) || !aligned16(w))
+    return SSD_ERR_UNSUPPORTED;
+  const int64_t runs = (seqlen + ssd::glue::kConvTok - 1) / ssd::glue::kConvTok;
+  if (runs > 65535 || batch > 65535) return SSD_ERR_UNSUPPORTED;
+  const dim3 grid(unsigned((cdim / vw + 127) / 128), unsigned(runs), unsigned(batch));
+#define SSD_CONV(T, KW)                                                                    \
+  ssd::glue::conv_silu_kernel<T, KW><<<grid, 128, 0, stream>>>(                            \
+      static_cast<const T*>(u), w, bias, static_cast<T*>(out), seqlen, cdim)
+#define SSD_CONV_K(T)                                                                      \
+  switch (kwidth) {                                                                        \
+    case 1: SSD_CONV(T, 1); break;                                                         \
+    case 2: SSD_CONV(T, 2); break;                                                         \
+    case 3: SSD_CONV(T, 3); break;                                                         \
+    case 4: SSD_CONV(T, 4); break;                                                         \
+    case 5: SSD_CONV(T, 5); break;                                                         \
+    case 6: SSD_CONV(T, 6); break;                                                         \
+    case 7: SSD_CONV(T, 7); break;                                                         \
+    default: SSD_CONV(T, 8); break;                                                        \
+  }
+  if (io == SSD_BF16) { SSD_CONV_K(__nv_bfloat16) }
+  else { SSD_CONV_K(float) }
+#undef SSD_CONV_K
+#undef SSD_CONV
   return launched();
 }
 
@@ -590,9 +601,10 @@ ssd_status ssd_dt_softplus(const float* raw, const float* bias, float* dt, int64
   const int64_t n = batch * seqlen * nheads;
   if (dt != raw && overlaps(dt, size_t(n) * 4, raw, size_t(n) * 4)) return SSD_ERR_INVALID_ARG;
   if (overlaps(dt, size_t(n) * 4, bias, size_t(nheads) * 4)) return SSD_ERR_INVALID_ARG;
-  if ((n + 255) / 256 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
-  ssd::glue::dt_softplus_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(raw, bias, dt, n,
-                                                                               nheads);
+  const int64_t nthr = (n + 7) / 8;
+  if ((nthr + 255) / 256 > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+  ssd::glue::dt_softplus_kernel<<<unsigned((nthr + 255) / 256), 256, 0, stream>>>(
+      raw, bias, dt, n, nheads, aligned16(raw) && aligned16(dt));
   return launched();
 }
 

@@ -17,9 +17,12 @@ Contents
                 the LTI convolution kernel, and closed forms of special cases.
 ``glue``        float64 definitions of the block steps around the layer (short causal
                 convolution + SiLU, dt softplus, SiLU output gate).
+``selective``   the selective scan with a per-state transition (the first Mamba generation).
+``backward``    the layer's gradients (reverse-mode adjoint of the recurrence).
 
-Every function is pinned by ``tests/test_oracle.py`` (``glue`` by
-``tests/test_oracle_glue.py``); no function is "parity unpinned".
+Every function is pinned: ``tests/test_oracle.py``, ``tests/test_oracle_glue.py``,
+``tests/test_oracle_selective.py``, ``tests/test_oracle_backward.py``; no function is "parity
+unpinned".
 """
 import ctypes
 import os

@@ -8,169 +8,175 @@
 //   y_t[d] = sum_n C_t[g,n] h_t[n] + D[d] x_t[d]
 //
 // Unlike the scalar-transition layer there is no matrix form to put on the tensor cores: every
-// (token, channel, state) needs its own exp, so the kernel is bound by the MUFU ex2 rate.
+// (token, channel, state) needs its own exp, so the kernel is bound by the SFU's ex2 rate.
 //
-// Layout of the work: one warp per batch row and 8 channels; four lanes per channel, each lane
-// holding 4 of the 16 states in registers for the whole sequence.  The warp streams its inputs
-// in chunks of 32 tokens: 16-byte global loads one chunk ahead into registers, unpacked to
-// float32 in the warp's own shared-memory tiles; y is staged the same way and written with
-// 16-byte stores.  Warps are independent (one-warp CTAs, __syncwarp only), so the grid spreads
-// evenly over the SM sub-partitions whose ex2 units bound the kernel.
+// Layout of the work: one warp (one CTA) per batch row and 8 channels; four lanes per channel,
+// each lane holding 4 of the 16 states in registers for the whole sequence.  The inputs arrive
+// as TMA tiles of 32 tokens ({8 channels} of x and dt, {16 states} of B and C) in a two-stage
+// ring, so the loads cost the SM no per-row cache lookups (a plain 16-byte load of a 32-row
+// tile takes one L1 lookup per row, and with ~4 warps per scheduler those lookups, not the
+// exps, set the pace).  Rows past the end of the sequence are zero-filled by the TMA unit:
+// dt = 0 makes them exact identity steps (decay 1, no input).  y goes out the same way: staged
+// in shared memory (two buffers) and written by TMA stores, which drop rows past the end.
+// Every wait on a TMA barrier is bounded; on expiry the kernel latches the device status word,
+// waits (bounded) for its own copies in flight and returns without writing the final state.
 #pragma once
-#include "ssd_common.cuh"
+#include "tc_prims.cuh"
 
 namespace ssd {
 namespace sel {
 
-constexpr int kTok = 32;   // tokens per staged chunk
-constexpr int kCpw = 8;    // channels per warp
-constexpr int kN = 16;     // states per channel
-constexpr int kSpl = 4;    // states per lane (kN / lanes per channel)
+constexpr int kTok = 32;    // tokens per tile
+constexpr int kCpw = 8;     // channels per warp
+constexpr int kN = 16;      // states per channel
+constexpr int kSpl = 4;     // states per lane
+constexpr int kStages = 2;  // input tiles in flight
 
-// A [kTok][W] tile of T from global memory, row stride `ld` elements, moved through registers
-// (one chunk ahead) into a float32 shared-memory tile.  Rows at or past `rows` read as zero.
-template <typename T, int W>
-struct Tile {
-  static constexpr int EPV = 16 / int(sizeof(T));  // elements per 16-byte vector
-  static constexpr int VPR = W / EPV;              // vectors per row
-  static constexpr int NV = kTok * VPR / 32;       // vectors per lane
-  static_assert(kTok * VPR % 32 == 0, "tile must split evenly over the warp");
-  uint4 r[NV];
-
-  __device__ __forceinline__ void load(const T* base, int64_t ld, int rows, int lane) {
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int v = lane + 32 * j, row = v / VPR, col = (v % VPR) * EPV;
-      r[j] = row < rows ? __ldg(reinterpret_cast<const uint4*>(base + row * ld + col))
-                        : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  __device__ __forceinline__ void stage(float (*s)[W], int lane) const {
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int v = lane + 32 * j, row = v / VPR, col = (v % VPR) * EPV;
-      float4* d = reinterpret_cast<float4*>(&s[row][col]);
-      if constexpr (sizeof(T) == 4) {
-        d[0] = make_float4(__uint_as_float(r[j].x), __uint_as_float(r[j].y),
-                           __uint_as_float(r[j].z), __uint_as_float(r[j].w));
-      } else {
-        d[0] = make_float4(bf16lo(r[j].x), bf16hi(r[j].x), bf16lo(r[j].y), bf16hi(r[j].y));
-        d[1] = make_float4(bf16lo(r[j].z), bf16hi(r[j].z), bf16lo(r[j].w), bf16hi(r[j].w));
-      }
-    }
-  }
+template <typename T, typename TY>
+struct Smem {
+  static constexpr int kX = kTok * kCpw * int(sizeof(T));   // x tile   [32][8]
+  static constexpr int kDt = kTok * kCpw * 4;               // dt tile  [32][8] float32
+  static constexpr int kBC = kTok * kN * int(sizeof(T));    // B, C tiles [32][16]
+  static constexpr int kStage = kX + kDt + 2 * kBC;         // one TMA transaction
+  static constexpr int kY = kTok * kCpw * int(sizeof(TY));  // y tile   [32][8]
+  static constexpr int kBars = kStages * kStage + 2 * kY;   // offset of the barriers
+  static constexpr int kBytes = kBars + 64 + 128;           // + barriers + alignment slack
+  static_assert(kX % 128 == 0 && kDt % 128 == 0 && kBC % 128 == 0 && kY % 128 == 0,
+                "tiles must stay 128-byte aligned");
 };
 
-// y tile [kTok][kCpw] float32 in shared memory -> global rows (stride `ld`), rows < `rows`.
-template <typename TY>
-__device__ __forceinline__ void store_y(const float (*s)[kCpw], TY* base, int64_t ld, int rows,
-                                        int lane) {
-  if constexpr (sizeof(TY) == 4) {  // 32 rows x 2 float4
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int v = lane + 32 * j, row = v >> 1, col = (v & 1) * 4;
-      if (row < rows)
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + row * ld + col) =
-            *reinterpret_cast<const float4*>(&s[row][col]);
-    }
-  } else {  // 32 rows x one 16-byte vector of 8 bf16
-    if (lane < rows) {
-      const float4 a = *reinterpret_cast<const float4*>(&s[lane][0]);
-      const float4 b = *reinterpret_cast<const float4*>(&s[lane][4]);
-      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + lane * ld) =
-          make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                     pack_bf16x2(b.z, b.w));
-    }
-  }
+__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) {
+  return __uint_as_float(uint32_t(*reinterpret_cast<const unsigned short*>(p)) << 16);
+}
+__device__ __forceinline__ float load1(const float* p) { return *p; }
+__device__ __forceinline__ float load1(const __nv_bfloat16* p) { return bf16_at(p); }
+__device__ __forceinline__ float4 load4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
+}
+__device__ __forceinline__ void store1(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Allow the most recent bulk group to be pending; every older one has finished reading smem.
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
-// One warp per (batch row, 8 channels).  Preconditions (checked on the host): dstate == 16,
-// dim % 8 == 0, (dim / ngroups) % 8 == 0, every pointer 16-byte aligned.
+// Bounded wait that ignores the abort flag: used after an abort to let this CTA's own TMA
+// loads land before it exits.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_test_sleep(bar, parity, 20000u))
+    if (tc::globaltimer() - t0 > 1000000000ull) return;
+}
+
+// Preconditions (checked on the host): dstate == 16, dim % 8 == 0, (dim / ngroups) % 8 == 0,
+// 16-byte aligned pointers; the tensor maps are 3-D {inner, seqlen, batch} with boxes
+// {8, 32, 1} (x, dt, y) and {16, 32, 1} (B, C), no swizzle, zero fill.
 template <typename T, typename TY>
 __global__ void __launch_bounds__(32) selective_scan_kernel(
-    const T* __restrict__ x, const float* __restrict__ dt, const float* __restrict__ A,
-    const T* __restrict__ B, const T* __restrict__ C, const float* __restrict__ D,
-    const float* __restrict__ init, TY* __restrict__ y, float* __restrict__ fin,
+    const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdt,
+    const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mc,
+    const __grid_constant__ CUtensorMap my, const float* __restrict__ A,
+    const float* __restrict__ D, const float* __restrict__ init, float* __restrict__ fin,
     int64_t seqlen, int dim, int ngroups) {
-  __shared__ __align__(16) float xs[kTok][kCpw];
-  __shared__ __align__(16) float ds[kTok][kCpw];
-  __shared__ __align__(16) float bs[kTok][kN];
-  __shared__ __align__(16) float cs[kTok][kN];
-  __shared__ __align__(16) float ys[kTok][kCpw];
+  using S = Smem<T, TY>;
+  extern __shared__ uint8_t smraw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 127) &
+                                           ~uintptr_t(127));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + S::kBars);
+  __shared__ int abort_flag;
 
   const int lane = threadIdx.x;
   const int c = lane >> 2, q = lane & 3;  // channel within the warp, state quarter
   const int wpr = dim / kCpw;             // warps per batch row
-  const int64_t b = blockIdx.x / wpr;
+  const int b = int(blockIdx.x / wpr);
   const int d0 = int(blockIdx.x % wpr) * kCpw;
   const int d = d0 + c;
   const int g = d0 / (dim / ngroups);
+  const int nck = int((seqlen + kTok - 1) / kTok);
 
-  // per-lane constants: this lane's 4 decay rates in log2 units, the skip weight
-  float2 a2[2];
+  auto issue = [&](int k) {  // lane 0: the four input tiles of chunk k into stage k % kStages
+    uint64_t* bar = &full[k % kStages];
+    uint8_t* st = sm + (k % kStages) * S::kStage;
+    tc::mbar_arrive_expect_tx(bar, uint32_t(S::kStage));
+    tc::tma_load_3d(st, &mx, bar, d0, k * kTok, b);
+    tc::tma_load_3d(st + S::kX, &mdt, bar, d0, k * kTok, b);
+    tc::tma_load_3d(st + S::kX + S::kDt, &mb, bar, g * kN, k * kTok, b);
+    tc::tma_load_3d(st + S::kX + S::kDt + S::kBC, &mc, bar, g * kN, k * kTok, b);
+  };
+  if (lane == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) tc::mbar_init(&full[s], 1);
+    tc::fence_mbar_init();
+    for (int k = 0; k < kStages && k < nck; ++k) issue(k);
+  }
+  __syncwarp();
+
+  // per-lane constants: this lane's 4 decay rates in log2 units, the skip weight, the state
+  float a2[kSpl];
   {
     const float4 av = *reinterpret_cast<const float4*>(A + int64_t(d) * kN + q * kSpl);
-    a2[0] = make_float2(av.x * kLog2e, av.y * kLog2e);
-    a2[1] = make_float2(av.z * kLog2e, av.w * kLog2e);
+    a2[0] = av.x * kLog2e; a2[1] = av.y * kLog2e; a2[2] = av.z * kLog2e; a2[3] = av.w * kLog2e;
   }
   const float Dd = D ? D[d] : 0.f;
-  float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  const int64_t st = (b * dim + d) * kN + q * kSpl;  // this lane's slice of the state
+  float h[kSpl] = {0.f, 0.f, 0.f, 0.f};
+  const int64_t st_off = (int64_t(b) * dim + d) * kN + q * kSpl;
   if (init) {
-    const float4 iv = *reinterpret_cast<const float4*>(init + st);
-    h[0] = make_float2(iv.x, iv.y);
-    h[1] = make_float2(iv.z, iv.w);
+    const float4 iv = *reinterpret_cast<const float4*>(init + st_off);
+    h[0] = iv.x; h[1] = iv.y; h[2] = iv.z; h[3] = iv.w;
   }
 
-  const int64_t row0 = b * seqlen;  // first token row of this batch row
-  const int64_t gld = int64_t(ngroups) * kN;
-  Tile<T, kCpw> tx;
-  Tile<float, kCpw> td;
-  Tile<T, kN> tb, tc;
-  auto fetch = [&](int64_t t0) {
-    const int rows = int(seqlen - t0 < kTok ? seqlen - t0 : kTok);
-    tx.load(x + (row0 + t0) * dim + d0, dim, rows, lane);
-    td.load(dt + (row0 + t0) * dim + d0, dim, rows, lane);
-    tb.load(B + (row0 + t0) * gld + int64_t(g) * kN, gld, rows, lane);
-    tc.load(C + (row0 + t0) * gld + int64_t(g) * kN, gld, rows, lane);
-  };
-
-  fetch(0);
-  for (int64_t t0 = 0; t0 < seqlen; t0 += kTok) {
-    __syncwarp();  // the previous chunk's reads of the tiles (and of ys) are done
-    tx.stage(xs, lane);
-    td.stage(ds, lane);
-    tb.stage(bs, lane);
-    tc.stage(cs, lane);
+  int k = 0;
+  for (; k < nck; ++k) {
+    const int s = k % kStages;
+    const bool got = tc::mbar_wait(&full[s], uint32_t(k / kStages) & 1u, &abort_flag, 60);
+    if (__any_sync(0xffffffffu, !got)) break;
+    // y buffer k & 1 was last handed to the TMA store of chunk k - 2
+    if (lane == 0 && k >= 2) bulk_wait_read_all_but_one();
     __syncwarp();
-    if (t0 + kTok < seqlen) fetch(t0 + kTok);
-    // Rows past the end were staged as zeros: dt = 0 makes them identity steps (decay 1, no
-    // input), so the state carried out of the last chunk is exact without a per-token check.
+    const uint8_t* stg = sm + s * S::kStage;
+    const T* xs = reinterpret_cast<const T*>(stg);
+    const float* ds = reinterpret_cast<const float*>(stg + S::kX);
+    const T* bs = reinterpret_cast<const T*>(stg + S::kX + S::kDt);
+    const T* cs = reinterpret_cast<const T*>(stg + S::kX + S::kDt + S::kBC);
+    TY* ys = reinterpret_cast<TY*>(sm + kStages * S::kStage + (k & 1) * S::kY);
 #pragma unroll 4
     for (int t = 0; t < kTok; ++t) {
-      const float xv = xs[t][c], dv = ds[t][c];
-      const float4 bv = *reinterpret_cast<const float4*>(&bs[t][q * kSpl]);
-      const float4 cv = *reinterpret_cast<const float4*>(&cs[t][q * kSpl]);
-      const float2 dd = make_float2(dv, dv);
-      const float2 l0 = mul2(dd, a2[0]), l1 = mul2(dd, a2[1]);
-      const float2 e0 = make_float2(ex2(l0.x), ex2(l0.y)), e1 = make_float2(ex2(l1.x), ex2(l1.y));
+      const float xv = load1(xs + t * kCpw + c), dv = ds[t * kCpw + c];
+      const float4 bv = load4(bs + t * kN + q * kSpl);
+      const float4 cv = load4(cs + t * kN + q * kSpl);
       const float u = dv * xv;
-      const float2 uu = make_float2(u, u);
-      h[0] = fma2(e0, h[0], mul2(uu, make_float2(bv.x, bv.y)));
-      h[1] = fma2(e1, h[1], mul2(uu, make_float2(bv.z, bv.w)));
-      const float2 acc = fma2(make_float2(cv.z, cv.w), h[1], mul2(make_float2(cv.x, cv.y), h[0]));
-      float s = acc.x + acc.y;
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (q == 0) ys[t][c] = fmaf(Dd, xv, s);
+      h[0] = fmaf(ex2(dv * a2[0]), h[0], u * bv.x);
+      h[1] = fmaf(ex2(dv * a2[1]), h[1], u * bv.y);
+      h[2] = fmaf(ex2(dv * a2[2]), h[2], u * bv.z);
+      h[3] = fmaf(ex2(dv * a2[3]), h[3], u * bv.w);
+      float p = fmaf(cv.z, h[2], cv.x * h[0]) + fmaf(cv.w, h[3], cv.y * h[1]);
+      p += __shfl_xor_sync(0xffffffffu, p, 1);
+      p += __shfl_xor_sync(0xffffffffu, p, 2);
+      if (q == 0) store1(ys + t * kCpw + c, fmaf(Dd, xv, p));
     }
-    __syncwarp();
-    const int rows = int(seqlen - t0 < kTok ? seqlen - t0 : kTok);
-    store_y<TY>(ys, y + (row0 + t0) * dim + d0, dim, rows, lane);
+    tc::fence_proxy_async_smem();  // this lane's y writes -> visible to the TMA store
+    __syncwarp();                  // every lane is done with stage s and with ys
+    if (lane == 0) {
+      tc::tma_store_3d(&my, ys, d0, k * kTok, b);
+      tc::bulk_commit();
+      if (k + kStages < nck) issue(k + kStages);
+    }
   }
-  if (fin) {
-    *reinterpret_cast<float4*>(fin + st) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+  if (k < nck) {
+    // aborted at chunk k: chunks k .. min(k + kStages, nck) - 1 may still be landing
+    if (lane == 0)
+      for (int j = k; j < k + kStages && j < nck; ++j)
+        drain_wait(&full[j % kStages], uint32_t(j / kStages) & 1u);
+  } else if (fin) {
+    *reinterpret_cast<float4*>(fin + st_off) = make_float4(h[0], h[1], h[2], h[3]);
   }
+  if (lane == 0) tc::bulk_wait_all();
+  __syncwarp();
 }
 
 }  // namespace sel

@@ -167,6 +167,22 @@ bool make_dt_map(CUtensorMap* m, const float* dt, int64_t batch, int64_t seqlen,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view {inner, mid, outer} of a row-major tensor with a {box_inner, box_mid, 1} box, no
+// swizzle, zero fill outside the tensor (the selective scan's tiles).
+bool make_box_map(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint64_t es,
+                  uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_mid) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * es, inner * mid * es};
+  cuuint32_t box[3] = {box_inner, box_mid, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, type, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Dynamic shared-memory limits of the kernels, set once per device (the attribute applies to
 // the current device only).
 ssd_status set_smem_attrs() {
@@ -187,6 +203,13 @@ ssd_status set_smem_attrs() {
     ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
           cudaSuccess;
+    // the selective scan runs ~17 one-warp CTAs per SM: ask for the largest shared-memory
+    // carve-out so that shared memory does not cap them
+    for (auto f : {(const void*)ssd::sel::selective_scan_kernel<float, float>,
+                   (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, float>,
+                   (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, __nv_bfloat16>})
+      ok &= cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 int(cudaSharedmemCarveoutMaxShared)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem<2>)) ==
           cudaSuccess;
@@ -672,14 +695,28 @@ ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A
                         (const void*)init_state, (const void*)final_state})
     if (p && !aligned16(p)) return SSD_ERR_UNSUPPORTED;
   const int64_t warps = batch * (dim / sel::kCpw);
-  if (warps > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+  if (warps > INT32_MAX || seqlen > INT32_MAX - sel::kTok || batch > INT32_MAX)
+    return SSD_ERR_UNSUPPORTED;
+  const bool bf = io == SSD_BF16, ybf = y_dtype == SSD_BF16;
+  const CUtensorMapDataType tio = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const uint64_t L = uint64_t(seqlen), Bn = uint64_t(batch), GN = uint64_t(ngroups) * sel::kN;
+  CUtensorMap mx, mdt, mb, mc, my;
+  if (!make_box_map(&mx, x, tio, es, dim, L, Bn, sel::kCpw, sel::kTok) ||
+      !make_box_map(&mdt, dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, L, Bn, sel::kCpw,
+                    sel::kTok) ||
+      !make_box_map(&mb, B, tio, es, GN, L, Bn, sel::kN, sel::kTok) ||
+      !make_box_map(&mc, C, tio, es, GN, L, Bn, sel::kN, sel::kTok) ||
+      !make_box_map(&my, y, ybf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    ybf ? 2 : 4, dim, L, Bn, sel::kCpw, sel::kTok))
+    return SSD_ERR_CUDA;
+  if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
   const unsigned grid = unsigned(warps);
 #define SSD_SEL(T, TY)                                                                      \
-  sel::selective_scan_kernel<T, TY><<<grid, 32, 0, stream>>>(                               \
-      static_cast<const T*>(x), dt, A, static_cast<const T*>(B), static_cast<const T*>(C),  \
-      D, init_state, static_cast<TY*>(y), final_state, seqlen, dim, ngroups)
-  if (io == SSD_F32) SSD_SEL(float, float);
-  else if (y_dtype == SSD_F32) SSD_SEL(__nv_bfloat16, float);
+  sel::selective_scan_kernel<T, TY><<<grid, 32, sel::Smem<T, TY>::kBytes, stream>>>(        \
+      mx, mdt, mb, mc, my, A, D, init_state, final_state, seqlen, dim, ngroups)
+  if (!bf) SSD_SEL(float, float);
+  else if (!ybf) SSD_SEL(__nv_bfloat16, float);
   else SSD_SEL(__nv_bfloat16, __nv_bfloat16);
 #undef SSD_SEL
   return launched();

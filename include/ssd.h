@@ -228,7 +228,9 @@ ssd_status ssd_state_pass(float* states, const float* decay, const float* init_s
  *   u taken as 0 before t = 0 (no history).
  *   u, out : [batch, seqlen, cdim] in `io` (SSD_BF16 or SSD_F32), must not overlap; w
  *   [cdim, kwidth] float32, kwidth 1..8; bias [cdim] float32 or NULL.  cdim a multiple of 8
- *   (bf16) or 4 (f32) and u, out 16-byte aligned, else SSD_ERR_UNSUPPORTED.
+ *   (bf16) or 4 (f32), u, out and w 16-byte aligned, batch <= 65535 and seqlen <= 64 * 65535,
+ *   else SSD_ERR_UNSUPPORTED.  SiLU here uses the hardware exponential and an approximate
+ *   divide (a few float32 ulps).
  */
 ssd_status ssd_conv_silu(const void* u, const float* w, const float* bias, void* out,
                          int64_t batch, int64_t seqlen, int cdim, int kwidth, ssd_dtype io,
@@ -266,7 +268,9 @@ ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ss
  * All pointers are device memory owned by the caller; y and final_state must not overlap the
  * inputs.  Float32 arithmetic, hardware exp2 for the decays; asynchronous on `stream`.
  * Supported: dstate == 16, dim and dim / ngroups multiples of 8, every pointer 16-byte aligned
- * (else SSD_ERR_UNSUPPORTED).  Argument errors are returned before any launch.
+ * (else SSD_ERR_UNSUPPORTED).  Argument errors are returned before any launch; the kernel's
+ * waits on its TMA tiles are bounded, and an expired wait is reported by
+ * ssd_get_device_status (the final state is then not written).
  */
 ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
                                   const void* C, const float* D, const float* init_state,

@@ -75,7 +75,8 @@ Seg tc_segments(const Shape& s) {
   Seg sg;
   sg.nblk = int((s.seqlen + ssd::tc::kBlk - 1) / ssd::tc::kBlk);
   const int64_t pairs = s.batch * (s.nheads / 2);
-  int nseg = int(std::min<int64_t>(sg.nblk, std::max<int64_t>(1, (kUnitsTarget + pairs - 1) / pairs)));
+  int nseg = int(std::min<int64_t>(
+      sg.nblk, std::max<int64_t>(1, (kUnitsTarget + pairs - 1) / pairs)));
   sg.seg_blks = (sg.nblk + nseg - 1) / nseg;
   sg.nseg = (sg.nblk + sg.seg_blks - 1) / sg.seg_blks;
   return sg;
@@ -707,7 +708,8 @@ ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A
                     sel::kTok) ||
       !make_box_map(&mb, B, tio, es, GN, L, Bn, sel::kN, sel::kTok) ||
       !make_box_map(&mc, C, tio, es, GN, L, Bn, sel::kN, sel::kTok) ||
-      !make_box_map(&my, y, ybf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+      !make_box_map(&my, y,
+                    ybf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                     ybf ? 2 : 4, dim, L, Bn, sel::kCpw, sel::kTok))
     return SSD_ERR_CUDA;
   if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;

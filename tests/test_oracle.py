@@ -315,7 +315,8 @@ def test_input_distributions():
     inp = ssd_inputs.make_scan_inputs(1, seqlen=256)
     x = ssd_inputs.bf16_bits_to_f32(inp["x"]).astype(np.float64)
     assert abs(x.mean()) < 0.02 and abs(x.std() - 1) < 0.02
-    assert np.all(inp["dt"] > 0) and abs(inp["dt"].mean() - 0.1403) < 0.003  # E[softplus(N(-2,0.5))] = 0.1403
+    # E[softplus(N(-2, 0.5))] = 0.1403
+    assert np.all(inp["dt"] > 0) and abs(inp["dt"].mean() - 0.1403) < 0.003
     assert np.all((inp["A"] <= -1.0) & (inp["A"] >= -16.0))
     Bv = ssd_inputs.bf16_bits_to_f32(inp["B"]).astype(np.float64)
     assert abs(Bv.std() * math.sqrt(128) - 1) < 0.03

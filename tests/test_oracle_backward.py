@@ -47,7 +47,8 @@ def fd_pins(grad_fn, seed=0, **shape):
     rng = np.random.default_rng(seed + 100)
     for name in NAMES:
         v = rng.standard_normal(inp[name].shape)
-        # a step of ~1e-4 relative: float32 storage keeps 4 digits of it, and the realised step is used
+        # a step of ~1e-4 relative: float32 storage keeps 4 digits of it; the realised step
+        # is what the prediction uses
         eps = 1e-4 * max(1e-3, float(np.max(np.abs(inp[name]))))
         up, dn = dict(inp), dict(inp)
         up[name] = inp[name] + eps * v

@@ -173,3 +173,39 @@ def test_selective_binding_refuses_cpu_tensors(lib):
         ssd.selective_scan_fwd(x, torch.zeros(1, 4, 16), torch.zeros(16, 16),
                                torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16),
                                torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "ssd.h"
+int main(void) {
+  /* a plain C client: the header is valid C99 and every call links against libssd.so */
+  if (strncmp(ssd_version(), "ssd-b200", 8) != 0) return 1;
+  if (strcmp(ssd_status_string(SSD_OK), "SSD_OK") != 0) return 2;
+  if (ssd_chunk_scan_path(2, 300, 4, 64, 128, 1, 256, SSD_BF16) != SSD_PATH_TCGEN05) return 3;
+  if (ssd_chunk_scan_path(2, 300, 4, 64, 128, 1, 256, SSD_F32) != SSD_PATH_SIMT) return 4;
+  if (ssd_chunk_scan_workspace_size(2, 300, 4, 64, 128, 1, 256, SSD_BF16) == 0) return 5;
+  /* argument errors come back before anything touches a GPU */
+  if (ssd_step(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 4, 64, 128, 1, SSD_BF16,
+               SSD_F32, 0) != SSD_ERR_INVALID_ARG) return 6;
+  if (ssd_selective_scan_fwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 8, 64, 16,
+                             1, SSD_BF16, SSD_F32, 0) != SSD_ERR_INVALID_ARG) return 7;
+  printf("%s\n", ssd_version());
+  return 0;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_runs(lib, tmp_path):
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(ssd.LIB_PATH)
+    cuda_inc = os.path.join(os.path.dirname(os.path.dirname(ssd_build.NVCC)), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", cuda_inc, str(src), "-o", str(exe), "-L", libdir, "-l:libssd.so",
+                    f"-Wl,-rpath,{libdir}"], check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.startswith("ssd-b200")

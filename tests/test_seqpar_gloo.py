@@ -64,7 +64,8 @@ def _worker(rank, world, port, cuts, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("cuts", [[0, 150, 300], [0, 1, 300], [0, 97, 211, 300]])
+@pytest.mark.parametrize("cuts", [[0, 150, 300], [0, 1, 300], [0, 97, 211, 300],
+                                  [0, 50, 100, 220, 300]])
 def test_sliced_scan_equals_whole_scan(cuts):
     world = len(cuts) - 1
     ctx = mp.get_context("spawn")
@@ -89,3 +90,39 @@ def test_sliced_scan_equals_whole_scan(cuts):
     assert np.max(np.abs(y - y_ref)) <= 1e-9 * np.sqrt(np.mean(y_ref ** 2))
     for r in range(world):
         assert np.max(np.abs(out[r][1] - f_ref)) <= 1e-9 * np.sqrt(np.mean(f_ref ** 2))
+
+
+def _dying_worker(rank, world, port, q):
+    """Rank 1 leaves before the exchange; rank 0 must get an error, not wait for ever."""
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        os._exit(0)  # gone between steps, no collective in flight
+    from mamba_ssd_scan_03_b200.seqpar import seqpar_scan_fwd
+    inp = ssd_inputs.make_scan_inputs(dict(batch=1, seqlen=64, nheads=4, headdim=8, dstate=16,
+                                           ngroups=2, chunk=64, io="f32", init="zeros"), seed=3)
+    t = {k: torch.from_numpy(np.ascontiguousarray(inp[k][:, :32]))
+         for k in ("x", "dt", "B", "C")}
+    try:
+        seqpar_scan_fwd(t["x"], t["dt"], torch.from_numpy(inp["A"]), t["B"], t["C"],
+                        torch.from_numpy(inp["D"]), 64, ops=OracleOps())
+        q.put("no error")
+    except Exception as e:  # the collective fails: the peer is gone
+        q.put(type(e).__name__)
+
+
+def test_exchange_fails_cleanly_when_a_rank_is_gone():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert res != "no error", res

@@ -322,3 +322,17 @@ def test_input_distributions():
     assert abs(Bv.std() * math.sqrt(128) - 1) < 0.03
     ini = ssd_inputs.make_scan_inputs(2, seqlen=128, batch=1)["init"]
     assert abs(ini.std() - 0.1) < 0.005
+
+
+def test_bf16_rounding_of_y_alone_exceeds_the_bf16_bar():
+    """Why y is float32 by default: on the 2.7B-shape workload's distributions, rounding the
+    exact y to bf16 (nearest even) by itself already misses max|err| <= 2e-2 * RMS(y), because
+    D x with D ~ N(0, 1) gives y heavy tails (max|y| / RMS(y) ~ 10)."""
+    inp = ssd_inputs.make_scan_inputs(2, batch=1, seqlen=2048)
+    ids = np.arange(0, 80 * 64, 37, dtype=np.int64)
+    init = inp["init"].reshape(-1, 128)[ids]
+    y, _ = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], init=init,
+                       chains=ids)
+    yb = ssd_inputs.bf16_bits_to_f32(ssd_inputs.f32_to_bf16_bits(y.astype(np.float32)))
+    rms = np.sqrt(np.mean(y ** 2))
+    assert np.max(np.abs(yb - y)) > 2e-2 * rms

@@ -14,6 +14,8 @@ uczenia rozproszonego": only boundary states cross between devices).
     4. y_r = chunk_scan_fwd(own slice, init_state = H_in[r])         -- the full scan kernels
 
 Steps 1, 3 and 4 are the library's kernels (`ops` replaces them only in host-logic tests).
+A rank whose slice is empty contributes the identity step (S = 0, total decay 0) and returns
+an empty y.
 """
 import torch
 import torch.distributed as dist
@@ -25,6 +27,12 @@ class LibraryOps:
     def state(self, x, dt, A, B, chunk):
         from . import chunk_state_fwd
         return chunk_state_fwd(x, dt, A, B, chunk)
+
+    def identity(self, x, B):
+        """The summary of an empty slice: no input (S = 0) and no decay (total 0)."""
+        Bt, _, H, P = x.shape
+        S = torch.zeros((Bt, H, P, B.shape[3]), dtype=torch.float32, device=x.device)
+        return S, torch.zeros((Bt, H), dtype=torch.float32, device=x.device)
 
     def state_pass(self, states, decay, init_state):
         from . import state_pass
@@ -45,7 +53,8 @@ def seqpar_scan_fwd(x, dt, A, B, C, D, chunk, init_state=None, group=None, ops=N
     ops = LibraryOps() if ops is None else ops
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    S, decay = ops.state(x, dt, A, B, chunk)
+    empty = x.shape[1] == 0
+    S, decay = ops.identity(x, B) if empty else ops.state(x, dt, A, B, chunk)
     all_s = [torch.empty_like(S) for _ in range(world)]
     all_d = [torch.empty_like(decay) for _ in range(world)]
     dist.all_gather(all_s, S.contiguous(), group=group)
@@ -53,5 +62,7 @@ def seqpar_scan_fwd(x, dt, A, B, C, D, chunk, init_state=None, group=None, ops=N
     states = torch.stack(all_s)
     decays = torch.stack(all_d)
     final = ops.state_pass(states, decays, init_state)
+    if empty:
+        return torch.empty(x.shape, dtype=y_dtype, device=x.device), final
     y = ops.scan(x, dt, A, B, C, D, chunk, states[rank].contiguous(), y_dtype)
     return y, final

@@ -24,6 +24,11 @@ class OracleOps:
         decay = (dt.numpy().astype(np.float64) * A.numpy()[None, None, :]).sum(axis=1)
         return torch.from_numpy(h1), torch.from_numpy(decay)
 
+    def identity(self, x, B):
+        Bt, _, H, P = x.shape
+        return (torch.zeros((Bt, H, P, B.shape[3]), dtype=torch.float64),
+                torch.zeros((Bt, H), dtype=torch.float64))
+
     def state_pass(self, states, decay, init_state):
         run = torch.zeros_like(states[0]) if init_state is None else init_state.clone()
         for r in range(states.shape[0]):
@@ -65,7 +70,7 @@ def _worker(rank, world, port, cuts, q):
 
 
 @pytest.mark.parametrize("cuts", [[0, 150, 300], [0, 1, 300], [0, 97, 211, 300],
-                                  [0, 50, 100, 220, 300]])
+                                  [0, 50, 100, 220, 300], [0, 0, 300], [0, 150, 150, 300]])
 def test_sliced_scan_equals_whole_scan(cuts):
     world = len(cuts) - 1
     ctx = mp.get_context("spawn")

@@ -131,3 +131,30 @@ def test_exchange_fails_cleanly_when_a_rank_is_gone():
         if p.is_alive():
             p.kill()
     assert res != "no error", res
+
+
+def _cpu_tensor_worker(port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        from mamba_ssd_scan_03_b200.seqpar import seqpar_scan_fwd
+        x = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+        bc = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
+        try:
+            seqpar_scan_fwd(x, torch.zeros(1, 8, 2), torch.zeros(2), bc, bc, None, 256)
+            q.put("no error")
+        except (ValueError, RuntimeError) as e:
+            q.put(str(e))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_library_ops_refuse_host_tensors():
+    """The product path has no CPU fallback: host tensors are refused by the binding."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_cpu_tensor_worker, args=(_free_port(), q))
+    p.start()
+    res = q.get(timeout=120)
+    p.join(timeout=60)
+    assert res != "no error" and "CUDA" in res, res

@@ -156,3 +156,14 @@ def test_glue_pins_catch_mistakes(i):
     with np.errstate(all="ignore"):
         results = [ok for _, ok in pins(fn)]
     assert not all(results)
+
+
+def test_glue_input_recipe():
+    from ssd_inputs import make_glue_inputs
+    g = make_glue_inputs(2, 512, 64, 4, 8, 32, "f32")
+    assert abs(g["u"].std() - 1) < 0.02 and abs(g["z"].std() - 1) < 0.02
+    assert abs(g["w"].std() - 0.5) < 0.05  # N(0, 1) / sqrt(4)
+    assert np.all(g["dt_bias"] >= -6) and np.all(g["dt_bias"] <= -2)
+    h = make_glue_inputs(2, 512, 64, 4, 8, 32, "f32")
+    for k in ("u", "w", "conv_bias", "raw", "dt_bias", "y", "z"):
+        np.testing.assert_array_equal(g[k], h[k])

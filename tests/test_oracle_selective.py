@@ -156,3 +156,23 @@ def test_selective_variant_without_mistake_passes():
 def test_selective_pins_catch_mistakes(mistake):
     with np.errstate(all="ignore"):
         assert not all(pin(_variant(mistake)) for pin in PINS)
+
+
+def test_selective_input_recipe():
+    """The recipe the docstring of make_selective_inputs states: x ~ N(0,1), dt = softplus of
+    N(-2, 0.5) (mean 0.1403), A in [-16, -1] independent per (channel, state), B and C with
+    standard deviation 1/sqrt(16), init N(0, 0.1); deterministic for a seed."""
+    inp = ssd_inputs.make_selective_inputs(dict(name="t", batch=2, seqlen=2048, dim=64,
+                                                dstate=16, ngroups=1, io="f32",
+                                                init="normal0.1"))
+    assert abs(inp["x"].mean()) < 0.01 and abs(inp["x"].std() - 1) < 0.01
+    assert abs(inp["dt"].mean() - 0.1403) < 0.003 and np.all(inp["dt"] > 0)
+    assert np.all(inp["A"] <= -1) and np.all(inp["A"] >= -16)
+    assert len(np.unique(inp["A"])) == inp["A"].size  # a rate per (channel, state)
+    assert abs(inp["B"].std() - 0.25) < 0.01 and abs(inp["C"].std() - 0.25) < 0.01
+    assert abs(inp["init"].std() - 0.1) < 0.005
+    again = ssd_inputs.make_selective_inputs(dict(name="t", batch=2, seqlen=2048, dim=64,
+                                                  dstate=16, ngroups=1, io="f32",
+                                                  init="normal0.1"))
+    for k in ("x", "dt", "A", "B", "C", "D", "init"):
+        np.testing.assert_array_equal(inp[k], again[k])

@@ -109,6 +109,56 @@ ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, co
                               ssd_dtype y_dtype, void* workspace, size_t workspace_bytes,
                               cudaStream_t stream);
 
+/*
+ * ssd_chunk_scan_fwd on the tensor-core path with its plan and its kernels' bounded waits under
+ * the caller's control -- for tests and tuning; the pages have no counterpart.  opt == NULL (or
+ * all fields 0) is exactly ssd_chunk_scan_fwd.
+ *   max_ctas       cap on the walk's CTAs (0: one per SM).  Fewer CTAs than (batch row, head
+ *                  pair) sequences make ranges that start inside a sequence, so the published
+ *                  boundary states are exercised on small shapes.
+ *   plan           0 automatic; 1 whole sequences (no summary pass); 2 segments whose entering
+ *                  states come from a summary pass (seg_state + seg_pass) before the walk.
+ *   wait_limit_ns  limit of every bounded wait in the walk (0: 2 s; -1: no waiting, i.e. a
+ *                  wait whose event has not already happened gives up at once).  A wait that
+ *                  gives up makes the kernel latch SSD_ERR_DEVICE_TIMEOUT in the device status
+ *                  word, let its copies and MMAs land, free its tensor memory and return; y and
+ *                  final_state are then undefined, and the next call works normally.
+ * Only tensor-core shapes (else SSD_ERR_UNSUPPORTED); max_ctas < 0, plan outside 0..2 or
+ * wait_limit_ns < -1 return
+ * SSD_ERR_INVALID_ARG.  The workspace must hold ssd_chunk_scan_workspace_size_ex() bytes for
+ * the same options.
+ */
+typedef struct {
+  int max_ctas;
+  int plan;
+  int64_t wait_limit_ns;
+} ssd_scan_options;
+size_t ssd_chunk_scan_workspace_size_ex(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                        int dstate, int ngroups, int chunk, ssd_dtype io,
+                                        const ssd_scan_options* opt);
+ssd_status ssd_chunk_scan_fwd_ex(const void* x, const float* dt, const float* A, const void* B,
+                                 const void* C, const float* D, const float* init_state,
+                                 void* y, float* final_state, int64_t batch, int64_t seqlen,
+                                 int nheads, int headdim, int dstate, int ngroups, int chunk,
+                                 ssd_dtype io, ssd_dtype y_dtype, void* workspace,
+                                 size_t workspace_bytes, const ssd_scan_options* opt,
+                                 cudaStream_t stream);
+
+/*
+ * How ssd_chunk_scan_fwd (or _ex with `opt`) runs this shape on the tensor cores: the kernels it
+ * launches per call, the CTAs of its walk, and the segments each sequence is cut into (1: no
+ * summary pass).  Returns SSD_ERR_UNSUPPORTED for shapes that do not take the tensor-core path
+ * and SSD_ERR_INVALID_ARG for invalid ones or a NULL `info`.  Host only; launches nothing.
+ */
+typedef struct {
+  int launches;  /* kernels per call (the call also clears a few bytes of workspace with a memset) */
+  int ctas;      /* CTAs of the walk */
+  int segments;  /* segments per sequence */
+} ssd_plan_info;
+ssd_status ssd_chunk_scan_plan_info(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                    int dstate, int ngroups, int chunk, ssd_dtype io,
+                                    const ssd_scan_options* opt, ssd_plan_info* info);
+
 /* The same operation forced onto the float32 SIMT kernels (any supported shape), with its
  * own workspace query.  Used as a second GPU reference and for float32 io. */
 size_t ssd_chunk_scan_simt_workspace_size(int64_t batch, int64_t seqlen, int nheads,
@@ -149,17 +199,17 @@ ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A
  * Scratch comes from one fixed array of SSD_NOALLOC_SCRATCH_BYTES (32 MiB) that the library
  * holds in every GPU that loads it, until the process exits.  The call allocates nothing.
  *   - Shapes: the tensor-core shapes only (io = SSD_BF16, headdim 64, dstate 128, an even
- *     number of heads per group).  The sequence is cut into as many segments as the array can
- *     hold states for (one float32 headdim x dstate state per batch row, segment and head);
- *     when batch * nheads states (32 KiB each) do not fit even with one segment, the call
- *     returns SSD_ERR_UNSUPPORTED before launching anything.  Other shapes also return
- *     SSD_ERR_UNSUPPORTED.
+ *     number of heads per group).  The array holds the walk's bookkeeping and one published
+ *     boundary state (64 KiB) per CTA, plus, where sequences are cut into segments, one float32
+ *     headdim x dstate state per batch row, segment and head; the call uses fewer CTAs when that
+ *     does not fit, and returns SSD_ERR_UNSUPPORTED before launching anything when even a
+ *     single CTA's plan does not.  Other shapes also return SSD_ERR_UNSUPPORTED.
  *   - The first call on each device looks up the array's device address (and configures the
  *     kernels) for that device; make that first call before any stream capture.
  *   - Every call on a device shares the one array.  Calls whose kernels overlap on the GPU
  *     (different streams without ordering, or several host threads) race on it and give wrong
- *     results: order them.  Nothing in the array needs to start at zero; each call writes every
- *     scratch value before it reads it.
+ *     results: order them.  Each call clears the part that must start at zero (the ticket and
+ *     the ready flags) and writes every other scratch value before it reads it.
  * Arguments, layouts and the result are exactly those of ssd_chunk_scan_fwd.
  */
 #define SSD_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -169,6 +219,38 @@ ssd_status ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, const floa
                                       int64_t batch, int64_t seqlen, int nheads, int headdim,
                                       int dstate, int ngroups, int chunk, ssd_dtype io,
                                       ssd_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Gradients of ssd_chunk_scan_fwd (training backward), for L = sum(dy * y) + sum(dfinal *
+ * final_state): the chain rule applied to the recurrence, in the same blocked form as the
+ * forward ("Mamba-2 (2024): SSM e attention sono la stessa cosa", "Il trucco a blocchi": masked
+ * quadratic forms inside each chunk; between chunks only the forward state entering each chunk
+ * and the adjoint carried into it from the right).  The pages give no gradient formulas; the
+ * all-at-once (parallel) form is the one used for training ("State Space Model"
+ * (book.paithon.it), "Un sistema che riassume il passato").
+ *   Inputs: x, dt, A, B, C, D, init_state exactly as given to the forward (D and init_state may
+ *           be NULL); dy [batch, seqlen, nheads, headdim] float32; dfinal [batch, nheads,
+ *           headdim, dstate] float32 or NULL (zero).
+ *   Outputs (float32, device, caller-owned, none overlapping an input or another output):
+ *           dx [batch, seqlen, nheads, headdim]; ddt [batch, seqlen, nheads]; dA [nheads];
+ *           dB, dC [batch, seqlen, ngroups, dstate] (summed over the heads of each group);
+ *           dD [nheads] or NULL (not written); dinit [batch, nheads, headdim, dstate] or NULL.
+ *   io: SSD_F32 or SSD_BF16 (x, B, C).  Float32 CUDA-core arithmetic throughout, chunks of 64
+ *   tokens; the result does not depend on the chunk.  Deterministic (fixed summation orders).
+ *   Supported: headdim * dstate small enough for one chunk's tiles in shared memory (headdim 64
+ *   with dstate 128, or smaller), batch * nheads <= 65535; else SSD_ERR_UNSUPPORTED.
+ *   workspace: ssd_chunk_scan_bwd_workspace_size() bytes, 256-byte aligned.
+ * Asynchronous on `stream`; argument errors are returned before any launch.
+ */
+size_t ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int nheads,
+                                         int headdim, int dstate, int ngroups, ssd_dtype io);
+ssd_status ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, const void* B,
+                              const void* C, const float* D, const float* init_state,
+                              const float* dy, const float* dfinal, float* dx, float* ddt,
+                              float* dA, float* dB, float* dC, float* dD, float* dinit,
+                              int64_t batch, int64_t seqlen, int nheads, int headdim, int dstate,
+                              int ngroups, ssd_dtype io, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* ssd_status_string(ssd_status s);
@@ -216,9 +298,9 @@ ssd_status ssd_state_pass(float* states, const float* decay, const float* init_s
                           int headdim, int dstate, cudaStream_t stream);
 
 /*
- * Steps either side of the layer inside a Mamba block ("Puntata 205 -- State Space Models e
- * Mamba" (aiperbabbani.it), "Da S4 a Mamba": every Mamba block wraps the selective SSM with a
- * short convolution and a SiLU gate).  silu(v) = v / (1 + exp(-v)).  Float32 arithmetic,
+ * Steps either side of the layer inside a Mamba block ("State Space Models (SSM)"
+ * (ultralytics.com glossary), section "Da S4 a Mamba": every Mamba block wraps the selective
+ * SSM with a short convolution and a SiLU gate).  silu(v) = v / (1 + exp(-v)).  Float32 arithmetic,
  * outputs rounded to nearest even in their dtype; asynchronous on `stream`; argument errors are
  * returned before any launch.
  *
@@ -244,8 +326,10 @@ ssd_status ssd_dt_softplus(const float* raw, const float* bias, float* dt, int64
 
 /* ssd_gate_silu: the output gate out[i] = y[i] * silu(z[i]) over n elements (y as the layer
  *   writes it, [batch, seqlen, nheads, headdim]).  y float32; z in z_dtype (SSD_BF16 or SSD_F32);
- *   out in out_dtype (SSD_F32 or z_dtype; out may equal y when float32).  n a multiple of 8
- *   (bf16 z) or 4 (f32 z) and all pointers 16-byte aligned, else SSD_ERR_UNSUPPORTED. */
+ *   out in out_dtype (SSD_F32 or z_dtype).  out may equal y only when out_dtype is SSD_F32 (a
+ *   narrower out in place would overwrite y elements before they are read: SSD_ERR_INVALID_ARG);
+ *   otherwise it must not overlap y or z.  n a multiple of 8 (bf16 z) or 4 (f32 z) and all
+ *   pointers 16-byte aligned, else SSD_ERR_UNSUPPORTED. */
 ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ssd_dtype z_dtype,
                          ssd_dtype out_dtype, cudaStream_t stream);
 

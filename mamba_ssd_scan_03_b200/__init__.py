@@ -24,7 +24,10 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
 # The symbols include/ssd.h declares (tests check that the library exports each one).
 EXPORTS = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_path", "ssd_chunk_scan_fwd",
            "ssd_chunk_scan_simt_workspace_size", "ssd_chunk_scan_fwd_simt", "ssd_step",
-           "ssd_chunk_scan_fwd_noalloc", "ssd_chunk_state_fwd", "ssd_state_pass",
+           "ssd_chunk_scan_fwd_noalloc", "ssd_chunk_scan_workspace_size_ex",
+           "ssd_chunk_scan_fwd_ex", "ssd_chunk_scan_plan_info",
+           "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd", "ssd_chunk_state_fwd",
+           "ssd_state_pass",
            "ssd_conv_silu", "ssd_dt_softplus", "ssd_gate_silu", "ssd_selective_scan_fwd",
            "ssd_status_string",
            "ssd_get_device_status", "ssd_version")
@@ -46,6 +49,17 @@ _SHAPE = [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32]  # batch .. chunk, io
 _SCAN = [_vp] * 9 + [_i64, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
 
 
+class PlanInfo(ctypes.Structure):
+    """ssd_plan_info: kernels per call, CTAs of the walk, segments per sequence."""
+    _fields_ = [("launches", ctypes.c_int), ("ctas", ctypes.c_int), ("segments", ctypes.c_int)]
+
+
+class ScanOptions(ctypes.Structure):
+    """ssd_scan_options: the walk's plan and wait limit (tests and tuning; zeros = defaults)."""
+    _fields_ = [("max_ctas", ctypes.c_int), ("plan", ctypes.c_int),
+                ("wait_limit_ns", ctypes.c_int64)]
+
+
 def load():
     """Load libssd.so (raises if it has not been built)."""
     global _lib
@@ -64,8 +78,19 @@ def load():
     for fn in (lib.ssd_chunk_scan_fwd, lib.ssd_chunk_scan_fwd_simt):
         fn.restype = _i32
         fn.argtypes = _SCAN
+    lib.ssd_chunk_scan_workspace_size_ex.restype = _sz
+    lib.ssd_chunk_scan_workspace_size_ex.argtypes = _SHAPE + [ctypes.POINTER(ScanOptions)]
+    lib.ssd_chunk_scan_plan_info.restype = _i32
+    lib.ssd_chunk_scan_plan_info.argtypes = _SHAPE + [ctypes.POINTER(ScanOptions),
+                                                      ctypes.POINTER(PlanInfo)]
+    lib.ssd_chunk_scan_fwd_ex.restype = _i32
+    lib.ssd_chunk_scan_fwd_ex.argtypes = _SCAN[:-1] + [ctypes.POINTER(ScanOptions), _vp]
     lib.ssd_chunk_scan_fwd_noalloc.restype = _i32
     lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 9 + [_i64, _i64] + [_i32] * 7 + [_vp]
+    lib.ssd_chunk_scan_bwd_workspace_size.restype = _sz
+    lib.ssd_chunk_scan_bwd_workspace_size.argtypes = [_i64, _i64] + [_i32] * 5
+    lib.ssd_chunk_scan_bwd.restype = _i32
+    lib.ssd_chunk_scan_bwd.argtypes = [_vp] * 16 + [_i64, _i64] + [_i32] * 5 + [_vp, _sz, _vp]
     lib.ssd_chunk_state_fwd.restype = _i32
     lib.ssd_chunk_state_fwd.argtypes = [_vp] * 7 + [_i64, _i64] + [_i32] * 6 + [_vp, _sz, _vp]
     lib.ssd_state_pass.restype = _i32
@@ -150,12 +175,23 @@ def workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io=SS
     return fn(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io)
 
 
+def plan_info(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io=SSD_BF16, max_ctas=0,
+              plan=0):
+    """The tensor-core plan of a shape: dict(launches, ctas, segments)."""
+    info = PlanInfo()
+    opts = ScanOptions(int(max_ctas), int(plan), 0)
+    rc = load().ssd_chunk_scan_plan_info(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
+                                         io, ctypes.byref(opts), ctypes.byref(info))
+    _check(rc, "ssd_chunk_scan_plan_info")
+    return dict(launches=info.launches, ctas=info.ctas, segments=info.segments)
+
+
 def path(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io=SSD_BF16):
     return load().ssd_chunk_scan_path(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io)
 
 
 def _scan(entry, simt, x, dt, A, B, C, D, chunk, init_state, want_final, workspace, out,
-          final_out, y_dtype):
+          final_out, y_dtype, opts=None):
     lib = load()
     _need(x, "x")
     dev = x.device
@@ -176,15 +212,19 @@ def _scan(entry, simt, x, dt, A, B, C, D, chunk, init_state, want_final, workspa
         fin = final_out if final_out is not None else torch.empty(
             (Bt, H, P, N), dtype=torch.float32, device=dev)
         _need(fin, "final_state", torch.float32, (Bt, H, P, N), dev)
-    need = workspace_size(Bt, L, H, P, N, G, Q, io, simt=simt)
+    if opts is None:
+        need = workspace_size(Bt, L, H, P, N, G, Q, io, simt=simt)
+    else:
+        need = lib.ssd_chunk_scan_workspace_size_ex(Bt, L, H, P, N, G, Q, io, ctypes.byref(opts))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     _need(workspace, "workspace", torch.uint8, device=dev)
+    extra = () if opts is None else (ctypes.byref(opts),)
     with torch.cuda.device(dev):
         rc = entry(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
                    _ptr(y), _ptr(fin), Bt, L, H, P, N, G, Q, io, _code(y_dtype), _ptr(workspace),
-                   workspace.numel(), _stream(dev))
-    _check(rc, "ssd_chunk_scan_fwd_simt" if simt else "ssd_chunk_scan_fwd")
+                   workspace.numel(), *extra, _stream(dev))
+    _check(rc, getattr(entry, "__name__", "ssd_chunk_scan_fwd"))
     return y, fin
 
 
@@ -195,6 +235,16 @@ def chunk_scan_fwd(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
     dtype).  Returns (y, final_state)."""
     return _scan(load().ssd_chunk_scan_fwd, False, x, dt, A, B, C, D, chunk, init_state,
                  want_final, workspace, out, final_out, y_dtype)
+
+
+def chunk_scan_fwd_ex(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
+                      workspace=None, out=None, final_out=None, y_dtype=torch.float32,
+                      max_ctas=0, plan=0, wait_limit_ns=0):
+    """ssd_chunk_scan_fwd_ex: the tensor-core scan with its plan (max_ctas, plan 0 auto / 1
+    whole sequences / 2 segments) and the kernels' wait limit set by the caller (tests)."""
+    opts = ScanOptions(int(max_ctas), int(plan), int(wait_limit_ns))
+    return _scan(load().ssd_chunk_scan_fwd_ex, False, x, dt, A, B, C, D, chunk, init_state,
+                 want_final, workspace, out, final_out, y_dtype, opts)
 
 
 def chunk_scan_fwd_simt(x, dt, A, B, C, D, chunk, init_state=None, want_final=True,
@@ -238,6 +288,46 @@ def chunk_scan_fwd_noalloc(x, dt, A, B, C, D, chunk, init_state=None, want_final
             _ptr(fin), Bt, L, H, P, N, G, Q, io, _code(y_dtype), _stream(dev))
     _check(rc, "ssd_chunk_scan_fwd_noalloc")
     return y, fin
+
+
+def chunk_scan_bwd(x, dt, A, B, C, D, dy, init_state=None, dfinal=None, workspace=None):
+    """Gradients of L = sum(dy * y) + sum(dfinal * final_state) through the chunked scan.
+    Inputs as for chunk_scan_fwd; dy [B,L,H,P] f32; dfinal [B,H,P,N] f32 or None.  Returns a
+    dict of float32 tensors: x, dt, A, B, C, D, init (the gradient of each input)."""
+    lib = load()
+    _need(x, "x")
+    dev = x.device
+    Bt, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = _io(x)
+    _need(B, "B", x.dtype, (Bt, L, G, N), dev)
+    _need(C, "C", x.dtype, (Bt, L, G, N), dev)
+    _need(dt, "dt", torch.float32, (Bt, L, H), dev)
+    _need(A, "A", torch.float32, (H,), dev)
+    _need(dy, "dy", torch.float32, (Bt, L, H, P), dev)
+    if D is not None:
+        _need(D, "D", torch.float32, (H,), dev)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (Bt, H, P, N), dev)
+    if dfinal is not None:
+        _need(dfinal, "dfinal", torch.float32, (Bt, H, P, N), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"x": torch.empty((Bt, L, H, P), **f32), "dt": torch.empty((Bt, L, H), **f32),
+         "A": torch.empty((H,), **f32), "B": torch.empty((Bt, L, G, N), **f32),
+         "C": torch.empty((Bt, L, G, N), **f32), "D": torch.empty((H,), **f32),
+         "init": torch.empty((Bt, H, P, N), **f32)}
+    need = lib.ssd_chunk_scan_bwd_workspace_size(Bt, L, H, P, N, G, io)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.ssd_chunk_scan_bwd(
+            _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(dy),
+            _ptr(dfinal), _ptr(g["x"]), _ptr(g["dt"]), _ptr(g["A"]), _ptr(g["B"]), _ptr(g["C"]),
+            _ptr(g["D"]), _ptr(g["init"]), Bt, L, H, P, N, G, io, _ptr(workspace),
+            workspace.numel(), _stream(dev))
+    _check(rc, "ssd_chunk_scan_bwd")
+    return g
 
 
 def chunk_state_fwd(x, dt, A, B, chunk, init_state=None, workspace=None, final_out=None):

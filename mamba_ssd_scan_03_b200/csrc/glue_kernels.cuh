@@ -1,7 +1,7 @@
 // glue_kernels.cuh -- the steps either side of the SSD layer inside a Mamba block: a short
 // causal depthwise convolution with SiLU on the layer's inputs, the step size dt = softplus(raw
-// + bias), and the SiLU gate on the output.  "Puntata 205 -- State Space Models e Mamba"
-// (aiperbabbani.it), "Da S4 a Mamba": every Mamba block wraps the selective SSM with a short
+// + bias), and the SiLU gate on the output.  "State Space Models (SSM)" (ultralytics.com
+// glossary), section "Da S4 a Mamba": every Mamba block wraps the selective SSM with a short
 // convolution and a SiLU gate.  All three stream HBM once; float32 arithmetic.
 #pragma once
 #include "ssd_common.cuh"

@@ -10,6 +10,7 @@
 #include <mutex>
 #include <utility>
 
+#include "bwd_kernels.cuh"
 #include "glue_kernels.cuh"
 #include "pass_kernels.cuh"
 #include "selective_kernels.cuh"
@@ -21,8 +22,6 @@
 namespace {
 
 using ssd::tc::Seg;
-
-constexpr int kUnitsTarget = 8 * 148;  // tensor-core grids: ~8 CTAs per SM of a B200
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -71,14 +70,40 @@ bool tc_shape_ok(const Shape& s) {
          s.seqlen <= (int64_t(1) << 30) && s.batch <= (int64_t(1) << 20);
 }
 
+// Streaming multiprocessors of the current device (148 on a B200; also the answer when no
+// device can be queried, so that workspace queries work on a host without a GPU).
+int sm_count() {
+  constexpr int kMaxDev = 256;
+  static std::mutex mu;
+  static int cache[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return 148;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Segments of the summary-only pass (ssd_chunk_state_fwd): enough (batch, segment, head pair)
+// units to give every SM about eight.
 Seg tc_segments(const Shape& s) {
   Seg sg;
   sg.nblk = int((s.seqlen + ssd::tc::kBlk - 1) / ssd::tc::kBlk);
   const int64_t pairs = s.batch * (s.nheads / 2);
-  int nseg = int(std::min<int64_t>(
-      sg.nblk, std::max<int64_t>(1, (kUnitsTarget + pairs - 1) / pairs)));
+  const int64_t target = 8 * int64_t(sm_count());
+  int nseg = int(std::min<int64_t>(sg.nblk, std::max<int64_t>(1, (target + pairs - 1) / pairs)));
   sg.seg_blks = (sg.nblk + nseg - 1) / nseg;
   sg.nseg = (sg.nblk + sg.seg_blks - 1) / sg.seg_blks;
+  sg.useg = sg.nseg;
   return sg;
 }
 
@@ -100,7 +125,96 @@ SegScratch seg_scratch(const Shape& s, const Seg& sg, void* base) {
   r.decay = reinterpret_cast<float*>(p);
   return r;
 }
-size_t tc_workspace(const Shape& s) { return seg_scratch_bytes(s, tc_segments(s)); }
+
+// Options of the scan entry points (the defaults, all zero, are what ssd_chunk_scan_fwd uses).
+struct ScanOpts {
+  int max_ctas = 0;        // cap on the walk's CTAs (0: one per SM)
+  int plan = 0;            // 0 automatic, 1 whole sequences, 2 segments with summaries
+  int64_t wait_ns = 0;     // limit of every bounded wait in the walk (0: 2 s; -1: no waiting)
+};
+
+// The walk of ssd_chunk_scan_fwd on the tensor cores.  Whole sequences (no summary pass) when
+// there are about as many (batch row, head pair) sequences as CTAs; otherwise each sequence is
+// cut into segments whose entering states seg_state + seg_pass provide, so that the CTAs share
+// the work evenly.
+struct TcPlan {
+  ssd::tc::WalkPlan w;
+  Seg sg;  // sg.nseg > 1: seg_state over the first nseg - 1 segments and seg_pass run first
+};
+bool make_tc_plan(const Shape& s, const ScanOpts& o, TcPlan* out) {
+  const int nsm = sm_count();
+  const int cap = o.max_ctas > 0 ? std::min(nsm, o.max_ctas) : nsm;
+  const int64_t nblk = (s.seqlen + ssd::tc::kBlk - 1) / ssd::tc::kBlk;
+  const int64_t npair = s.nheads / 2, nseqs = s.batch * npair;
+  if (nblk > (int64_t(1) << 30) || nseqs * nblk > (int64_t(1) << 40)) return false;
+  const bool whole =
+      nblk == 1 || o.plan == 1 || (o.plan == 0 && nseqs * 5 >= int64_t(cap) * 4);
+  int64_t nseg = whole ? 1 : std::min<int64_t>(nblk, std::max<int64_t>(2, (cap + nseqs - 1) / nseqs));
+  const int64_t seg_blks = (nblk + nseg - 1) / nseg;
+  nseg = (nblk + seg_blks - 1) / seg_blks;
+  const int64_t total = nseqs * nblk;
+  // every range at least one segment long (a range inside one segment would wait on a chain of
+  // ranges) and at most kMaxItems - 2 segments long (its items fit the kernel's list)
+  int64_t nct = std::min<int64_t>(cap, nseqs * nseg);
+  const int64_t per = seg_blks * (ssd::tc::kMaxItems - 2);
+  nct = std::max<int64_t>(nct, (total + per - 1) / per);
+  while (nct > 1 && total / nct < seg_blks) --nct;
+  if ((total + nct - 1) / nct > per || nct > (int64_t(1) << 20)) return false;
+  TcPlan p;
+  p.w.total = total;
+  p.w.nblk = int(nblk);
+  p.w.seg_blks = int(seg_blks);
+  p.w.nseg = int(nseg);
+  p.w.npair = int(npair);
+  p.w.nct = int(nct);
+  p.w.wait_ns = o.wait_ns > 0 ? uint64_t(o.wait_ns) : (o.wait_ns < 0 ? 0ull : 2000000000ull);
+  p.sg.nblk = int(nblk);
+  p.sg.seg_blks = int(seg_blks);
+  p.sg.nseg = int(nseg);
+  p.sg.useg = int(nseg) - 1;
+  *out = p;
+  return true;
+}
+
+// Workspace of the walk: [ticket + one ready flag per range] | [one published state per range,
+// two heads] | (segments) [entering state per (batch, segment, head)] [log2-decay of each].
+struct WalkScratch {
+  unsigned* ticket;
+  int* flags;
+  float* slots;
+  float* states;
+  float* decay;
+  size_t header_bytes;
+};
+size_t walk_bytes(const Shape& s, const TcPlan& p) {
+  size_t n = align256(size_t(p.w.nct + 1) * 4) +
+             align256(size_t(p.w.nct) * ssd::tc::kSlotFloats * sizeof(float));
+  if (p.sg.nseg > 1) n += seg_scratch_bytes(s, p.sg);
+  return n;
+}
+WalkScratch walk_scratch(const Shape& s, const TcPlan& p, void* base) {
+  char* c = static_cast<char*>(base);
+  WalkScratch w{};
+  w.header_bytes = align256(size_t(p.w.nct + 1) * 4);
+  w.ticket = reinterpret_cast<unsigned*>(c);
+  w.flags = reinterpret_cast<int*>(c) + 1;
+  c += w.header_bytes;
+  w.slots = reinterpret_cast<float*>(c);
+  c += align256(size_t(p.w.nct) * ssd::tc::kSlotFloats * sizeof(float));
+  if (p.sg.nseg > 1) {
+    const SegScratch sc = seg_scratch(s, p.sg, c);
+    w.states = sc.states;
+    w.decay = sc.decay;
+  }
+  return w;
+}
+
+// ssd_chunk_scan_fwd and ssd_chunk_state_fwd share one workspace query: the larger need.
+size_t tc_workspace(const Shape& s, const ScanOpts& o = ScanOpts()) {
+  TcPlan p;
+  const size_t walk = make_tc_plan(s, o, &p) ? walk_bytes(s, p) : 0;
+  return std::max(walk, seg_scratch_bytes(s, tc_segments(s)));
+}
 
 size_t simt_workspace(const Shape& s) {
   const int64_t nchunks = (s.seqlen + s.chunk - 1) / s.chunk;
@@ -198,10 +312,10 @@ ssd_status set_smem_attrs() {
   std::lock_guard<std::mutex> lock(mu);
   if (done[dev] == 0) {
     bool ok = true;
-    ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<float>,
+    ok &= cudaFuncSetAttribute(ssd::tc::scan_walk_kernel<float>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
           cudaSuccess;
-    ok &= cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<__nv_bfloat16>,
+    ok &= cudaFuncSetAttribute(ssd::tc::scan_walk_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
           cudaSuccess;
     // the selective scan runs ~17 one-warp CTAs per SM: ask for the largest shared-memory
@@ -214,6 +328,10 @@ ssd_status set_smem_attrs() {
     ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem<2>)) ==
           cudaSuccess;
+    for (auto f : {(const void*)ssd::bwd::chunk_bwd_kernel<float>,
+                   (const void*)ssd::bwd::chunk_bwd_kernel<__nv_bfloat16>})
+      ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) ==
+            cudaSuccess;
     for (auto f : {(const void*)ssd::simt::chunk_out_kernel<float, float>,
                    (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16, float>,
                    (const void*)ssd::simt::chunk_out_kernel<__nv_bfloat16, __nv_bfloat16>,
@@ -257,9 +375,10 @@ ssd_status validate_scan(const Shape& s, const ScanArgs& a, size_t need) {
   const size_t nbc = size_t(s.batch) * s.seqlen * s.ngroups * s.dstate * es;
   const size_t ndt = size_t(s.batch) * s.seqlen * s.nheads * 4;
   const size_t nst = size_t(s.batch) * s.nheads * s.headdim * s.dstate * 4;
+  const size_t nh = size_t(s.nheads) * 4;
   if (overlaps(a.y, ny, a.x, nx) || overlaps(a.y, ny, a.B, nbc) || overlaps(a.y, ny, a.C, nbc) ||
-      overlaps(a.y, ny, a.dt, ndt) || overlaps(a.y, ny, a.init, nst) ||
-      overlaps(a.y, ny, a.fin, nst))
+      overlaps(a.y, ny, a.dt, ndt) || overlaps(a.y, ny, a.A, nh) || overlaps(a.y, ny, a.D, nh) ||
+      overlaps(a.y, ny, a.init, nst) || overlaps(a.y, ny, a.fin, nst))
     return SSD_ERR_INVALID_ARG;
   if (a.fin && a.fin != a.init &&
       (overlaps(a.fin, nst, a.init, nst) || overlaps(a.fin, nst, a.x, nx) ||
@@ -305,50 +424,78 @@ ssd_status run_simt(const Shape& s, const ScanArgs& a, bool with_output = true) 
   return launched();
 }
 
-// with_output = false: the states only (seg_state and seg_pass), for ssd_chunk_state_fwd
-ssd_status run_tc_segments(const Shape& s, const ScanArgs& a, const Seg& sg, void* scratch,
-                           bool with_output = true) {
-  const SegScratch w = seg_scratch(s, sg, scratch);
-  CUtensorMap mx, mb, mc, my;
-  const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
-  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch))
-    return SSD_ERR_CUDA;
-  if (with_output && (!make_map(&mc, a.C, GN, s.seqlen, s.batch) ||
-                      !make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32)))
-    return SSD_ERR_CUDA;
+// seg_state over the first sg.useg segments of every sequence (persistent, one CTA per SM).
+ssd_status launch_seg_state(const Shape& s, const ScanArgs& a, const Seg& sg, const CUtensorMap& mx,
+                            const CUtensorMap& mb, float* states, float* decay) {
   const int hpg = s.nheads / s.ngroups;
-  const unsigned grid = unsigned(s.batch * sg.nseg * (s.nheads / 2));
-  int dev = 0, nsm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return SSD_ERR_CUDA;
+  const int64_t units = s.batch * int64_t(sg.useg) * (s.nheads / 2);
+  if (units <= 0) return SSD_OK;
   CUtensorMap mdt;
   std::memset(&mdt, 0, sizeof mdt);
   const int dt_tma = make_dt_map(&mdt, a.dt, s.batch, s.seqlen, s.nheads) ? 1 : 0;
   // two heads per unit: four (one B tile for four heads) measured slower at the 2.7B shape
   // (two 96 KB stages instead of three of 64 KB, and half as many units to balance over SMs)
-  ssd::tc::seg_state_kernel<2><<<std::min<unsigned>(grid, unsigned(nsm)),
+  ssd::tc::seg_state_kernel<2><<<unsigned(std::min<int64_t>(units, sm_count())),
                                  ssd::tc::SegCfg<2>::kThreads, kSegSmem<2>, a.stream>>>(
-      mx, mb, mdt, dt_tma, a.dt, a.A, w.states, w.decay, s.seqlen, s.nheads, hpg, sg,
-      int(grid));
-  if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  const int64_t nvec = s.batch * s.nheads * int64_t(64) * 128 / 4;
-  ssd::tc::seg_pass_kernel<<<unsigned((nvec + ssd::tc::kPassThreads - 1) / ssd::tc::kPassThreads),
-                             ssd::tc::kPassThreads, 0, a.stream>>>(
-      w.states, w.decay, a.init, a.fin, int(s.batch), s.nheads, sg.nseg);
-  if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  if (!with_output) return SSD_OK;
-  if (a.ydt == SSD_F32)
-    ssd::tc::chunk_out_kernel<float><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
-        mx, mb, mc, my, a.dt, a.A, a.D, w.states, s.seqlen, s.nheads, hpg, sg);
-  else
-    ssd::tc::chunk_out_kernel<__nv_bfloat16><<<grid, ssd::tc::kOutThreads, kTcSmem, a.stream>>>(
-        mx, mb, mc, my, a.dt, a.A, a.D, w.states, s.seqlen, s.nheads, hpg, sg);
+      mx, mb, mdt, dt_tma, a.dt, a.A, states, decay, s.seqlen, s.nheads, hpg, sg, int(units));
   return launched();
 }
 
-ssd_status run_tc(const Shape& s, const ScanArgs& a) {
-  return run_tc_segments(s, a, tc_segments(s), a.ws);
+ssd_status launch_seg_pass(const Shape& s, const ScanArgs& a, const Seg& sg, float* states,
+                           const float* decay, float* fin) {
+  const int64_t nvec = s.batch * s.nheads * int64_t(64) * 128 / 4;
+  ssd::tc::seg_pass_kernel<<<unsigned((nvec + ssd::tc::kPassThreads - 1) / ssd::tc::kPassThreads),
+                             ssd::tc::kPassThreads, 0, a.stream>>>(
+      states, decay, a.init, fin, int(s.batch), s.nheads, sg.nseg, sg.useg);
+  return launched();
+}
+
+// The states only (seg_state over every segment, seg_pass with the final state), for
+// ssd_chunk_state_fwd.
+ssd_status run_tc_state(const Shape& s, const ScanArgs& a, void* scratch) {
+  const Seg sg = tc_segments(s);
+  const SegScratch w = seg_scratch(s, sg, scratch);
+  CUtensorMap mx, mb;
+  const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
+  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch))
+    return SSD_ERR_CUDA;
+  ssd_status st = launch_seg_state(s, a, sg, mx, mb, w.states, w.decay);
+  if (st != SSD_OK) return st;
+  return launch_seg_pass(s, a, sg, w.states, w.decay, a.fin);
+}
+
+// The scan: (segments only) seg_state + seg_pass, then the walk.
+ssd_status run_tc_walk(const Shape& s, const ScanArgs& a, const TcPlan& p, void* scratch) {
+  const WalkScratch w = walk_scratch(s, p, scratch);
+  CUtensorMap mx, mb, mc, my;
+  const uint64_t HP = uint64_t(s.nheads) * 64, GN = uint64_t(s.ngroups) * 128;
+  if (!make_map(&mx, a.x, HP, s.seqlen, s.batch) || !make_map(&mb, a.B, GN, s.seqlen, s.batch) ||
+      !make_map(&mc, a.C, GN, s.seqlen, s.batch) ||
+      !make_map(&my, a.y, HP, s.seqlen, s.batch, a.ydt == SSD_F32))
+    return SSD_ERR_CUDA;
+  // the ticket and the ready flags start at zero every call
+  if (cudaMemsetAsync(w.ticket, 0, w.header_bytes, a.stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SSD_ERR_CUDA;
+  }
+  if (p.sg.nseg > 1) {
+    ssd_status st = launch_seg_state(s, a, p.sg, mx, mb, w.states, w.decay);
+    if (st != SSD_OK) return st;
+    st = launch_seg_pass(s, a, p.sg, w.states, w.decay, nullptr);
+    if (st != SSD_OK) return st;
+  }
+  const int hpg = s.nheads / s.ngroups;
+  if (a.ydt == SSD_F32)
+    ssd::tc::scan_walk_kernel<float><<<unsigned(p.w.nct), ssd::tc::kWalkThreads, kTcSmem,
+                                       a.stream>>>(
+        mx, mb, mc, my, a.dt, a.A, a.D, a.init, w.states, a.fin, w.slots, w.flags, w.ticket,
+        s.seqlen, s.nheads, hpg, p.w);
+  else
+    ssd::tc::scan_walk_kernel<__nv_bfloat16><<<unsigned(p.w.nct), ssd::tc::kWalkThreads, kTcSmem,
+                                               a.stream>>>(
+        mx, mb, mc, my, a.dt, a.A, a.D, a.init, w.states, a.fin, w.slots, w.flags, w.ticket,
+        s.seqlen, s.nheads, hpg, p.w);
+  return launched();
 }
 
 ssd_status run_simt_any(const Shape& s, const ScanArgs& a) {
@@ -387,6 +534,83 @@ ssd_status validate_state(const Shape& s, const ScanArgs& a, float* total_decay,
       return SSD_ERR_INVALID_ARG;
   }
   return SSD_OK;
+}
+
+// ---- backward ---------------------------------------------------------------------------
+// Workspace: cs [B, H, nc, kQ] | forward entering states [B, nc, H, P, N] | adjoints (same) |
+// per-head dB, dC rows [B, L, H, N] each | dA, dD partials [B, nc, H] each.
+size_t bwd_workspace(const Shape& s) {
+  const int64_t nc = (s.seqlen + ssd::bwd::kQ - 1) / ssd::bwd::kQ;
+  const size_t st = size_t(s.batch) * nc * s.nheads * size_t(s.headdim) * s.dstate * 4;
+  const size_t rows = size_t(s.batch) * s.seqlen * s.nheads * size_t(s.dstate) * 4;
+  const size_t part = size_t(s.batch) * nc * s.nheads * 4;
+  return align256(size_t(s.batch) * s.nheads * nc * ssd::bwd::kQ * 4) + 2 * align256(st) +
+         2 * align256(rows) + 2 * align256(part);
+}
+
+bool bwd_supported(const Shape& s) {
+  const size_t smem = ssd::bwd::BwdSmem::floats(s.headdim, s.dstate) * sizeof(float);
+  return smem <= 227 * 1024 && s.batch * s.nheads <= 65535 &&
+         (s.seqlen + ssd::bwd::kQ - 1) / ssd::bwd::kQ <= (int64_t(1) << 30);
+}
+
+template <typename T>
+ssd_status run_bwd(const Shape& s, const ScanArgs& a, const float* dy, const float* dfinal,
+                   float* dx, float* ddt, float* dA, float* dB, float* dC, float* dD,
+                   float* dinit) {
+  namespace bw = ssd::bwd;
+  const int64_t nc = (s.seqlen + bw::kQ - 1) / bw::kQ;
+  const size_t st = size_t(s.batch) * nc * s.nheads * size_t(s.headdim) * s.dstate * 4;
+  const size_t rows = size_t(s.batch) * s.seqlen * s.nheads * size_t(s.dstate) * 4;
+  const size_t part = size_t(s.batch) * nc * s.nheads * 4;
+  char* w = static_cast<char*>(a.ws);
+  float* cs = reinterpret_cast<float*>(w);
+  w += align256(size_t(s.batch) * s.nheads * nc * bw::kQ * 4);
+  float* hst = reinterpret_cast<float*>(w);
+  w += align256(st);
+  float* adj = reinterpret_cast<float*>(w);
+  w += align256(st);
+  float* dbh = reinterpret_cast<float*>(w);
+  w += align256(rows);
+  float* dch = reinterpret_cast<float*>(w);
+  w += align256(rows);
+  float* dA_part = reinterpret_cast<float*>(w);
+  w += align256(part);
+  float* dD_part = reinterpret_cast<float*>(w);
+  const dim3 grid(unsigned(nc), unsigned(s.batch * s.nheads));
+  const int P = s.headdim, N = s.dstate;
+  // forward: within-chunk cumsums, chunk states, and the state entering every chunk
+  ssd::simt::cumsum_kernel<<<grid, bw::kQ, 0, a.stream>>>(a.dt, a.A, cs, s.seqlen, s.nheads,
+                                                          bw::kQ, int(nc));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  ssd::simt::chunk_state_kernel<T><<<grid, 256, 16 * size_t(P + N) * sizeof(float), a.stream>>>(
+      static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), cs, hst, s.seqlen, s.nheads,
+      P, N, s.ngroups, bw::kQ, int(nc));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const int64_t nel = s.batch * s.nheads * int64_t(P) * N;
+  ssd::simt::state_pass_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
+      hst, cs, a.init, nullptr, s.batch, s.nheads, P, N, bw::kQ, int(nc));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  // backward: adjoint summaries, the adjoint entering every chunk from the right, then chunks
+  bw::adj_state_kernel<T><<<grid, bw::kThreads, 16 * size_t(P + N) * sizeof(float), a.stream>>>(
+      dy, static_cast<const T*>(a.C), cs, adj, s.seqlen, s.nheads, P, N, s.ngroups, int(nc));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  bw::adj_pass_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
+      adj, cs, dfinal, dinit, s.batch, s.nheads, P, N, int(nc));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  bw::chunk_bwd_kernel<T><<<grid, bw::kThreads, bw::BwdSmem::floats(P, N) * sizeof(float),
+                            a.stream>>>(
+      static_cast<const T*>(a.x), a.dt, a.A, static_cast<const T*>(a.B),
+      static_cast<const T*>(a.C), a.D, dy, cs, hst, adj, dx, ddt, dbh, dch, dA_part, dD_part,
+      s.seqlen, s.nheads, P, N, s.ngroups, int(nc));
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  const int64_t ngn = s.batch * s.seqlen * s.ngroups * int64_t(N);
+  bw::group_sum_kernel<float><<<unsigned((ngn + 255) / 256), 256, 0, a.stream>>>(
+      dbh, dch, dB, dC, s.batch * s.seqlen, s.nheads, s.ngroups, N);
+  if (launched() != SSD_OK) return SSD_ERR_CUDA;
+  bw::head_sum_kernel<<<unsigned((s.nheads + 127) / 128), 128, 0, a.stream>>>(
+      dA_part, dD_part, dA, dD, s.batch * nc, s.nheads);
+  return launched();
 }
 
 }  // namespace
@@ -428,14 +652,80 @@ ssd_status ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, co
   if (st != SSD_OK) return st;
   const bool tc = tc_shape_ok(s);
   if (!tc && !simt_supported(s)) return SSD_ERR_UNSUPPORTED;
+  TcPlan plan;
+  if (tc && !make_tc_plan(s, ScanOpts(), &plan)) return SSD_ERR_UNSUPPORTED;
   st = validate_scan(s, a, tc ? tc_workspace(s) : simt_workspace(s));
   if (st != SSD_OK) return st;
   if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
   if (tc) {
     if (!tc_pointers_ok(a)) return SSD_ERR_UNSUPPORTED;
-    return run_tc(s, a);
+    return run_tc_walk(s, a, plan, a.ws);
   }
   return run_simt_any(s, a);
+}
+
+size_t ssd_chunk_scan_workspace_size_ex(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                        int dstate, int ngroups, int chunk, ssd_dtype io,
+                                        const ssd_scan_options* opt) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  if (check_shape(s) != SSD_OK || !tc_shape_ok(s)) return 0;
+  ScanOpts o;
+  if (opt) {
+    o.max_ctas = opt->max_ctas;
+    o.plan = opt->plan;
+    o.wait_ns = opt->wait_limit_ns;
+  }
+  return tc_workspace(s, o);
+}
+
+ssd_status ssd_chunk_scan_plan_info(int64_t batch, int64_t seqlen, int nheads, int headdim,
+                                    int dstate, int ngroups, int chunk, ssd_dtype io,
+                                    const ssd_scan_options* opt, ssd_plan_info* info) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  if (!info || check_shape(s) != SSD_OK) return SSD_ERR_INVALID_ARG;
+  if (!tc_shape_ok(s)) return SSD_ERR_UNSUPPORTED;
+  ScanOpts o;
+  if (opt) {
+    o.max_ctas = opt->max_ctas;
+    o.plan = opt->plan;
+    o.wait_ns = opt->wait_limit_ns;
+  }
+  TcPlan p;
+  if (!make_tc_plan(s, o, &p)) return SSD_ERR_UNSUPPORTED;
+  info->launches = p.sg.nseg > 1 ? 3 : 1;
+  info->ctas = p.w.nct;
+  info->segments = p.w.nseg;
+  return SSD_OK;
+}
+
+ssd_status ssd_chunk_scan_fwd_ex(const void* x, const float* dt, const float* A, const void* B,
+                                 const void* C, const float* D, const float* init_state,
+                                 void* y, float* final_state, int64_t batch, int64_t seqlen,
+                                 int nheads, int headdim, int dstate, int ngroups, int chunk,
+                                 ssd_dtype io, ssd_dtype y_dtype, void* workspace,
+                                 size_t workspace_bytes, const ssd_scan_options* opt,
+                                 cudaStream_t stream) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, chunk, io};
+  const ScanArgs a{y_dtype, x, B, C, dt, A, D, init_state, y, final_state, workspace,
+                   workspace_bytes, stream};
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  ScanOpts o;
+  if (opt) {
+    if (opt->max_ctas < 0 || opt->plan < 0 || opt->plan > 2 || opt->wait_limit_ns < -1)
+      return SSD_ERR_INVALID_ARG;
+    o.max_ctas = opt->max_ctas;
+    o.plan = opt->plan;
+    o.wait_ns = opt->wait_limit_ns;
+  }
+  if (!tc_shape_ok(s)) return SSD_ERR_UNSUPPORTED;
+  TcPlan plan;
+  if (!make_tc_plan(s, o, &plan)) return SSD_ERR_UNSUPPORTED;
+  st = validate_scan(s, a, tc_workspace(s, o));
+  if (st != SSD_OK) return st;
+  if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
+  if (!tc_pointers_ok(a)) return SSD_ERR_UNSUPPORTED;
+  return run_tc_walk(s, a, plan, a.ws);
 }
 
 ssd_status ssd_chunk_scan_fwd_simt(const void* x, const float* dt, const float* A,
@@ -475,9 +765,12 @@ ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A
   const size_t nx = size_t(batch) * nheads * headdim * es;
   const size_t ny = size_t(batch) * nheads * headdim * (y_dtype == SSD_BF16 ? 2 : 4);
   const size_t nbc = size_t(batch) * ngroups * dstate * es;
+  const size_t ndt = size_t(batch) * nheads * 4, nh = size_t(nheads) * 4;
   if (overlaps(y, ny, state, nst) || overlaps(y, ny, x, nx) || overlaps(y, ny, B, nbc) ||
-      overlaps(y, ny, C, nbc) || overlaps(state, nst, x, nx) || overlaps(state, nst, B, nbc) ||
-      overlaps(state, nst, C, nbc))
+      overlaps(y, ny, C, nbc) || overlaps(y, ny, dt, ndt) || overlaps(y, ny, A, nh) ||
+      overlaps(y, ny, D, nh) || overlaps(state, nst, x, nx) || overlaps(state, nst, B, nbc) ||
+      overlaps(state, nst, C, nbc) || overlaps(state, nst, dt, ndt) ||
+      overlaps(state, nst, A, nh) || overlaps(state, nst, D, nh))
     return SSD_ERR_INVALID_ARG;
   const int hpg = nheads / ngroups;
   const unsigned grid = unsigned(batch * nheads);
@@ -515,6 +808,64 @@ ssd_status ssd_step(float* state, const void* x, const float* dt, const float* A
   return launched();
 }
 
+size_t ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int nheads,
+                                         int headdim, int dstate, int ngroups, ssd_dtype io) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, 64, io};
+  if (check_shape(s) != SSD_OK || !bwd_supported(s)) return 0;
+  return bwd_workspace(s);
+}
+
+ssd_status ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, const void* B,
+                              const void* C, const float* D, const float* init_state,
+                              const float* dy, const float* dfinal, float* dx, float* ddt,
+                              float* dA, float* dB, float* dC, float* dD, float* dinit,
+                              int64_t batch, int64_t seqlen, int nheads, int headdim, int dstate,
+                              int ngroups, ssd_dtype io, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  const Shape s{batch, seqlen, nheads, headdim, dstate, ngroups, 64, io};
+  ssd_status st = check_shape(s);
+  if (st != SSD_OK) return st;
+  if (!bwd_supported(s)) return SSD_ERR_UNSUPPORTED;
+  for (const void* p : {x, (const void*)dt, (const void*)A, B, C, (const void*)dy, (const void*)dx,
+                        (const void*)ddt, (const void*)dA, (const void*)dB, (const void*)dC})
+    if (!is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)D, (const void*)init_state, (const void*)dfinal,
+                        (const void*)dD, (const void*)dinit})
+    if (p && !is_device_ptr(p)) return SSD_ERR_INVALID_ARG;
+  const size_t es = io == SSD_BF16 ? 2 : 4;
+  const size_t ntok = size_t(batch) * seqlen;
+  const size_t nx = ntok * nheads * headdim * es, nxf = ntok * nheads * headdim * 4;
+  const size_t ndt = ntok * nheads * 4, nbc = ntok * ngroups * dstate * es;
+  const size_t nbcf = ntok * ngroups * dstate * 4, nh = size_t(nheads) * 4;
+  const size_t nst = size_t(batch) * nheads * headdim * dstate * 4;
+  const std::pair<const void*, size_t> ins[] = {{x, nx}, {dt, ndt}, {A, nh}, {B, nbc}, {C, nbc},
+                                                {D, nh}, {init_state, nst}, {dy, nxf},
+                                                {dfinal, nst}};
+  const std::pair<const void*, size_t> outs[] = {{dx, nxf}, {ddt, ndt}, {dA, nh}, {dB, nbcf},
+                                                 {dC, nbcf}, {dD, nh}, {dinit, nst}};
+  for (const auto& o : outs) {
+    for (const auto& i : ins)
+      if (overlaps(o.first, o.second, i.first, i.second)) return SSD_ERR_INVALID_ARG;
+    for (const auto& o2 : outs)
+      if (&o2 != &o && overlaps(o.first, o.second, o2.first, o2.second))
+        return SSD_ERR_INVALID_ARG;
+  }
+  const size_t need = bwd_workspace(s);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      !is_device_ptr(workspace))
+    return SSD_ERR_WORKSPACE;
+  for (const auto& o : outs)
+    if (overlaps(workspace, need, o.first, o.second)) return SSD_ERR_INVALID_ARG;
+  for (const auto& i : ins)
+    if (overlaps(workspace, need, i.first, i.second)) return SSD_ERR_INVALID_ARG;
+  if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
+  const ScanArgs a{SSD_F32, x, B, C, dt, A, D, init_state, nullptr, nullptr, workspace,
+                   workspace_bytes, stream};
+  if (io == SSD_BF16)
+    return run_bwd<__nv_bfloat16>(s, a, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit);
+  return run_bwd<float>(s, a, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit);
+}
+
 const char* ssd_status_string(ssd_status s) {
   switch (s) {
     case SSD_OK: return "SSD_OK";
@@ -544,7 +895,7 @@ ssd_status ssd_chunk_state_fwd(const void* x, const float* dt, const float* A, c
   if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
   if (tc) {
     if (!aligned16(x) || !aligned16(B)) return SSD_ERR_UNSUPPORTED;
-    st = run_tc_segments(s, a, tc_segments(s), a.ws, false);
+    st = run_tc_state(s, a, a.ws);
   } else {
     st = s.io == SSD_F32 ? run_simt<float, float>(s, a, false)
                          : run_simt<__nv_bfloat16, float>(s, a, false);
@@ -640,6 +991,9 @@ ssd_status ssd_gate_silu(const float* y, const void* z, void* out, int64_t n, ss
   if (!is_device_ptr(y) || !is_device_ptr(z) || !is_device_ptr(out)) return SSD_ERR_INVALID_ARG;
   const size_t nz = size_t(n) * (z_dtype == SSD_BF16 ? 2 : 4);
   const size_t no = size_t(n) * (out_dtype == SSD_BF16 ? 2 : 4);
+  // in place over y only with a float32 out: a narrower out would let one thread overwrite y
+  // elements that a lower-index thread has not read yet
+  if (out == static_cast<const void*>(y) && out_dtype != SSD_F32) return SSD_ERR_INVALID_ARG;
   if ((out != static_cast<const void*>(y) && overlaps(out, no, y, size_t(n) * 4)) ||
       overlaps(out, no, z, nz))
     return SSD_ERR_INVALID_ARG;
@@ -739,9 +1093,10 @@ const char* ssd_version(void) { return "ssd-b200 0.1 sm_100a"; }
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------------------
-// ssd_chunk_scan_fwd_noalloc: the tensor-core scan with its scratch (the per-segment states and
-// decays) in a fixed device array instead of a caller workspace, for callers that cannot
-// allocate device memory.  The array lives in every GPU that loads this library until exit.
+// ssd_chunk_scan_fwd_noalloc: the tensor-core scan with its scratch (the walk's ticket, ready
+// flags and published boundary states, and the segments' entering states where the walk needs
+// them) in a fixed device array instead of a caller workspace, for callers that cannot allocate
+// device memory.  The array lives in every GPU that loads this library until exit.
 // ---------------------------------------------------------------------------------------------
 namespace {
 
@@ -770,10 +1125,10 @@ ssd_status noalloc_setup(void** scratch) {
         cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSegSmem<2>)) ==
             cudaSuccess &&
-        cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<float>,
+        cudaFuncSetAttribute(ssd::tc::scan_walk_kernel<float>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
             cudaSuccess &&
-        cudaFuncSetAttribute(ssd::tc::chunk_out_kernel<__nv_bfloat16>,
+        cudaFuncSetAttribute(ssd::tc::scan_walk_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
             cudaSuccess;
     if (!ok) {
@@ -786,19 +1141,15 @@ ssd_status noalloc_setup(void** scratch) {
   return SSD_OK;
 }
 
-
-
-// The usual segmentation, with fewer (longer) segments when their states would not fit in
-// `cap` bytes.  Returns false when even one segment per sequence does not fit.
-bool segments_within(const Shape& s, size_t cap, Seg* out) {
-  Seg sg = tc_segments(s);
-  for (int nseg = sg.nseg; nseg >= 1; --nseg) {
-    Seg t;
-    t.nblk = sg.nblk;
-    t.seg_blks = (t.nblk + nseg - 1) / nseg;
-    t.nseg = (t.nblk + t.seg_blks - 1) / t.seg_blks;
-    if (seg_scratch_bytes(s, t) <= cap) {
-      *out = t;
+// The usual plan, or one with fewer CTAs (fewer published states, and fewer segments where
+// there are any) when its scratch would not fit in `cap` bytes.  False when none fits.
+bool plan_within(const Shape& s, size_t cap, TcPlan* out) {
+  for (int ctas = sm_count(); ctas >= 1; ctas /= 2) {
+    ScanOpts o;
+    o.max_ctas = ctas;
+    TcPlan p;
+    if (make_tc_plan(s, o, &p) && walk_bytes(s, p) <= cap) {
+      *out = p;
       return true;
     }
   }
@@ -817,13 +1168,13 @@ extern "C" ssd_status ssd_chunk_scan_fwd_noalloc(
   ssd_status st = check_shape(s);
   if (st != SSD_OK) return st;
   if (!tc_shape_ok(s)) return SSD_ERR_UNSUPPORTED;
-  Seg sg;
-  if (!segments_within(s, SSD_NOALLOC_SCRATCH_BYTES, &sg)) return SSD_ERR_UNSUPPORTED;
+  TcPlan plan;
+  if (!plan_within(s, SSD_NOALLOC_SCRATCH_BYTES, &plan)) return SSD_ERR_UNSUPPORTED;
   st = validate_scan(s, a, 0);
   if (st != SSD_OK) return st;
   if (!tc_pointers_ok(a)) return SSD_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   st = noalloc_setup(&scratch);
   if (st != SSD_OK) return st;
-  return run_tc_segments(s, a, sg, scratch);
+  return run_tc_walk(s, a, plan, scratch);
 }

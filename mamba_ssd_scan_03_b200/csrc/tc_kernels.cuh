@@ -1,17 +1,21 @@
 // tc_kernels.cuh -- the chunked scan on sm_100a tensor cores (bf16 io, headdim 64, dstate 128).
 //
-// The sequence of each (batch row, head) is cut into 128-token blocks (the tcgen05 M=128 tile)
-// and the blocks into segments of consecutive blocks.  Three kernels, in stream order:
+// The sequence of each (batch row, head pair) is cut into 128-token blocks (the tcgen05 M=128
+// tile).  The output pass, scan_walk, walks blocks in order with the running state resident in
+// TMEM.  Per block: G = C B^T (once for both heads), masked diagonal tile (L o G o dt) X,
+// off-diagonal C H, skip term D x, y store, then H <- exp(cs_end) H + B^T (w*x) in place.
+//
+// The walk's work is cut into equal ranges of blocks, one per CTA.  When there are at least
+// about as many (batch row, head pair) sequences as SMs, a range starting inside a sequence gets
+// its entering state from the CTA that walked the sequence's head (published through L2), and
+// nothing else runs.  With fewer, longer sequences each is cut into segments first:
 //
 //  seg_state   per (b, segment, head pair): S_seg = sum_{t in seg} exp(sum_{k>t in seg} a_k)
 //              dt_t B_t x_t^T, one long-K GEMM on the tensor cores (A = B^T, B = w*x, K =
-//              tokens), plus the segment's total log-decay.  Reads x and B once.  Persistent.
+//              tokens), plus the segment's total log-decay.  Persistent.
 //  seg_pass    per state element: passes the state along the segments: H_in(seg) = state
-//              entering each segment, and final_state.
-//  chunk_out   per (b, segment, head pair): walks the segment's blocks in order with the
-//              running state resident in TMEM.  Per block: G = C B^T (once for both heads),
-//              masked diagonal tile (L o G o dt) X, off-diagonal C H, skip term D x, y store,
-//              then H <- exp(cs_end) H + B^T (w*x) in place.
+//              entering each segment.
+//  scan_walk   as above, with the segments' entering states from seg_pass.
 //
 // "Mamba-2 (2024): SSM e attention sono la stessa cosa" (paithon.it), "Il trucco a blocchi":
 // quadratic attention-like form inside blocks, state summary passed between blocks.
@@ -38,7 +42,8 @@ constexpr uint32_t kTile = 16384;  // one 128-row x 128-byte swizzled region
 struct Seg {
   int nblk;      // 128-token blocks per sequence
   int seg_blks;  // blocks per segment
-  int nseg;      // segments per sequence
+  int nseg;      // segments per sequence (stride of the per-segment state and decay arrays)
+  int useg;      // leading segments per sequence that seg_state summarises (<= nseg)
 };
 
 // Inclusive scan over the 128 threads of one half of a 256-thread CTA (warps 0-3 form half 0,
@@ -128,8 +133,8 @@ struct SegUnit {
 __device__ __forceinline__ SegUnit seg_unit(int u, int nq, const Seg& sg) {
   SegUnit r;
   r.hq = u % nq;
-  r.seg = (u / nq) % sg.nseg;
-  r.b = u / (nq * sg.nseg);
+  r.seg = (u / nq) % sg.useg;
+  r.b = u / (nq * sg.useg);
   r.blk0 = r.seg * sg.seg_blks;
   r.nb = min(sg.nblk, r.blk0 + sg.seg_blks) - r.blk0;
   return r;
@@ -469,13 +474,15 @@ __global__ void __launch_bounds__(SegCfg<HU>::kThreads, 1) seg_state_kernel(
 // seg_pass: the state passing between segments.  One thread per float4 of a (batch, head)
 // state, all segments: H_in(0) = init, H_in(s + 1) = 2^decay(s) H_in(s) + S(s).  seg_states
 // is overwritten in place with H_in; final_state receives the state after the last segment
-// (it may alias init_state: each element is read before it is written, by one thread).
+// (it may alias init_state: each element is read before it is written, by one thread).  Only
+// the first `useg` segments carry a summary S(s); with useg = nseg - 1 the entering state of
+// the last segment is still written, and final_state must be NULL (the walk produces it).
 // Segments are taken eight at a time so that eight loads are in flight per thread.
 // =============================================================================================
 constexpr int kPassThreads = 256;
 __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
     float* __restrict__ seg_states, const float* __restrict__ seg_decay,
-    const float* init_state, float* final_state, int batch, int nheads, int nseg) {
+    const float* init_state, float* final_state, int batch, int nheads, int nseg, int useg) {
   constexpr int kVec = kP * kN / 4;  // float4 per (batch, head) state
   const int64_t e = int64_t(blockIdx.x) * kPassThreads + threadIdx.x;
   if (e >= int64_t(batch) * nheads * kVec) return;
@@ -493,9 +500,12 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      if (s0 + i < nseg) {
+      if (s0 + i < useg) {
         v[i] = *reinterpret_cast<const float4*>(base + (s0 + i) * stride);
         a[i] = ex2(dbase[int64_t(s0 + i) * nheads]);
+      } else {
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        a[i] = 1.f;
       }
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -509,23 +519,42 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 }
 
 // =============================================================================================
-// chunk_out: grid = batch * nseg * (nheads / 2), block = 640 threads in five roles:
-//   warps 0-15  compute (512 threads).  Thread (row = tid % 128, q = tid / 128): token row
-//               `row` of a block (state row n = row in the state passes) and a quarter of the
-//               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and
-//               the epilogue; G column groups q and q + 4 for the masks.  Four warps share
-//               each TMEM lane quarter, so every phase is spread over all 16 warps.
-//   warp 16     TMA producer (lane 0): C, x (single buffers), B (double buffer) per block.
-//   warp 17     MMA issuer (lane 0).
-//   warp 18     y writer (lane 0): TMA stores of each block's staged y.
-//   warp 19     cumsums: loads each block's dt of the two heads and writes its log2 cumsums
-//               to shared memory, up to two blocks ahead (lane l: rows 4l .. 4l+3).
-// Per block k the compute warps write the masks (MMA: diagonal tiles), then the state pass
-// (MMA: C H), then X' (MMA: state update) and the epilogue.  The masks come first so that the
-// previous block's y stores, which read the staging buffer the state pass overwrites, drain
-// while they are computed.  Roles hand blocks to each other through mbarriers only; a thread
-// is never more than one phase of a barrier ahead of the slowest, because every barrier it
-// waits on next needs an arrival that the slowest makes after its own previous wait.
+// scan_walk: the output pass.  The blocks of all (batch row, head pair) sequences, laid end to
+// end (block k of sequence s at position s * nblk + k), are cut into `nct` equal ranges, one per
+// CTA (taken by an atomic ticket in launch order).  A CTA walks its range block by block with
+// the running state resident in TMEM; the range splits into items at segment boundaries (a
+// segment is a stretch of a sequence whose entering state is known before the walk: the
+// initial state for the first, a seg_state/seg_pass summary for the others).  An item that
+// starts inside a segment continues the previous range's last item: that CTA walks its last item
+// FIRST and publishes the state it ends with; this CTA walks such an item LAST and reads that
+// state.  A CTA thus only ever waits on a lower ticket's first item, which waits on nothing.
+// With at least as many sequences as CTAs every segment is a whole sequence and there is no
+// summary pass at all: x is read once and no state leaves the L2 except final_state.
+//
+// Per block k (G = C B^T once for both heads; masks; diagonal tiles (L o G o dt) X; off-
+// diagonal C H; skip term D x; y store; then H <- exp(cs_end) H + B^T (w*x) in place), with
+// block = 768 threads in specialised roles, so that the CUDA-core phases of a block run side by
+// side and overlap the tensor-core work instead of following one another:
+//   warps 0-3   state group (thread = state row n = TMEM lane): per block, the bf16 high/low
+//               copy of H for C H and H <- exp(cs_end) H; per item, the entering state into TMEM
+//               and the exit state out of it (final_state or the published slot).
+//   warps 4-11  X' and epilogue group (thread = token row t of one head, all 64 p): X' = w x in
+//               place once the diagonal MMAs have read x; then y = Diag + exp(cs_t) Off + D x
+//               staged in shared memory.
+//   warps 12-19 mask group (thread = token row t, four of G's eight 16-column groups): the two
+//               heads' bf16 masked tiles written over G in TMEM.
+//   warp 20     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block.
+//   warp 21     MMA issuer (lane 0): G, then the diagonal tiles and C H in whichever order their
+//               inputs are ready, then the state update.
+//   warp 22     y writer (lane 0): TMA stores of each block's staged y.
+//   warp 23     cumsums: each block's dt of the two heads -> log2 cumsums and the factors the
+//               other groups use, one block ahead (lane l: rows 4l .. 4l+3).
+// Roles hand blocks to each other through mbarriers only (blocks are numbered across items, so
+// the rings run on from one item to the next); a thread is never more than one phase of a
+// barrier ahead of the slowest, because every barrier it waits on next needs an arrival that
+// the slowest makes after its own previous wait.  The last block of an item whose exit state is
+// kept also sends the bf16 remainder of X' through the tensor core (written over C's tiles once
+// C H is done), so that state carries about 16 bits of the block's input.
 // Shared memory (1024-aligned, 12 x 16 KB):
 //   sC   2 tiles  C, K-major (rows t), n halves
 //   sB   4 tiles  B, rows s, n halves, two slots (blocks k % 2): K-major for G = C B^T,
@@ -542,8 +571,6 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 // =============================================================================================
 constexpr uint32_t kOffC = 0, kOffB = 2 * kTile, kOffX = 6 * kTile, kOffHh = 8 * kTile,
                    kOffHl = 10 * kTile, kSmemTiles = 12 * kTile;
-constexpr int kComputeThreads = 512;
-constexpr int kOutThreads = kComputeThreads + 128;
 
 // y staging (in sHh/sHl) and its TMA stores.  Float32 y: 4 boxes {32 p, 128 t} (one per
 // thread quarter q: head q/2, p-half q%2), 128B-swizzled.  Bf16 y: 2 boxes {64 p, 128 t} (one
@@ -558,6 +585,14 @@ template <> struct ystage<float> {
     for (int i = 0; i < 4; ++i)
       *reinterpret_cast<float4*>(box + swz(t, half * 4 + i)) =
           make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  // thread (t, head j) writes y[t, p0 .. p0+8) (p0 a multiple of 8)
+  static __device__ __forceinline__ void put8(uint8_t* stage, int t, int j, int p0,
+                                              const float (&v)[8]) {
+    uint8_t* box = stage + (2 * j + (p0 >> 5)) * kTile;
+    const int c = (p0 & 31) >> 2;
+    *reinterpret_cast<float4*>(box + swz(t, c)) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(box + swz(t, c + 1)) = make_float4(v[4], v[5], v[6], v[7]);
   }
   static __device__ __forceinline__ void store(const CUtensorMap* map, const uint8_t* stage,
                                                int h0, int t0, int b) {
@@ -578,6 +613,12 @@ template <> struct ystage<__nv_bfloat16> {
         make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
                    pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
   }
+  static __device__ __forceinline__ void put8(uint8_t* stage, int t, int j, int p0,
+                                              const float (&v)[8]) {
+    *reinterpret_cast<uint4*>(stage + j * kTile + swz(t, p0 >> 3)) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                   pack_bf16x2(v[6], v[7]));
+  }
   static __device__ __forceinline__ void store(const CUtensorMap* map, const uint8_t* stage,
                                                int h0, int t0, int b) {
 #pragma unroll
@@ -585,61 +626,167 @@ template <> struct ystage<__nv_bfloat16> {
   }
 };
 
-// mbarriers of chunk_out (all in shared memory)
-struct OutBars {
+// The plan of one call's walk (host-computed).
+struct WalkPlan {
+  int64_t total;  // batch * npair * nblk: every block of every (batch row, head pair) sequence
+  int nblk;       // 128-token blocks per sequence
+  int seg_blks;   // blocks per segment
+  int nseg;       // segments per sequence (1: the entering state of a sequence is init_state)
+  int npair;      // head pairs
+  int nct;        // ranges (= CTAs)
+  uint64_t wait_ns;  // limit of every bounded wait (2 s in production; 0: no waiting)
+};
+// Where an item's entering state comes from and where its exit state goes.
+enum : int { kSrcInit = 0, kSrcSeg = 1, kSrcSlot = 2 };
+enum : int { kDstNone = 0, kDstFinal = 1, kDstSlot = 2 };
+struct WalkItem {
+  int seq, k0, k1, src, dst;  // sequence b * npair + pair, blocks [k0, k1)
+};
+constexpr int kMaxItems = 16;
+constexpr int kSlotFloats = 2 * kP * kN;  // one published state: two heads, [j][p][n]
+
+// The items of range r in walk order (the publishing item first, the waiting one last), written
+// to `out` (shared memory).  Returns their number, or -1 if there are more than kMaxItems (the
+// host plans fewer).  Three passes over the range, one per class, so no local list is needed.
+__device__ int walk_items(const WalkPlan& pl, int r, bool has_final, WalkItem* out) {
+  const int64_t g0 = pl.total * r / pl.nct, g1 = pl.total * (r + 1) / pl.nct;
+  int m = 0;
+  for (int cls = 0; cls < 3; ++cls) {
+    for (int64_t g = g0; g < g1;) {
+      WalkItem w;
+      w.seq = int(g / pl.nblk);
+      w.k0 = int(g % pl.nblk);
+      const int seg = w.k0 / pl.seg_blks;
+      const int seg_end = min((seg + 1) * pl.seg_blks, pl.nblk);
+      w.k1 = int(g1 - g < int64_t(seg_end - w.k0) ? w.k0 + (g1 - g) : int64_t(seg_end));
+      w.src = (w.k0 % pl.seg_blks) ? kSrcSlot : (pl.nseg > 1 ? kSrcSeg : kSrcInit);
+      w.dst = w.k1 < seg_end ? kDstSlot : ((w.k1 == pl.nblk && has_final) ? kDstFinal : kDstNone);
+      const int c = w.dst == kDstSlot ? 0 : (w.src == kSrcSlot ? 2 : 1);
+      if (c == cls) {
+        if (m == kMaxItems) return -1;
+        out[m++] = w;
+      }
+      g += w.k1 - w.k0;
+    }
+  }
+  return m;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait (warp-collective) until *flag != 0: lane 0 polls, then every lane acquires.  The
+// limit works as in mbar_wait (0: give up unless the flag is already set).
+__device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort, unsigned site,
+                                          uint64_t limit_ns) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    const uint64_t t0 = globaltimer();
+    while (ld_acquire_gpu(flag) == 0) {
+      if (*abort) {
+        ok = 0;
+        break;
+      }
+      if (limit_ns == 0 || globaltimer() - t0 > limit_ns) {
+        latch_status(SSD_ERR_DEVICE_TIMEOUT, site);
+        *abort = 1;
+        ok = 0;
+        break;
+      }
+      __nanosleep(256);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) (void)ld_acquire_gpu(flag);
+  return ok != 0;
+}
+
+// Warp roles of the walk (768 threads).
+constexpr int kWarpE = 4;     // warps 0-3: state group
+constexpr int kWarpM = 12;    // warps 4-11: X' and epilogue group; warps 12-19: mask group
+constexpr int kWarpTma = 20, kWarpMma = 21, kWarpY = 22, kWarpCs = 23;
+constexpr int kHThreads = 128, kEThreads = 256, kMThreads = 256;
+constexpr int kWalkThreads = 768;
+
+// The cumsum warp's per-block values, two buffers (block k in buffer k % 2), two heads.  Read
+// and written as float4 (16-byte aligned rows).
+struct __align__(16) WalkCs {
+  float cs[2][2][kBlk];  // inclusive log2 cumsum of dt A within the block
+  float cl[2][2][kBlk];  // cs - log2(dt) (+inf where dt = 0)
+  float v[2][2][kBlk];   // exp(cs_{s|15} - cs_s) dt_s (masks, factorized form)
+  float e[2][2][kBlk];   // exp(cs_t) (epilogue)
+  float w[2][2][kBlk];   // exp(cs_end - cs_t) dt_t (X')
+  float alpha[2][2];     // exp(cs_end) (state pass)
+};
+static_assert(offsetof(WalkCs, cl) % 16 == 0 && offsetof(WalkCs, v) % 16 == 0 &&
+                  offsetof(WalkCs, e) % 16 == 0 && offsetof(WalkCs, w) % 16 == 0,
+              "WalkCs rows must stay 16-byte aligned");
+
+// mbarriers of the walk (all in shared memory)
+struct WalkBars {
   uint64_t c_full, b_full[2], x_full;        // TMA -> consumers
   uint64_t c_empty, b_empty[2], x_empty;     // MMA completion -> producer
-  uint64_t g_done, d_done, o_done, st_done;  // MMA completion -> compute
-  uint64_t m0_ready, m1_ready, h_ready, xp_ready;  // compute -> MMA issuer
-  uint64_t y_staged, stage_free;             // compute <-> y writer
-  uint64_t cs_full[2], cs_empty[2];          // cumsum warp <-> compute (per cumsum buffer)
+  uint64_t g_done, d_done, o_done, st_done;  // MMA completion -> compute groups
+  uint64_t m_ready, h_ready, xp_ready;       // masks / state pass / X' -> MMA issuer
+  uint64_t y_staged;                         // epilogue -> y writer and MMA issuer
+  uint64_t stage_free;                       // y writer -> state group
+  uint64_t cs_full[2], cs_empty[2];          // cumsum warp <-> compute groups
+  uint64_t pub;                              // state group: exit state written (published item)
   uint64_t drain;
 };
 
 template <typename TY>
-__global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
+__global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
     const float* __restrict__ dt, const float* __restrict__ A, const float* __restrict__ D,
-    const float* __restrict__ h_in, int64_t seqlen, int nheads, int heads_per_group, Seg sg) {
+    const float* init_state, const float* seg_hin, float* final_state, float* slots,
+    int* flags, unsigned* ticket, int64_t seqlen, int nheads, int heads_per_group,
+    WalkPlan pl) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ OutBars bars;
+  __shared__ WalkBars bars;
   __shared__ uint32_t tmem_base_sh;
-  // per block (two buffers, block k in buffer k % 2) and head: log2 cumsums cs, cl = cs -
-  // log2(dt) (+inf where dt = 0), v_s = exp(cs_{s|15} - cs_s) dt_s
-  __shared__ __align__(16) float cs_sh[2][2][kBlk];
-  __shared__ __align__(16) float cl_sh[2][2][kBlk];
-  __shared__ __align__(16) float v_sh[2][2][kBlk];
+  __shared__ __align__(16) WalkCs cs;  // per block (two buffers, block k % 2) and head
+  __shared__ WalkItem items_sh[kMaxItems];
+  __shared__ int nitems_sh, nblocks_sh, range_sh;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int npair = nheads / 2;
-  const int unit = blockIdx.x;
-  const int hp = unit % npair;
-  const int seg = (unit / npair) % sg.nseg;
-  const int b = unit / (npair * sg.nseg);
-  const int h0 = hp * 2;
-  const int g = h0 / heads_per_group;
-  const int blk0 = seg * sg.seg_blks;
-  const int nb = min(sg.nblk, blk0 + sg.seg_blks) - blk0;
   volatile int* abort_v = &abort_flag;
   uint32_t n_c = 0, n_x = 0, n_b[2] = {0, 0};  // the producer's loads issued per barrier
+  const uint64_t lim = pl.wait_ns;
 
   if (tid == 0) {
     abort_flag = 0;
+    const int r = int(atomicAdd(ticket, 1u));
+    int n = r < pl.nct ? walk_items(pl, r, final_state != nullptr, items_sh) : 0;
+    if (n < 0) {
+      latch_status(SSD_ERR_UNSUPPORTED, 70);
+      n = 0;
+    }
+    int nb = 0;
+    for (int i = 0; i < n; ++i) nb += items_sh[i].k1 - items_sh[i].k0;
+    range_sh = r;
+    nitems_sh = n;
+    nblocks_sh = nb;
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
-    for (int i = 0; i < int(sizeof(OutBars) / 8); ++i) mbar_init(all + i, 1);
-    mbar_init(&bars.m0_ready, kComputeThreads);
-    mbar_init(&bars.m1_ready, kComputeThreads);
-    mbar_init(&bars.h_ready, kComputeThreads);
-    mbar_init(&bars.xp_ready, kComputeThreads);
-    mbar_init(&bars.y_staged, kComputeThreads);
+    for (int i = 0; i < int(sizeof(WalkBars) / 8); ++i) mbar_init(all + i, 1);
+    mbar_init(&bars.m_ready, kMThreads);
+    mbar_init(&bars.h_ready, kHThreads);
+    mbar_init(&bars.xp_ready, kEThreads);
+    mbar_init(&bars.y_staged, kEThreads);
+    mbar_init(&bars.pub, kHThreads);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.cs_full[i], 32);
-      mbar_init(&bars.cs_empty[i], kComputeThreads);
+      mbar_init(&bars.cs_empty[i], kHThreads + kEThreads + kMThreads);
     }
     fence_mbar_init();
   }
@@ -650,49 +797,54 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
   const uint32_t tmem = tmem_base_sh;
   const uint32_t tH = tmem, tD = tmem + 128, tO = tmem + 256, tG = tmem + 384;
   const uint32_t sbase = smem_u32(smem);
+  const int nit = nitems_sh, nbt = nblocks_sh, range = range_sh;
 
-  if (warp == 16) {
+  if (warp == kWarpTma) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_c);
-      auto load_c = [&](int k) {
-        const int t0 = (blk0 + k) * kBlk;
-        ++n_c;
-        mbar_arrive_expect_tx(&bars.c_full, 2 * kTile);
-        tma_load_3d(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b);
-        tma_load_3d(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b);
-      };
-      auto load_b = [&](int k) {
-        const int t0 = (blk0 + k) * kBlk;
-        uint8_t* dst = smem + kOffB + (k & 1) * 2 * kTile;
-        ++n_b[k & 1];
-        mbar_arrive_expect_tx(&bars.b_full[k & 1], 2 * kTile);
-        tma_load_3d(dst, &tm_b, &bars.b_full[k & 1], g * kN, t0, b);
-        tma_load_3d(dst + kTile, &tm_b, &bars.b_full[k & 1], g * kN + 64, t0, b);
-      };
-      auto load_x = [&](int k) {
-        const int t0 = (blk0 + k) * kBlk;
-        ++n_x;
-        mbar_arrive_expect_tx(&bars.x_full, 2 * kTile);
-        tma_load_3d(smem + kOffX, &tm_x, &bars.x_full, h0 * kP, t0, b);
-        tma_load_3d(smem + kOffX + kTile, &tm_x, &bars.x_full, (h0 + 1) * kP, t0, b);
-      };
-      if (nb > 0) { load_c(0); load_b(0); load_x(0); }
-      if (nb > 1) load_b(1);
-      for (int k = 0; k + 1 < nb; ++k) {
-        if (!mbar_wait(&bars.c_empty, k & 1, abort_v, 31)) break;  // C H of block k done
-        load_c(k + 1);
-        if (!mbar_wait(&bars.x_empty, k & 1, abort_v, 32)) break;  // state MMA of block k done
-        load_x(k + 1);
-        if (k + 2 < nb) {
-          if (!mbar_wait(&bars.b_empty[k & 1], (k >> 1) & 1, abort_v, 33)) break;
-          load_b(k + 2);
+      int j = 0;
+      bool ok = true;
+      for (int it = 0; it < nit && ok; ++it) {
+        const WalkItem w = items_sh[it];
+        const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
+        const int g = h0 / heads_per_group;
+        for (int k = w.k0; k < w.k1; ++k, ++j) {
+          const int t0 = k * kBlk;
+          // B of block j into slot j % 2 once block j - 2's G and state MMAs are done
+          if (j >= 2 && !mbar_wait(&bars.b_empty[j & 1], ((j - 2) >> 1) & 1, abort_v, 33, lim)) {
+            ok = false;
+            break;
+          }
+          uint8_t* bdst = smem + kOffB + (j & 1) * 2 * kTile;
+          ++n_b[j & 1];
+          mbar_arrive_expect_tx(&bars.b_full[j & 1], 2 * kTile);
+          tma_load_3d(bdst, &tm_b, &bars.b_full[j & 1], g * kN, t0, b);
+          tma_load_3d(bdst + kTile, &tm_b, &bars.b_full[j & 1], g * kN + 64, t0, b);
+          // C once block j - 1's G and C H are done
+          if (j >= 1 && !mbar_wait(&bars.c_empty, (j - 1) & 1, abort_v, 31, lim)) {
+            ok = false;
+            break;
+          }
+          ++n_c;
+          mbar_arrive_expect_tx(&bars.c_full, 2 * kTile);
+          tma_load_3d(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b);
+          tma_load_3d(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b);
+          // x once block j - 1's diagonal and state MMAs are done
+          if (j >= 1 && !mbar_wait(&bars.x_empty, (j - 1) & 1, abort_v, 32, lim)) {
+            ok = false;
+            break;
+          }
+          ++n_x;
+          mbar_arrive_expect_tx(&bars.x_full, 2 * kTile);
+          tma_load_3d(smem + kOffX, &tm_x, &bars.x_full, h0 * kP, t0, b);
+          tma_load_3d(smem + kOffX + kTile, &tm_x, &bars.x_full, (h0 + 1) * kP, t0, b);
         }
       }
     }
-  } else if (warp == 17) {
+  } else if (warp == kWarpMma) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
       const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
@@ -708,173 +860,454 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       const uint64_t dHh = sdesc(sbase + kOffHh, kTile, 1024);
       const uint64_t dHl = sdesc(sbase + kOffHl, kTile, 1024);
       auto kmaj = [](int kk) { return uint64_t(((kk >> 2) * kTile + (kk & 3) * 32) >> 4); };
-      for (int k = 0; k < nb; ++k) {
+      const uint64_t dXlo = sdesc(sbase + kOffC, kTile, 1024);  // X' low part over C's tiles
+      int it = 0, kend = nit > 0 ? items_sh[0].k1 - items_sh[0].k0 : 0;
+      for (int k = 0; k < nbt; ++k) {
         const uint32_t par = k & 1;
         const uint64_t bslot = (k & 1) ? uint64_t((2 * kTile) >> 4) : 0u;
-        if (k > 0 && !mbar_wait(&bars.d_done, par ^ 1, abort_v, 41)) break;  // G region free
-        if (!mbar_wait(&bars.c_full, par, abort_v, 42)) break;
-        if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43)) break;
+        // the last block of an item whose exit state is kept also sends X's bf16 remainder
+        while (it < nit && k >= kend) {
+          ++it;
+          if (it < nit) kend += items_sh[it].k1 - items_sh[it].k0;
+        }
+        const bool lo = it < nit && k == kend - 1 && items_sh[it].dst != kDstNone;
+        if (k > 0 && !mbar_wait(&bars.d_done, par ^ 1, abort_v, 41, lim)) break;  // G free
+        if (!mbar_wait(&bars.c_full, par, abort_v, 42, lim)) break;
+        if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43, lim)) break;
         tc_fence_after();
         // G = C B^T (M = t, N = s, K = n)
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk)
           mma_ss(tG, dC + kmaj(kk), dBk + bslot + kmaj(kk), id_g, kk > 0 ? 1u : 0u);
         mma_commit(&bars.g_done);
-        // Diag_h = M_h X_h (M = t, N = p, K = s), A = head h's bf16 mask in TMEM (columns
-        // 8h .. 8h+7 of each 16-column group); head 0 while head 1's mask is being written
-        if (!mbar_wait(&bars.x_full, par, abort_v, 45)) break;
-        auto diag = [&](int h) {
+        // the diagonal and off-diagonal accumulators are free once block k - 1's epilogue has
+        // read them; x of block k must have landed
+        if (k > 0 && !mbar_wait(&bars.y_staged, par ^ 1, abort_v, 49, lim)) break;
+        if (!mbar_wait(&bars.x_full, par, abort_v, 45, lim)) break;
+        // Diag_h = M_h X_h (M = t, N = p, K = s; A = head h's bf16 mask in TMEM, columns
+        // 8h .. 8h+7 of each 16-column group) and Off = C (Hhi + Hlo) (M = t, N = (head, p),
+        // K = n), in whichever order the masks and the state pass finish
+        bool dd = false, oo = false, fail = false;
+        const uint64_t t0 = globaltimer();
+        while (!(dd && oo)) {
+          if (!dd && mbar_test(&bars.m_ready, par)) {
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk)
-            mma_ts(tD + h * 64, tG + kk * 16 + h * 8, dX + h * (kTile >> 4) + kk * 128, id_diag,
-                   kk > 0 ? 1u : 0u);
-        };
-        if (!mbar_wait(&bars.m0_ready, par, abort_v, 46)) break;
-        tc_fence_after();
-        diag(0);
-        if (!mbar_wait(&bars.m1_ready, par, abort_v, 48)) break;
-        tc_fence_after();
-        diag(1);
-        mma_commit(&bars.d_done);
-        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n)
-        if (!mbar_wait(&bars.h_ready, par, abort_v, 44)) break;
-        tc_fence_after();
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
-          mma_ss(tO, dC + kmaj(kk), dHh + kk * 128, id_off, kk > 0 ? 1u : 0u);
-          mma_ss(tO, dC + kmaj(kk), dHl + kk * 128, id_off, 1u);
+              for (int kk = 0; kk < kBlk / 16; ++kk)
+                mma_ts(tD + h * 64, tG + kk * 16 + h * 8, dX + h * (kTile >> 4) + kk * 128,
+                       id_diag, kk > 0 ? 1u : 0u);
+            mma_commit(&bars.d_done);
+            dd = true;
+          }
+          if (!oo && mbar_test(&bars.h_ready, par)) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kN / 16; ++kk) {
+              mma_ss(tO, dC + kmaj(kk), dHh + kk * 128, id_off, kk > 0 ? 1u : 0u);
+              mma_ss(tO, dC + kmaj(kk), dHl + kk * 128, id_off, 1u);
+            }
+            mma_commit(&bars.o_done);
+            oo = true;
+          }
+          if (dd && oo) break;
+          if (*abort_v) {
+            fail = true;
+            break;
+          }
+          if (lim == 0 || globaltimer() - t0 > lim) {
+            latch_status(SSD_ERR_DEVICE_TIMEOUT, 46);
+            *abort_v = 1;
+            fail = true;
+            break;
+          }
+          __nanosleep(64);
         }
-        mma_commit(&bars.o_done);
-        mma_commit(&bars.c_empty);
-        // H += B^T X' (M = n, N = (head, p), K = t)
-        if (!mbar_wait(&bars.xp_ready, par, abort_v, 47)) break;
+        if (fail) break;
+        if (!lo) mma_commit(&bars.c_empty);  // G and C H of block k have read C
+        // H += B^T X' (M = n, N = (head, p), K = t), plus B^T X'_lo from C's tiles
+        if (!mbar_wait(&bars.xp_ready, par, abort_v, 47, lim)) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
           mma_ss(tH, dBm + bslot + kk * 128, dX + kk * 128, id_st, 1u);
+          if (lo) mma_ss(tH, dBm + bslot + kk * 128, dXlo + kk * 128, id_st, 1u);
+        }
+        if (lo) mma_commit(&bars.c_empty);
         mma_commit(&bars.st_done);
         mma_commit(&bars.x_empty);
         mma_commit(&bars.b_empty[k & 1]);
       }
     }
-  } else if (warp == 18) {
+  } else if (warp == kWarpY) {
     // ------------------------------ y writer ------------------------------
     if (lane == 0) {
       prefetch_tmap(&tm_y);
       const uint8_t* stage = smem + kOffHh;
-      for (int k = 0; k < nb; ++k) {
-        if (!mbar_wait(&bars.y_staged, k & 1, abort_v, 61)) break;
-        ystage<TY>::store(&tm_y, stage, h0, (blk0 + k) * kBlk, b);
-        bulk_commit();
-        bulk_wait_read();  // the staging buffer may be reused once the stores have read it
-        mbar_arrive(&bars.stage_free);
+      int j = 0;
+      bool ok = true;
+      for (int it = 0; it < nit && ok; ++it) {
+        const WalkItem w = items_sh[it];
+        const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
+        for (int k = w.k0; k < w.k1; ++k, ++j) {
+          if (!mbar_wait(&bars.y_staged, j & 1, abort_v, 61, lim)) {
+            ok = false;
+            break;
+          }
+          ystage<TY>::store(&tm_y, stage, h0, k * kBlk, b);
+          bulk_commit();
+          bulk_wait_read();  // the staging buffer may be reused once the stores have read it
+          mbar_arrive(&bars.stage_free);
+        }
       }
       bulk_wait_all();
     }
-  } else if (warp == 19) {
+  } else if (warp == kWarpCs) {
     // ------------------------------ cumsums ------------------------------
     // Per block and head: cs_t = inclusive log2 cumsum of dt A (within the block), cl_t =
-    // cs_t - log2(dt_t) (+inf where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15.
-    const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
-    const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
+    // cs_t - log2(dt_t) (+inf where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15
+    // (the masks), e_t = exp(cs_t) (the epilogue), w_t = exp(cs_end - cs_t) dt_t (X') and
+    // alpha = exp(cs_end) (the state pass).  The next block's dt is loaded meanwhile.
     float v[8];  // dt of rows 4 lane + r, head h at v[2r + h]
-    auto load = [&](int kb) {
+    auto load = [&](int it, int kb) {
+      const WalkItem w = items_sh[it];
+      const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
+      const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const int64_t tok = int64_t(blk0 + kb) * kBlk + 4 * lane + r;
+        const int64_t tok = int64_t(kb) * kBlk + 4 * lane + r;
         const bool in = tok < seqlen;
         v[2 * r] = in ? dtb[tok * nheads] : 0.f;
         v[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
       }
     };
-    load(0);
+    if (nit > 0) load(0, items_sh[0].k0);
     const float inf = __int_as_float(0x7f800000);
-    for (int kb = 0; kb < nb; ++kb) {
-      const int bf = kb & 1;
-      if (kb >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars.cs_empty[bf], ((kb - 2) >> 1) & 1,
-                                                        abort_v, 58)))
-        break;  // warp-uniform, so every lane reaches the same __syncwarp
+    int j = 0;
+    bool ok = true;
+    for (int it = 0; it < nit && ok; ++it) {
+      const WalkItem w = items_sh[it];
+      const int h0 = (w.seq % pl.npair) * 2;
+      const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
+      for (int kb = w.k0; kb < w.k1; ++kb, ++j) {
+        const int bf = j & 1;
+        if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars.cs_empty[bf], ((j - 2) >> 1) & 1,
+                                                         abort_v, 58, lim))) {
+          ok = false;  // warp-uniform, so every lane reaches the same __syncwarp
+          break;
+        }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float d0 = v[h], d1 = v[2 + h], d2 = v[4 + h], d3 = v[6 + h];
-        float c0 = d0 * al[h];
-        float c1 = fmaf(d1, al[h], c0);
-        float c2 = fmaf(d2, al[h], c1);
-        float c3 = fmaf(d3, al[h], c2);
-        const float off = warp_inclusive_scan(c3) - c3;
-        c0 += off;
-        c1 += off;
-        c2 += off;
-        c3 += off;
-        const float l0 = d0 > 0.f ? c0 - __log2f(d0) : inf;
-        const float l1 = d1 > 0.f ? c1 - __log2f(d1) : inf;
-        const float l2 = d2 > 0.f ? c2 - __log2f(d2) : inf;
-        const float l3 = d3 > 0.f ? c3 - __log2f(d3) : inf;
-        const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
-        *reinterpret_cast<float4*>(&cs_sh[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
-        *reinterpret_cast<float4*>(&cl_sh[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
-        *reinterpret_cast<float4*>(&v_sh[bf][h][4 * lane]) =
-            make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
+        for (int h = 0; h < 2; ++h) {
+          const float d0 = v[h], d1 = v[2 + h], d2 = v[4 + h], d3 = v[6 + h];
+          float c0 = d0 * al[h];
+          float c1 = fmaf(d1, al[h], c0);
+          float c2 = fmaf(d2, al[h], c1);
+          float c3 = fmaf(d3, al[h], c2);
+          const float off = warp_inclusive_scan(c3) - c3;
+          c0 += off;
+          c1 += off;
+          c2 += off;
+          c3 += off;
+          const float l0 = d0 > 0.f ? c0 - __log2f(d0) : inf;
+          const float l1 = d1 > 0.f ? c1 - __log2f(d1) : inf;
+          const float l2 = d2 > 0.f ? c2 - __log2f(d2) : inf;
+          const float l3 = d3 > 0.f ? c3 - __log2f(d3) : inf;
+          const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
+          const float ce = __shfl_sync(0xffffffffu, c3, 31);        // cs at the block's end
+          *reinterpret_cast<float4*>(&cs.cs[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
+          *reinterpret_cast<float4*>(&cs.cl[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
+          *reinterpret_cast<float4*>(&cs.v[bf][h][4 * lane]) =
+              make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
+          *reinterpret_cast<float4*>(&cs.e[bf][h][4 * lane]) =
+              make_float4(ex2(c0), ex2(c1), ex2(c2), ex2(c3));
+          *reinterpret_cast<float4*>(&cs.w[bf][h][4 * lane]) =
+              make_float4(ex2(ce - l0), ex2(ce - l1), ex2(ce - l2), ex2(ce - l3));
+          if (lane == 0) cs.alpha[bf][h] = ex2(ce);
+        }
+        mbar_arrive_warp(&bars.cs_full[bf]);
+        if (kb + 1 < w.k1) load(it, kb + 1);
+        else if (it + 1 < nit) load(it + 1, items_sh[it + 1].k0);
       }
-      mbar_arrive_warp(&bars.cs_full[bf]);
-      if (kb + 1 < nb) load(kb + 1);
+    }
+  } else if (warp < kWarpE) {
+    // ------------------------------ state group (warps 0-3) ------------------------------
+    // Thread n = tid: state row n (TMEM lane n), all 128 columns (head, p).  Per block: the bf16
+    // high/low copy of H for C H (sHh/sHl), then H <- alpha H in place; per item: the entering
+    // state into TMEM and the exit state out of it.
+    const int n = tid;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    bool ok = true, stop = false;
+    int k = 0;
+    for (int it = 0; it < nit && !stop; ++it) {
+      const WalkItem w = items_sh[it];
+      const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
+      // ---- entering state -> TMEM once the previous item's last state MMA is done ----
+      if (k > 0) ok = ok && mbar_wait(&bars.st_done, (k - 1) & 1, abort_v, 71, lim);
+      ok = __all_sync(0xffffffffu, ok);
+      const float* src = nullptr;
+      int64_t hstride = int64_t(kP) * kN;  // from head h0 to h0 + 1
+      if (w.src == kSrcSlot) {
+        if (ok) ok = flag_wait(flags + (range - 1), abort_v, 74, lim);
+        src = slots + int64_t(range - 1) * kSlotFloats + n;
+      } else if (w.src == kSrcSeg) {
+        const int seg = w.k0 / pl.seg_blks;
+        src = seg_hin + ((int64_t(b) * pl.nseg + seg) * nheads + h0) * kP * kN + n;
+      } else if (init_state) {
+        src = init_state + (int64_t(b) * nheads + h0) * kP * kN + n;
+      }
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {  // 16 columns (head c / 4, p = 16 (c % 4) ..) at a time
+          uint32_t r[16];
+          if (src) {
+            const float* sp = src + (c >> 2) * hstride + (c & 3) * 16 * kN;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(sp[e * kN]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = 0u;
+          }
+          tmem_st16(tH + lane_off + c * 16, r);
+        }
+        tmem_wait_st();
+      }
+      for (int kb = w.k0; kb < w.k1; ++kb, ++k) {
+        const uint32_t par = k & 1;
+        const int bf = k & 1;
+        ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 50, lim);
+        const float al0 = cs.alpha[bf][0], al1 = cs.alpha[bf][1];
+        mbar_arrive_warp(&bars.cs_empty[bf]);
+        // H of block k is complete once block k - 1's state MMA is; sHh/sHl are free once block
+        // k - 1's y stores (staged there) have read them
+        if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51, lim);
+        if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55, lim);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {  // 32 columns: head c / 2, p in [32 (c % 2), +32)
+            const int j = c >> 1;
+            const float al = j ? al1 : al0;
+            uint8_t* hh = smem + kOffHh + j * kTile;
+            uint8_t* hl = smem + kOffHl + j * kTile;
+            uint32_t ra[16], rb[16];
+            tmem_ld16(tH + lane_off + c * 32, ra);
+            tmem_ld16(tH + lane_off + c * 32 + 16, rb);
+            tmem_wait_ld();
+            const int ch = (c & 1) * 4;  // 16-byte chunk of the 128-byte row
+#define SSD_HSPLIT(R, C0)                                                                     \
+  {                                                                                           \
+    uint32_t hi[8], lo[8];                                                                    \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
+        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
+    *reinterpret_cast<uint4*>(hh + swz(n, C0)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);      \
+    *reinterpret_cast<uint4*>(hh + swz(n, C0 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);  \
+    *reinterpret_cast<uint4*>(hl + swz(n, C0)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);      \
+    *reinterpret_cast<uint4*>(hl + swz(n, C0 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);  \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e) {                                          \
+      const float2 sc = mul2(make_float2(__uint_as_float(R[2 * e]),                          \
+                                         __uint_as_float(R[2 * e + 1])), make_float2(al, al)); \
+      R[2 * e] = __float_as_uint(sc.x);                                                       \
+      R[2 * e + 1] = __float_as_uint(sc.y);                                                   \
+    }                                                                                         \
+  }
+            SSD_HSPLIT(ra, ch)
+            SSD_HSPLIT(rb, ch + 2)
+#undef SSD_HSPLIT
+            tmem_st16(tH + lane_off + c * 32, ra);
+            tmem_st16(tH + lane_off + c * 32 + 16, rb);
+          }
+          tmem_wait_st();
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive_warp(&bars.h_ready);
+        if (__any_sync(0xffffffffu, !ok || *abort_v)) {
+          stop = true;
+          break;
+        }
+      }
+      if (stop) break;
+      // ---- the item's exit state: final_state, or the slot the next range reads ----
+      if (w.dst != kDstNone) {
+        ok = ok && mbar_wait(&bars.st_done, (k - 1) & 1, abort_v, 72, lim);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          float* dst = w.dst == kDstFinal
+                           ? final_state + (int64_t(b) * nheads + h0) * kP * kN + n
+                           : slots + int64_t(range) * kSlotFloats + n;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tH + lane_off + c * 16, r);
+            tmem_wait_ld();
+            float* d = dst + (c >> 2) * hstride + (c & 3) * 16 * kN;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) d[e * kN] = __uint_as_float(r[e]);
+          }
+        }
+        tc_fence_before();
+        if (w.dst == kDstSlot) {
+          __threadfence();
+          mbar_arrive_warp(&bars.pub);
+          if (tid == 0 && mbar_wait(&bars.pub, 0, abort_v, 73, lim)) {
+            __threadfence();
+            st_release_gpu(flags + range, 1);
+          }
+        }
+      }
+      if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
+    }
+  } else if (warp < kWarpM) {
+    // ------------------------------ X' and epilogue group (warps 4-11) ------------------------
+    // Thread (row t = 32 (warp % 4) + lane, head j = (warp - 4) / 4): token row t of head j, all
+    // 64 p.  Per block: X' = w x in place over the x tile once the diagonal MMAs have read it
+    // (x itself stays in registers for the skip term), then y_t = Diag + e_t Off + D x_t staged
+    // in shared memory for the y writer.
+    const int wq = warp & 3, j = (warp - kWarpE) >> 2;
+    const int t = wq * 32 + lane;
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    uint8_t* stage = smem + kOffHh;
+    uint8_t* xrow = smem + kOffX + j * kTile;
+    bool ok = true, stop = false;
+    int k = 0;
+    for (int it = 0; it < nit && !stop; ++it) {
+      const WalkItem w = items_sh[it];
+      const int h0 = (w.seq % pl.npair) * 2;
+      const float Dh = D ? D[h0 + j] : 0.f;
+      for (int kb = w.k0; kb < w.k1; ++kb, ++k) {
+        const uint32_t par = k & 1;
+        const int bf = k & 1;
+        ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 53, lim);
+        ok = ok && mbar_wait(&bars.d_done, par, abort_v, 54, lim);
+        ok = __all_sync(0xffffffffu, ok);
+        uint32_t xw[32];
+        if (ok) {
+          tc_fence_after();
+          const float wj = cs.w[bf][j][t];
+          const float2 ww = make_float2(wj, wj);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4* pch = reinterpret_cast<uint4*>(xrow + swz(t, c));
+            const uint4 v = *pch;
+            xw[4 * c] = v.x;
+            xw[4 * c + 1] = v.y;
+            xw[4 * c + 2] = v.z;
+            xw[4 * c + 3] = v.w;
+            *pch = make_uint4(scale_bf16x2(v.x, ww), scale_bf16x2(v.y, ww), scale_bf16x2(v.z, ww),
+                              scale_bf16x2(v.w, ww));
+          }
+          fence_proxy_async_smem();
+        }
+        // the last block of an item whose exit state is kept also sends the bf16 remainder of
+        // X' (over C's tiles, free once C H is done), so that the state it leaves carries ~16
+        // bits of the block's input: its X' is handed over only then
+        const bool lo = kb == w.k1 - 1 && w.dst != kDstNone;
+        if (!lo) mbar_arrive_warp(&bars.xp_ready);
+        ok = ok && mbar_wait(&bars.o_done, par, abort_v, 57, lim);
+        ok = __all_sync(0xffffffffu, ok);
+        if (lo) {
+          if (ok) {
+            tc_fence_after();
+            const float wj = cs.w[bf][j][t];
+            uint8_t* lrow = smem + kOffC + j * kTile;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t hi4[4], lo4[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t xv = xw[4 * c + i];
+                split2(bf16lo(xv) * wj, bf16hi(xv) * wj, hi4[i], lo4[i]);
+              }
+              *reinterpret_cast<uint4*>(lrow + swz(t, c)) =
+                  make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+            }
+            fence_proxy_async_smem();
+          }
+          mbar_arrive_warp(&bars.xp_ready);
+        }
+        if (ok) {
+          tc_fence_after();
+          const float ej = cs.e[bf][j][t];
+          const float2 ee = make_float2(ej, ej), dd2 = make_float2(Dh, Dh);
+#pragma unroll
+          for (int pc = 0; pc < 8; ++pc) {  // 8 columns p in [8 pc, +8)
+            uint32_t rd[8], ro[8];
+            tmem_ld8(tD + lane_off + j * 64 + pc * 8, rd);
+            tmem_ld8(tO + lane_off + j * 64 + pc * 8, ro);
+            tmem_wait_ld();
+            float yv[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t xv = xw[pc * 4 + e];
+              const float2 a = fma2(ee, make_float2(__uint_as_float(ro[2 * e]),
+                                                    __uint_as_float(ro[2 * e + 1])),
+                                    make_float2(__uint_as_float(rd[2 * e]),
+                                                __uint_as_float(rd[2 * e + 1])));
+              const float2 yy = fma2(dd2, make_float2(bf16lo(xv), bf16hi(xv)), a);
+              yv[2 * e] = yy.x;
+              yv[2 * e + 1] = yy.y;
+            }
+            ystage<TY>::put8(stage, t, j, pc * 8, yv);
+          }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive_warp(&bars.y_staged);
+        mbar_arrive_warp(&bars.cs_empty[bf]);
+        if (__any_sync(0xffffffffu, !ok || *abort_v)) {
+          stop = true;
+          break;
+        }
+      }
     }
   } else {
-    // ------------------------------ compute warps ------------------------------
-    const int row = tid & 127, q = tid >> 7;
-    const int j = q >> 1, p0 = (q & 1) * 32;        // head and p-range of the state/epilogue
-    const int wq = warp & 3;                        // TMEM lane quarter of this warp
+    // ------------------------------ mask group (warps 12-19) ------------------------------
+    // Thread (row t = 32 (warp % 4) + lane, hf = (warp - 12) / 4): the 16-column groups
+    // cg = hf, hf + 2, hf + 4, hf + 6 of G (two at a time).  M_h[t, s] = G[t, s] exp(cs_t -
+    // cs_s) dt_s for s <= t, in bf16, written over TMEM columns 8h .. 8h+7 of the group.  Each
+    // warp takes one branch per group: the factorized product where all its rows are past the
+    // group, the exact exponent where some row meets it, zeros where none reaches it.
+    const int wq = warp & 3, hf = (warp - kWarpM) >> 2;
+    const int t = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    // entering state of the segment -> TMEM (lane n = row, columns (j, p0 .. p0+32))
-    {
-      const float* src =
-          h_in + (((int64_t(b) * sg.nseg + seg) * nheads + h0 + j) * kP + p0) * kN + row;
-#pragma unroll
-      for (int pc = 0; pc < 2; ++pc) {
-        uint32_t r[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(src[(pc * 16 + e) * kN]);
-        tmem_st16(tH + lane_off + j * 64 + p0 + pc * 16, r);
-      }
-      tmem_wait_st();
-    }
-    const float Dh = D ? D[h0 + j] : 0.f;
     bool ok = true;
-    uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
-    const int t = row;
-    const int wlast = wq * 32 + 31;                 // last row of this warp
-    const bool live0 = q * 16 <= wlast, live1 = (q + 4) * 16 <= wlast;
-    const uint32_t gaddr0 = tG + lane_off + q * 16, gaddr1 = gaddr0 + 64;
-    for (int k = 0; k < nb; ++k) {
+    for (int k = 0; k < nbt; ++k) {
       const uint32_t par = k & 1;
       const int bf = k & 1;
-      ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 50);
-      // ---- masked tiles.  Thread (row t, q) owns the 16-column groups q and q + 4 of G
-      //      (columns [16q, 16q+16) and [16q+64, 16q+80)), which spreads the rows' diagonal
-      //      groups over all warps.  M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for s <= t, in
-      //      bf16, written over TMEM columns 8h .. 8h+7 of the group.  Each warp takes one
-      //      branch per group: the factorized product where all its rows are past the group,
-      //      the exact exponent where some row meets it, zeros where none reaches it ----
-      float gv[32];
-      ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52);
-      if (ok && live0) {
+      ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 56, lim);
+      ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52, lim);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
         tc_fence_after();
-        uint32_t r0[16], r1[16];
-        tmem_ld16(gaddr0, r0);
-        if (live1) tmem_ld16(gaddr1, r1);
-        tmem_wait_ld();
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+          const int ga = hf + 4 * pass, gb = ga + 2;
+          const bool live_a = ga * 16 <= wq * 32 + 31, live_b = gb * 16 <= wq * 32 + 31;
+          float gv[32];
+          if (live_a) {
+            uint32_t r0[16], r1[16];
+            tmem_ld16(tG + lane_off + ga * 16, r0);
+            if (live_b) tmem_ld16(tG + lane_off + gb * 16, r1);
+            tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) { gv[e] = __uint_as_float(r0[e]); gv[16 + e] = __uint_as_float(r1[e]); }
-      }
-      // one 16-column group (gg = 0: group q, gg = 1: group q + 4) of head h's mask, packed
+            for (int e = 0; e < 16; ++e) {
+              gv[e] = __uint_as_float(r0[e]);
+              gv[16 + e] = live_b ? __uint_as_float(r1[e]) : 0.f;
+            }
+          }
+          // one 16-column group (GG = 0: ga, 1: gb) of head H's mask, packed into R[8]
 #define SSD_MASK_GROUP(H, GG, R)                                                               \
   {                                                                                            \
-    const int s0 = (q + 4 * (GG)) * 16;                                                        \
-    const bool live = (GG) ? live1 : live0;                                                    \
+    const int s0 = ((GG) ? gb : ga) * 16;                                                      \
+    const bool live = (GG) ? live_b : live_a;                                                  \
     if (wq * 32 >= s0 + 15) {                                                                  \
-      const float u = ex2(cs_sh[bf][H][t] - cs_sh[bf][H][s0 + 15]);                            \
+      const float u = ex2(cs.cs[bf][H][t] - cs.cs[bf][H][s0 + 15]);                            \
       const float2 uu = make_float2(u, u);                                                     \
-      const float4* vp = reinterpret_cast<const float4*>(&v_sh[bf][H][s0]);                    \
+      const float4* vp = reinterpret_cast<const float4*>(&cs.v[bf][H][s0]);                    \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 vv = vp[e4];                                                              \
         const float* gq = &gv[(GG) * 16 + 4 * e4];                                             \
@@ -884,9 +1317,9 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
         R[2 * e4 + 1] = pack_bf16x2(c.x, c.y);                                                 \
       }                                                                                        \
     } else if (live) {                                                                         \
-      const float ct = cs_sh[bf][H][t];                                                        \
+      const float ct = cs.cs[bf][H][t];                                                        \
       const float2 cc = make_float2(ct, ct);                                                   \
-      const float4* cp = reinterpret_cast<const float4*>(&cl_sh[bf][H][s0]);                   \
+      const float4* cp = reinterpret_cast<const float4*>(&cs.cl[bf][H][s0]);                   \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 cl = cp[e4];                                                              \
         const int s = s0 + 4 * e4;                                                             \
@@ -902,126 +1335,36 @@ __global__ void __launch_bounds__(kOutThreads, 1) chunk_out_kernel(
       _Pragma("unroll") for (int e = 0; e < 8; ++e) R[e] = 0u;                                \
     }                                                                                          \
   }
-      // head 0, then head 1 (its own TMEM columns, so no wait for the first diagonal MMA)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (ok) {
-          uint32_t r0[8], r1[8];
-          if (hh == 0) {
-            SSD_MASK_GROUP(0, 0, r0)
-            SSD_MASK_GROUP(0, 1, r1)
-          } else {
-            SSD_MASK_GROUP(1, 0, r0)
-            SSD_MASK_GROUP(1, 1, r1)
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t ra[8], rb[8];
+            if (hh == 0) {
+              SSD_MASK_GROUP(0, 0, ra)
+              SSD_MASK_GROUP(0, 1, rb)
+            } else {
+              SSD_MASK_GROUP(1, 0, ra)
+              SSD_MASK_GROUP(1, 1, rb)
+            }
+            tmem_st8(tG + lane_off + ga * 16 + hh * 8, ra);
+            tmem_st8(tG + lane_off + gb * 16 + hh * 8, rb);
           }
-          tmem_st8(gaddr0 + hh * 8, r0);
-          tmem_st8(gaddr1 + hh * 8, r1);
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        mbar_arrive_warp(hh == 0 ? &bars.m0_ready : &bars.m1_ready);
-      }
 #undef SSD_MASK_GROUP
-      // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
-      //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA and
-      //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
-      if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51);
-      if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55);
-      if (ok) {
-        tc_fence_after();
-        const float al = ex2(cs_sh[bf][j][kBlk - 1]);
-        uint8_t* hh = smem + kOffHh + j * kTile;
-        uint8_t* hl = smem + kOffHl + j * kTile;
-        uint32_t ra[16], rb[16];
-        tmem_ld16(tH + lane_off + j * 64 + p0, ra);
-        tmem_wait_ld();
-#define SSD_HPASS(R, PC)                                                                      \
-  {                                                                                           \
-    uint32_t hi[8], lo[8];                                                                    \
-    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
-        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
-    const int ch = (p0 >> 3) + (PC) * 2;                                                      \
-    *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);    \
-    *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
-    *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
-    *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
-    _Pragma("unroll") for (int e = 0; e < 8; ++e) {                                          \
-      const float2 sc = mul2(make_float2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1])), \
-                             make_float2(al, al));                                            \
-      R[2 * e] = __float_as_uint(sc.x);                                                       \
-      R[2 * e + 1] = __float_as_uint(sc.y);                                                   \
-    }                                                                                         \
-    tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
-  }
-        SSD_HPASS(ra, 0)
-        tmem_ld16(tH + lane_off + j * 64 + p0 + 16, rb);
-        tmem_wait_ld();
-        SSD_HPASS(rb, 1)
-#undef SSD_HPASS
+        }
         tmem_wait_st();
-        fence_proxy_async_smem();
       }
       tc_fence_before();
-      mbar_arrive_warp(&bars.h_ready);
-      // ---- once the diagonal MMAs are done: X' = w x in place for the state MMA (row t,
-      //      head j, p in [p0, p0+32)); then, once C H is done too, y_t = Diag + exp(cs_t) Off
-      //      + D x_t staged in shared memory and written by TMA ----
-      ok = ok && mbar_wait(&bars.d_done, par, abort_v, 54);
-      uint32_t xw[16];
-      if (ok) {
-        tc_fence_after();
-        const float wj = ex2(cs_sh[bf][j][kBlk - 1] - cl_sh[bf][j][t]);
-        uint8_t* xrow = smem + kOffX + j * kTile;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint4* pch = reinterpret_cast<uint4*>(xrow + swz(t, (p0 >> 3) + cc));
-          const uint4 v = *pch;
-          xw[cc * 4 + 0] = v.x; xw[cc * 4 + 1] = v.y; xw[cc * 4 + 2] = v.z; xw[cc * 4 + 3] = v.w;
-          const float2 ww = make_float2(wj, wj);
-          *pch = make_uint4(scale_bf16x2(v.x, ww), scale_bf16x2(v.y, ww), scale_bf16x2(v.z, ww),
-                            scale_bf16x2(v.w, ww));
-        }
-        fence_proxy_async_smem();
-      }
-      mbar_arrive_warp(&bars.xp_ready);
-      ok = ok && mbar_wait(&bars.o_done, par, abort_v, 57);
-      if (ok) {
-        tc_fence_after();
-        const float ej = ex2(cs_sh[bf][j][t]);
-#pragma unroll
-        for (int pc = 0; pc < 2; ++pc) {
-          uint32_t rd[16], ro[16];
-          tmem_ld16(tD + lane_off + j * 64 + p0 + pc * 16, rd);
-          tmem_ld16(tO + lane_off + j * 64 + p0 + pc * 16, ro);
-          tmem_wait_ld();
-          float yv[16];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t xv = xw[pc * 8 + e];
-            const float2 dd = fma2(make_float2(ej, ej),
-                                   make_float2(__uint_as_float(ro[2 * e]), __uint_as_float(ro[2 * e + 1])),
-                                   make_float2(__uint_as_float(rd[2 * e]), __uint_as_float(rd[2 * e + 1])));
-            const float2 yy = fma2(make_float2(Dh, Dh), make_float2(bf16lo(xv), bf16hi(xv)), dd);
-            yv[2 * e] = yy.x;
-            yv[2 * e + 1] = yy.y;
-          }
-          ystage<TY>::put16(stage, t, q, pc, yv);
-        }
-        fence_proxy_async_smem();
-      }
-      tc_fence_before();
-      mbar_arrive_warp(&bars.y_staged);
-      mbar_arrive_warp(&bars.cs_empty[bf]);  // done with block k's cumsums and TMEM reads
+      mbar_arrive_warp(&bars.m_ready);
+      mbar_arrive_warp(&bars.cs_empty[bf]);
       if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
     }
   }
   // ------------------------------ teardown ------------------------------
   __syncthreads();
-  if (*abort_v && warp == 17 && lane == 0) {  // let every issued MMA land before leaving
+  if (*abort_v && warp == kWarpMma && lane == 0) {  // let every issued MMA land before leaving
     mma_commit(&bars.drain);
     drain(&bars.drain, 0);
   }
-  if (*abort_v && warp == 16 && lane == 0) {  // and every issued copy
+  if (*abort_v && warp == kWarpTma && lane == 0) {  // and every issued copy
     if (n_c) drain(&bars.c_full, (n_c - 1) & 1);
     if (n_x) drain(&bars.x_full, (n_x - 1) & 1);
     for (int i = 0; i < 2; ++i)

@@ -82,23 +82,22 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Wait for phase `parity` of `bar` to complete, giving up after `limit_ns` nanoseconds or as
-// soon as *abort is set by another thread of the CTA.  On expiry: latch the device status
+// Wait for phase `parity` of `bar` to complete, giving up once `limit_ns` nanoseconds have
+// passed (checked before every sleep; limit 0: give up unless the phase is already complete) or
+// as soon as *abort is set by another thread of the CTA.  On expiry: latch the device status
 // word (SSD_ERR_DEVICE_TIMEOUT with `site`), set *abort, and return false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned site, uint64_t limit_ns = 2000000000ull) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test_sleep(bar, parity, 20000u)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
-        latch_status(SSD_ERR_DEVICE_TIMEOUT, site);
-        *abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (*abort) return false;
+    if (limit_ns == 0 || globaltimer() - t0 > limit_ns) {
+      latch_status(SSD_ERR_DEVICE_TIMEOUT, site);
+      *abort = 1;
+      return false;
     }
+    if (mbar_test_sleep(bar, parity, 20000u)) return true;
   }
 }
 
@@ -228,6 +227,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(

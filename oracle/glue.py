@@ -1,7 +1,7 @@
 """Float64 definitions of the steps either side of the SSD layer in a Mamba block -- TEST
 INFRASTRUCTURE (only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` may use it).
 
-"Puntata 205 -- State Space Models e Mamba" (aiperbabbani.it), section "Da S4 a Mamba": the
+"State Space Models (SSM)" (ultralytics.com glossary), section "Da S4 a Mamba": the
 selective SSM sits inside a block that runs its input through a short convolution, derives the
 step size from the input, and gates the output with a SiLU branch.  The pages name these steps
 but give no formula beyond that; the readings taken here are the plainest ones:

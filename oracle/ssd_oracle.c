@@ -28,7 +28,7 @@
  *  - input-dependent Delta, B, C (selectivity): same page, section
  *    "Mamba (Gu & Dao, dicembre 2023): selective scan".
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - the initial state is the state before token 0, so token 0 decays it once;
  *  - dt and A are used as given (no softplus or clamp inside);
  *  - inputs stored as bf16 or f32 are widened exactly to double.

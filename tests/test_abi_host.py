@@ -127,6 +127,76 @@ def test_sliced_scan_binding_refuses_cpu_tensors(lib):
         ssd.state_pass(torch.zeros(2, 1, 2, 64, 128), torch.zeros(2, 1, 2))
 
 
+def test_walk_plans_on_host(lib):
+    # one walk over whole sequences when there are about as many (batch row, head pair)
+    # sequences as SMs (a host without a GPU plans for 148); segments with a summary pass
+    # (seg_state + seg_pass + walk) when there are fewer
+    assert ssd.plan_info(4, 8192, 80, 64, 128, 1, 256) == dict(launches=1, ctas=148, segments=1)
+    p = ssd.plan_info(8, 2048, 24, 64, 128, 1, 256)
+    assert p["launches"] == 3 and p["segments"] >= 2 and p["ctas"] <= 148
+    p = ssd.plan_info(1, 1 << 20, 24, 64, 128, 1, 256)
+    assert p["launches"] == 3 and p["ctas"] == 148 and 8192 / p["segments"] <= 8192 * 12 / 148
+    # forced plans and CTA caps
+    assert ssd.plan_info(2, 1000, 4, 64, 128, 1, 256, max_ctas=3, plan=1) == \
+        dict(launches=1, ctas=3, segments=1)
+    assert ssd.plan_info(2, 1000, 4, 64, 128, 1, 256, max_ctas=3, plan=2)["segments"] >= 2
+    # every range is at least one segment long: one sequence of 47 blocks over 9 CTAs in
+    # segments of 6 blocks leaves 7 CTAs
+    p = ssd.plan_info(1, 6000, 2, 64, 128, 1, 256, max_ctas=9, plan=2)
+    assert p == dict(launches=3, ctas=7, segments=8)
+    # not a tensor-core shape / invalid
+    with pytest.raises(ssd.SSDError):
+        ssd.plan_info(1, 256, 4, 16, 16, 1, 64, ssd.SSD_F32)
+    with pytest.raises(ssd.SSDError):
+        ssd.plan_info(1, 256, 4, 64, 128, 1, 100)
+
+
+def test_scan_ex_rejects_bad_options_on_host(lib):
+    import ctypes
+    shape = [2, 300, 4, 64, 128, 1, 256, 1, 0]
+    for opts in [(-1, 0, 0), (0, 3, 0), (0, -1, 0), (0, 0, -2)]:
+        o = ssd.ScanOptions(*opts)
+        assert lib.ssd_chunk_scan_fwd_ex(*([None] * 9), *shape, None, 0, ctypes.byref(o),
+                                         None) == 1
+    # valid options, NULL pointers: still an argument error, nothing launched
+    o = ssd.ScanOptions(3, 1, -1)
+    assert lib.ssd_chunk_scan_fwd_ex(*([None] * 9), *shape, None, 0, ctypes.byref(o), None) == 1
+    # the float32 SIMT shapes have no tensor-core plan
+    assert lib.ssd_chunk_scan_fwd_ex(*([None] * 9), 1, 256, 4, 16, 16, 1, 64, 0, 0, None, 0,
+                                     None, None) == 2
+    # the workspace of a forced segment plan covers the segments' states
+    o1, o2 = ssd.ScanOptions(0, 1, 0), ssd.ScanOptions(0, 2, 0)
+    w1 = lib.ssd_chunk_scan_workspace_size_ex(4, 8192, 80, 64, 128, 1, 256, 1, ctypes.byref(o1))
+    w2 = lib.ssd_chunk_scan_workspace_size_ex(4, 8192, 80, 64, 128, 1, 256, 1, ctypes.byref(o2))
+    assert w1 > 0 and w2 >= w1
+
+
+def test_backward_rejects_bad_arguments_on_host(lib):
+    # ssd_chunk_scan_bwd(x, dt, A, B, C, D, init, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit,
+    #                    batch, seqlen, nheads, headdim, dstate, ngroups, io, ws, bytes, stream)
+    shape = [2, 300, 4, 64, 128, 1, 1]
+    assert lib.ssd_chunk_scan_bwd(*([None] * 16), *shape, None, 0, None) == 1  # NULL pointers
+    bad = list(shape)
+    bad[2], bad[5] = 3, 2  # 3 heads in 2 groups
+    assert lib.ssd_chunk_scan_bwd(*([None] * 16), *bad, None, 0, None) == 1
+    bad = list(shape)
+    bad[6] = 9  # io
+    assert lib.ssd_chunk_scan_bwd(*([None] * 16), *bad, None, 0, None) == 1
+    # tiles too large for one chunk in shared memory
+    assert lib.ssd_chunk_scan_bwd(*([None] * 16), 1, 128, 2, 128, 256, 1, 1, None, 0,
+                                  None) == 2
+    assert lib.ssd_chunk_scan_bwd_workspace_size(2, 300, 4, 64, 128, 1, 1) > 0
+    assert lib.ssd_chunk_scan_bwd_workspace_size(2, 300, 4, 64, 128, 3, 1) == 0
+
+
+def test_backward_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        ssd.chunk_scan_bwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 128),
+                           torch.zeros(1, 4, 1, 128), None, torch.zeros(1, 4, 2, 64))
+
+
 def test_glue_entry_points_reject_bad_arguments_on_host(lib):
     # ssd_conv_silu(u, w, bias, out, batch, seqlen, cdim, kwidth, io, stream)
     assert lib.ssd_conv_silu(None, None, None, None, 1, 8, 64, 4, 1, None) == 1  # NULL pointers

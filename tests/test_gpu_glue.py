@@ -79,6 +79,23 @@ def test_gate_silu(io, out_dtype):
     assert ssd.device_status() == 0
 
 
+def test_gate_silu_refuses_narrow_output_in_place():
+    """out == y with a bf16 out would overwrite y elements that other threads have not read yet
+    (a bf16 group of 8 covers the bytes of the first 4 float32 inputs of the same group):
+    SSD_ERR_INVALID_ARG before any launch, and y is untouched."""
+    y = torch.randn(4096, device="cuda")
+    y0 = y.clone()
+    z = torch.randn(4096, device="cuda").to(torch.bfloat16)
+    lib = ssd.load()
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = lib.ssd_gate_silu(y.data_ptr(), z.data_ptr(), y.data_ptr(), y.numel(), ssd.SSD_BF16,
+                           ssd.SSD_BF16, stream)
+    assert rc == 1  # SSD_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0)
+    assert ssd.device_status() == 0
+
+
 def test_glue_refuses_unsupported():
     u = torch.zeros(1, 4, 6, device="cuda", dtype=torch.bfloat16)  # 6 channels: not 8-aligned
     with pytest.raises(ssd.SSDError):

@@ -40,11 +40,11 @@ def check_full(inp, y, fin, tol=None):
     return ey, ef
 
 
-def small(io="bf16", seed=7, **shape):
+def small(io="bf16", seed=7, A_range=None, **shape):
     cfg = dict(batch=1, seqlen=256, nheads=4, headdim=64, dstate=128, ngroups=1, chunk=256,
                io=io, init="normal0.1")
     cfg.update(shape)
-    return ssd_inputs.make_scan_inputs(cfg, seed=seed)
+    return ssd_inputs.make_scan_inputs(cfg, seed=seed, A_range=A_range)
 
 
 # ---- the tiny float32 workload, every element ------------------------------------------------
@@ -86,12 +86,80 @@ def test_simt_path_small(io, shape):
 
 
 @pytest.mark.parametrize("chunk", [64, 128, 256])
-@pytest.mark.parametrize("simt", [False, True])
-def test_chunk_size_invariance(chunk, simt):
+def test_chunk_size_invariance(chunk):
     """The output does not depend on the block length (the duality's point); every admissible
-    chunk gives the oracle's answer, including a partial last chunk."""
+    chunk gives the oracle's answer, including a partial last chunk.  Only the SIMT kernels use
+    `chunk` as their block length: the tensor-core path evaluates 128-token blocks (the tcgen05
+    M = 128 tile) whatever the argument, so repeating it per chunk would rerun one computation."""
     inp = small(seed=11, batch=2, seqlen=700, nheads=4)
-    y, fin = run(inp, dev_inputs(inp), chunk=chunk, simt=simt)
+    y, fin = run(inp, dev_inputs(inp), chunk=chunk, simt=True)
+    check_full(inp, y, fin)
+
+
+def test_tensor_core_path_ignores_chunk():
+    """The tensor-core path's blocks are 128 tokens for every admissible chunk: bit-identical."""
+    inp = small(seed=11, batch=2, seqlen=700, nheads=4)
+    t = dev_inputs(inp)
+    ys = [run(inp, t, chunk=q) for q in (64, 128, 256)]
+    check_full(inp, *ys[0])
+    for y, fin in ys[1:]:
+        assert torch.equal(y, ys[0][0]) and torch.equal(fin, ys[0][1])
+
+
+# ---- the walk's plans ------------------------------------------------------------------------
+# plan 1: whole sequences, cut into ranges across CTAs, so that a range starting inside a
+# sequence takes the state published by the CTA that walked the sequence's head; plan 2: segments
+# whose entering states come from the summary pass, with ranges that also start inside segments.
+@pytest.mark.parametrize("plan,max_ctas,shape", [
+    (1, 3, dict(batch=2, seqlen=1000, nheads=4)),            # 4 x 8 blocks over 3 CTAs
+    (1, 3, dict(batch=1, seqlen=2100, nheads=8, ngroups=2)),  # 4 x 17 blocks, ragged tail
+    (1, 2, dict(batch=3, seqlen=300, nheads=2, init="zeros")),
+    (1, 5, dict(batch=2, seqlen=4500, nheads=6)),            # 6 x 36 blocks over 5 CTAs
+    (2, 5, dict(batch=1, seqlen=3000, nheads=4)),            # 3 segments of 8, ranges of 9.6
+    (2, 0, dict(batch=2, seqlen=777, nheads=6)),             # one-block segments
+    (2, 9, dict(batch=1, seqlen=6000, nheads=2)),            # one sequence, 9 segments
+])
+def test_walk_plans(plan, max_ctas, shape):
+    inp = small(seed=21 + max_ctas, **shape)
+    t = dev_inputs(inp)
+    y, fin = ssd.chunk_scan_fwd_ex(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], 256,
+                                   init_state=t["init"], max_ctas=max_ctas, plan=plan)
+    torch.cuda.synchronize()
+    assert ssd.device_status() == 0
+    check_full(inp, y, fin)
+
+
+def test_walk_plans_agree():
+    """Whole sequences and segments walk the same blocks with the same arithmetic per block;
+    only where the entering state of a stretch comes from differs."""
+    inp = small(seed=29, batch=2, seqlen=2000, nheads=4)
+    t = dev_inputs(inp)
+    out = []
+    for plan, ctas in ((1, 0), (1, 3), (2, 6)):
+        out.append(ssd.chunk_scan_fwd_ex(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], 256,
+                                         init_state=t["init"], max_ctas=ctas, plan=plan))
+    torch.cuda.synchronize()
+    assert ssd.device_status() == 0
+    for y, fin in out[1:]:
+        assert rel_err(to_np(y), to_np(out[0][0])) <= TOL["bf16"]
+        assert rel_err(to_np(fin), to_np(out[0][1])) <= TOL["bf16"]
+    check_full(inp, *out[0])
+
+
+@pytest.mark.parametrize("plan", [1, 2])
+def test_device_timeout_is_reported_and_recovered(plan):
+    """A wait that gives up: with no waiting allowed every CTA's first wait on an event that has
+    not happened yet expires.  The kernel latches SSD_ERR_DEVICE_TIMEOUT, lets its copies and
+    MMAs land, frees its tensor memory and returns; the next normal call on the same stream
+    is correct."""
+    inp = small(seed=33, batch=2, seqlen=1000, nheads=4)
+    t = dev_inputs(inp)
+    ssd.chunk_scan_fwd_ex(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], 256,
+                          init_state=t["init"], max_ctas=3, plan=plan, wait_limit_ns=-1)
+    torch.cuda.synchronize()
+    assert ssd.device_status() == 5  # SSD_ERR_DEVICE_TIMEOUT
+    assert ssd.device_status() == 0  # read and cleared
+    y, fin = run(inp, t)
     check_full(inp, y, fin)
 
 
@@ -113,6 +181,24 @@ def test_initial_state_only():
     inp = small(seed=12, batch=2, seqlen=640, nheads=4)
     inp["x"] = np.zeros_like(inp["x"])
     y, fin = run(inp, dev_inputs(inp))
+    check_full(inp, y, fin)
+
+
+@pytest.mark.parametrize("plan,max_ctas", [(0, 0), (1, 2), (2, 4)])
+def test_initial_state_only_survives(plan, max_ctas):
+    """x = 0 with slow decays (A in [-0.5, -0.05]) over three and a half blocks: the initial state
+    carries through every block and through the hand-offs between CTAs, and the final state is
+    far from underflow (so its check has teeth)."""
+    inp = small(seed=18, batch=2, seqlen=450, nheads=4, A_range=(0.05, 0.5))
+    inp["x"] = np.zeros_like(inp["x"])
+    t = dev_inputs(inp)
+    y, fin = ssd.chunk_scan_fwd_ex(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], 256,
+                                   init_state=t["init"], max_ctas=max_ctas, plan=plan)
+    torch.cuda.synchronize()
+    assert ssd.device_status() == 0
+    _, fo = oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                        init=inp["init"])
+    assert np.sqrt(np.mean(fo ** 2)) > 1e-3  # the state has not decayed away
     check_full(inp, y, fin)
 
 
@@ -256,16 +342,30 @@ def test_full_size_workload(cfg_idx, n_chains):
 
 
 def test_million_token_context():
+    """2^20 tokens, 24 heads: 256 sampled chains (and their final states) against the oracle,
+    compared 64 chains at a time; the RMS is taken over all compared elements."""
     inp = ssd_inputs.make_scan_inputs(3)
     cfg = inp["cfg"]
     t = dev_inputs(inp)
     y, fin = run(inp, t)
-    ids, b, h, p = sample_chains(cfg, 24, seed=3)
-    yo, fo = oracle_chains(inp, ids, b, h, p)
-    yg = to_np(y[torch.as_tensor(b), :, torch.as_tensor(h), torch.as_tensor(p)])
-    fg = to_np(fin[torch.as_tensor(b), torch.as_tensor(h), torch.as_tensor(p)])
-    assert rel_err(yg, yo) <= TOL["bf16"]
-    assert rel_err(fg, fo) <= TOL["bf16"]
+    ids, b, h, p = sample_chains(cfg, 256, seed=3)
+    max_y = max_f = 0.0
+    sq_y = sq_f = 0.0
+    n_y = n_f = 0
+    for s in range(0, len(ids), 64):
+        sl = slice(s, s + 64)
+        yo, fo = oracle_chains(inp, ids[sl], b[sl], h[sl], p[sl])
+        bb, hh, pp = (torch.as_tensor(v[sl]) for v in (b, h, p))
+        yg = to_np(y[bb, :, hh, pp])
+        fg = to_np(fin[bb, hh, pp])
+        max_y = max(max_y, float(np.max(np.abs(yg - yo))))
+        max_f = max(max_f, float(np.max(np.abs(fg - fo))))
+        sq_y += float(np.sum(yo ** 2))
+        sq_f += float(np.sum(fo ** 2))
+        n_y += yo.size
+        n_f += fo.size
+    assert max_y <= TOL["bf16"] * np.sqrt(sq_y / n_y)
+    assert max_f <= TOL["bf16"] * np.sqrt(sq_f / n_f)
 
 
 @pytest.mark.parametrize("simt", [False, True])

@@ -3,8 +3,9 @@
 
 Called through the C ABI and compared with ssd_chunk_scan_fwd on the same inputs, within the
 bf16 tolerance the parity tests use, on two calls in a row (the second call reuses the array the
-first one left behind).  This file is collected last so that a run stopping at the first failure
-has already run every other test; it also passes alone in a fresh process.
+first one left behind), and with the float64 oracle on sampled chains.  This file is collected
+last so that a run stopping at the first failure has already run every other test; it also
+passes alone in a fresh process.
 """
 import ctypes
 
@@ -13,7 +14,7 @@ import torch
 
 import mamba_ssd_scan_03_b200 as ssd
 import ssd_inputs
-from gpu_util import TOL, dev_inputs, rel_err, to_np
+from gpu_util import TOL, dev_inputs, oracle_chains, rel_err, sample_chains, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -31,10 +32,8 @@ def _noalloc_call(t, shape, y, fin):
 
 
 @pytest.mark.parametrize("shape", [
-    dict(batch=2, seqlen=1500, nheads=8),
-    # 320 heads x 32 KiB states per segment: the 32 MiB array holds 3 segments where the
-    # workspace path uses 8, so the two entry points cut the sequence differently
-    dict(batch=4, seqlen=2048, nheads=80),
+    dict(batch=2, seqlen=1500, nheads=8),      # segments with a summary pass
+    dict(batch=4, seqlen=2048, nheads=80),     # whole sequences handed between CTAs
 ])
 def test_noalloc_matches_workspace_entry_point(shape):
     cfg = dict(headdim=64, dstate=128, ngroups=1, chunk=256, io="bf16", init="normal0.1")
@@ -54,12 +53,20 @@ def test_noalloc_matches_workspace_entry_point(shape):
         assert ssd.device_status() == 0
         assert rel_err(to_np(y), to_np(y_ref)) <= TOL["bf16"], call
         assert rel_err(to_np(fin), to_np(f_ref)) <= TOL["bf16"], call
+    # and against the float64 oracle on sampled (b, h, p) chains
+    ids, b, h, p = sample_chains(cfg, 48, seed=5)
+    yo, fo = oracle_chains(inp, ids, b, h, p)
+    bb, hh, pp = (torch.as_tensor(v) for v in (b, h, p))
+    assert rel_err(to_np(y[bb, :, hh, pp]), yo) <= TOL["bf16"]
+    assert rel_err(to_np(fin[bb, hh, pp]), fo) <= TOL["bf16"]
 
 
 def test_noalloc_rejects_what_does_not_fit():
-    # 16 x 80 states of 32 KiB = 40 MiB > the 32 MiB array: rejected before any launch
+    # 256 x 40 one-block sequences: a CTA walks at most 14 of them, so the walk needs at least
+    # 732 CTAs and as many published 64 KiB states (46 MiB > the 32 MiB array): rejected before
+    # any launch
     lib = ssd.load()
-    rc = lib.ssd_chunk_scan_fwd_noalloc(*([None] * 9), 16, 1024, 80, 64, 128, 1, 256,
+    rc = lib.ssd_chunk_scan_fwd_noalloc(*([None] * 9), 256, 128, 80, 64, 128, 1, 256,
                                         ssd.SSD_BF16, ssd.SSD_F32, None)
     assert rc == 2  # SSD_ERR_UNSUPPORTED
     # float32 io has no tensor-core path, so no fixed-scratch variant either

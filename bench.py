@@ -285,6 +285,45 @@ def time_scan(c, dev, seed, y_dtype, steps, warmup, hbm):
             "steps": steps, "l2": "flushed before every timed call (256 MB write)"}
 
 
+def time_backward(c, dev, seed, steps, warmup, hbm):
+    """Mean time of one ssd_chunk_scan_bwd (all seven gradients) over a device-seeded workload,
+    each call timed alone after an L2 flush."""
+    import torch
+    import mamba_ssd_scan_03_b200 as ssd
+    t = device_scan_inputs(c, dev, seed)
+    g = torch.Generator(device=dev).manual_seed(seed + 7)
+    dy = torch.randn(t["x"].shape, generator=g, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(1, ssd.load().ssd_chunk_scan_bwd_workspace_size(
+        c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["ngroups"], 1)),
+        dtype=torch.uint8, device=dev)
+
+    def once():
+        ssd.chunk_scan_bwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], dy,
+                           init_state=t["init"], workspace=ws)
+
+    for _ in range(warmup):
+        once()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        once()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    assert ssd.device_status() == 0
+    ms = statistics.mean(times)
+    tok = c["batch"] * c["seqlen"]
+    del t, dy, flush, ws
+    torch.cuda.empty_cache()
+    return {"ms": round(ms, 5), "tokens_per_s": round(tok / (ms * 1e-3), 1),
+            "kernels": "float32 CUDA cores (cumsum, chunk states, state pass, adjoint summaries, "
+                       "adjoint pass, per-chunk gradients, group and head sums: 8 launches)",
+            "steps": steps, "l2": "flushed before every timed call (256 MB write)"}
+
+
 def scan_extras(dev, hbm, steps=5, warmup=3):
     """The other scan workloads: the 130M-layer and million-token shapes, the 2.7B layer with
     bf16 y, and the length sweep at the 2.7B layer's heads (batch 1)."""
@@ -296,6 +335,7 @@ def scan_extras(dev, hbm, steps=5, warmup=3):
     out[c3["name"]] = time_scan(c3, dev, 2103, torch.float32, steps, warmup, hbm)
     c2 = ssd_inputs.resolve(SCAN_CFG)
     out[c2["name"] + "_bf16y"] = time_scan(c2, dev, 2102, torch.bfloat16, steps, warmup, hbm)
+    out[c1["name"] + "_backward"] = time_backward(c1, dev, 2111, steps, warmup, hbm)
     sweep = []
     for L in (4096, 32768, 131072, 524288):
         c = dict(c2, batch=1, seqlen=L, init="zeros", name=f"sweep_{L}")

@@ -533,28 +533,31 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 //
 // Per block k (G = C B^T once for both heads; masks; diagonal tiles (L o G o dt) X; off-
 // diagonal C H; skip term D x; y store; then H <- exp(cs_end) H + B^T (w*x) in place), with
-// block = 768 threads in specialised roles, so that the CUDA-core phases of a block run side by
-// side and overlap the tensor-core work instead of following one another:
-//   warps 0-3   state group (thread = state row n = TMEM lane): per block, the bf16 high/low
-//               copy of H for C H and H <- exp(cs_end) H; per item, the entering state into TMEM
-//               and the exit state out of it (final_state or the published slot).
-//   warps 4-11  X' and epilogue group (thread = token row t of one head, all 64 p): X' = w x in
-//               place once the diagonal MMAs have read x; then y = Diag + exp(cs_t) Off + D x
-//               staged in shared memory.
-//   warps 12-19 mask group (thread = token row t, four of G's eight 16-column groups): the two
-//               heads' bf16 masked tiles written over G in TMEM.
-//   warp 20     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block.
-//   warp 21     MMA issuer (lane 0): G, then the diagonal tiles and C H in whichever order their
-//               inputs are ready, then the state update.
-//   warp 22     y writer (lane 0): TMA stores of each block's staged y.
-//   warp 23     cumsums: each block's dt of the two heads -> log2 cumsums and the factors the
-//               other groups use, one block ahead (lane l: rows 4l .. 4l+3).
-// Roles hand blocks to each other through mbarriers only (blocks are numbered across items, so
-// the rings run on from one item to the next); a thread is never more than one phase of a
-// barrier ahead of the slowest, because every barrier it waits on next needs an arrival that
-// the slowest makes after its own previous wait.  The last block of an item whose exit state is
-// kept also sends the bf16 remainder of X' through the tensor core (written over C's tiles once
-// C H is done), so that state carries about 16 bits of the block's input.
+// block = 640 threads in five roles:
+//   warps 0-15  compute (512 threads).  Thread (row = tid % 128, q = tid / 128): token row
+//               `row` of a block (state row n = row in the state passes) and a quarter of the
+//               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and
+//               the epilogue; G column groups q and q + 4 for the masks.  Four warps share
+//               each TMEM lane quarter, so every phase is spread over all 16 warps (a phase's
+//               latency, not only its instructions, bounds the block).  They also load each
+//               item's entering state into TMEM and store its exit state.
+//   warp 16     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block, and x
+//               of the block after next into L2.
+//   warp 17     MMA issuer (lane 0).
+//   warp 18     y writer (lane 0): TMA stores of each block's staged y, in two groups (one per
+//               head) whose halves of the staging buffer are handed back separately.
+//   warp 19     cumsums: loads each block's dt of the two heads and writes its log2 cumsums
+//               to shared memory, up to two blocks ahead (lane l: rows 4l .. 4l+3).
+// Per block the compute warps write the masks (MMA: diagonal tiles), then the state pass
+// (MMA: C H), then X' (MMA: state update) and the epilogue.  The masks come first so that the
+// previous block's y stores, which read the staging buffer the state pass overwrites, drain
+// while they are computed.  The last block of an item whose exit state is kept also sends the
+// bf16 remainder of X' through the tensor core (written over C's tiles once C H is done), so
+// that state carries about 16 bits of the block's input.  Roles hand blocks to each other
+// through mbarriers only (blocks are numbered across items, so the rings run on from one item to
+// the next); a thread is never more than one phase of a barrier ahead of the slowest, because
+// every barrier it waits on next needs an arrival that the slowest makes after its own previous
+// wait.
 // Shared memory (1024-aligned, 12 x 16 KB):
 //   sC   2 tiles  C, K-major (rows t), n halves
 //   sB   4 tiles  B, rows s, n halves, two slots (blocks k % 2): K-major for G = C B^T,
@@ -600,6 +603,16 @@ template <> struct ystage<float> {
     for (int q = 0; q < 4; ++q)
       tma_store_3d(map, stage + q * kTile, (h0 + q / 2) * kP + (q % 2) * 32, t0, b);
   }
+  // part 0: the boxes over the staging's tiles 0 and 2 (sHh and sHl of head 0); part 1: tiles 1
+  // and 3 (head 1)
+  static __device__ __forceinline__ void store_part(const CUtensorMap* map, const uint8_t* stage,
+                                                    int h0, int t0, int b, int part) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int q = part + 2 * i;
+      tma_store_3d(map, stage + q * kTile, (h0 + q / 2) * kP + (q % 2) * 32, t0, b);
+    }
+  }
 };
 template <> struct ystage<__nv_bfloat16> {
   static __device__ __forceinline__ void put16(uint8_t* stage, int t, int q, int half,
@@ -623,6 +636,11 @@ template <> struct ystage<__nv_bfloat16> {
                                                int h0, int t0, int b) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) tma_store_3d(map, stage + j * kTile, (h0 + j) * kP, t0, b);
+  }
+  // part j: head j's box, over the staging's tile j
+  static __device__ __forceinline__ void store_part(const CUtensorMap* map, const uint8_t* stage,
+                                                    int h0, int t0, int b, int part) {
+    tma_store_3d(map, stage + part * kTile, (h0 + part) * kP, t0, b);
   }
 };
 
@@ -706,37 +724,19 @@ __device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort, 
   return ok != 0;
 }
 
-// Warp roles of the walk (768 threads).
-constexpr int kWarpE = 4;     // warps 0-3: state group
-constexpr int kWarpM = 12;    // warps 4-11: X' and epilogue group; warps 12-19: mask group
-constexpr int kWarpTma = 20, kWarpMma = 21, kWarpY = 22, kWarpCs = 23;
-constexpr int kHThreads = 128, kEThreads = 256, kMThreads = 256;
-constexpr int kWalkThreads = 768;
-
-// The cumsum warp's per-block values, two buffers (block k in buffer k % 2), two heads.  Read
-// and written as float4 (16-byte aligned rows).
-struct __align__(16) WalkCs {
-  float cs[2][2][kBlk];  // inclusive log2 cumsum of dt A within the block
-  float cl[2][2][kBlk];  // cs - log2(dt) (+inf where dt = 0)
-  float v[2][2][kBlk];   // exp(cs_{s|15} - cs_s) dt_s (masks, factorized form)
-  float e[2][2][kBlk];   // exp(cs_t) (epilogue)
-  float w[2][2][kBlk];   // exp(cs_end - cs_t) dt_t (X')
-  float alpha[2][2];     // exp(cs_end) (state pass)
-};
-static_assert(offsetof(WalkCs, cl) % 16 == 0 && offsetof(WalkCs, v) % 16 == 0 &&
-                  offsetof(WalkCs, e) % 16 == 0 && offsetof(WalkCs, w) % 16 == 0,
-              "WalkCs rows must stay 16-byte aligned");
+constexpr int kComputeThreads = 512;
+constexpr int kWalkThreads = kComputeThreads + 128;
 
 // mbarriers of the walk (all in shared memory)
-struct WalkBars {
+struct OutBars {
   uint64_t c_full, b_full[2], x_full;        // TMA -> consumers
   uint64_t c_empty, b_empty[2], x_empty;     // MMA completion -> producer
-  uint64_t g_done, d_done, o_done, st_done;  // MMA completion -> compute groups
-  uint64_t m_ready, h_ready, xp_ready;       // masks / state pass / X' -> MMA issuer
-  uint64_t y_staged;                         // epilogue -> y writer and MMA issuer
-  uint64_t stage_free;                       // y writer -> state group
-  uint64_t cs_full[2], cs_empty[2];          // cumsum warp <-> compute groups
-  uint64_t pub;                              // state group: exit state written (published item)
+  uint64_t g_done, d_done, o_done, st_done;  // MMA completion -> compute
+  uint64_t m0_ready, m1_ready, h_ready, xp_ready;  // compute -> MMA issuer
+  uint64_t y_staged;                         // compute -> y writer
+  uint64_t stage_free[2];                    // y writer -> compute (halves of the staging)
+  uint64_t cs_full[2], cs_empty[2];          // cumsum warp <-> compute (per cumsum buffer)
+  uint64_t pub;                              // compute: exit state written (published item)
   uint64_t drain;
 };
 
@@ -751,9 +751,13 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ WalkBars bars;
+  __shared__ OutBars bars;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ __align__(16) WalkCs cs;  // per block (two buffers, block k % 2) and head
+  // per block (two buffers, block k in buffer k % 2) and head: log2 cumsums cs, cl = cs -
+  // log2(dt) (+inf where dt = 0), v_s = exp(cs_{s|15} - cs_s) dt_s
+  __shared__ __align__(16) float cs_sh[2][2][kBlk];
+  __shared__ __align__(16) float cl_sh[2][2][kBlk];
+  __shared__ __align__(16) float v_sh[2][2][kBlk];
   __shared__ WalkItem items_sh[kMaxItems];
   __shared__ int nitems_sh, nblocks_sh, range_sh;
   __shared__ int abort_flag;
@@ -762,7 +766,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
   const int warp = tid >> 5, lane = tid & 31;
   volatile int* abort_v = &abort_flag;
   uint32_t n_c = 0, n_x = 0, n_b[2] = {0, 0};  // the producer's loads issued per barrier
-  const uint64_t lim = pl.wait_ns;
 
   if (tid == 0) {
     abort_flag = 0;
@@ -778,15 +781,16 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     nitems_sh = n;
     nblocks_sh = nb;
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
-    for (int i = 0; i < int(sizeof(WalkBars) / 8); ++i) mbar_init(all + i, 1);
-    mbar_init(&bars.m_ready, kMThreads);
-    mbar_init(&bars.h_ready, kHThreads);
-    mbar_init(&bars.xp_ready, kEThreads);
-    mbar_init(&bars.y_staged, kEThreads);
-    mbar_init(&bars.pub, kHThreads);
+    for (int i = 0; i < int(sizeof(OutBars) / 8); ++i) mbar_init(all + i, 1);
+    mbar_init(&bars.m0_ready, kComputeThreads);
+    mbar_init(&bars.m1_ready, kComputeThreads);
+    mbar_init(&bars.h_ready, kComputeThreads);
+    mbar_init(&bars.xp_ready, kComputeThreads);
+    mbar_init(&bars.y_staged, kComputeThreads);
+    mbar_init(&bars.pub, kComputeThreads);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.cs_full[i], 32);
-      mbar_init(&bars.cs_empty[i], kHThreads + kEThreads + kMThreads);
+      mbar_init(&bars.cs_empty[i], kComputeThreads);
     }
     fence_mbar_init();
   }
@@ -799,12 +803,30 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
   const uint32_t sbase = smem_u32(smem);
   const int nit = nitems_sh, nbt = nblocks_sh, range = range_sh;
 
-  if (warp == kWarpTma) {
+  if (warp == 16) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_c);
+      // x of block jj (both heads) into L2, a couple of blocks ahead: its load into shared
+      // memory waits for the previous block's state MMA, and then hits L2
+      auto prefetch_x = [&](int jj) {
+        int acc = 0;
+        for (int i = 0; i < nit; ++i) {
+          const int len = items_sh[i].k1 - items_sh[i].k0;
+          if (jj < acc + len) {
+            const int pb = items_sh[i].seq / pl.npair, ph = (items_sh[i].seq % pl.npair) * 2;
+            const int pt = (items_sh[i].k0 + jj - acc) * kBlk;
+            tma_prefetch_3d(&tm_x, ph * kP, pt, pb);
+            tma_prefetch_3d(&tm_x, (ph + 1) * kP, pt, pb);
+            return;
+          }
+          acc += len;
+        }
+      };
+      constexpr int kAhead = 2;
+      for (int jj = 1; jj < kAhead; ++jj) prefetch_x(jj);
       int j = 0;
       bool ok = true;
       for (int it = 0; it < nit && ok; ++it) {
@@ -813,8 +835,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         const int g = h0 / heads_per_group;
         for (int k = w.k0; k < w.k1; ++k, ++j) {
           const int t0 = k * kBlk;
+          prefetch_x(j + kAhead);
           // B of block j into slot j % 2 once block j - 2's G and state MMAs are done
-          if (j >= 2 && !mbar_wait(&bars.b_empty[j & 1], ((j - 2) >> 1) & 1, abort_v, 33, lim)) {
+          if (j >= 2 && !mbar_wait(&bars.b_empty[j & 1], ((j - 2) >> 1) & 1, abort_v, 33, pl.wait_ns)) {
             ok = false;
             break;
           }
@@ -823,8 +846,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           mbar_arrive_expect_tx(&bars.b_full[j & 1], 2 * kTile);
           tma_load_3d(bdst, &tm_b, &bars.b_full[j & 1], g * kN, t0, b);
           tma_load_3d(bdst + kTile, &tm_b, &bars.b_full[j & 1], g * kN + 64, t0, b);
-          // C once block j - 1's G and C H are done
-          if (j >= 1 && !mbar_wait(&bars.c_empty, (j - 1) & 1, abort_v, 31, lim)) {
+          // C once block j - 1's C H is done
+          if (j >= 1 && !mbar_wait(&bars.c_empty, (j - 1) & 1, abort_v, 31, pl.wait_ns)) {
             ok = false;
             break;
           }
@@ -832,8 +855,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           mbar_arrive_expect_tx(&bars.c_full, 2 * kTile);
           tma_load_3d(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b);
           tma_load_3d(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b);
-          // x once block j - 1's diagonal and state MMAs are done
-          if (j >= 1 && !mbar_wait(&bars.x_empty, (j - 1) & 1, abort_v, 32, lim)) {
+          // x once block j - 1's state MMA is done
+          if (j >= 1 && !mbar_wait(&bars.x_empty, (j - 1) & 1, abort_v, 32, pl.wait_ns)) {
             ok = false;
             break;
           }
@@ -844,7 +867,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         }
       }
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == 17) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
       const uint32_t id_g = idesc_bf16(128, 128, 0, 0);
@@ -871,63 +894,43 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           if (it < nit) kend += items_sh[it].k1 - items_sh[it].k0;
         }
         const bool lo = it < nit && k == kend - 1 && items_sh[it].dst != kDstNone;
-        if (k > 0 && !mbar_wait(&bars.d_done, par ^ 1, abort_v, 41, lim)) break;  // G free
-        if (!mbar_wait(&bars.c_full, par, abort_v, 42, lim)) break;
-        if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43, lim)) break;
+        if (k > 0 && !mbar_wait(&bars.d_done, par ^ 1, abort_v, 41, pl.wait_ns)) break;  // G region free
+        if (!mbar_wait(&bars.c_full, par, abort_v, 42, pl.wait_ns)) break;
+        if (!mbar_wait(&bars.b_full[k & 1], (k >> 1) & 1, abort_v, 43, pl.wait_ns)) break;
         tc_fence_after();
         // G = C B^T (M = t, N = s, K = n)
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk)
           mma_ss(tG, dC + kmaj(kk), dBk + bslot + kmaj(kk), id_g, kk > 0 ? 1u : 0u);
         mma_commit(&bars.g_done);
-        // the diagonal and off-diagonal accumulators are free once block k - 1's epilogue has
-        // read them; x of block k must have landed
-        if (k > 0 && !mbar_wait(&bars.y_staged, par ^ 1, abort_v, 49, lim)) break;
-        if (!mbar_wait(&bars.x_full, par, abort_v, 45, lim)) break;
-        // Diag_h = M_h X_h (M = t, N = p, K = s; A = head h's bf16 mask in TMEM, columns
-        // 8h .. 8h+7 of each 16-column group) and Off = C (Hhi + Hlo) (M = t, N = (head, p),
-        // K = n), in whichever order the masks and the state pass finish
-        bool dd = false, oo = false, fail = false;
-        const uint64_t t0 = globaltimer();
-        while (!(dd && oo)) {
-          if (!dd && mbar_test(&bars.m_ready, par)) {
-            tc_fence_after();
+        // Diag_h = M_h X_h (M = t, N = p, K = s), A = head h's bf16 mask in TMEM (columns
+        // 8h .. 8h+7 of each 16-column group); head 0 while head 1's mask is being written
+        if (!mbar_wait(&bars.x_full, par, abort_v, 45, pl.wait_ns)) break;
+        auto diag = [&](int h) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+          for (int kk = 0; kk < kBlk / 16; ++kk)
+            mma_ts(tD + h * 64, tG + kk * 16 + h * 8, dX + h * (kTile >> 4) + kk * 128, id_diag,
+                   kk > 0 ? 1u : 0u);
+        };
+        if (!mbar_wait(&bars.m0_ready, par, abort_v, 46, pl.wait_ns)) break;
+        tc_fence_after();
+        diag(0);
+        if (!mbar_wait(&bars.m1_ready, par, abort_v, 48, pl.wait_ns)) break;
+        tc_fence_after();
+        diag(1);
+        mma_commit(&bars.d_done);
+        // Off = C (Hhi + Hlo) (M = t, N = (head, p), K = n)
+        if (!mbar_wait(&bars.h_ready, par, abort_v, 44, pl.wait_ns)) break;
+        tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < kBlk / 16; ++kk)
-                mma_ts(tD + h * 64, tG + kk * 16 + h * 8, dX + h * (kTile >> 4) + kk * 128,
-                       id_diag, kk > 0 ? 1u : 0u);
-            mma_commit(&bars.d_done);
-            dd = true;
-          }
-          if (!oo && mbar_test(&bars.h_ready, par)) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kN / 16; ++kk) {
-              mma_ss(tO, dC + kmaj(kk), dHh + kk * 128, id_off, kk > 0 ? 1u : 0u);
-              mma_ss(tO, dC + kmaj(kk), dHl + kk * 128, id_off, 1u);
-            }
-            mma_commit(&bars.o_done);
-            oo = true;
-          }
-          if (dd && oo) break;
-          if (*abort_v) {
-            fail = true;
-            break;
-          }
-          if (lim == 0 || globaltimer() - t0 > lim) {
-            latch_status(SSD_ERR_DEVICE_TIMEOUT, 46);
-            *abort_v = 1;
-            fail = true;
-            break;
-          }
-          __nanosleep(64);
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          mma_ss(tO, dC + kmaj(kk), dHh + kk * 128, id_off, kk > 0 ? 1u : 0u);
+          mma_ss(tO, dC + kmaj(kk), dHl + kk * 128, id_off, 1u);
         }
-        if (fail) break;
-        if (!lo) mma_commit(&bars.c_empty);  // G and C H of block k have read C
+        mma_commit(&bars.o_done);
+        if (!lo) mma_commit(&bars.c_empty);
         // H += B^T X' (M = n, N = (head, p), K = t), plus B^T X'_lo from C's tiles
-        if (!mbar_wait(&bars.xp_ready, par, abort_v, 47, lim)) break;
+        if (!mbar_wait(&bars.xp_ready, par, abort_v, 47, pl.wait_ns)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
@@ -940,7 +943,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         mma_commit(&bars.b_empty[k & 1]);
       }
     }
-  } else if (warp == kWarpY) {
+  } else if (warp == 18) {
     // ------------------------------ y writer ------------------------------
     if (lane == 0) {
       prefetch_tmap(&tm_y);
@@ -951,26 +954,32 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         const WalkItem w = items_sh[it];
         const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
         for (int k = w.k0; k < w.k1; ++k, ++j) {
-          if (!mbar_wait(&bars.y_staged, j & 1, abort_v, 61, lim)) {
+          if (!mbar_wait(&bars.y_staged, j & 1, abort_v, 61, pl.wait_ns)) {
             ok = false;
             break;
           }
-          ystage<TY>::store(&tm_y, stage, h0, k * kBlk, b);
+          // two store groups; each half of the staging buffer (head 0's sHh/sHl tiles, then head
+          // 1's) is handed back once its group has read it
+          ystage<TY>::store_part(&tm_y, stage, h0, k * kBlk, b, 0);
           bulk_commit();
-          bulk_wait_read();  // the staging buffer may be reused once the stores have read it
-          mbar_arrive(&bars.stage_free);
+          ystage<TY>::store_part(&tm_y, stage, h0, k * kBlk, b, 1);
+          bulk_commit();
+          bulk_wait_read_1();
+          mbar_arrive(&bars.stage_free[0]);
+          bulk_wait_read();
+          mbar_arrive(&bars.stage_free[1]);
         }
       }
       bulk_wait_all();
     }
-  } else if (warp == kWarpCs) {
+  } else if (warp == 19) {
     // ------------------------------ cumsums ------------------------------
     // Per block and head: cs_t = inclusive log2 cumsum of dt A (within the block), cl_t =
-    // cs_t - log2(dt_t) (+inf where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15
-    // (the masks), e_t = exp(cs_t) (the epilogue), w_t = exp(cs_end - cs_t) dt_t (X') and
-    // alpha = exp(cs_end) (the state pass).  The next block's dt is loaded meanwhile.
+    // cs_t - log2(dt_t) (+inf where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15.
+    // The next block's dt is loaded while the current one is processed.
     float v[8];  // dt of rows 4 lane + r, head h at v[2r + h]
     auto load = [&](int it, int kb) {
+      if (it >= nit) return;
       const WalkItem w = items_sh[it];
       const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
       const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
@@ -993,7 +1002,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
       for (int kb = w.k0; kb < w.k1; ++kb, ++j) {
         const int bf = j & 1;
         if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars.cs_empty[bf], ((j - 2) >> 1) & 1,
-                                                         abort_v, 58, lim))) {
+                                                         abort_v, 58, pl.wait_ns))) {
           ok = false;  // warp-uniform, so every lane reaches the same __syncwarp
           break;
         }
@@ -1014,300 +1023,90 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           const float l2 = d2 > 0.f ? c2 - __log2f(d2) : inf;
           const float l3 = d3 > 0.f ? c3 - __log2f(d3) : inf;
           const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
-          const float ce = __shfl_sync(0xffffffffu, c3, 31);        // cs at the block's end
-          *reinterpret_cast<float4*>(&cs.cs[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
-          *reinterpret_cast<float4*>(&cs.cl[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
-          *reinterpret_cast<float4*>(&cs.v[bf][h][4 * lane]) =
+          *reinterpret_cast<float4*>(&cs_sh[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
+          *reinterpret_cast<float4*>(&cl_sh[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
+          *reinterpret_cast<float4*>(&v_sh[bf][h][4 * lane]) =
               make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
-          *reinterpret_cast<float4*>(&cs.e[bf][h][4 * lane]) =
-              make_float4(ex2(c0), ex2(c1), ex2(c2), ex2(c3));
-          *reinterpret_cast<float4*>(&cs.w[bf][h][4 * lane]) =
-              make_float4(ex2(ce - l0), ex2(ce - l1), ex2(ce - l2), ex2(ce - l3));
-          if (lane == 0) cs.alpha[bf][h] = ex2(ce);
         }
         mbar_arrive_warp(&bars.cs_full[bf]);
         if (kb + 1 < w.k1) load(it, kb + 1);
         else if (it + 1 < nit) load(it + 1, items_sh[it + 1].k0);
       }
     }
-  } else if (warp < kWarpE) {
-    // ------------------------------ state group (warps 0-3) ------------------------------
-    // Thread n = tid: state row n (TMEM lane n), all 128 columns (head, p).  Per block: the bf16
-    // high/low copy of H for C H (sHh/sHl), then H <- alpha H in place; per item: the entering
-    // state into TMEM and the exit state out of it.
-    const int n = tid;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+  } else {
+    // ------------------------------ compute warps ------------------------------
+    const int row = tid & 127, q = tid >> 7;
+    const int j = q >> 1, p0 = (q & 1) * 32;        // head and p-range of the state/epilogue
+    const int wq = warp & 3;                        // TMEM lane quarter of this warp
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
     bool ok = true, stop = false;
-    int k = 0;
+    uint8_t* stage = smem + kOffHh;                 // y staging (sHh + sHl)
+    const int t = row;
+    const int wlast = wq * 32 + 31;                 // last row of this warp
+    const bool live0 = q * 16 <= wlast, live1 = (q + 4) * 16 <= wlast;
+    const uint32_t gaddr0 = tG + lane_off + q * 16, gaddr1 = gaddr0 + 64;
+    int k = 0;                                      // blocks walked so far (all items)
     for (int it = 0; it < nit && !stop; ++it) {
       const WalkItem w = items_sh[it];
       const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
-      // ---- entering state -> TMEM once the previous item's last state MMA is done ----
-      if (k > 0) ok = ok && mbar_wait(&bars.st_done, (k - 1) & 1, abort_v, 71, lim);
-      ok = __all_sync(0xffffffffu, ok);
+      // ---- the item's entering state -> TMEM (lane n = row, columns (j, p0 .. p0+32)), once
+      //      the previous item's last state MMA is done ----
+      if (k > 0) ok = ok && mbar_wait(&bars.st_done, (k - 1) & 1, abort_v, 71, pl.wait_ns);
       const float* src = nullptr;
-      int64_t hstride = int64_t(kP) * kN;  // from head h0 to h0 + 1
+      ok = __all_sync(0xffffffffu, ok);
       if (w.src == kSrcSlot) {
-        if (ok) ok = flag_wait(flags + (range - 1), abort_v, 74, lim);
-        src = slots + int64_t(range - 1) * kSlotFloats + n;
+        if (ok) ok = flag_wait(flags + (range - 1), abort_v, 74, pl.wait_ns);
+        src = slots + int64_t(range - 1) * kSlotFloats + (j * kP + p0) * kN + row;
       } else if (w.src == kSrcSeg) {
         const int seg = w.k0 / pl.seg_blks;
-        src = seg_hin + ((int64_t(b) * pl.nseg + seg) * nheads + h0) * kP * kN + n;
+        src = seg_hin + (((int64_t(b) * pl.nseg + seg) * nheads + h0 + j) * kP + p0) * kN + row;
       } else if (init_state) {
-        src = init_state + (int64_t(b) * nheads + h0) * kP * kN + n;
+        src = init_state + ((int64_t(b) * nheads + h0 + j) * kP + p0) * kN + row;
       }
+      ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {  // 16 columns (head c / 4, p = 16 (c % 4) ..) at a time
+#pragma unroll
+        for (int pc = 0; pc < 2; ++pc) {
           uint32_t r[16];
-          if (src) {
-            const float* sp = src + (c >> 2) * hstride + (c & 3) * 16 * kN;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(sp[e * kN]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = 0u;
-          }
-          tmem_st16(tH + lane_off + c * 16, r);
+          for (int e = 0; e < 16; ++e) r[e] = src ? __float_as_uint(src[(pc * 16 + e) * kN]) : 0u;
+          tmem_st16(tH + lane_off + j * 64 + p0 + pc * 16, r);
         }
         tmem_wait_st();
       }
-      for (int kb = w.k0; kb < w.k1; ++kb, ++k) {
-        const uint32_t par = k & 1;
-        const int bf = k & 1;
-        ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 50, lim);
-        const float al0 = cs.alpha[bf][0], al1 = cs.alpha[bf][1];
-        mbar_arrive_warp(&bars.cs_empty[bf]);
-        // H of block k is complete once block k - 1's state MMA is; sHh/sHl are free once block
-        // k - 1's y stores (staged there) have read them
-        if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51, lim);
-        if (k > 0) ok = ok && mbar_wait(&bars.stage_free, par ^ 1, abort_v, 55, lim);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {  // 32 columns: head c / 2, p in [32 (c % 2), +32)
-            const int j = c >> 1;
-            const float al = j ? al1 : al0;
-            uint8_t* hh = smem + kOffHh + j * kTile;
-            uint8_t* hl = smem + kOffHl + j * kTile;
-            uint32_t ra[16], rb[16];
-            tmem_ld16(tH + lane_off + c * 32, ra);
-            tmem_ld16(tH + lane_off + c * 32 + 16, rb);
-            tmem_wait_ld();
-            const int ch = (c & 1) * 4;  // 16-byte chunk of the 128-byte row
-#define SSD_HSPLIT(R, C0)                                                                     \
-  {                                                                                           \
-    uint32_t hi[8], lo[8];                                                                    \
-    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
-        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
-    *reinterpret_cast<uint4*>(hh + swz(n, C0)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);      \
-    *reinterpret_cast<uint4*>(hh + swz(n, C0 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);  \
-    *reinterpret_cast<uint4*>(hl + swz(n, C0)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);      \
-    *reinterpret_cast<uint4*>(hl + swz(n, C0 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);  \
-    _Pragma("unroll") for (int e = 0; e < 8; ++e) {                                          \
-      const float2 sc = mul2(make_float2(__uint_as_float(R[2 * e]),                          \
-                                         __uint_as_float(R[2 * e + 1])), make_float2(al, al)); \
-      R[2 * e] = __float_as_uint(sc.x);                                                       \
-      R[2 * e + 1] = __float_as_uint(sc.y);                                                   \
-    }                                                                                         \
-  }
-            SSD_HSPLIT(ra, ch)
-            SSD_HSPLIT(rb, ch + 2)
-#undef SSD_HSPLIT
-            tmem_st16(tH + lane_off + c * 32, ra);
-            tmem_st16(tH + lane_off + c * 32 + 16, rb);
-          }
-          tmem_wait_st();
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        mbar_arrive_warp(&bars.h_ready);
-        if (__any_sync(0xffffffffu, !ok || *abort_v)) {
-          stop = true;
-          break;
-        }
-      }
-      if (stop) break;
-      // ---- the item's exit state: final_state, or the slot the next range reads ----
-      if (w.dst != kDstNone) {
-        ok = ok && mbar_wait(&bars.st_done, (k - 1) & 1, abort_v, 72, lim);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-          tc_fence_after();
-          float* dst = w.dst == kDstFinal
-                           ? final_state + (int64_t(b) * nheads + h0) * kP * kN + n
-                           : slots + int64_t(range) * kSlotFloats + n;
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tH + lane_off + c * 16, r);
-            tmem_wait_ld();
-            float* d = dst + (c >> 2) * hstride + (c & 3) * 16 * kN;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) d[e * kN] = __uint_as_float(r[e]);
-          }
-        }
-        tc_fence_before();
-        if (w.dst == kDstSlot) {
-          __threadfence();
-          mbar_arrive_warp(&bars.pub);
-          if (tid == 0 && mbar_wait(&bars.pub, 0, abort_v, 73, lim)) {
-            __threadfence();
-            st_release_gpu(flags + range, 1);
-          }
-        }
-      }
-      if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
-    }
-  } else if (warp < kWarpM) {
-    // ------------------------------ X' and epilogue group (warps 4-11) ------------------------
-    // Thread (row t = 32 (warp % 4) + lane, head j = (warp - 4) / 4): token row t of head j, all
-    // 64 p.  Per block: X' = w x in place over the x tile once the diagonal MMAs have read it
-    // (x itself stays in registers for the skip term), then y_t = Diag + e_t Off + D x_t staged
-    // in shared memory for the y writer.
-    const int wq = warp & 3, j = (warp - kWarpE) >> 2;
-    const int t = wq * 32 + lane;
-    const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    uint8_t* stage = smem + kOffHh;
-    uint8_t* xrow = smem + kOffX + j * kTile;
-    bool ok = true, stop = false;
-    int k = 0;
-    for (int it = 0; it < nit && !stop; ++it) {
-      const WalkItem w = items_sh[it];
-      const int h0 = (w.seq % pl.npair) * 2;
       const float Dh = D ? D[h0 + j] : 0.f;
       for (int kb = w.k0; kb < w.k1; ++kb, ++k) {
         const uint32_t par = k & 1;
         const int bf = k & 1;
-        ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 53, lim);
-        ok = ok && mbar_wait(&bars.d_done, par, abort_v, 54, lim);
+        ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 50, pl.wait_ns);
+        // ---- masked tiles.  Thread (row t, q) owns the 16-column groups q and q + 4 of G
+        //      (columns [16q, 16q+16) and [16q+64, 16q+80)), which spreads the rows' diagonal
+        //      groups over all warps.  M_h[t, s] = G[t, s] exp(cs_t - cs_s) dt_s for s <= t, in
+        //      bf16, written over TMEM columns 8h .. 8h+7 of the group.  Each warp takes one
+        //      branch per group: the factorized product where all its rows are past the group,
+        //      the exact exponent where some row meets it, zeros where none reaches it ----
+        float gv[32];
+        ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52, pl.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
-        uint32_t xw[32];
-        if (ok) {
+        if (ok && live0) {
           tc_fence_after();
-          const float wj = cs.w[bf][j][t];
-          const float2 ww = make_float2(wj, wj);
+          uint32_t r0[16], r1[16];
+          tmem_ld16(gaddr0, r0);
+          if (live1) tmem_ld16(gaddr1, r1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4* pch = reinterpret_cast<uint4*>(xrow + swz(t, c));
-            const uint4 v = *pch;
-            xw[4 * c] = v.x;
-            xw[4 * c + 1] = v.y;
-            xw[4 * c + 2] = v.z;
-            xw[4 * c + 3] = v.w;
-            *pch = make_uint4(scale_bf16x2(v.x, ww), scale_bf16x2(v.y, ww), scale_bf16x2(v.z, ww),
-                              scale_bf16x2(v.w, ww));
-          }
-          fence_proxy_async_smem();
+          for (int e = 0; e < 16; ++e) { gv[e] = __uint_as_float(r0[e]); gv[16 + e] = __uint_as_float(r1[e]); }
         }
-        // the last block of an item whose exit state is kept also sends the bf16 remainder of
-        // X' (over C's tiles, free once C H is done), so that the state it leaves carries ~16
-        // bits of the block's input: its X' is handed over only then
-        const bool lo = kb == w.k1 - 1 && w.dst != kDstNone;
-        if (!lo) mbar_arrive_warp(&bars.xp_ready);
-        ok = ok && mbar_wait(&bars.o_done, par, abort_v, 57, lim);
-        ok = __all_sync(0xffffffffu, ok);
-        if (lo) {
-          if (ok) {
-            tc_fence_after();
-            const float wj = cs.w[bf][j][t];
-            uint8_t* lrow = smem + kOffC + j * kTile;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint32_t hi4[4], lo4[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint32_t xv = xw[4 * c + i];
-                split2(bf16lo(xv) * wj, bf16hi(xv) * wj, hi4[i], lo4[i]);
-              }
-              *reinterpret_cast<uint4*>(lrow + swz(t, c)) =
-                  make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
-            }
-            fence_proxy_async_smem();
-          }
-          mbar_arrive_warp(&bars.xp_ready);
-        }
-        if (ok) {
-          tc_fence_after();
-          const float ej = cs.e[bf][j][t];
-          const float2 ee = make_float2(ej, ej), dd2 = make_float2(Dh, Dh);
-#pragma unroll
-          for (int pc = 0; pc < 8; ++pc) {  // 8 columns p in [8 pc, +8)
-            uint32_t rd[8], ro[8];
-            tmem_ld8(tD + lane_off + j * 64 + pc * 8, rd);
-            tmem_ld8(tO + lane_off + j * 64 + pc * 8, ro);
-            tmem_wait_ld();
-            float yv[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t xv = xw[pc * 4 + e];
-              const float2 a = fma2(ee, make_float2(__uint_as_float(ro[2 * e]),
-                                                    __uint_as_float(ro[2 * e + 1])),
-                                    make_float2(__uint_as_float(rd[2 * e]),
-                                                __uint_as_float(rd[2 * e + 1])));
-              const float2 yy = fma2(dd2, make_float2(bf16lo(xv), bf16hi(xv)), a);
-              yv[2 * e] = yy.x;
-              yv[2 * e + 1] = yy.y;
-            }
-            ystage<TY>::put8(stage, t, j, pc * 8, yv);
-          }
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        mbar_arrive_warp(&bars.y_staged);
-        mbar_arrive_warp(&bars.cs_empty[bf]);
-        if (__any_sync(0xffffffffu, !ok || *abort_v)) {
-          stop = true;
-          break;
-        }
-      }
-    }
-  } else {
-    // ------------------------------ mask group (warps 12-19) ------------------------------
-    // Thread (row t = 32 (warp % 4) + lane, hf = (warp - 12) / 4): the 16-column groups
-    // cg = hf, hf + 2, hf + 4, hf + 6 of G (two at a time).  M_h[t, s] = G[t, s] exp(cs_t -
-    // cs_s) dt_s for s <= t, in bf16, written over TMEM columns 8h .. 8h+7 of the group.  Each
-    // warp takes one branch per group: the factorized product where all its rows are past the
-    // group, the exact exponent where some row meets it, zeros where none reaches it.
-    const int wq = warp & 3, hf = (warp - kWarpM) >> 2;
-    const int t = wq * 32 + lane;
-    const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    bool ok = true;
-    for (int k = 0; k < nbt; ++k) {
-      const uint32_t par = k & 1;
-      const int bf = k & 1;
-      ok = ok && mbar_wait(&bars.cs_full[bf], (k >> 1) & 1, abort_v, 56, lim);
-      ok = ok && mbar_wait(&bars.g_done, par, abort_v, 52, lim);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-          const int ga = hf + 4 * pass, gb = ga + 2;
-          const bool live_a = ga * 16 <= wq * 32 + 31, live_b = gb * 16 <= wq * 32 + 31;
-          float gv[32];
-          if (live_a) {
-            uint32_t r0[16], r1[16];
-            tmem_ld16(tG + lane_off + ga * 16, r0);
-            if (live_b) tmem_ld16(tG + lane_off + gb * 16, r1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              gv[e] = __uint_as_float(r0[e]);
-              gv[16 + e] = live_b ? __uint_as_float(r1[e]) : 0.f;
-            }
-          }
-          // one 16-column group (GG = 0: ga, 1: gb) of head H's mask, packed into R[8]
+        // one 16-column group (gg = 0: group q, gg = 1: group q + 4) of head h's mask, packed
 #define SSD_MASK_GROUP(H, GG, R)                                                               \
   {                                                                                            \
-    const int s0 = ((GG) ? gb : ga) * 16;                                                      \
-    const bool live = (GG) ? live_b : live_a;                                                  \
+    const int s0 = (q + 4 * (GG)) * 16;                                                        \
+    const bool live = (GG) ? live1 : live0;                                                    \
     if (wq * 32 >= s0 + 15) {                                                                  \
-      const float u = ex2(cs.cs[bf][H][t] - cs.cs[bf][H][s0 + 15]);                            \
+      const float u = ex2(cs_sh[bf][H][t] - cs_sh[bf][H][s0 + 15]);                            \
       const float2 uu = make_float2(u, u);                                                     \
-      const float4* vp = reinterpret_cast<const float4*>(&cs.v[bf][H][s0]);                    \
+      const float4* vp = reinterpret_cast<const float4*>(&v_sh[bf][H][s0]);                    \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 vv = vp[e4];                                                              \
         const float* gq = &gv[(GG) * 16 + 4 * e4];                                             \
@@ -1317,9 +1116,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         R[2 * e4 + 1] = pack_bf16x2(c.x, c.y);                                                 \
       }                                                                                        \
     } else if (live) {                                                                         \
-      const float ct = cs.cs[bf][H][t];                                                        \
+      const float ct = cs_sh[bf][H][t];                                                        \
       const float2 cc = make_float2(ct, ct);                                                   \
-      const float4* cp = reinterpret_cast<const float4*>(&cs.cl[bf][H][s0]);                   \
+      const float4* cp = reinterpret_cast<const float4*>(&cl_sh[bf][H][s0]);                   \
       _Pragma("unroll") for (int e4 = 0; e4 < 4; ++e4) {                                      \
         const float4 cl = cp[e4];                                                              \
         const int s = s0 + 4 * e4;                                                             \
@@ -1335,36 +1134,185 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
       _Pragma("unroll") for (int e = 0; e < 8; ++e) R[e] = 0u;                                \
     }                                                                                          \
   }
+        // head 0, then head 1 (its own TMEM columns, so no wait for the first diagonal MMA)
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t ra[8], rb[8];
+        for (int hh = 0; hh < 2; ++hh) {
+          if (ok) {
+            uint32_t r0[8], r1[8];
             if (hh == 0) {
-              SSD_MASK_GROUP(0, 0, ra)
-              SSD_MASK_GROUP(0, 1, rb)
+              SSD_MASK_GROUP(0, 0, r0)
+              SSD_MASK_GROUP(0, 1, r1)
             } else {
-              SSD_MASK_GROUP(1, 0, ra)
-              SSD_MASK_GROUP(1, 1, rb)
+              SSD_MASK_GROUP(1, 0, r0)
+              SSD_MASK_GROUP(1, 1, r1)
             }
-            tmem_st8(tG + lane_off + ga * 16 + hh * 8, ra);
-            tmem_st8(tG + lane_off + gb * 16 + hh * 8, rb);
+            tmem_st8(gaddr0 + hh * 8, r0);
+            tmem_st8(gaddr1 + hh * 8, r1);
+            tmem_wait_st();
           }
-#undef SSD_MASK_GROUP
+          tc_fence_before();
+          mbar_arrive_warp(hh == 0 ? &bars.m0_ready : &bars.m1_ready);
         }
-        tmem_wait_st();
+#undef SSD_MASK_GROUP
+        // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
+        //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA and
+        //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
+        if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51, pl.wait_ns);
+        if (k > 0) ok = ok && mbar_wait(&bars.stage_free[j], par ^ 1, abort_v, 55, pl.wait_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          const float al = ex2(cs_sh[bf][j][kBlk - 1]);
+          uint8_t* hh = smem + kOffHh + j * kTile;
+          uint8_t* hl = smem + kOffHl + j * kTile;
+          uint32_t ra[16], rb[16];
+          tmem_ld16(tH + lane_off + j * 64 + p0, ra);
+          tmem_wait_ld();
+#define SSD_HPASS(R, PC)                                                                      \
+  {                                                                                           \
+    uint32_t hi[8], lo[8];                                                                    \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e)                                            \
+        split2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1]), hi[e], lo[e]);      \
+    const int ch = (p0 >> 3) + (PC) * 2;                                                      \
+    *reinterpret_cast<uint4*>(hh + swz(row, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);    \
+    *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
+    *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
+    *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
+    _Pragma("unroll") for (int e = 0; e < 8; ++e) {                                          \
+      const float2 sc = mul2(make_float2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1])), \
+                             make_float2(al, al));                                            \
+      R[2 * e] = __float_as_uint(sc.x);                                                       \
+      R[2 * e + 1] = __float_as_uint(sc.y);                                                   \
+    }                                                                                         \
+    tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
+  }
+          SSD_HPASS(ra, 0)
+          tmem_ld16(tH + lane_off + j * 64 + p0 + 16, rb);
+          tmem_wait_ld();
+          SSD_HPASS(rb, 1)
+#undef SSD_HPASS
+          tmem_wait_st();
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive_warp(&bars.h_ready);
+        // ---- once the diagonal MMAs are done: X' = w x in place for the state MMA (row t,
+        //      head j, p in [p0, p0+32)); then, once C H is done too, y_t = Diag + exp(cs_t) Off
+        //      + D x_t staged in shared memory and written by TMA ----
+        ok = ok && mbar_wait(&bars.d_done, par, abort_v, 54, pl.wait_ns);
+        uint32_t xw[16];
+        if (ok) {
+          tc_fence_after();
+          const float wj = ex2(cs_sh[bf][j][kBlk - 1] - cl_sh[bf][j][t]);
+          uint8_t* xrow = smem + kOffX + j * kTile;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint4* pch = reinterpret_cast<uint4*>(xrow + swz(t, (p0 >> 3) + cc));
+            const uint4 v = *pch;
+            xw[cc * 4 + 0] = v.x; xw[cc * 4 + 1] = v.y; xw[cc * 4 + 2] = v.z; xw[cc * 4 + 3] = v.w;
+            const float2 ww = make_float2(wj, wj);
+            *pch = make_uint4(scale_bf16x2(v.x, ww), scale_bf16x2(v.y, ww), scale_bf16x2(v.z, ww),
+                              scale_bf16x2(v.w, ww));
+          }
+          fence_proxy_async_smem();
+        }
+        // the last block of an item whose exit state is kept also sends the bf16 remainder of
+        // X' (over C's tiles, free once C H is done): its X' is handed over only then
+        const bool lo = kb == w.k1 - 1 && w.dst != kDstNone;
+        if (!lo) mbar_arrive_warp(&bars.xp_ready);
+        ok = ok && mbar_wait(&bars.o_done, par, abort_v, 57, pl.wait_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (lo) {
+          if (ok) {
+            tc_fence_after();
+            const float wj = ex2(cs_sh[bf][j][kBlk - 1] - cl_sh[bf][j][t]);
+            uint8_t* lrow = smem + kOffC + j * kTile;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t hi4[4], lo4[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t xv = xw[cc * 4 + i];
+                split2(bf16lo(xv) * wj, bf16hi(xv) * wj, hi4[i], lo4[i]);
+              }
+              *reinterpret_cast<uint4*>(lrow + swz(t, (p0 >> 3) + cc)) =
+                  make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+            }
+            fence_proxy_async_smem();
+          }
+          mbar_arrive_warp(&bars.xp_ready);
+        }
+        if (ok) {
+          tc_fence_after();
+          const float ej = ex2(cs_sh[bf][j][t]);
+#pragma unroll
+          for (int pc = 0; pc < 2; ++pc) {
+            uint32_t rd[16], ro[16];
+            tmem_ld16(tD + lane_off + j * 64 + p0 + pc * 16, rd);
+            tmem_ld16(tO + lane_off + j * 64 + p0 + pc * 16, ro);
+            tmem_wait_ld();
+            float yv[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t xv = xw[pc * 8 + e];
+              const float2 dd = fma2(make_float2(ej, ej),
+                                     make_float2(__uint_as_float(ro[2 * e]), __uint_as_float(ro[2 * e + 1])),
+                                     make_float2(__uint_as_float(rd[2 * e]), __uint_as_float(rd[2 * e + 1])));
+              const float2 yy = fma2(make_float2(Dh, Dh), make_float2(bf16lo(xv), bf16hi(xv)), dd);
+              yv[2 * e] = yy.x;
+              yv[2 * e + 1] = yy.y;
+            }
+            ystage<TY>::put16(stage, t, q, pc, yv);
+          }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive_warp(&bars.y_staged);
+        mbar_arrive_warp(&bars.cs_empty[bf]);  // done with block k's cumsums and TMEM reads
+        if (__any_sync(0xffffffffu, !ok || *abort_v)) {
+          stop = true;
+          break;
+        }
       }
-      tc_fence_before();
-      mbar_arrive_warp(&bars.m_ready);
-      mbar_arrive_warp(&bars.cs_empty[bf]);
+      if (stop) break;
+      // ---- the item's exit state: final_state, or the slot the next range reads ----
+      if (w.dst != kDstNone) {
+        ok = ok && mbar_wait(&bars.st_done, (k - 1) & 1, abort_v, 72, pl.wait_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          float* dst = w.dst == kDstFinal
+                           ? final_state + ((int64_t(b) * nheads + h0 + j) * kP + p0) * kN + row
+                           : slots + int64_t(range) * kSlotFloats + (j * kP + p0) * kN + row;
+#pragma unroll
+          for (int pc = 0; pc < 2; ++pc) {
+            uint32_t r[16];
+            tmem_ld16(tH + lane_off + j * 64 + p0 + pc * 16, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[(pc * 16 + e) * kN] = __uint_as_float(r[e]);
+          }
+        }
+        tc_fence_before();
+        if (w.dst == kDstSlot) {
+          __threadfence();
+          mbar_arrive_warp(&bars.pub);
+          if (tid == 0 && mbar_wait(&bars.pub, 0, abort_v, 73, pl.wait_ns)) {
+            __threadfence();
+            st_release_gpu(flags + range, 1);
+          }
+        }
+      }
       if (__any_sync(0xffffffffu, !ok || *abort_v)) break;
     }
   }
   // ------------------------------ teardown ------------------------------
   __syncthreads();
-  if (*abort_v && warp == kWarpMma && lane == 0) {  // let every issued MMA land before leaving
+  if (*abort_v && warp == 17 && lane == 0) {  // let every issued MMA land before leaving
     mma_commit(&bars.drain);
     drain(&bars.drain, 0);
   }
-  if (*abort_v && warp == kWarpTma && lane == 0) {  // and every issued copy
+  if (*abort_v && warp == 16 && lane == 0) {  // and every issued copy
     if (n_c) drain(&bars.c_full, (n_c - 1) & 1);
     if (n_x) drain(&bars.x_full, (n_x - 1) & 1);
     for (int i = 0; i < 2; ++i)

@@ -606,11 +606,12 @@ template <> struct ystage<float> {
   // part 0: the boxes over the staging's tiles 0 and 2 (sHh and sHl of head 0); part 1: tiles 1
   // and 3 (head 1)
   static __device__ __forceinline__ void store_part(const CUtensorMap* map, const uint8_t* stage,
-                                                    int h0, int t0, int b, int part) {
+                                                    int h0, int t0, int b, int part,
+                                                    uint64_t policy) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int q = part + 2 * i;
-      tma_store_3d(map, stage + q * kTile, (h0 + q / 2) * kP + (q % 2) * 32, t0, b);
+      tma_store_3d_hint(map, stage + q * kTile, (h0 + q / 2) * kP + (q % 2) * 32, t0, b, policy);
     }
   }
 };
@@ -639,8 +640,9 @@ template <> struct ystage<__nv_bfloat16> {
   }
   // part j: head j's box, over the staging's tile j
   static __device__ __forceinline__ void store_part(const CUtensorMap* map, const uint8_t* stage,
-                                                    int h0, int t0, int b, int part) {
-    tma_store_3d(map, stage + part * kTile, (h0 + part) * kP, t0, b);
+                                                    int h0, int t0, int b, int part,
+                                                    uint64_t policy) {
+    tma_store_3d_hint(map, stage + part * kTile, (h0 + part) * kP, t0, b, policy);
   }
 };
 
@@ -809,6 +811,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_c);
+      // B and C tiles are read again by the other head pairs' CTAs: kept in L2; x is read once
+      const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
       // x of block jj (both heads) into L2, a couple of blocks ahead: its load into shared
       // memory waits for the previous block's state MMA, and then hits L2
       auto prefetch_x = [&](int jj) {
@@ -844,8 +848,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           uint8_t* bdst = smem + kOffB + (j & 1) * 2 * kTile;
           ++n_b[j & 1];
           mbar_arrive_expect_tx(&bars.b_full[j & 1], 2 * kTile);
-          tma_load_3d(bdst, &tm_b, &bars.b_full[j & 1], g * kN, t0, b);
-          tma_load_3d(bdst + kTile, &tm_b, &bars.b_full[j & 1], g * kN + 64, t0, b);
+          tma_load_3d_hint(bdst, &tm_b, &bars.b_full[j & 1], g * kN, t0, b, keep);
+          tma_load_3d_hint(bdst + kTile, &tm_b, &bars.b_full[j & 1], g * kN + 64, t0, b, keep);
           // C once block j - 1's C H is done
           if (j >= 1 && !mbar_wait(&bars.c_empty, (j - 1) & 1, abort_v, 31, pl.wait_ns)) {
             ok = false;
@@ -853,8 +857,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           }
           ++n_c;
           mbar_arrive_expect_tx(&bars.c_full, 2 * kTile);
-          tma_load_3d(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b);
-          tma_load_3d(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b);
+          tma_load_3d_hint(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b, keep);
+          tma_load_3d_hint(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b, keep);
           // x once block j - 1's state MMA is done
           if (j >= 1 && !mbar_wait(&bars.x_empty, (j - 1) & 1, abort_v, 32, pl.wait_ns)) {
             ok = false;
@@ -862,8 +866,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           }
           ++n_x;
           mbar_arrive_expect_tx(&bars.x_full, 2 * kTile);
-          tma_load_3d(smem + kOffX, &tm_x, &bars.x_full, h0 * kP, t0, b);
-          tma_load_3d(smem + kOffX + kTile, &tm_x, &bars.x_full, (h0 + 1) * kP, t0, b);
+          tma_load_3d_hint(smem + kOffX, &tm_x, &bars.x_full, h0 * kP, t0, b, stream);
+          tma_load_3d_hint(smem + kOffX + kTile, &tm_x, &bars.x_full, (h0 + 1) * kP, t0, b,
+                           stream);
         }
       }
     }
@@ -947,6 +952,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     // ------------------------------ y writer ------------------------------
     if (lane == 0) {
       prefetch_tmap(&tm_y);
+      const uint64_t stream = l2_evict_first();  // y is not read again here
       const uint8_t* stage = smem + kOffHh;
       int j = 0;
       bool ok = true;
@@ -960,9 +966,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
           }
           // two store groups; each half of the staging buffer (head 0's sHh/sHl tiles, then head
           // 1's) is handed back once its group has read it
-          ystage<TY>::store_part(&tm_y, stage, h0, k * kBlk, b, 0);
+          ystage<TY>::store_part(&tm_y, stage, h0, k * kBlk, b, 0, stream);
           bulk_commit();
-          ystage<TY>::store_part(&tm_y, stage, h0, k * kBlk, b, 1);
+          ystage<TY>::store_part(&tm_y, stage, h0, k * kBlk, b, 1, stream);
           bulk_commit();
           bulk_wait_read_1();
           mbar_arrive(&bars.stage_free[0]);

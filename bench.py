@@ -80,20 +80,21 @@ def step_bytes(c, y_bytes=4):
     return 2 * st + x + y + bc + c["batch"] * c["nheads"] * 4 + 2 * c["nheads"] * 4
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per scan call (sum over its kernels)
-# and per decode step, from one ncu capture of `python bench.py --profile ...` (profiles/), with
-# the hash of the device-code headers of those kernels (KERNEL_SOURCES) they were taken on:
-# reported only while those sources match.
-KERNEL_SOURCES = ("ssd_common.cuh", "tc_prims.cuh", "tc_kernels.cuh", "step_kernels.cuh")
-MEASURED_TRAFFIC = {"scan": (1633198592, "73cb014a6c26db98"),
-                    "decode": (1291061248, "73cb014a6c26db98")}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per scan call and per decode step,
+# from ncu captures of `python bench.py --profile ...` (profiles/), each with the hash of the
+# device-code headers of its kernels (KERNEL_SOURCES[kind]) it was taken on: reported only while
+# those sources match.
+KERNEL_SOURCES = {"scan": ("ssd_common.cuh", "tc_prims.cuh", "tc_kernels.cuh"),
+                  "decode": ("ssd_common.cuh", "step_kernels.cuh")}
+MEASURED_TRAFFIC = {"scan": (None, None),
+                    "decode": (1291061248, "1418c01d203c6f57")}
 
 
-def kernel_source_hash():
+def kernel_source_hash(kind):
     import hashlib
     d = os.path.join(ROOT, "mamba_ssd_scan_03_b200", "csrc")
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kind]:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
@@ -101,7 +102,7 @@ def kernel_source_hash():
 
 def measured_traffic(kind):
     nbytes, src = MEASURED_TRAFFIC[kind]
-    return nbytes if nbytes is not None and src == kernel_source_hash() else None
+    return nbytes if nbytes is not None and src == kernel_source_hash(kind) else None
 
 
 # B200 HBM3e bandwidth from the spec sheet (8 TB/s): a second denominator next to the measured

@@ -542,12 +542,14 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 //               latency, not only its instructions, bounds the block).  They also load each
 //               item's entering state into TMEM and store its exit state.
 //   warp 16     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block, and x
-//               of the block after next into L2.
+//               of the block after next into L2; and, with the whole warp, the cumsums: each
+//               block's dt of the two heads and its log2 cumsums in shared memory, up to two
+//               blocks ahead (lane l: rows 4l .. 4l+3).
 //   warp 17     MMA issuer (lane 0).
 //   warp 18     y writer (lane 0): TMA stores of each block's staged y, in two groups (one per
 //               head) whose halves of the staging buffer are handed back separately.
-//   warp 19     cumsums: loads each block's dt of the two heads and writes its log2 cumsums
-//               to shared memory, up to two blocks ahead (lane l: rows 4l .. 4l+3).
+// Warp w issues from scheduler w % 4; the compute warps of TMEM lane quarter 3 carry the most
+// mask work, so the three role warps sit on the other three schedulers.
 // Per block the compute warps write the masks (MMA: diagonal tiles), then the state pass
 // (MMA: C H), then X' (MMA: state update) and the epilogue.  The masks come first so that the
 // previous block's y stores, which read the staging buffer the state pass overwrites, drain
@@ -727,7 +729,7 @@ __device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort, 
 }
 
 constexpr int kComputeThreads = 512;
-constexpr int kWalkThreads = kComputeThreads + 128;
+constexpr int kWalkThreads = kComputeThreads + 96;
 
 // mbarriers of the walk (all in shared memory)
 struct OutBars {
@@ -806,64 +808,127 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
   const int nit = nitems_sh, nbt = nblocks_sh, range = range_sh;
 
   if (warp == 16) {
-    // ------------------------------ TMA producer ------------------------------
+    // ------------------------------ TMA producer (lane 0) and cumsums (whole warp) -----------
+    // Per block: B (double buffer), the block's cumsums, C, x.  Cumsums, per block and head:
+    // cs_t = inclusive log2 cumsum of dt A (within the block), cl_t = cs_t - log2(dt_t) (+inf
+    // where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15 (lane l: rows 4l .. 4l+3);
+    // the next block's dt is loaded while the current one is processed.  The cumsums of block j
+    // wait for block j - 2's compute to finish, which comes before block j - 1's C H, so the
+    // C and x loads after them are not held back.
+    const uint64_t keep = l2_evict_last(), stream = l2_evict_first();  // B/C reread, x once
+    // x of block jj (both heads) into L2, a couple of blocks ahead: its load into shared memory
+    // waits for the previous block's state MMA, and then hits L2
+    auto prefetch_x = [&](int jj) {
+      int acc = 0;
+      for (int i = 0; i < nit; ++i) {
+        const int len = items_sh[i].k1 - items_sh[i].k0;
+        if (jj < acc + len) {
+          const int pb = items_sh[i].seq / pl.npair, ph = (items_sh[i].seq % pl.npair) * 2;
+          const int pt = (items_sh[i].k0 + jj - acc) * kBlk;
+          tma_prefetch_3d(&tm_x, ph * kP, pt, pb);
+          tma_prefetch_3d(&tm_x, (ph + 1) * kP, pt, pb);
+          return;
+        }
+        acc += len;
+      }
+    };
+    constexpr int kAhead = 2;
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_c);
-      // B and C tiles are read again by the other head pairs' CTAs: kept in L2; x is read once
-      const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
-      // x of block jj (both heads) into L2, a couple of blocks ahead: its load into shared
-      // memory waits for the previous block's state MMA, and then hits L2
-      auto prefetch_x = [&](int jj) {
-        int acc = 0;
-        for (int i = 0; i < nit; ++i) {
-          const int len = items_sh[i].k1 - items_sh[i].k0;
-          if (jj < acc + len) {
-            const int pb = items_sh[i].seq / pl.npair, ph = (items_sh[i].seq % pl.npair) * 2;
-            const int pt = (items_sh[i].k0 + jj - acc) * kBlk;
-            tma_prefetch_3d(&tm_x, ph * kP, pt, pb);
-            tma_prefetch_3d(&tm_x, (ph + 1) * kP, pt, pb);
-            return;
-          }
-          acc += len;
-        }
-      };
-      constexpr int kAhead = 2;
       for (int jj = 1; jj < kAhead; ++jj) prefetch_x(jj);
-      int j = 0;
-      bool ok = true;
-      for (int it = 0; it < nit && ok; ++it) {
-        const WalkItem w = items_sh[it];
-        const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
-        const int g = h0 / heads_per_group;
-        for (int k = w.k0; k < w.k1; ++k, ++j) {
-          const int t0 = k * kBlk;
-          prefetch_x(j + kAhead);
-          // B of block j into slot j % 2 once block j - 2's G and state MMAs are done
-          if (j >= 2 && !mbar_wait(&bars.b_empty[j & 1], ((j - 2) >> 1) & 1, abort_v, 33, pl.wait_ns)) {
-            ok = false;
-            break;
-          }
+    }
+    float v[8];  // dt of rows 4 lane + r, head h at v[2r + h]
+    auto load_dt = [&](int it, int kb) {
+      if (it >= nit) return;
+      const WalkItem w = items_sh[it];
+      const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
+      const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int64_t tok = int64_t(kb) * kBlk + 4 * lane + r;
+        const bool in = tok < seqlen;
+        v[2 * r] = in ? dtb[tok * nheads] : 0.f;
+        v[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
+      }
+    };
+    if (nit > 0) load_dt(0, items_sh[0].k0);
+    const float inf = __int_as_float(0x7f800000);
+    // bounded wait by every lane, the same verdict in all of them
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, unsigned site) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, site, pl.wait_ns));
+    };
+    int j = 0;
+    bool ok = true;
+    for (int it = 0; it < nit && ok; ++it) {
+      const WalkItem w = items_sh[it];
+      const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
+      const int g = h0 / heads_per_group;
+      const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
+      for (int k = w.k0; k < w.k1; ++k, ++j) {
+        const int t0 = k * kBlk;
+        if (lane == 0) prefetch_x(j + kAhead);
+        // B of block j into slot j % 2 once block j - 2's G and state MMAs are done
+        if (j >= 2 && !wait_all(&bars.b_empty[j & 1], ((j - 2) >> 1) & 1, 33)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
           uint8_t* bdst = smem + kOffB + (j & 1) * 2 * kTile;
           ++n_b[j & 1];
           mbar_arrive_expect_tx(&bars.b_full[j & 1], 2 * kTile);
           tma_load_3d_hint(bdst, &tm_b, &bars.b_full[j & 1], g * kN, t0, b, keep);
           tma_load_3d_hint(bdst + kTile, &tm_b, &bars.b_full[j & 1], g * kN + 64, t0, b, keep);
-          // C once block j - 1's C H is done
-          if (j >= 1 && !mbar_wait(&bars.c_empty, (j - 1) & 1, abort_v, 31, pl.wait_ns)) {
-            ok = false;
-            break;
-          }
+        }
+        // cumsums of block j into buffer j % 2 once block j - 2's compute is done with it
+        const int bf = j & 1;
+        if (j >= 2 && !wait_all(&bars.cs_empty[bf], ((j - 2) >> 1) & 1, 58)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float d0 = v[h], d1 = v[2 + h], d2 = v[4 + h], d3 = v[6 + h];
+          float c0 = d0 * al[h];
+          float c1 = fmaf(d1, al[h], c0);
+          float c2 = fmaf(d2, al[h], c1);
+          float c3 = fmaf(d3, al[h], c2);
+          const float off = warp_inclusive_scan(c3) - c3;
+          c0 += off;
+          c1 += off;
+          c2 += off;
+          c3 += off;
+          const float l0 = d0 > 0.f ? c0 - __log2f(d0) : inf;
+          const float l1 = d1 > 0.f ? c1 - __log2f(d1) : inf;
+          const float l2 = d2 > 0.f ? c2 - __log2f(d2) : inf;
+          const float l3 = d3 > 0.f ? c3 - __log2f(d3) : inf;
+          const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
+          *reinterpret_cast<float4*>(&cs_sh[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
+          *reinterpret_cast<float4*>(&cl_sh[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
+          *reinterpret_cast<float4*>(&v_sh[bf][h][4 * lane]) =
+              make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
+        }
+        mbar_arrive_warp(&bars.cs_full[bf]);
+        if (k + 1 < w.k1) load_dt(it, k + 1);
+        else if (it + 1 < nit) load_dt(it + 1, items_sh[it + 1].k0);
+        // C once block j - 1's C H is done
+        if (j >= 1 && !wait_all(&bars.c_empty, (j - 1) & 1, 31)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
           ++n_c;
           mbar_arrive_expect_tx(&bars.c_full, 2 * kTile);
           tma_load_3d_hint(smem + kOffC, &tm_c, &bars.c_full, g * kN, t0, b, keep);
           tma_load_3d_hint(smem + kOffC + kTile, &tm_c, &bars.c_full, g * kN + 64, t0, b, keep);
-          // x once block j - 1's state MMA is done
-          if (j >= 1 && !mbar_wait(&bars.x_empty, (j - 1) & 1, abort_v, 32, pl.wait_ns)) {
-            ok = false;
-            break;
-          }
+        }
+        // x once block j - 1's state MMA is done
+        if (j >= 1 && !wait_all(&bars.x_empty, (j - 1) & 1, 32)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
           ++n_x;
           mbar_arrive_expect_tx(&bars.x_full, 2 * kTile);
           tma_load_3d_hint(smem + kOffX, &tm_x, &bars.x_full, h0 * kP, t0, b, stream);
@@ -977,67 +1042,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         }
       }
       bulk_wait_all();
-    }
-  } else if (warp == 19) {
-    // ------------------------------ cumsums ------------------------------
-    // Per block and head: cs_t = inclusive log2 cumsum of dt A (within the block), cl_t =
-    // cs_t - log2(dt_t) (+inf where dt = 0), v_s = exp(cs_r(s) - cs_s) dt_s with r(s) = s | 15.
-    // The next block's dt is loaded while the current one is processed.
-    float v[8];  // dt of rows 4 lane + r, head h at v[2r + h]
-    auto load = [&](int it, int kb) {
-      if (it >= nit) return;
-      const WalkItem w = items_sh[it];
-      const int b = w.seq / pl.npair, h0 = (w.seq % pl.npair) * 2;
-      const float* dtb = dt + int64_t(b) * seqlen * nheads + h0;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int64_t tok = int64_t(kb) * kBlk + 4 * lane + r;
-        const bool in = tok < seqlen;
-        v[2 * r] = in ? dtb[tok * nheads] : 0.f;
-        v[2 * r + 1] = in ? dtb[tok * nheads + 1] : 0.f;
-      }
-    };
-    if (nit > 0) load(0, items_sh[0].k0);
-    const float inf = __int_as_float(0x7f800000);
-    int j = 0;
-    bool ok = true;
-    for (int it = 0; it < nit && ok; ++it) {
-      const WalkItem w = items_sh[it];
-      const int h0 = (w.seq % pl.npair) * 2;
-      const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
-      for (int kb = w.k0; kb < w.k1; ++kb, ++j) {
-        const int bf = j & 1;
-        if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars.cs_empty[bf], ((j - 2) >> 1) & 1,
-                                                         abort_v, 58, pl.wait_ns))) {
-          ok = false;  // warp-uniform, so every lane reaches the same __syncwarp
-          break;
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float d0 = v[h], d1 = v[2 + h], d2 = v[4 + h], d3 = v[6 + h];
-          float c0 = d0 * al[h];
-          float c1 = fmaf(d1, al[h], c0);
-          float c2 = fmaf(d2, al[h], c1);
-          float c3 = fmaf(d3, al[h], c2);
-          const float off = warp_inclusive_scan(c3) - c3;
-          c0 += off;
-          c1 += off;
-          c2 += off;
-          c3 += off;
-          const float l0 = d0 > 0.f ? c0 - __log2f(d0) : inf;
-          const float l1 = d1 > 0.f ? c1 - __log2f(d1) : inf;
-          const float l2 = d2 > 0.f ? c2 - __log2f(d2) : inf;
-          const float l3 = d3 > 0.f ? c3 - __log2f(d3) : inf;
-          const float cr = __shfl_sync(0xffffffffu, c3, lane | 3);  // cs at row (4 lane) | 15
-          *reinterpret_cast<float4*>(&cs_sh[bf][h][4 * lane]) = make_float4(c0, c1, c2, c3);
-          *reinterpret_cast<float4*>(&cl_sh[bf][h][4 * lane]) = make_float4(l0, l1, l2, l3);
-          *reinterpret_cast<float4*>(&v_sh[bf][h][4 * lane]) =
-              make_float4(ex2(cr - l0), ex2(cr - l1), ex2(cr - l2), ex2(cr - l3));
-        }
-        mbar_arrive_warp(&bars.cs_full[bf]);
-        if (kb + 1 < w.k1) load(it, kb + 1);
-        else if (it + 1 < nit) load(it + 1, items_sh[it + 1].k0);
-      }
     }
   } else {
     // ------------------------------ compute warps ------------------------------

@@ -147,8 +147,14 @@ bool make_tc_plan(const Shape& s, const ScanOpts& o, TcPlan* out) {
   const int64_t nblk = (s.seqlen + ssd::tc::kBlk - 1) / ssd::tc::kBlk;
   const int64_t npair = s.nheads / 2, nseqs = s.batch * npair;
   if (nblk > (int64_t(1) << 30) || nseqs * nblk > (int64_t(1) << 40)) return false;
+  // Whole sequences (one launch: a CTA walks max(nblk, total / cap) blocks) unless the segment
+  // plan finishes sooner: its walk spreads total / cap blocks over every CTA, but its two
+  // summary kernels cost about kSegOverheadBlocks blocks' time (measured on the 130M-layer,
+  // 4K x 80-head and 1M-token shapes on B200).
+  constexpr int64_t kSegOverheadBlocks = 9;
+  const int64_t share = (nseqs * nblk + cap - 1) / cap;
   const bool whole =
-      nblk == 1 || o.plan == 1 || (o.plan == 0 && nseqs * 5 >= int64_t(cap) * 4);
+      nblk == 1 || o.plan == 1 || (o.plan == 0 && nblk <= share + kSegOverheadBlocks);
   int64_t nseg = whole ? 1 : std::min<int64_t>(nblk, std::max<int64_t>(2, (cap + nseqs - 1) / nseqs));
   const int64_t seg_blks = (nblk + nseg - 1) / nseg;
   nseg = (nblk + seg_blks - 1) / seg_blks;

@@ -816,8 +816,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     // wait for block j - 2's compute to finish, which comes before block j - 1's C H, so the
     // C and x loads after them are not held back.
     const uint64_t keep = l2_evict_last(), stream = l2_evict_first();  // B/C reread, x once
-    // x of block jj (both heads) into L2, a couple of blocks ahead: its load into shared memory
-    // waits for the previous block's state MMA, and then hits L2
+    // x of block jj (both heads) into L2, a block ahead: its load into shared memory waits for
+    // the previous block's state MMA, and then hits L2 (two blocks ahead measured slower, three
+    // slower still)
     auto prefetch_x = [&](int jj) {
       int acc = 0;
       for (int i = 0; i < nit; ++i) {
@@ -832,12 +833,11 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         acc += len;
       }
     };
-    constexpr int kAhead = 2;
+    constexpr int kAhead = 1;
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_c);
-      for (int jj = 1; jj < kAhead; ++jj) prefetch_x(jj);
     }
     float v[8];  // dt of rows 4 lane + r, head h at v[2r + h]
     auto load_dt = [&](int it, int kb) {

@@ -128,11 +128,14 @@ def test_sliced_scan_binding_refuses_cpu_tensors(lib):
 
 
 def test_walk_plans_on_host(lib):
-    # one walk over whole sequences when there are about as many (batch row, head pair)
-    # sequences as SMs (a host without a GPU plans for 148); segments with a summary pass
-    # (seg_state + seg_pass + walk) when there are fewer
+    # one walk over whole sequences unless a sequence is longer than every CTA's share of all
+    # blocks plus the segment plan's overhead (9 blocks; a host without a GPU plans for 148
+    # SMs); segments with a summary pass (seg_state + seg_pass + walk) otherwise
     assert ssd.plan_info(4, 8192, 80, 64, 128, 1, 256) == dict(launches=1, ctas=148, segments=1)
-    p = ssd.plan_info(8, 2048, 24, 64, 128, 1, 256)
+    # 130M layer: 96 sequences of 16 blocks, share 11 -> whole sequences on 96 CTAs
+    assert ssd.plan_info(8, 2048, 24, 64, 128, 1, 256) == dict(launches=1, ctas=96, segments=1)
+    # 40 sequences of 32 blocks, share 9 -> segments
+    p = ssd.plan_info(1, 4096, 80, 64, 128, 1, 256)
     assert p["launches"] == 3 and p["segments"] >= 2 and p["ctas"] <= 148
     p = ssd.plan_info(1, 1 << 20, 24, 64, 128, 1, 256)
     assert p["launches"] == 3 and p["ctas"] == 148 and 8192 / p["segments"] <= 8192 * 12 / 148

@@ -48,17 +48,16 @@ constexpr int kQ = 64;         // tokens per chunk of the backward (the result d
 constexpr int kThreads = 256;
 
 // ---- 1. adjoint summaries: grid (nchunks, batch * nheads), block 256 ------------------------
-// S'_c[p, n] = sum_{t in c} exp(cs_t) dy_t[p] C_t[n], stored [b][c][h][p][n].
+// S'_c[p, n] = sum_{t in c} exp(cs_t) dy_t[p] C_t[n], stored [b][c][h][p][n] (outer_sum).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) adj_state_kernel(
+__global__ void __launch_bounds__(kOuterThreads) adj_state_kernel(
     const float* __restrict__ dy, const T* __restrict__ Cm, const float* __restrict__ cs,
     float* __restrict__ adj, int64_t seqlen, int nheads, int headdim, int dstate, int ngroups,
     int nchunks) {
-  constexpr int TS = 16;   // tokens per shared-memory tile
-  constexpr int OPT = 16;  // outputs per thread per pass
   extern __shared__ float sm[];
-  float* ys = sm;                 // [TS][headdim]  exp(cs_t) dy_t
-  float* cb = sm + TS * headdim;  // [TS][dstate]   C_t
+  const int P4 = round4(headdim), N4 = round4(dstate);
+  float* us = sm;                    // [TS][P4]  exp(cs_t) dy_t
+  float* vs = sm + kOuterTS * P4;    // [TS][N4]  C_t
   const int c = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = int(bh % nheads);
@@ -66,45 +65,24 @@ __global__ void __launch_bounds__(kThreads) adj_state_kernel(
   const int g = h / (nheads / ngroups);
   const float* csb = cs + (bh * nchunks + c) * kQ;
   const int64_t t0 = int64_t(c) * kQ;
-  const int nout = headdim * dstate;
-  float* out = adj + ((b * nchunks + c) * nheads + h) * int64_t(nout);
-  for (int base = 0; base < nout; base += kThreads * OPT) {
-    float acc[OPT];
-#pragma unroll
-    for (int i = 0; i < OPT; ++i) acc[i] = 0.f;
-    for (int s0 = 0; s0 < kQ; s0 += TS) {
-      __syncthreads();
-      for (int i = threadIdx.x; i < TS * headdim; i += kThreads) {
-        const int s = i / headdim, p = i % headdim;
-        const int64_t tok = t0 + s0 + s;
-        ys[i] = tok < seqlen ? expf(csb[s0 + s]) * dy[((b * seqlen + tok) * nheads + h) * headdim + p]
-                             : 0.f;
-      }
-      for (int i = threadIdx.x; i < TS * dstate; i += kThreads) {
-        const int s = i / dstate, n = i % dstate;
-        const int64_t tok = t0 + s0 + s;
-        cb[i] = tok < seqlen
-                    ? io_traits<T>::load(Cm, ((b * seqlen + tok) * ngroups + g) * dstate + n)
-                    : 0.f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < OPT; ++i) {
-        const int o = base + i * kThreads + threadIdx.x;  // o = p * dstate + n
-        if (o < nout) {
-          const int p = o / dstate, n = o % dstate;
-          float a = acc[i];
-          for (int s = 0; s < TS; ++s) a = fmaf(ys[s * headdim + p], cb[s * dstate + n], a);
-          acc[i] = a;
-        }
-      }
+  float* out = adj + ((b * nchunks + c) * nheads + h) * int64_t(headdim) * dstate;
+  auto stage = [&](int s0, float* u, float* v) {
+    for (int i = threadIdx.x; i < kOuterTS * P4; i += kOuterThreads) {
+      const int s = i / P4, p = i % P4;
+      const int64_t tok = t0 + s0 + s;
+      u[i] = p < headdim && tok < seqlen
+                 ? expf(csb[s0 + s]) * dy[((b * seqlen + tok) * nheads + h) * headdim + p]
+                 : 0.f;
     }
-#pragma unroll
-    for (int i = 0; i < OPT; ++i) {
-      const int o = base + i * kThreads + threadIdx.x;
-      if (o < nout) out[o] = acc[i];
+    for (int i = threadIdx.x; i < kOuterTS * N4; i += kOuterThreads) {
+      const int s = i / N4, n = i % N4;
+      const int64_t tok = t0 + s0 + s;
+      v[i] = n < dstate && tok < seqlen
+                 ? io_traits<T>::load(Cm, ((b * seqlen + tok) * ngroups + g) * dstate + n)
+                 : 0.f;
     }
-  }
+  };
+  outer_sum(stage, kQ, headdim, dstate, out, us, vs);
 }
 
 // ---- 2. adjoint passing: one thread per state element, chunks last to first ------------------
@@ -121,27 +99,119 @@ __global__ void adj_pass_kernel(float* __restrict__ adj, const float* __restrict
   const int h = int(bh % nheads);
   const int64_t b = bh / nheads;
   float run = dfinal ? dfinal[e] : 0.f;
-  for (int c = nchunks - 1; c >= 0; --c) {
-    float* slot = adj + ((b * nchunks + c) * nheads + h) * per_bh + pn;
-    const float s = *slot;
-    *slot = run;
-    run = fmaf(expf(cs[(bh * nchunks + c) * kQ + kQ - 1]), run, s);
+  float* base = adj + (b * nchunks * nheads + h) * per_bh + pn;  // chunk c: + c * cstride
+  const int64_t cstride = int64_t(nheads) * per_bh;
+  const float* last = cs + bh * nchunks * kQ + kQ - 1;  // chunk c's last cumsum: + c * kQ
+  // kBatch chunks' loads in flight at once, then the recurrence over them (last chunk first)
+  constexpr int kBatch = 8;
+  for (int c0 = nchunks - 1; c0 >= 0; c0 -= kBatch) {
+    float sv[kBatch], lv[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t c = c0 - i;
+      if (c >= 0) {
+        sv[i] = base[c * cstride];
+        lv[i] = last[c * kQ];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t c = c0 - i;
+      if (c >= 0) {
+        base[c * cstride] = run;
+        run = fmaf(expf(lv[i]), run, sv[i]);
+      }
+    }
   }
   if (dinit) dinit[e] = run;
 }
 
 // ---- 3. per-chunk gradients: grid (nchunks, batch * nheads), block 256 ------------------------
-// Shared memory (floats): x [kQ][P + 1], dy [kQ][P], B [kQ][N + 1], C [kQ][N]; H, R [N][P + 1];
-// CB, XY, L [kQ][kQ]; per-token scalars.  The padded rows keep both the row and the column
-// walks over x, B, H and R free of bank conflicts.
+// Every product of the chunk is a small matrix product from shared memory, 4 x 4 outputs per
+// thread and product (thread (a, b) = (tid / 16, tid % 16): rows 4a .. 4a+3, columns
+// 4b .. 4b+3 of each 64-column pass) with float4 operand loads.
+// Shared memory (floats; rows padded to multiples of 4 plus 4, which keeps float4 rows aligned
+// and spreads the strided row walks over the banks):
+//   x, dy [kQ][P4 + 4]; B, C [kQ][N4 + 4]; H, R [P4][N4 + 4] (as stored: [p][n]);
+//   three [kQ][kQ] tables, first C.B, x.dy and L, then (in place) M[tau][t] = L (C_tau . B_t),
+//   N2[tau][t] = L[tau][t] (x_t . dy_tau) and K2[t][s] = dt_s N2[t][s];
+//   row and column partials of K [16][kQ] each; per-token scalars.
 // Outputs: dx [b, t, h, p]; ddt [b, t, h]; the head's dB and dC rows into dbh, dch
 // [b, t, h, n] (summed over the group by the reduce kernel); partial dA and dD per (b, c, h).
 struct BwdSmem {
+  static __host__ __device__ int px(int P) { return round4(P) + 4; }
+  static __host__ __device__ int nx(int N) { return round4(N) + 4; }
   static __host__ __device__ size_t floats(int P, int N) {
-    return size_t(kQ) * (2 * P + 2 * N + 2) + 2 * size_t(N) * (P + 1) + 3 * size_t(kQ) * kQ +
-           8 * kQ + 64;
+    return size_t(kQ) * 2 * (px(P) + nx(N)) + 2 * size_t(round4(P)) * nx(N) +
+           3 * size_t(kQ) * kQ + 2 * 16 * size_t(kQ) + 8 * kQ + 64;
   }
 };
+
+// acc[i][j] += sum_{k0 <= k < k1} A[m0 + i][k] B[k][n0 + j]   (k0, k1 multiples of 4)
+__device__ __forceinline__ void mm_nn(float (&acc)[4][4], const float* A, int sa, const float* B,
+                                      int sb, int m0, int n0, int k0, int k1) {
+  for (int k = k0; k < k1; k += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * sa + k);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 bv = *reinterpret_cast<const float4*>(B + (k + u) * sb + n0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float av = u == 0 ? a[i].x : u == 1 ? a[i].y : u == 2 ? a[i].z : a[i].w;
+        acc[i][0] = fmaf(av, bv.x, acc[i][0]);
+        acc[i][1] = fmaf(av, bv.y, acc[i][1]);
+        acc[i][2] = fmaf(av, bv.z, acc[i][2]);
+        acc[i][3] = fmaf(av, bv.w, acc[i][3]);
+      }
+    }
+  }
+}
+// acc[i][j] += sum_{k0 <= k < k1} A[k][m0 + i] B[k][n0 + j]
+__device__ __forceinline__ void mm_tn(float (&acc)[4][4], const float* A, int sa, const float* B,
+                                      int sb, int m0, int n0, int k0, int k1) {
+  for (int k = k0; k < k1; ++k) {
+    const float4 av = *reinterpret_cast<const float4*>(A + k * sa + m0);
+    const float4 bv = *reinterpret_cast<const float4*>(B + k * sb + n0);
+    const float aa[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[i][0] = fmaf(aa[i], bv.x, acc[i][0]);
+      acc[i][1] = fmaf(aa[i], bv.y, acc[i][1]);
+      acc[i][2] = fmaf(aa[i], bv.z, acc[i][2]);
+      acc[i][3] = fmaf(aa[i], bv.w, acc[i][3]);
+    }
+  }
+}
+// acc[i][j] += sum_{k0 <= k < k1} A[m0 + i][k] B[n0 + j][k]   (k0, k1 multiples of 4)
+__device__ __forceinline__ void mm_nt(float (&acc)[4][4], const float* A, int sa, const float* B,
+                                      int sb, int m0, int n0, int k0, int k1) {
+  for (int k = k0; k < k1; k += 4) {
+    float4 a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * sa + k);
+      b[i] = *reinterpret_cast<const float4*>(B + (n0 + i) * sb + k);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float v = acc[i][j];
+        v = fmaf(a[i].x, b[j].x, v);
+        v = fmaf(a[i].y, b[j].y, v);
+        v = fmaf(a[i].z, b[j].z, v);
+        acc[i][j] = fmaf(a[i].w, b[j].w, v);
+      }
+  }
+}
+__device__ __forceinline__ void zero4x4(float (&acc)[4][4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
@@ -153,17 +223,20 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
     float* __restrict__ dA_part, float* __restrict__ dD_part, int64_t seqlen, int nheads,
     int headdim, int dstate, int ngroups, int nchunks) {
   extern __shared__ float sm[];
-  const int P = headdim, N = dstate, P1 = headdim + 1, N1 = dstate + 1;
-  float* xs = sm;                  // [kQ][P1]
-  float* ys = xs + kQ * P1;        // [kQ][P]   dy
-  float* bs = ys + kQ * P;         // [kQ][N1]
-  float* cm = bs + kQ * N1;        // [kQ][N]
-  float* hs = cm + kQ * N;         // [N][P1]   H (forward state entering the chunk)
-  float* rs = hs + N * P1;         // [N][P1]   R (adjoint carried in from the right)
-  float* CB = rs + N * P1;         // [tau][s]  C_tau . B_s
-  float* XY = CB + kQ * kQ;        // [s][tau]  x_s . dy_tau
-  float* Ls = XY + kQ * kQ;        // [tau][s]  exp(cs_tau - cs_s), s <= tau (else 0)
-  float* csv = Ls + kQ * kQ;       // [kQ] cs
+  const int P = headdim, N = dstate, P4 = round4(P), N4 = round4(N);
+  const int PX = BwdSmem::px(P), NX = BwdSmem::nx(N);
+  float* xs = sm;                  // [kQ][PX]  x
+  float* ys = xs + kQ * PX;        // [kQ][PX]  dy
+  float* bs = ys + kQ * PX;        // [kQ][NX]  B
+  float* cm = bs + kQ * NX;        // [kQ][NX]  C
+  float* hs = cm + kQ * NX;        // [P4][NX]  H (forward state entering the chunk)
+  float* rs = hs + P4 * NX;        // [P4][NX]  R (adjoint carried in from the right)
+  float* T1 = rs + P4 * NX;        // [tau][s]  C_tau . B_s, then M
+  float* T2 = T1 + kQ * kQ;        // [s][tau]  x_s . dy_tau, then K2 [t][s]
+  float* T3 = T2 + kQ * kQ;        // [tau][s]  L, then N2
+  float* rowP = T3 + kQ * kQ;      // [16][kQ]  partial row sums of K (by column tile)
+  float* colP = rowP + 16 * kQ;    // [16][kQ]  partial column sums of K (by row tile)
+  float* csv = colP + 16 * kQ;     // [kQ] cs
   float* dts = csv + kQ;           // [kQ] dt
   float* term1 = dts + kQ;         // [kQ] x_t . (G_t B_t)
   float* vv = term1 + kQ;          // [kQ] v_t
@@ -174,6 +247,7 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   float* red = dyx + kQ;           // [64] block reduction scratch
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ta = tid >> 4, tb = tid & 15;  // this thread's row tile and column tile
   const int c = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = int(bh % nheads);
@@ -185,28 +259,29 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   const float Dh = D ? D[h] : 0.f;
   const float* csb = cs + (bh * nchunks + c) * kQ;
 
-  // ---- load the chunk ----
-  for (int i = tid; i < kQ * P; i += kThreads) {
-    const int t = i / P, p = i % P;
-    const bool in = t < nvalid;
+  // ---- load the chunk (zeros in the padding and past the sequence's end) ----
+  for (int i = tid; i < kQ * PX; i += kThreads) {
+    const int t = i / PX, p = i % PX;
+    const bool in = t < nvalid && p < P;
     const int64_t off = ((b * seqlen + t0 + t) * nheads + h) * P + p;
-    xs[t * P1 + p] = in ? io_traits<T>::load(x, off) : 0.f;
+    xs[i] = in ? io_traits<T>::load(x, off) : 0.f;
     ys[i] = in ? dy[off] : 0.f;
   }
-  for (int i = tid; i < kQ * N; i += kThreads) {
-    const int t = i / N, n = i % N;
-    const bool in = t < nvalid;
+  for (int i = tid; i < kQ * NX; i += kThreads) {
+    const int t = i / NX, n = i % NX;
+    const bool in = t < nvalid && n < N;
     const int64_t off = ((b * seqlen + t0 + t) * ngroups + g) * N + n;
-    bs[t * N1 + n] = in ? io_traits<T>::load(Bm, off) : 0.f;
+    bs[i] = in ? io_traits<T>::load(Bm, off) : 0.f;
     cm[i] = in ? io_traits<T>::load(Cm, off) : 0.f;
   }
   {
     const float* hsrc = hstates + ((b * nchunks + c) * nheads + h) * int64_t(P) * N;
     const float* rsrc = adj + ((b * nchunks + c) * nheads + h) * int64_t(P) * N;
-    for (int i = tid; i < P * N; i += kThreads) {  // global [p][n] -> shared [n][p]
-      const int p = i / N, n = i % N;
-      hs[n * P1 + p] = hsrc[i];
-      rs[n * P1 + p] = rsrc[i];
+    for (int i = tid; i < P4 * NX; i += kThreads) {  // global [p][n] -> shared [p][n]
+      const int p = i / NX, n = i % NX;
+      const bool in = p < P && n < N;
+      hs[i] = in ? hsrc[int64_t(p) * N + n] : 0.f;
+      rs[i] = in ? rsrc[int64_t(p) * N + n] : 0.f;
     }
   }
   for (int t = tid; t < kQ; t += kThreads) {
@@ -216,98 +291,176 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   __syncthreads();
   const float cs_end = csv[kQ - 1];
 
-  // ---- the chunk's quadratic tables (lower triangle s <= tau) ----
-  for (int i = tid; i < kQ * kQ; i += kThreads) {
-    const int tau = i / kQ, s = i % kQ;
-    float cbv = 0.f, xyv = 0.f, lv = 0.f;
-    if (s <= tau) {
-      for (int n = 0; n < N; ++n) cbv = fmaf(cm[tau * N + n], bs[s * N1 + n], cbv);
-      for (int p = 0; p < P; ++p) xyv = fmaf(xs[s * P1 + p], ys[tau * P + p], xyv);
-      lv = expf(csv[tau] - csv[s]);
+  // ---- the chunk's quadratic tables: C.B, x.dy and L (4 x 4 per thread) ----
+  {
+    float cb[4][4], xy[4][4];
+    zero4x4(cb);
+    zero4x4(xy);
+    mm_nt(cb, cm, NX, bs, NX, 4 * ta, 4 * tb, 0, N4);  // [tau][s]
+    mm_nt(xy, xs, PX, ys, PX, 4 * ta, 4 * tb, 0, P4);  // [s][tau]
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 4 * ta + i;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = 4 * tb + j;
+        T1[r * kQ + q] = cb[i][j];
+        T2[r * kQ + q] = xy[i][j];
+        T3[r * kQ + q] = q <= r ? expf(csv[r] - csv[q]) : 0.f;
+      }
     }
-    CB[tau * kQ + s] = cbv;
-    XY[s * kQ + tau] = xyv;
-    Ls[tau * kQ + s] = lv;
+  }
+  __syncthreads();
+  // ---- M, N2, K2 in place; the row and column sums of K = K2 (C.B), in a fixed order ----
+  {
+    float mv[4][4], n2[4][4], k2[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tau = 4 * ta + i;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = 4 * tb + j;
+        const float lv = T3[tau * kQ + s], cbv = T1[tau * kQ + s];
+        mv[i][j] = lv * cbv;
+        n2[i][j] = lv * T2[s * kQ + tau];
+        k2[i][j] = dts[s] * n2[i][j];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float rsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rsum = fmaf(k2[i][j], T1[(4 * ta + i) * kQ + 4 * tb + j], rsum);
+      rowP[tb * kQ + 4 * ta + i] = rsum;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float csum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) csum = fmaf(k2[i][j], T1[(4 * ta + i) * kQ + 4 * tb + j], csum);
+      colP[ta * kQ + 4 * tb + j] = csum;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int o = (4 * ta + i) * kQ + 4 * tb + j;
+        T1[o] = mv[i][j];
+        T2[o] = k2[i][j];
+        T3[o] = n2[i][j];
+      }
+  }
+  for (int i = tid; i < 2 * kQ; i += kThreads) {
+    const int r = i % kQ;
+    const float* part = i < kQ ? rowP : colP;
+    float sum = 0.f;
+    for (int k = 0; k < 16; ++k) sum += part[k * kQ + r];
+    (i < kQ ? rowK : colK)[r] = sum;
   }
   __syncthreads();
 
-  // ---- per token t (one warp per token, lanes over p): G_t B_t, dx, x.GB, v_t, w_t, dy.x ----
-  for (int t = warp; t < kQ; t += kThreads / 32) {
-    const float er = expf(cs_end - csv[t]);  // exp(cs_end - cs_t)
-    const float et = expf(csv[t]);
-    float s1 = 0.f, sv = 0.f, sw = 0.f, sd = 0.f;
-    for (int p = lane; p < P; p += 32) {
-      float q = 0.f;
-      for (int tau = t; tau < kQ; ++tau)
-        q = fmaf(Ls[tau * kQ + t] * CB[tau * kQ + t], ys[tau * P + p], q);
-      float rb = 0.f, hc = 0.f;
-      for (int n = 0; n < N; ++n) {
-        rb = fmaf(rs[n * P1 + p], bs[t * N1 + n], rb);
-        hc = fmaf(hs[n * P1 + p], cm[t * N + n], hc);
+  // ---- per token t (rows 4ta..), p (columns): q = sum_tau M[tau][t] dy_tau + er_t R B_t;
+  //      dx, and the per-token sums x.q, x.(R B), dy.(H C), dy.x ----
+  {
+    float s1[4] = {0.f, 0.f, 0.f, 0.f}, sv[4] = {0.f, 0.f, 0.f, 0.f};
+    float sw[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c0 = 0; c0 < P4; c0 += 64) {
+      const int p0 = c0 + 4 * tb;
+      if (p0 >= P4) continue;
+      float q[4][4], rb[4][4], hc[4][4];
+      zero4x4(q);
+      zero4x4(rb);
+      zero4x4(hc);
+      mm_tn(q, T1, kQ, ys, PX, 4 * ta, p0, 4 * ta, kQ);
+      mm_nt(rb, bs, NX, rs, NX, 4 * ta, p0, 0, N4);
+      mm_nt(hc, cm, NX, hs, NX, 4 * ta, p0, 0, N4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * ta + i;
+        const float er = expf(cs_end - csv[t]);
+        float o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float qv = fmaf(er, rb[i][j], q[i][j]);
+          const float xv = xs[t * PX + p0 + j], yv = ys[t * PX + p0 + j];
+          o[j] = fmaf(dts[t], qv, Dh * yv);
+          s1[i] = fmaf(xv, qv, s1[i]);
+          sv[i] = fmaf(xv, rb[i][j], sv[i]);
+          sw[i] = fmaf(yv, hc[i][j], sw[i]);
+          sd[i] = fmaf(yv, xv, sd[i]);
+        }
+        if (t < nvalid) {
+          float* dst = dx + ((b * seqlen + t0 + t) * nheads + h) * P + p0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (p0 + j < P) dst[j] = o[j];
+        }
       }
-      q = fmaf(er, rb, q);
-      const float xv = xs[t * P1 + p], yv = ys[t * P + p];
-      if (t < nvalid)
-        dx[((b * seqlen + t0 + t) * nheads + h) * P + p] = fmaf(dts[t], q, Dh * yv);
-      s1 = fmaf(xv, q, s1);
-      sv = fmaf(xv, rb, sv);
-      sw = fmaf(yv, hc, sw);
-      sd = fmaf(yv, xv, sd);
     }
-    s1 = warp_sum(s1);
-    sv = warp_sum(sv);
-    sw = warp_sum(sw);
-    sd = warp_sum(sd);
-    if (lane == 0) {
-      term1[t] = s1;
-      vv[t] = er * dts[t] * sv;
-      ww[t] = et * sw;
-      dyx[t] = sd;
+    // sum over the 16 column tiles (lanes tb = 0..15 of this half-warp), in a fixed order
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) {
+        s1[i] += __shfl_xor_sync(0xffffffffu, s1[i], off);
+        sv[i] += __shfl_xor_sync(0xffffffffu, sv[i], off);
+        sw[i] += __shfl_xor_sync(0xffffffffu, sw[i], off);
+        sd[i] += __shfl_xor_sync(0xffffffffu, sd[i], off);
+      }
+      if (tb == 0) {
+        const int t = 4 * ta + i;
+        term1[t] = s1[i];
+        vv[t] = expf(cs_end - csv[t]) * dts[t] * sv[i];
+        ww[t] = expf(csv[t]) * sw[i];
+        dyx[t] = sd[i];
+      }
     }
   }
 
-  // ---- per (t, n): this head's dB_t and dC_t ----
-  for (int i = tid; i < kQ * N; i += kThreads) {
-    const int t = i / N, n = i % N;
-    if (t >= nvalid) continue;
-    const float er = expf(cs_end - csv[t]);
-    // dB_t[n] = dt_t [sum_{tau >= t} L[tau, t] XY[t, tau] C_tau[n] + er (R^T x_t)[n]]
-    float sb = 0.f;
-    for (int tau = t; tau < kQ; ++tau)
-      sb = fmaf(Ls[tau * kQ + t] * XY[t * kQ + tau], cm[tau * N + n], sb);
-    float xr = 0.f, yh = 0.f;
-    for (int p = 0; p < P; ++p) {
-      xr = fmaf(xs[t * P1 + p], rs[n * P1 + p], xr);
-      yh = fmaf(ys[t * P + p], hs[n * P1 + p], yh);
+  // ---- per (t, n): this head's dB_t = dt_t (er_t R^T x_t + sum_tau N2[tau][t] C_tau) and
+  //      dC_t = exp(cs_t) H^T dy_t + sum_s K2[t][s] B_s ----
+  for (int c0 = 0; c0 < N4; c0 += 64) {
+    const int n0 = c0 + 4 * tb;
+    if (n0 >= N4) continue;
+    {
+      float sb[4][4], xr[4][4];
+      zero4x4(sb);
+      zero4x4(xr);
+      mm_tn(sb, T3, kQ, cm, NX, 4 * ta, n0, 4 * ta, kQ);
+      mm_nn(xr, xs, PX, rs, NX, 4 * ta, n0, 0, P4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * ta + i;
+        if (t >= nvalid) continue;
+        const float er = expf(cs_end - csv[t]);
+        float* dst = dbh + ((b * seqlen + t0 + t) * nheads + h) * N + n0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (n0 + j < N) dst[j] = dts[t] * fmaf(er, xr[i][j], sb[i][j]);
+      }
     }
-    // dC_t[n] = sum_{s <= t} L[t, s] dt_s XY[s, t] B_s[n] + exp(cs_t) (H^T dy_t)[n]
-    float sc = 0.f;
-    for (int s = 0; s <= t; ++s)
-      sc = fmaf(Ls[t * kQ + s] * dts[s] * XY[s * kQ + t], bs[s * N1 + n], sc);
-    const int64_t off = ((b * seqlen + t0 + t) * nheads + h) * N + n;
-    dbh[off] = dts[t] * fmaf(er, xr, sb);
-    dch[off] = fmaf(expf(csv[t]), yh, sc);
-  }
-  // ---- K's row and column sums ----
-  for (int i = tid; i < 2 * kQ; i += kThreads) {
-    const int r = i % kQ;
-    float sum = 0.f;
-    if (i < kQ) {  // row tau = r: sum over s <= tau
-      for (int s = 0; s <= r; ++s)
-        sum = fmaf(Ls[r * kQ + s] * dts[s], XY[s * kQ + r] * CB[r * kQ + s], sum);
-      rowK[r] = sum;
-    } else {  // column s = r: sum over tau >= s
-      for (int tau = r; tau < kQ; ++tau)
-        sum = fmaf(Ls[tau * kQ + r] * dts[r], XY[r * kQ + tau] * CB[tau * kQ + r], sum);
-      colK[r] = sum;
+    {
+      float sc[4][4], yh[4][4];
+      zero4x4(sc);
+      zero4x4(yh);
+      mm_nn(sc, T2, kQ, bs, NX, 4 * ta, n0, 0, 4 * ta + 4);
+      mm_nn(yh, ys, PX, hs, NX, 4 * ta, n0, 0, P4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * ta + i;
+        if (t >= nvalid) continue;
+        const float et = expf(csv[t]);
+        float* dst = dch + ((b * seqlen + t0 + t) * nheads + h) * N + n0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (n0 + j < N) dst[j] = fmaf(et, yh[i][j], sc[i][j]);
+      }
     }
   }
   // exp(cs_end) <R, H>
   float rh = 0.f;
-  for (int i = tid; i < P * N; i += kThreads) {
-    const int n = i / P, p = i % P;
-    rh = fmaf(rs[n * P1 + p], hs[n * P1 + p], rh);
-  }
+  for (int i = tid; i < P4 * NX; i += kThreads) rh = fmaf(rs[i], hs[i], rh);
   rh = warp_sum(rh);
   if (lane == 0) red[warp] = rh;
   __syncthreads();

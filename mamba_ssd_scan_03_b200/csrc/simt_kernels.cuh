@@ -40,16 +40,17 @@ __global__ void cumsum_kernel(const float* __restrict__ dt, const float* __restr
 }
 
 // ---- 2. chunk states: grid (nchunks, batch*nheads), block 256 --------------------------------
+// S_c[p, n] stored [b][c][h][p][n]: the outer-product sum of (w_s x_s) and B_s over the chunk,
+// 4 x 4 outputs per thread (outer_sum).
 template <typename T>
-__global__ void __launch_bounds__(256) chunk_state_kernel(
+__global__ void __launch_bounds__(kOuterThreads) chunk_state_kernel(
     const T* __restrict__ x, const float* __restrict__ dt, const T* __restrict__ Bm,
     const float* __restrict__ cs, float* __restrict__ states, int64_t seqlen, int nheads,
     int headdim, int dstate, int ngroups, int chunk, int nchunks) {
-  constexpr int TS = 16;   // tokens per smem tile
-  constexpr int OPT = 16;  // outputs per thread per pass
   extern __shared__ float sm[];
-  float* xs = sm;                    // [TS][headdim]
-  float* bs = sm + TS * headdim;     // [TS][dstate]
+  const int P4 = round4(headdim), N4 = round4(dstate);
+  float* us = sm;                    // [TS][P4]  w_s x_s
+  float* vs = sm + kOuterTS * P4;    // [TS][N4]  B_s
   const int c = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = int(bh % nheads);
@@ -58,49 +59,27 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(
   const float* csb = cs + (bh * nchunks + c) * chunk;
   const float cs_end = csb[chunk - 1];
   const int64_t t0 = int64_t(c) * chunk;
-  const int nout = headdim * dstate;
-  float* out = states + ((b * nchunks + c) * nheads + h) * int64_t(nout);
-  for (int base = 0; base < nout; base += 256 * OPT) {
-    float acc[OPT];
-#pragma unroll
-    for (int i = 0; i < OPT; ++i) acc[i] = 0.0f;
-    for (int s0 = 0; s0 < chunk; s0 += TS) {
-      __syncthreads();
-      for (int i = threadIdx.x; i < TS * headdim; i += 256) {
-        const int s = i / headdim, p = i % headdim;
-        const int64_t tok = t0 + s0 + s;
-        float v = 0.0f;
-        if (tok < seqlen) {
-          const float w = expf(cs_end - csb[s0 + s]) * dt[(b * seqlen + tok) * nheads + h];
-          v = w * io_traits<T>::load(x, ((b * seqlen + tok) * nheads + h) * headdim + p);
-        }
-        xs[i] = v;
+  float* out = states + ((b * nchunks + c) * nheads + h) * int64_t(headdim) * dstate;
+  auto stage = [&](int s0, float* u, float* v) {
+    for (int i = threadIdx.x; i < kOuterTS * P4; i += kOuterThreads) {
+      const int s = i / P4, p = i % P4;
+      const int64_t tok = t0 + s0 + s;
+      float val = 0.0f;
+      if (p < headdim && s0 + s < chunk && tok < seqlen) {
+        const float w = expf(cs_end - csb[s0 + s]) * dt[(b * seqlen + tok) * nheads + h];
+        val = w * io_traits<T>::load(x, ((b * seqlen + tok) * nheads + h) * headdim + p);
       }
-      for (int i = threadIdx.x; i < TS * dstate; i += 256) {
-        const int s = i / dstate, n = i % dstate;
-        const int64_t tok = t0 + s0 + s;
-        bs[i] = tok < seqlen
-                    ? io_traits<T>::load(Bm, ((b * seqlen + tok) * ngroups + g) * dstate + n)
-                    : 0.0f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < OPT; ++i) {
-        const int o = base + i * 256 + threadIdx.x;  // o = p * dstate + n
-        if (o < nout) {
-          const int p = o / dstate, n = o % dstate;
-          float a = acc[i];
-          for (int s = 0; s < TS; ++s) a = fmaf(xs[s * headdim + p], bs[s * dstate + n], a);
-          acc[i] = a;
-        }
-      }
+      u[i] = val;
     }
-#pragma unroll
-    for (int i = 0; i < OPT; ++i) {
-      const int o = base + i * 256 + threadIdx.x;
-      if (o < nout) out[o] = acc[i];
+    for (int i = threadIdx.x; i < kOuterTS * N4; i += kOuterThreads) {
+      const int s = i / N4, n = i % N4;
+      const int64_t tok = t0 + s0 + s;
+      v[i] = n < dstate && s0 + s < chunk && tok < seqlen
+                 ? io_traits<T>::load(Bm, ((b * seqlen + tok) * ngroups + g) * dstate + n)
+                 : 0.0f;
     }
-  }
+  };
+  outer_sum(stage, chunk, headdim, dstate, out, us, vs);
 }
 
 // ---- 3. state passing: one thread per state element, sequential over chunks -------------------
@@ -116,12 +95,30 @@ __global__ void state_pass_kernel(float* __restrict__ states, const float* __res
   const int h = int(bh % nheads);
   const int64_t b = bh / nheads;
   float run = init_state ? init_state[e] : 0.0f;
-  for (int c = 0; c < nchunks; ++c) {
-    float* slot = states + ((b * nchunks + c) * nheads + h) * per_bh + pn;
-    const float s = *slot;
-    *slot = run;
-    const float decay = expf(cs[(bh * nchunks + c) * chunk + chunk - 1]);
-    run = fmaf(decay, run, s);
+  float* base = states + (b * nchunks * nheads + h) * per_bh + pn;  // chunk c: + c * cstride
+  const int64_t cstride = int64_t(nheads) * per_bh;
+  const float* last = cs + bh * nchunks * chunk + chunk - 1;  // chunk c's last cumsum: + c * chunk
+  // kBatch chunks' loads in flight at once (they do not depend on the running state), then the
+  // recurrence over them in order
+  constexpr int kBatch = 8;
+  for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+    float sv[kBatch], lv[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t c = c0 + i;
+      if (c < nchunks) {
+        sv[i] = base[c * cstride];
+        lv[i] = last[c * chunk];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t c = c0 + i;
+      if (c < nchunks) {
+        base[c * cstride] = run;
+        run = fmaf(expf(lv[i]), run, sv[i]);
+      }
+    }
   }
   if (final_state) final_state[e] = run;
 }

@@ -92,4 +92,69 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return d;
 }
 
+// ---- register-tiled outer-product sums (float32 CUDA cores) ----------------------------------
+// out[p * N + n] = sum over a chunk's tokens s of u_s[p] v_s[n], for a P x N output, by a block
+// of kOuterThreads threads, 4 x 4 outputs per thread and tile (two 16-byte shared loads per 16
+// FMAs).  stage(s0, us, vs) fills kOuterTS token rows: us [kOuterTS][P4], vs [kOuterTS][N4]
+// (P4, N4: P and N rounded up to multiples of 4; the padding and rows past the chunk's end
+// hold zeros).  Shared memory: outer_smem_floats(P, N).
+constexpr int kOuterTS = 16, kOuterThreads = 256, kOuterTiles = 2;
+__host__ __device__ inline int round4(int v) { return (v + 3) & ~3; }
+__host__ __device__ inline size_t outer_smem_floats(int P, int N) {
+  return size_t(kOuterTS) * (round4(P) + round4(N));
+}
+template <typename Stage>
+__device__ __forceinline__ void outer_sum(const Stage& stage, int ntok, int P, int N,
+                                          float* __restrict__ out, float* us, float* vs) {
+  const int P4 = round4(P), N4 = round4(N);
+  const int ntn = N4 / 4, ntiles = (P4 / 4) * ntn;
+  for (int base = 0; base < ntiles; base += kOuterThreads * kOuterTiles) {
+    float acc[kOuterTiles][4][4];
+    int tp[kOuterTiles], tn[kOuterTiles];
+#pragma unroll
+    for (int k = 0; k < kOuterTiles; ++k) {
+      const int idx = base + k * kOuterThreads + int(threadIdx.x);
+      tp[k] = idx < ntiles ? idx / ntn : -1;
+      tn[k] = idx % ntn;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[k][i][j] = 0.f;
+    }
+    for (int s0 = 0; s0 < ntok; s0 += kOuterTS) {
+      __syncthreads();
+      stage(s0, us, vs);
+      __syncthreads();
+#pragma unroll 4
+      for (int s = 0; s < kOuterTS; ++s) {
+#pragma unroll
+        for (int k = 0; k < kOuterTiles; ++k) {
+          if (tp[k] < 0) continue;
+          const float4 u = *reinterpret_cast<const float4*>(us + s * P4 + 4 * tp[k]);
+          const float4 v = *reinterpret_cast<const float4*>(vs + s * N4 + 4 * tn[k]);
+          const float uu[4] = {u.x, u.y, u.z, u.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[k][i][j] = fmaf(uu[i], vv[j], acc[k][i][j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kOuterTiles; ++k) {
+      if (tp[k] < 0) continue;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int p = 4 * tp[k] + i;
+        if (p >= P) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int n = 4 * tn[k] + j;
+          if (n < N) out[int64_t(p) * N + n] = acc[k][i][j];
+        }
+      }
+    }
+  }
+}
+
 }  // namespace ssd

@@ -412,8 +412,8 @@ ssd_status run_simt(const Shape& s, const ScanArgs& a, bool with_output = true) 
   ssd::simt::cumsum_kernel<<<grid, s.chunk, 0, a.stream>>>(a.dt, a.A, cs, s.seqlen, s.nheads,
                                                            s.chunk, int(nchunks));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  const size_t sm_state = 16 * size_t(s.headdim + s.dstate) * sizeof(float);
-  ssd::simt::chunk_state_kernel<T><<<grid, 256, sm_state, a.stream>>>(
+  const size_t sm_state = ssd::outer_smem_floats(s.headdim, s.dstate) * sizeof(float);
+  ssd::simt::chunk_state_kernel<T><<<grid, ssd::kOuterThreads, sm_state, a.stream>>>(
       static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), cs, states, s.seqlen,
       s.nheads, s.headdim, s.dstate, s.ngroups, s.chunk, int(nchunks));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
@@ -589,7 +589,8 @@ ssd_status run_bwd(const Shape& s, const ScanArgs& a, const float* dy, const flo
   ssd::simt::cumsum_kernel<<<grid, bw::kQ, 0, a.stream>>>(a.dt, a.A, cs, s.seqlen, s.nheads,
                                                           bw::kQ, int(nc));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  ssd::simt::chunk_state_kernel<T><<<grid, 256, 16 * size_t(P + N) * sizeof(float), a.stream>>>(
+  const size_t sm_outer = ssd::outer_smem_floats(P, N) * sizeof(float);
+  ssd::simt::chunk_state_kernel<T><<<grid, ssd::kOuterThreads, sm_outer, a.stream>>>(
       static_cast<const T*>(a.x), a.dt, static_cast<const T*>(a.B), cs, hst, s.seqlen, s.nheads,
       P, N, s.ngroups, bw::kQ, int(nc));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
@@ -598,7 +599,7 @@ ssd_status run_bwd(const Shape& s, const ScanArgs& a, const float* dy, const flo
       hst, cs, a.init, nullptr, s.batch, s.nheads, P, N, bw::kQ, int(nc));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   // backward: adjoint summaries, the adjoint entering every chunk from the right, then chunks
-  bw::adj_state_kernel<T><<<grid, bw::kThreads, 16 * size_t(P + N) * sizeof(float), a.stream>>>(
+  bw::adj_state_kernel<T><<<grid, ssd::kOuterThreads, sm_outer, a.stream>>>(
       dy, static_cast<const T*>(a.C), cs, adj, s.seqlen, s.nheads, P, N, s.ngroups, int(nc));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
   bw::adj_pass_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(

@@ -46,6 +46,7 @@ namespace bwd {
 
 constexpr int kQ = 64;         // tokens per chunk of the backward (the result does not depend on it)
 constexpr int kThreads = 256;
+constexpr int kBwdThreads = 512;  // chunk_bwd: two halves of 256 threads
 
 // ---- 1. adjoint summaries: grid (nchunks, batch * nheads), block 256 ------------------------
 // S'_c[p, n] = sum_{t in c} exp(cs_t) dy_t[p] C_t[n], stored [b][c][h][p][n] (outer_sum).
@@ -55,9 +56,9 @@ __global__ void __launch_bounds__(kOuterThreads) adj_state_kernel(
     float* __restrict__ adj, int64_t seqlen, int nheads, int headdim, int dstate, int ngroups,
     int nchunks) {
   extern __shared__ float sm[];
-  const int P4 = round4(headdim), N4 = round4(dstate);
+  const int P4 = round4(headdim), N4 = round4(dstate), TS = outer_ts(headdim, dstate);
   float* us = sm;                    // [TS][P4]  exp(cs_t) dy_t
-  float* vs = sm + kOuterTS * P4;    // [TS][N4]  C_t
+  float* vs = sm + TS * P4;          // [TS][N4]  C_t
   const int c = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = int(bh % nheads);
@@ -66,20 +67,28 @@ __global__ void __launch_bounds__(kOuterThreads) adj_state_kernel(
   const float* csb = cs + (bh * nchunks + c) * kQ;
   const int64_t t0 = int64_t(c) * kQ;
   float* out = adj + ((b * nchunks + c) * nheads + h) * int64_t(headdim) * dstate;
-  auto stage = [&](int s0, float* u, float* v) {
-    for (int i = threadIdx.x; i < kOuterTS * P4; i += kOuterThreads) {
-      const int s = i / P4, p = i % P4;
+  const bool vy = vec4_ok(dy, headdim), vc = vec4_ok(Cm, dstate);
+  auto stage = [&](int s0, int ts, float* u, float* v) {  // four columns per step
+    const int gp = P4 / 4, gn = N4 / 4;
+    for (int i = threadIdx.x; i < ts * gp; i += kOuterThreads) {
+      const int s = i / gp, p = (i % gp) * 4;
       const int64_t tok = t0 + s0 + s;
-      u[i] = p < headdim && tok < seqlen
-                 ? expf(csb[s0 + s]) * dy[((b * seqlen + tok) * nheads + h) * headdim + p]
-                 : 0.f;
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (tok < seqlen) {
+        const float w = expf(csb[s0 + s]);
+        load4_row(dy, ((b * seqlen + tok) * nheads + h) * headdim + p, p, headdim, vy, e);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) e[q] *= w;
+      }
+      *reinterpret_cast<float4*>(u + s * P4 + p) = make_float4(e[0], e[1], e[2], e[3]);
     }
-    for (int i = threadIdx.x; i < kOuterTS * N4; i += kOuterThreads) {
-      const int s = i / N4, n = i % N4;
+    for (int i = threadIdx.x; i < ts * gn; i += kOuterThreads) {
+      const int s = i / gn, n = (i % gn) * 4;
       const int64_t tok = t0 + s0 + s;
-      v[i] = n < dstate && tok < seqlen
-                 ? io_traits<T>::load(Cm, ((b * seqlen + tok) * ngroups + g) * dstate + n)
-                 : 0.f;
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (tok < seqlen)
+        load4_row(Cm, ((b * seqlen + tok) * ngroups + g) * dstate + n, n, dstate, vc, e);
+      *reinterpret_cast<float4*>(v + s * N4 + n) = make_float4(e[0], e[1], e[2], e[3]);
     }
   };
   outer_sum(stage, kQ, headdim, dstate, out, us, vs);
@@ -126,10 +135,11 @@ __global__ void adj_pass_kernel(float* __restrict__ adj, const float* __restrict
   if (dinit) dinit[e] = run;
 }
 
-// ---- 3. per-chunk gradients: grid (nchunks, batch * nheads), block 256 ------------------------
+// ---- 3. per-chunk gradients: grid (nchunks, batch * nheads), block 512 ------------------------
 // Every product of the chunk is a small matrix product from shared memory, 4 x 4 outputs per
-// thread and product (thread (a, b) = (tid / 16, tid % 16): rows 4a .. 4a+3, columns
-// 4b .. 4b+3 of each 64-column pass) with float4 operand loads.
+// thread and product (thread (a, b) = (i / 16, i % 16) of a half, i = tid % 256: rows
+// 4a .. 4a+3, columns 4b .. 4b+3 of each 64-column pass) with float4 operand loads.  The two
+// halves of the block take independent products: C.B / x.dy, the dx terms / H C, dB / dC.
 // Shared memory (floats; rows padded to multiples of 4 plus 4, which keeps float4 rows aligned
 // and spreads the strided row walks over the banks):
 //   x, dy [kQ][P4 + 4]; B, C [kQ][N4 + 4]; H, R [P4][N4 + 4] (as stored: [p][n]);
@@ -214,7 +224,7 @@ __device__ __forceinline__ void zero4x4(float (&acc)[4][4]) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
+__global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     const T* __restrict__ x, const float* __restrict__ dt, const float* __restrict__ A,
     const T* __restrict__ Bm, const T* __restrict__ Cm, const float* __restrict__ D,
     const float* __restrict__ dy, const float* __restrict__ cs,
@@ -247,7 +257,8 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   float* red = dyx + kQ;           // [64] block reduction scratch
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ta = tid >> 4, tb = tid & 15;  // this thread's row tile and column tile
+  const int half = tid >> 8;                        // which half of the block
+  const int ta = (tid & 255) >> 4, tb = tid & 15;  // this thread's row tile and column tile
   const int c = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = int(bh % nheads);
@@ -260,14 +271,14 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   const float* csb = cs + (bh * nchunks + c) * kQ;
 
   // ---- load the chunk (zeros in the padding and past the sequence's end) ----
-  for (int i = tid; i < kQ * PX; i += kThreads) {
+  for (int i = tid; i < kQ * PX; i += kBwdThreads) {
     const int t = i / PX, p = i % PX;
     const bool in = t < nvalid && p < P;
     const int64_t off = ((b * seqlen + t0 + t) * nheads + h) * P + p;
     xs[i] = in ? io_traits<T>::load(x, off) : 0.f;
     ys[i] = in ? dy[off] : 0.f;
   }
-  for (int i = tid; i < kQ * NX; i += kThreads) {
+  for (int i = tid; i < kQ * NX; i += kBwdThreads) {
     const int t = i / NX, n = i % NX;
     const bool in = t < nvalid && n < N;
     const int64_t off = ((b * seqlen + t0 + t) * ngroups + g) * N + n;
@@ -277,14 +288,14 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   {
     const float* hsrc = hstates + ((b * nchunks + c) * nheads + h) * int64_t(P) * N;
     const float* rsrc = adj + ((b * nchunks + c) * nheads + h) * int64_t(P) * N;
-    for (int i = tid; i < P4 * NX; i += kThreads) {  // global [p][n] -> shared [p][n]
+    for (int i = tid; i < P4 * NX; i += kBwdThreads) {  // global [p][n] -> shared [p][n]
       const int p = i / NX, n = i % NX;
       const bool in = p < P && n < N;
       hs[i] = in ? hsrc[int64_t(p) * N + n] : 0.f;
       rs[i] = in ? rsrc[int64_t(p) * N + n] : 0.f;
     }
   }
-  for (int t = tid; t < kQ; t += kThreads) {
+  for (int t = tid; t < kQ; t += kBwdThreads) {
     csv[t] = csb[t];
     dts[t] = t < nvalid ? dt[(b * seqlen + t0 + t) * nheads + h] : 0.f;
   }
@@ -293,20 +304,19 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
 
   // ---- the chunk's quadratic tables: C.B, x.dy and L (4 x 4 per thread) ----
   {
-    float cb[4][4], xy[4][4];
-    zero4x4(cb);
-    zero4x4(xy);
-    mm_nt(cb, cm, NX, bs, NX, 4 * ta, 4 * tb, 0, N4);  // [tau][s]
-    mm_nt(xy, xs, PX, ys, PX, 4 * ta, 4 * tb, 0, P4);  // [s][tau]
+    float acc[4][4];
+    zero4x4(acc);
+    if (half == 0) mm_nt(acc, cm, NX, bs, NX, 4 * ta, 4 * tb, 0, N4);  // C.B [tau][s]
+    else mm_nt(acc, xs, PX, ys, PX, 4 * ta, 4 * tb, 0, P4);            // x.dy [s][tau]
+    float* dst = half == 0 ? T1 : T2;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = 4 * ta + i;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int q = 4 * tb + j;
-        T1[r * kQ + q] = cb[i][j];
-        T2[r * kQ + q] = xy[i][j];
-        T3[r * kQ + q] = q <= r ? expf(csv[r] - csv[q]) : 0.f;
+        dst[r * kQ + q] = acc[i][j];
+        if (half == 0) T3[r * kQ + q] = q <= r ? expf(csv[r] - csv[q]) : 0.f;
       }
     }
   }
@@ -314,6 +324,7 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   // ---- M, N2, K2 in place; the row and column sums of K = K2 (C.B), in a fixed order ----
   {
     float mv[4][4], n2[4][4], k2[4][4];
+    if (half == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int tau = 4 * ta + i;
@@ -340,18 +351,21 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
       for (int i = 0; i < 4; ++i) csum = fmaf(k2[i][j], T1[(4 * ta + i) * kQ + 4 * tb + j], csum);
       colP[ta * kQ + 4 * tb + j] = csum;
     }
+    }
     __syncthreads();
+    if (half == 0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int o = (4 * ta + i) * kQ + 4 * tb + j;
-        T1[o] = mv[i][j];
-        T2[o] = k2[i][j];
-        T3[o] = n2[i][j];
-      }
+        for (int j = 0; j < 4; ++j) {
+          const int o = (4 * ta + i) * kQ + 4 * tb + j;
+          T1[o] = mv[i][j];
+          T2[o] = k2[i][j];
+          T3[o] = n2[i][j];
+        }
+    }
   }
-  for (int i = tid; i < 2 * kQ; i += kThreads) {
+  for (int i = tid; i < 2 * kQ; i += kBwdThreads) {
     const int r = i % kQ;
     const float* part = i < kQ ? rowP : colP;
     float sum = 0.f;
@@ -360,42 +374,49 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   }
   __syncthreads();
 
-  // ---- per token t (rows 4ta..), p (columns): q = sum_tau M[tau][t] dy_tau + er_t R B_t;
-  //      dx, and the per-token sums x.q, x.(R B), dy.(H C), dy.x ----
+  // ---- per token t (rows 4ta..), p (columns).  Half 0: q = sum_tau M[tau][t] dy_tau +
+  //      er_t R B_t, dx, and the per-token sums x.q, x.(R B), dy.x; half 1: dy.(H C) ----
   {
     float s1[4] = {0.f, 0.f, 0.f, 0.f}, sv[4] = {0.f, 0.f, 0.f, 0.f};
     float sw[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
     for (int c0 = 0; c0 < P4; c0 += 64) {
       const int p0 = c0 + 4 * tb;
       if (p0 >= P4) continue;
-      float q[4][4], rb[4][4], hc[4][4];
-      zero4x4(q);
-      zero4x4(rb);
-      zero4x4(hc);
-      mm_tn(q, T1, kQ, ys, PX, 4 * ta, p0, 4 * ta, kQ);
-      mm_nt(rb, bs, NX, rs, NX, 4 * ta, p0, 0, N4);
-      mm_nt(hc, cm, NX, hs, NX, 4 * ta, p0, 0, N4);
+      if (half == 0) {
+        float q[4][4], rb[4][4];
+        zero4x4(q);
+        zero4x4(rb);
+        mm_tn(q, T1, kQ, ys, PX, 4 * ta, p0, 4 * ta, kQ);
+        mm_nt(rb, bs, NX, rs, NX, 4 * ta, p0, 0, N4);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = 4 * ta + i;
-        const float er = expf(cs_end - csv[t]);
-        float o[4];
+        for (int i = 0; i < 4; ++i) {
+          const int t = 4 * ta + i;
+          const float er = expf(cs_end - csv[t]);
+          float o[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float qv = fmaf(er, rb[i][j], q[i][j]);
-          const float xv = xs[t * PX + p0 + j], yv = ys[t * PX + p0 + j];
-          o[j] = fmaf(dts[t], qv, Dh * yv);
-          s1[i] = fmaf(xv, qv, s1[i]);
-          sv[i] = fmaf(xv, rb[i][j], sv[i]);
-          sw[i] = fmaf(yv, hc[i][j], sw[i]);
-          sd[i] = fmaf(yv, xv, sd[i]);
+          for (int j = 0; j < 4; ++j) {
+            const float qv = fmaf(er, rb[i][j], q[i][j]);
+            const float xv = xs[t * PX + p0 + j], yv = ys[t * PX + p0 + j];
+            o[j] = fmaf(dts[t], qv, Dh * yv);
+            s1[i] = fmaf(xv, qv, s1[i]);
+            sv[i] = fmaf(xv, rb[i][j], sv[i]);
+            sd[i] = fmaf(yv, xv, sd[i]);
+          }
+          if (t < nvalid) {
+            float* dst = dx + ((b * seqlen + t0 + t) * nheads + h) * P + p0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (p0 + j < P) dst[j] = o[j];
+          }
         }
-        if (t < nvalid) {
-          float* dst = dx + ((b * seqlen + t0 + t) * nheads + h) * P + p0;
+      } else {
+        float hc[4][4];
+        zero4x4(hc);
+        mm_nt(hc, cm, NX, hs, NX, 4 * ta, p0, 0, N4);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (p0 + j < P) dst[j] = o[j];
-        }
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sw[i] = fmaf(ys[(4 * ta + i) * PX + p0 + j], hc[i][j], sw[i]);
       }
     }
     // sum over the 16 column tiles (lanes tb = 0..15 of this half-warp), in a fixed order
@@ -410,20 +431,23 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
       }
       if (tb == 0) {
         const int t = 4 * ta + i;
-        term1[t] = s1[i];
-        vv[t] = expf(cs_end - csv[t]) * dts[t] * sv[i];
-        ww[t] = expf(csv[t]) * sw[i];
-        dyx[t] = sd[i];
+        if (half == 0) {
+          term1[t] = s1[i];
+          vv[t] = expf(cs_end - csv[t]) * dts[t] * sv[i];
+          dyx[t] = sd[i];
+        } else {
+          ww[t] = expf(csv[t]) * sw[i];
+        }
       }
     }
   }
 
-  // ---- per (t, n): this head's dB_t = dt_t (er_t R^T x_t + sum_tau N2[tau][t] C_tau) and
-  //      dC_t = exp(cs_t) H^T dy_t + sum_s K2[t][s] B_s ----
+  // ---- per (t, n): this head's dB_t = dt_t (er_t R^T x_t + sum_tau N2[tau][t] C_tau) (half 0)
+  //      and dC_t = exp(cs_t) H^T dy_t + sum_s K2[t][s] B_s (half 1) ----
   for (int c0 = 0; c0 < N4; c0 += 64) {
     const int n0 = c0 + 4 * tb;
     if (n0 >= N4) continue;
-    {
+    if (half == 0) {
       float sb[4][4], xr[4][4];
       zero4x4(sb);
       zero4x4(xr);
@@ -439,8 +463,7 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
         for (int j = 0; j < 4; ++j)
           if (n0 + j < N) dst[j] = dts[t] * fmaf(er, xr[i][j], sb[i][j]);
       }
-    }
-    {
+    } else {
       float sc[4][4], yh[4][4];
       zero4x4(sc);
       zero4x4(yh);
@@ -460,14 +483,14 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(
   }
   // exp(cs_end) <R, H>
   float rh = 0.f;
-  for (int i = tid; i < P4 * NX; i += kThreads) rh = fmaf(rs[i], hs[i], rh);
+  for (int i = tid; i < P4 * NX; i += kBwdThreads) rh = fmaf(rs[i], hs[i], rh);
   rh = warp_sum(rh);
   if (lane == 0) red[warp] = rh;
   __syncthreads();
   // ---- one warp: the per-token sums, ddt, and this chunk's dA and dD partials ----
   if (warp == 0) {
     float rht = 0.f;
-    for (int w = 0; w < kThreads / 32; ++w) rht += red[w];
+    for (int w = 0; w < kBwdThreads / 32; ++w) rht += red[w];
     const float cst = expf(cs_end) * rht;
     // S_t = S_{t-1} + colK[t] - rowK[t-1]; W_t = sum_{tau >= t} w; V_t = sum_{s <= t} v.  Lane l
     // takes tokens 2l, 2l+1; the running sums are warp scans.

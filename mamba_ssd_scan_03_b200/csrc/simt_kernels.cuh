@@ -48,9 +48,9 @@ __global__ void __launch_bounds__(kOuterThreads) chunk_state_kernel(
     const float* __restrict__ cs, float* __restrict__ states, int64_t seqlen, int nheads,
     int headdim, int dstate, int ngroups, int chunk, int nchunks) {
   extern __shared__ float sm[];
-  const int P4 = round4(headdim), N4 = round4(dstate);
+  const int P4 = round4(headdim), N4 = round4(dstate), TS = outer_ts(headdim, dstate);
   float* us = sm;                    // [TS][P4]  w_s x_s
-  float* vs = sm + kOuterTS * P4;    // [TS][N4]  B_s
+  float* vs = sm + TS * P4;          // [TS][N4]  B_s
   const int c = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = int(bh % nheads);
@@ -60,23 +60,28 @@ __global__ void __launch_bounds__(kOuterThreads) chunk_state_kernel(
   const float cs_end = csb[chunk - 1];
   const int64_t t0 = int64_t(c) * chunk;
   float* out = states + ((b * nchunks + c) * nheads + h) * int64_t(headdim) * dstate;
-  auto stage = [&](int s0, float* u, float* v) {
-    for (int i = threadIdx.x; i < kOuterTS * P4; i += kOuterThreads) {
-      const int s = i / P4, p = i % P4;
+  const bool vx = vec4_ok(x, headdim), vb = vec4_ok(Bm, dstate);
+  auto stage = [&](int s0, int ts, float* u, float* v) {  // four columns per step
+    const int gp = P4 / 4, gn = N4 / 4;
+    for (int i = threadIdx.x; i < ts * gp; i += kOuterThreads) {
+      const int s = i / gp, p = (i % gp) * 4;
       const int64_t tok = t0 + s0 + s;
-      float val = 0.0f;
-      if (p < headdim && s0 + s < chunk && tok < seqlen) {
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (s0 + s < chunk && tok < seqlen) {
         const float w = expf(cs_end - csb[s0 + s]) * dt[(b * seqlen + tok) * nheads + h];
-        val = w * io_traits<T>::load(x, ((b * seqlen + tok) * nheads + h) * headdim + p);
+        load4_row(x, ((b * seqlen + tok) * nheads + h) * headdim + p, p, headdim, vx, e);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) e[q] *= w;
       }
-      u[i] = val;
+      *reinterpret_cast<float4*>(u + s * P4 + p) = make_float4(e[0], e[1], e[2], e[3]);
     }
-    for (int i = threadIdx.x; i < kOuterTS * N4; i += kOuterThreads) {
-      const int s = i / N4, n = i % N4;
+    for (int i = threadIdx.x; i < ts * gn; i += kOuterThreads) {
+      const int s = i / gn, n = (i % gn) * 4;
       const int64_t tok = t0 + s0 + s;
-      v[i] = n < dstate && s0 + s < chunk && tok < seqlen
-                 ? io_traits<T>::load(Bm, ((b * seqlen + tok) * ngroups + g) * dstate + n)
-                 : 0.0f;
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      if (s0 + s < chunk && tok < seqlen)
+        load4_row(Bm, ((b * seqlen + tok) * ngroups + g) * dstate + n, n, dstate, vb, e);
+      *reinterpret_cast<float4*>(v + s * N4 + n) = make_float4(e[0], e[1], e[2], e[3]);
     }
   };
   outer_sum(stage, chunk, headdim, dstate, out, us, vs);

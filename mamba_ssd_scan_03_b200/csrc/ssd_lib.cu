@@ -605,7 +605,7 @@ ssd_status run_bwd(const Shape& s, const ScanArgs& a, const float* dy, const flo
   bw::adj_pass_kernel<<<unsigned((nel + 255) / 256), 256, 0, a.stream>>>(
       adj, cs, dfinal, dinit, s.batch, s.nheads, P, N, int(nc));
   if (launched() != SSD_OK) return SSD_ERR_CUDA;
-  bw::chunk_bwd_kernel<T><<<grid, bw::kThreads, bw::BwdSmem::floats(P, N) * sizeof(float),
+  bw::chunk_bwd_kernel<T><<<grid, bw::kBwdThreads, bw::BwdSmem::floats(P, N) * sizeof(float),
                             a.stream>>>(
       static_cast<const T*>(a.x), a.dt, a.A, static_cast<const T*>(a.B),
       static_cast<const T*>(a.C), a.D, dy, cs, hst, adj, dx, ddt, dbh, dch, dA_part, dD_part,

@@ -140,33 +140,47 @@ __global__ void adj_pass_kernel(float* __restrict__ adj, const float* __restrict
 // thread and product (thread (a, b) = (i / 16, i % 16) of a half, i = tid % 256: rows
 // 4a .. 4a+3, columns 4b .. 4b+3 of each 64-column pass) with float4 operand loads.  The two
 // halves of the block take independent products: C.B / x.dy, the dx terms / H C, dB / dC.
-// Shared memory (floats; rows padded to multiples of 4 plus 4, which keeps float4 rows aligned
-// and spreads the strided row walks over the banks):
-//   x, dy [kQ][P4 + 4]; B, C [kQ][N4 + 4]; H, R [P4][N4 + 4] (as stored: [p][n]);
-//   three [kQ][kQ] tables, first C.B, x.dy and L, then (in place) M[tau][t] = L (C_tau . B_t),
-//   N2[tau][t] = L[tau][t] (x_t . dy_tau) and K2[t][s] = dt_s N2[t][s];
-//   row and column partials of K [16][kQ] each; per-token scalars.
+// Shared memory (floats; rows of P4 or N4, the widths rounded up to multiples of 4):
+//   x, dy [kQ][P4]; B, C [kQ][N4]; H, R [P4][N4] (as stored: [p][n]);
+//   three [kQ][kQ] tables, first C.B, (x.dy)^T and L, then (in place) M[tau][t] =
+//   L (C_tau . B_t), N2[tau][t] = L[tau][t] (x_t . dy_tau) and K2[t][s] = dt_s N2[t][s];
+//   row and column partials of K; per-token scalars.
+// x, B, H and R are read as four rows at a time by the lanes of a quarter-warp (the right-hand
+// operand of the x.y^T-shaped products), rows 4 apart: their 16-byte groups are XOR-swizzled by
+// bits of the row (swz), so those reads, and every other walk over them, hit distinct banks.
 // Outputs: dx [b, t, h, p]; ddt [b, t, h]; the head's dB and dC rows into dbh, dch
 // [b, t, h, n] (summed over the group by the reduce kernel); partial dA and dD per (b, c, h).
 struct BwdSmem {
-  static __host__ __device__ int px(int P) { return round4(P) + 4; }
-  static __host__ __device__ int nx(int N) { return round4(N) + 4; }
+  static __host__ __device__ int px(int P) { return round4(P); }
+  static __host__ __device__ int nx(int N) { return round4(N); }
   static __host__ __device__ size_t floats(int P, int N) {
     return size_t(kQ) * 2 * (px(P) + nx(N)) + 2 * size_t(round4(P)) * nx(N) +
            3 * size_t(kQ) * kQ + 2 * 16 * size_t(kQ) + 8 * kQ + 64;
   }
 };
+// The XOR swizzle of a row of `groups` 16-byte groups: the largest of 7, 3, 1, 0 that keeps the
+// XOR inside the row.
+__device__ __forceinline__ int swz_mask(int groups) {
+  return groups % 8 == 0 ? 7 : (groups % 4 == 0 ? 3 : (groups % 2 == 0 ? 1 : 0));
+}
+// physical column of (row, col): the 16-byte group XOR (row / 4) & mask
+__device__ __forceinline__ int swz(int row, int col, int mask) {
+  return ((((col >> 2) ^ ((row >> 2) & mask))) << 2) | (col & 3);
+}
 
-// acc[i][j] += sum_{k0 <= k < k1} A[m0 + i][k] B[k][n0 + j]   (k0, k1 multiples of 4)
-__device__ __forceinline__ void mm_nn(float (&acc)[4][4], const float* A, int sa, const float* B,
-                                      int sb, int m0, int n0, int k0, int k1) {
+// The products: am, bm are the operands' swizzle masks (0: plain rows).
+// acc[i][j] += sum_{k0 <= k < k1} A[m0 + i][k] B[k][n0 + j]   (k0, k1, m0, n0 multiples of 4)
+__device__ __forceinline__ void mm_nn(float (&acc)[4][4], const float* A, int sa, int am,
+                                      const float* B, int sb, int bm, int m0, int n0, int k0,
+                                      int k1) {
   for (int k = k0; k < k1; k += 4) {
     float4 a[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * sa + k);
+    for (int i = 0; i < 4; ++i)
+      a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * sa + swz(m0 + i, k, am));
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float4 bv = *reinterpret_cast<const float4*>(B + (k + u) * sb + n0);
+      const float4 bv = *reinterpret_cast<const float4*>(B + (k + u) * sb + swz(k + u, n0, bm));
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float av = u == 0 ? a[i].x : u == 1 ? a[i].y : u == 2 ? a[i].z : a[i].w;
@@ -179,11 +193,12 @@ __device__ __forceinline__ void mm_nn(float (&acc)[4][4], const float* A, int sa
   }
 }
 // acc[i][j] += sum_{k0 <= k < k1} A[k][m0 + i] B[k][n0 + j]
-__device__ __forceinline__ void mm_tn(float (&acc)[4][4], const float* A, int sa, const float* B,
-                                      int sb, int m0, int n0, int k0, int k1) {
+__device__ __forceinline__ void mm_tn(float (&acc)[4][4], const float* A, int sa, int am,
+                                      const float* B, int sb, int bm, int m0, int n0, int k0,
+                                      int k1) {
   for (int k = k0; k < k1; ++k) {
-    const float4 av = *reinterpret_cast<const float4*>(A + k * sa + m0);
-    const float4 bv = *reinterpret_cast<const float4*>(B + k * sb + n0);
+    const float4 av = *reinterpret_cast<const float4*>(A + k * sa + swz(k, m0, am));
+    const float4 bv = *reinterpret_cast<const float4*>(B + k * sb + swz(k, n0, bm));
     const float aa[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -195,14 +210,15 @@ __device__ __forceinline__ void mm_tn(float (&acc)[4][4], const float* A, int sa
   }
 }
 // acc[i][j] += sum_{k0 <= k < k1} A[m0 + i][k] B[n0 + j][k]   (k0, k1 multiples of 4)
-__device__ __forceinline__ void mm_nt(float (&acc)[4][4], const float* A, int sa, const float* B,
-                                      int sb, int m0, int n0, int k0, int k1) {
+__device__ __forceinline__ void mm_nt(float (&acc)[4][4], const float* A, int sa, int am,
+                                      const float* B, int sb, int bm, int m0, int n0, int k0,
+                                      int k1) {
   for (int k = k0; k < k1; k += 4) {
     float4 a[4], b[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * sa + k);
-      b[i] = *reinterpret_cast<const float4*>(B + (n0 + i) * sb + k);
+      a[i] = *reinterpret_cast<const float4*>(A + (m0 + i) * sa + swz(m0 + i, k, am));
+      b[i] = *reinterpret_cast<const float4*>(B + (n0 + i) * sb + swz(n0 + i, k, bm));
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -242,9 +258,9 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
   float* hs = cm + kQ * NX;        // [P4][NX]  H (forward state entering the chunk)
   float* rs = hs + P4 * NX;        // [P4][NX]  R (adjoint carried in from the right)
   float* T1 = rs + P4 * NX;        // [tau][s]  C_tau . B_s, then M
-  float* T2 = T1 + kQ * kQ;        // [s][tau]  x_s . dy_tau, then K2 [t][s]
+  float* T2 = T1 + kQ * kQ;        // [tau][s]  x_s . dy_tau, then K2 [t][s]
   float* T3 = T2 + kQ * kQ;        // [tau][s]  L, then N2
-  float* rowP = T3 + kQ * kQ;      // [16][kQ]  partial row sums of K (by column tile)
+  float* rowP = T3 + kQ * kQ;      // [kQ][16]  partial row sums of K (by column tile)
   float* colP = rowP + 16 * kQ;    // [16][kQ]  partial column sums of K (by row tile)
   float* csv = colP + 16 * kQ;     // [kQ] cs
   float* dts = csv + kQ;           // [kQ] dt
@@ -269,20 +285,21 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
   const float Ah = A[h];
   const float Dh = D ? D[h] : 0.f;
   const float* csb = cs + (bh * nchunks + c) * kQ;
+  const int mP = swz_mask(PX / 4), mN = swz_mask(NX / 4);  // swizzles of x and of B, H, R
 
   // ---- load the chunk (zeros in the padding and past the sequence's end) ----
   for (int i = tid; i < kQ * PX; i += kBwdThreads) {
     const int t = i / PX, p = i % PX;
     const bool in = t < nvalid && p < P;
     const int64_t off = ((b * seqlen + t0 + t) * nheads + h) * P + p;
-    xs[i] = in ? io_traits<T>::load(x, off) : 0.f;
+    xs[t * PX + swz(t, p, mP)] = in ? io_traits<T>::load(x, off) : 0.f;
     ys[i] = in ? dy[off] : 0.f;
   }
   for (int i = tid; i < kQ * NX; i += kBwdThreads) {
     const int t = i / NX, n = i % NX;
     const bool in = t < nvalid && n < N;
     const int64_t off = ((b * seqlen + t0 + t) * ngroups + g) * N + n;
-    bs[i] = in ? io_traits<T>::load(Bm, off) : 0.f;
+    bs[t * NX + swz(t, n, mN)] = in ? io_traits<T>::load(Bm, off) : 0.f;
     cm[i] = in ? io_traits<T>::load(Cm, off) : 0.f;
   }
   {
@@ -291,8 +308,9 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     for (int i = tid; i < P4 * NX; i += kBwdThreads) {  // global [p][n] -> shared [p][n]
       const int p = i / NX, n = i % NX;
       const bool in = p < P && n < N;
-      hs[i] = in ? hsrc[int64_t(p) * N + n] : 0.f;
-      rs[i] = in ? rsrc[int64_t(p) * N + n] : 0.f;
+      const int o = p * NX + swz(p, n, mN);
+      hs[o] = in ? hsrc[int64_t(p) * N + n] : 0.f;
+      rs[o] = in ? rsrc[int64_t(p) * N + n] : 0.f;
     }
   }
   for (int t = tid; t < kQ; t += kBwdThreads) {
@@ -302,12 +320,12 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
   __syncthreads();
   const float cs_end = csv[kQ - 1];
 
-  // ---- the chunk's quadratic tables: C.B, x.dy and L (4 x 4 per thread) ----
+  // ---- the chunk's quadratic tables: C.B, (x.dy)^T and L (4 x 4 per thread) ----
   {
     float acc[4][4];
     zero4x4(acc);
-    if (half == 0) mm_nt(acc, cm, NX, bs, NX, 4 * ta, 4 * tb, 0, N4);  // C.B [tau][s]
-    else mm_nt(acc, xs, PX, ys, PX, 4 * ta, 4 * tb, 0, P4);            // x.dy [s][tau]
+    if (half == 0) mm_nt(acc, cm, NX, 0, bs, NX, mN, 4 * ta, 4 * tb, 0, N4);  // C.B [tau][s]
+    else mm_nt(acc, ys, PX, 0, xs, PX, mP, 4 * ta, 4 * tb, 0, P4);  // x_s . dy_tau [tau][s]
     float* dst = half == 0 ? T1 : T2;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -333,7 +351,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
         const int s = 4 * tb + j;
         const float lv = T3[tau * kQ + s], cbv = T1[tau * kQ + s];
         mv[i][j] = lv * cbv;
-        n2[i][j] = lv * T2[s * kQ + tau];
+        n2[i][j] = lv * T2[tau * kQ + s];
         k2[i][j] = dts[s] * n2[i][j];
       }
     }
@@ -342,7 +360,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
       float rsum = 0.f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) rsum = fmaf(k2[i][j], T1[(4 * ta + i) * kQ + 4 * tb + j], rsum);
-      rowP[tb * kQ + 4 * ta + i] = rsum;
+      rowP[(4 * ta + i) * 16 + tb] = rsum;
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -367,10 +385,14 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
   }
   for (int i = tid; i < 2 * kQ; i += kBwdThreads) {
     const int r = i % kQ;
-    const float* part = i < kQ ? rowP : colP;
     float sum = 0.f;
-    for (int k = 0; k < 16; ++k) sum += part[k * kQ + r];
-    (i < kQ ? rowK : colK)[r] = sum;
+    if (i < kQ) {
+      for (int k = 0; k < 16; ++k) sum += rowP[r * 16 + k];
+      rowK[r] = sum;
+    } else {
+      for (int k = 0; k < 16; ++k) sum += colP[k * kQ + r];
+      colK[r] = sum;
+    }
   }
   __syncthreads();
 
@@ -386,8 +408,8 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
         float q[4][4], rb[4][4];
         zero4x4(q);
         zero4x4(rb);
-        mm_tn(q, T1, kQ, ys, PX, 4 * ta, p0, 4 * ta, kQ);
-        mm_nt(rb, bs, NX, rs, NX, 4 * ta, p0, 0, N4);
+        mm_tn(q, T1, kQ, 0, ys, PX, 0, 4 * ta, p0, 4 * ta, kQ);
+        mm_nt(rb, bs, NX, mN, rs, NX, mN, 4 * ta, p0, 0, N4);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = 4 * ta + i;
@@ -396,7 +418,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const float qv = fmaf(er, rb[i][j], q[i][j]);
-            const float xv = xs[t * PX + p0 + j], yv = ys[t * PX + p0 + j];
+            const float xv = xs[t * PX + swz(t, p0 + j, mP)], yv = ys[t * PX + p0 + j];
             o[j] = fmaf(dts[t], qv, Dh * yv);
             s1[i] = fmaf(xv, qv, s1[i]);
             sv[i] = fmaf(xv, rb[i][j], sv[i]);
@@ -412,7 +434,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
       } else {
         float hc[4][4];
         zero4x4(hc);
-        mm_nt(hc, cm, NX, hs, NX, 4 * ta, p0, 0, N4);
+        mm_nt(hc, cm, NX, 0, hs, NX, mN, 4 * ta, p0, 0, N4);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -451,8 +473,8 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
       float sb[4][4], xr[4][4];
       zero4x4(sb);
       zero4x4(xr);
-      mm_tn(sb, T3, kQ, cm, NX, 4 * ta, n0, 4 * ta, kQ);
-      mm_nn(xr, xs, PX, rs, NX, 4 * ta, n0, 0, P4);
+      mm_tn(sb, T3, kQ, 0, cm, NX, 0, 4 * ta, n0, 4 * ta, kQ);
+      mm_nn(xr, xs, PX, mP, rs, NX, mN, 4 * ta, n0, 0, P4);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = 4 * ta + i;
@@ -467,8 +489,8 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
       float sc[4][4], yh[4][4];
       zero4x4(sc);
       zero4x4(yh);
-      mm_nn(sc, T2, kQ, bs, NX, 4 * ta, n0, 0, 4 * ta + 4);
-      mm_nn(yh, ys, PX, hs, NX, 4 * ta, n0, 0, P4);
+      mm_nn(sc, T2, kQ, 0, bs, NX, mN, 4 * ta, n0, 0, 4 * ta + 4);
+      mm_nn(yh, ys, PX, 0, hs, NX, mN, 4 * ta, n0, 0, P4);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = 4 * ta + i;
@@ -481,7 +503,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
       }
     }
   }
-  // exp(cs_end) <R, H>
+  // exp(cs_end) <R, H> (R and H share one layout)
   float rh = 0.f;
   for (int i = tid; i < P4 * NX; i += kBwdThreads) rh = fmaf(rs[i], hs[i], rh);
   rh = warp_sum(rh);

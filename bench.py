@@ -18,8 +18,9 @@ the data path; times are the max over ranks.
 cores, each step a bounded sample of the same workload (batch row 0: 80 heads x 64 channels
 x 8192 tokens), and reports the same metric.
 
---profile scan|decode runs only W + K calls of that workload and prints nothing else: the
-command the launch lists and ncu captures under profiles/ were taken with.
+--profile scan|decode|backward runs only W + K calls of that workload (backward: the gradients
+at the 130M-layer shape) and prints nothing else: the command the launch lists and ncu captures
+under profiles/ were taken with.
 
 --glue times the block steps around the layer at the 2.7B shape (short convolution + SiLU over
 the 5376 x/B/C channels, dt softplus, SiLU output gate over y) and prints one JSON line with
@@ -86,7 +87,10 @@ def step_bytes(c, y_bytes=4):
 # those sources match.
 KERNEL_SOURCES = {"scan": ("ssd_common.cuh", "tc_prims.cuh", "tc_kernels.cuh"),
                   "decode": ("ssd_common.cuh", "step_kernels.cuh")}
-MEASURED_TRAFFIC = {"scan": (None, None),
+# scan: from the 4 x 2048-token capture, per-block reads x4 plus the initial state, and y x4 plus
+# the final state less the 46.8 MB of y still dirty in L2 when the kernel exits (read 377.8 MB,
+# write 634.8 MB; profiles/scan_walk_2p7b_ncu.md)
+MEASURED_TRAFFIC = {"scan": (1012601200, "574e2e69e6126a19"),
                     "decode": (1291061248, "1418c01d203c6f57")}
 
 
@@ -570,6 +574,14 @@ def run_profile(args):
         for _ in range(args.warmup + args.steps):
             ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], c["chunk"],
                                init_state=t["init"])
+    elif args.profile == "backward":
+        c = ssd_inputs.resolve(1)  # the 130M-layer shape, float32 dy
+        t = device_scan_inputs(c, dev, 1101)
+        g = torch.Generator(device=dev).manual_seed(1108)
+        dy = torch.randn(t["x"].shape, generator=g, device=dev)
+        for _ in range(args.warmup + args.steps):
+            ssd.chunk_scan_bwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], dy,
+                               init_state=t["init"])
     else:
         dec = ssd_inputs.make_decode_inputs(DECODE_CFG)
         st = to_dev(dec["state"], False, dev)
@@ -701,7 +713,7 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per scan call (null when not measured)")
     ap.add_argument("--decode-traffic", type=float, default=None)
-    ap.add_argument("--profile", choices=["scan", "decode"], default=None)
+    ap.add_argument("--profile", choices=["scan", "decode", "backward"], default=None)
     ap.add_argument("--glue", action="store_true")
     ap.add_argument("--selective", action="store_true")
     ap.add_argument("--seqlen", type=int, default=None,

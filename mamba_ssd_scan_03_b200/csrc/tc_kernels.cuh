@@ -5,10 +5,10 @@
 // TMEM.  Per block: G = C B^T (once for both heads), masked diagonal tile (L o G o dt) X,
 // off-diagonal C H, skip term D x, y store, then H <- exp(cs_end) H + B^T (w*x) in place.
 //
-// The walk's work is cut into equal ranges of blocks, one per CTA.  When there are at least
-// about as many (batch row, head pair) sequences as SMs, a range starting inside a sequence gets
-// its entering state from the CTA that walked the sequence's head (published through L2), and
-// nothing else runs.  With fewer, longer sequences each is cut into segments first:
+// The walk's work is cut into equal ranges of blocks, one per CTA.  Unless a sequence is much
+// longer than every CTA's share of all blocks, a range starting inside a sequence gets its
+// entering state from the CTA that walked the sequence's head (published through L2), and
+// nothing else runs.  With few, long sequences each is cut into segments first:
 //
 //  seg_state   per (b, segment, head pair): S_seg = sum_{t in seg} exp(sum_{k>t in seg} a_k)
 //              dt_t B_t x_t^T, one long-K GEMM on the tensor cores (A = B^T, B = w*x, K =
@@ -528,12 +528,12 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 // starts inside a segment continues the previous range's last item: that CTA walks its last item
 // FIRST and publishes the state it ends with; this CTA walks such an item LAST and reads that
 // state.  A CTA thus only ever waits on a lower ticket's first item, which waits on nothing.
-// With at least as many sequences as CTAs every segment is a whole sequence and there is no
-// summary pass at all: x is read once and no state leaves the L2 except final_state.
+// When every segment is a whole sequence there is no summary pass at all: x is read once and no
+// state leaves the L2 except final_state.
 //
 // Per block k (G = C B^T once for both heads; masks; diagonal tiles (L o G o dt) X; off-
 // diagonal C H; skip term D x; y store; then H <- exp(cs_end) H + B^T (w*x) in place), with
-// block = 640 threads in five roles:
+// block = 608 threads in four roles:
 //   warps 0-15  compute (512 threads).  Thread (row = tid % 128, q = tid / 128): token row
 //               `row` of a block (state row n = row in the state passes) and a quarter of the
 //               columns: head j = q / 2 with p in [32 (q % 2), +32) for the state pass, X' and
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 //               latency, not only its instructions, bounds the block).  They also load each
 //               item's entering state into TMEM and store its exit state.
 //   warp 16     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block, and x
-//               of the block after next into L2; and, with the whole warp, the cumsums: each
+//               of the next block into L2; and, with the whole warp, the cumsums: each
 //               block's dt of the two heads and its log2 cumsums in shared memory, up to two
 //               blocks ahead (lane l: rows 4l .. 4l+3).
 //   warp 17     MMA issuer (lane 0).

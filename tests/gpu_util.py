@@ -60,6 +60,20 @@ def sample_chains(cfg, n, seed=0):
     return ids, b, h, p
 
 
+def stratified_chains(cfg, per_pair, seed=0):
+    """per_pair distinct channels p of every (batch row, head) pair: every head pair, and so every
+    CTA range of the walk and every hand-off between ranges, is among the compared chains."""
+    Bt, H, P = cfg["batch"], cfg["nheads"], cfg["headdim"]
+    rng = np.random.default_rng(seed)
+    ids = []
+    for bb in range(Bt):
+        for hh in range(H):
+            for pp in rng.choice(P, size=min(per_pair, P), replace=False):
+                ids.append((bb * H + hh) * P + int(pp))
+    ids = np.unique(np.asarray(ids, dtype=np.int64))
+    return ids, ids // (P * H), (ids // P) % H, ids % P
+
+
 def oracle_chains(inp, ids, b, h, p):
     init = None if inp["init"] is None else inp["init"][b, h, p]
     return oracle.scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], init=init,

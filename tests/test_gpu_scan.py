@@ -15,7 +15,7 @@ import mamba_ssd_scan_03_b200 as ssd
 import oracle
 import ssd_inputs
 from gpu_util import (TOL, bf16_excess, dev_inputs, oracle_chains, rel_err, sample_chains,
-                      to_dev, to_np)
+                      stratified_chains, to_dev, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -323,13 +323,16 @@ def test_device_argument_errors():
 
 
 # ---- full-size workloads: sampled chains, the launch configuration bench.py times -------------
-@pytest.mark.parametrize("cfg_idx,n_chains", [(1, 96), (2, 96)])
-def test_full_size_workload(cfg_idx, n_chains):
+@pytest.mark.parametrize("cfg_idx,per_pair", [(1, 4), (2, 3)])
+def test_full_size_workload(cfg_idx, per_pair):
+    """Configs 1 and 2 at full size, in bench.py's launch configuration: 768 and 960 chains (a few
+    channels of every (batch row, head) pair) and their final states against the oracle."""
     inp = ssd_inputs.make_scan_inputs(cfg_idx)
     cfg = inp["cfg"]
     t = dev_inputs(inp)
     y, fin = run(inp, t)
-    ids, b, h, p = sample_chains(cfg, n_chains, seed=cfg_idx)
+    ids, b, h, p = stratified_chains(cfg, per_pair, seed=cfg_idx)
+    assert len(ids) == cfg["batch"] * cfg["nheads"] * per_pair
     yo, fo = oracle_chains(inp, ids, b, h, p)
     yg = to_np(y[torch.as_tensor(b), :, torch.as_tensor(h), torch.as_tensor(p)])
     fg = to_np(fin[torch.as_tensor(b), torch.as_tensor(h), torch.as_tensor(p)])

@@ -47,10 +47,12 @@ __device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.f +
 
 // out[b,t,c] = silu(bias[c] + sum_{k<K} w[c,k] u[b, t-K+1+k, c]), u = 0 before t = 0.
 // One thread per (batch row, 16-byte group of channels, run of kConvTok tokens): its weights
-// and bias sit in registers, the last K-1 input rows in a register window, and each input row
-// is read once with a 16-byte load (a warp reads 32 neighbouring groups: 512 contiguous bytes).
-// The K-1 rows before the run are read again by the previous run's thread (K-1 of kConvTok).
-constexpr int kConvTok = 64;
+// and bias sit in registers, the last K-1 input rows in a register window, and the run's rows
+// are read kConvStep at a time, their 16-byte loads issued together (a warp reads 32
+// neighbouring groups: 512 contiguous bytes per row), so that a thread keeps several loads in
+// flight.  The K-1 rows before the run are read again by the previous run's thread (K-1 of
+// kConvTok).
+constexpr int kConvTok = 64, kConvStep = 4;
 
 template <typename T, int K>
 __global__ void __launch_bounds__(128) conv_silu_kernel(const T* __restrict__ u,
@@ -59,6 +61,7 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(const T* __restrict__ u,
                                                         T* __restrict__ out, int64_t seqlen,
                                                         int cdim) {
   constexpr int VW = vec<T>::VW;
+  constexpr int W = K - 1 + kConvStep;  // window rows: K - 1 before the step, then the step's
   const int cg = blockIdx.x * blockDim.x + threadIdx.x;
   if (cg >= cdim / VW) return;
   const int c0 = cg * VW;
@@ -81,7 +84,7 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(const T* __restrict__ u,
 #pragma unroll
   for (int j = 0; j < VW; ++j) bv[j] = bias ? bias[c0 + j] : 0.f;
 
-  float win[K][VW];  // win[k] = input row t-K+1+k; rows before t = 0 are zero
+  float win[W][VW];  // win[k] = input row t-K+1+k; rows before t = 0 (and past the end) zero
 #pragma unroll
   for (int k = 0; k < K - 1; ++k) {
     const int64_t ts = t0 - (K - 1) + k;
@@ -91,21 +94,33 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(const T* __restrict__ u,
       for (int j = 0; j < VW; ++j) win[k][j] = 0.f;
     }
   }
-  for (int64_t t = t0; t < t1; ++t) {
-    vec<T>::load(ub + t * cdim, win[K - 1]);
-    float o[VW];
+  for (int64_t t = t0; t < t1; t += kConvStep) {
 #pragma unroll
-    for (int j = 0; j < VW; ++j) {
-      float acc = bv[j];
+    for (int i = 0; i < kConvStep; ++i) {
+      if (t + i < t1) vec<T>::load(ub + (t + i) * cdim, win[K - 1 + i]);
+      else {
 #pragma unroll
-      for (int k = 0; k < K; ++k) acc = fmaf(wr[j][k], win[k][j], acc);
-      o[j] = silu_fast(acc);
+        for (int j = 0; j < VW; ++j) win[K - 1 + i][j] = 0.f;
+      }
     }
-    vec<T>::store(ob + t * cdim, o);
+#pragma unroll
+    for (int i = 0; i < kConvStep; ++i) {
+      if (t + i < t1) {
+        float o[VW];
+#pragma unroll
+        for (int j = 0; j < VW; ++j) {
+          float acc = bv[j];
+#pragma unroll
+          for (int k = 0; k < K; ++k) acc = fmaf(wr[j][k], win[i + k][j], acc);
+          o[j] = silu_fast(acc);
+        }
+        vec<T>::store(ob + (t + i) * cdim, o);
+      }
+    }
 #pragma unroll
     for (int k = 0; k < K - 1; ++k)
 #pragma unroll
-      for (int j = 0; j < VW; ++j) win[k][j] = win[k + 1][j];
+      for (int j = 0; j < VW; ++j) win[k][j] = win[k + kConvStep][j];
   }
 }
 

@@ -324,11 +324,14 @@ ssd_status set_smem_attrs() {
     ok &= cudaFuncSetAttribute(ssd::tc::scan_walk_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) ==
           cudaSuccess;
-    // the selective scan runs ~17 one-warp CTAs per SM: ask for the largest shared-memory
+    // the selective scan runs many small CTAs per SM: ask for the largest shared-memory
     // carve-out so that shared memory does not cap them
-    for (auto f : {(const void*)ssd::sel::selective_scan_kernel<float, float>,
-                   (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, float>,
-                   (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, __nv_bfloat16>})
+#define SSD_SEL_FNS(W)                                                                     \
+  (const void*)ssd::sel::selective_scan_kernel<float, float, W>,                           \
+      (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, float, W>,               \
+      (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, __nv_bfloat16, W>
+    for (auto f : {SSD_SEL_FNS(1), SSD_SEL_FNS(2), SSD_SEL_FNS(4)})
+#undef SSD_SEL_FNS
       ok &= cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  int(cudaSharedmemCarveoutMaxShared)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
@@ -1053,34 +1056,45 @@ ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A
   namespace sel = ssd::sel;
   if (dstate != sel::kN || dim % sel::kCpw != 0 || (dim / ngroups) % sel::kCpw != 0)
     return SSD_ERR_UNSUPPORTED;
+  // warps per CTA: the most (up to four) whose 8-channel slices stay inside one group
+  const int cpg = dim / ngroups;
+  const int wpc = cpg % (4 * sel::kCpw) == 0 ? 4 : (cpg % (2 * sel::kCpw) == 0 ? 2 : 1);
+  const int cw = wpc * sel::kCpw;
   for (const void* p : {x, (const void*)dt, (const void*)A, B, C, (const void*)y,
                         (const void*)init_state, (const void*)final_state})
     if (p && !aligned16(p)) return SSD_ERR_UNSUPPORTED;
-  const int64_t warps = batch * (dim / sel::kCpw);
-  if (warps > INT32_MAX || seqlen > INT32_MAX - sel::kTok || batch > INT32_MAX)
+  const int64_t ctas = batch * (dim / cw);
+  if (ctas > INT32_MAX || seqlen > INT32_MAX - sel::kTok || batch > INT32_MAX)
     return SSD_ERR_UNSUPPORTED;
   const bool bf = io == SSD_BF16, ybf = y_dtype == SSD_BF16;
   const CUtensorMapDataType tio = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const uint64_t L = uint64_t(seqlen), Bn = uint64_t(batch), GN = uint64_t(ngroups) * sel::kN;
   CUtensorMap mx, mdt, mb, mc, my;
-  if (!make_box_map(&mx, x, tio, es, dim, L, Bn, sel::kCpw, sel::kTok) ||
-      !make_box_map(&mdt, dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, L, Bn, sel::kCpw,
+  if (!make_box_map(&mx, x, tio, es, dim, L, Bn, uint32_t(cw), sel::kTok) ||
+      !make_box_map(&mdt, dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dim, L, Bn, uint32_t(cw),
                     sel::kTok) ||
       !make_box_map(&mb, B, tio, es, GN, L, Bn, sel::kN, sel::kTok) ||
       !make_box_map(&mc, C, tio, es, GN, L, Bn, sel::kN, sel::kTok) ||
       !make_box_map(&my, y,
                     ybf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                    ybf ? 2 : 4, dim, L, Bn, sel::kCpw, sel::kTok))
+                    ybf ? 2 : 4, dim, L, Bn, uint32_t(cw), sel::kTok))
     return SSD_ERR_CUDA;
   if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
-  const unsigned grid = unsigned(warps);
-#define SSD_SEL(T, TY)                                                                      \
-  sel::selective_scan_kernel<T, TY><<<grid, 32, sel::Smem<T, TY>::kBytes, stream>>>(        \
+  const unsigned grid = unsigned(ctas);
+#define SSD_SEL(T, TY, W)                                                                   \
+  sel::selective_scan_kernel<T, TY, W><<<grid, 32 * W, sel::Smem<T, TY, W>::kBytes, stream>>>( \
       mx, mdt, mb, mc, my, A, D, init_state, final_state, seqlen, dim, ngroups)
-  if (!bf) SSD_SEL(float, float);
-  else if (!ybf) SSD_SEL(__nv_bfloat16, float);
-  else SSD_SEL(__nv_bfloat16, __nv_bfloat16);
+#define SSD_SEL_W(T, TY)                 \
+  do {                                   \
+    if (wpc == 4) SSD_SEL(T, TY, 4);     \
+    else if (wpc == 2) SSD_SEL(T, TY, 2); \
+    else SSD_SEL(T, TY, 1);              \
+  } while (0)
+  if (!bf) SSD_SEL_W(float, float);
+  else if (!ybf) SSD_SEL_W(__nv_bfloat16, float);
+  else SSD_SEL_W(__nv_bfloat16, __nv_bfloat16);
+#undef SSD_SEL_W
 #undef SSD_SEL
   return launched();
 }

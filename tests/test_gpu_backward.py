@@ -65,6 +65,7 @@ def check(inp, dy, dfin, got, with_init=True, with_D=True, tol=TOL, skip=()):
     dict(batch=2, seqlen=130, nheads=6, headdim=32, dstate=64, ngroups=3),
     dict(batch=1, seqlen=64, nheads=2, headdim=64, dstate=128),             # one chunk
     dict(batch=3, seqlen=1, nheads=2, headdim=16, dstate=32),               # one token
+    dict(batch=2, seqlen=100, nheads=2, headdim=18, dstate=30),             # widths not /4
 ])
 def test_backward_small(io, shape):
     inp, dy, dfin = make(40 + shape["seqlen"], io=io, **shape)

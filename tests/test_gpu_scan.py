@@ -78,6 +78,11 @@ def test_tensor_core_path_small(shape):
     dict(batch=2, seqlen=300, nheads=4),
     dict(batch=1, seqlen=513, nheads=4, ngroups=4),  # one group per head
     dict(batch=2, seqlen=200, nheads=3, headdim=24, dstate=40, ngroups=1),
+    # wide states (the chunk summaries stage 32 and 16 tokens at a time) and widths that are
+    # not multiples of four (element-by-element loads, padded rows)
+    dict(batch=1, seqlen=150, nheads=2, headdim=32, dstate=256, ngroups=1),
+    dict(batch=1, seqlen=100, nheads=2, headdim=16, dstate=512, ngroups=2),
+    dict(batch=2, seqlen=90, nheads=2, headdim=18, dstate=30, ngroups=1),
 ])
 def test_simt_path_small(io, shape):
     inp = small(io=io, **shape)

@@ -1165,14 +1165,14 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
         }
 #undef SSD_MASK_GROUP
         // ---- state pass (lane n = row, columns (j, p0 .. p0+32)): bf16 high/low copy of H for
-        //      C H, then H <- exp(cs_end) H in place.  Needs the previous block's state MMA and
-        //      the previous block's y stores to have read the staging buffer (sHh/sHl) ----
+        //      C H (the decay H <- exp(cs_end) H follows in the X' phase).  Needs the previous
+        //      block's state MMA and the previous block's y stores to have read the staging
+        //      buffer (sHh/sHl) ----
         if (k > 0) ok = ok && mbar_wait(&bars.st_done, par ^ 1, abort_v, 51, pl.wait_ns);
         if (k > 0) ok = ok && mbar_wait(&bars.stage_free[j], par ^ 1, abort_v, 55, pl.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           tc_fence_after();
-          const float al = ex2(cs_sh[bf][j][kBlk - 1]);
           uint8_t* hh = smem + kOffHh + j * kTile;
           uint8_t* hl = smem + kOffHl + j * kTile;
           uint32_t ra[16], rb[16];
@@ -1188,20 +1188,12 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     *reinterpret_cast<uint4*>(hh + swz(row, ch + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]); \
     *reinterpret_cast<uint4*>(hl + swz(row, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);    \
     *reinterpret_cast<uint4*>(hl + swz(row, ch + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]); \
-    _Pragma("unroll") for (int e = 0; e < 8; ++e) {                                          \
-      const float2 sc = mul2(make_float2(__uint_as_float(R[2 * e]), __uint_as_float(R[2 * e + 1])), \
-                             make_float2(al, al));                                            \
-      R[2 * e] = __float_as_uint(sc.x);                                                       \
-      R[2 * e + 1] = __float_as_uint(sc.y);                                                   \
-    }                                                                                         \
-    tmem_st16(tH + lane_off + j * 64 + p0 + (PC) * 16, R);                                   \
   }
           SSD_HPASS(ra, 0)
           tmem_ld16(tH + lane_off + j * 64 + p0 + 16, rb);
           tmem_wait_ld();
           SSD_HPASS(rb, 1)
 #undef SSD_HPASS
-          tmem_wait_st();
           fence_proxy_async_smem();
         }
         tc_fence_before();
@@ -1225,6 +1217,25 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
                               scale_bf16x2(v.w, ww));
           }
           fence_proxy_async_smem();
+          // H <- exp(cs_end) H in TMEM before the state MMA adds B^T X' (done here, off the
+          // masks -> state pass -> C H -> next C chain, which only needs H's bf16 copy)
+          const float al = ex2(cs_sh[bf][j][kBlk - 1]);
+#pragma unroll
+          for (int pc = 0; pc < 2; ++pc) {
+            uint32_t r[16];
+            tmem_ld16(tH + lane_off + j * 64 + p0 + pc * 16, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 sc = mul2(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
+                                     make_float2(al, al));
+              r[2 * e] = __float_as_uint(sc.x);
+              r[2 * e + 1] = __float_as_uint(sc.y);
+            }
+            tmem_st16(tH + lane_off + j * 64 + p0 + pc * 16, r);
+          }
+          tmem_wait_st();
+          tc_fence_before();
         }
         // the last block of an item whose exit state is kept also sends the bf16 remainder of
         // X' (over C's tiles, free once C H is done): its X' is handed over only then

@@ -111,22 +111,26 @@ __global__ void adj_pass_kernel(float* __restrict__ adj, const float* __restrict
   float* base = adj + (b * nchunks * nheads + h) * per_bh + pn;  // chunk c: + c * cstride
   const int64_t cstride = int64_t(nheads) * per_bh;
   const float* last = cs + bh * nchunks * kQ + kQ - 1;  // chunk c's last cumsum: + c * kQ
-  // kBatch chunks' loads in flight at once, then the recurrence over them (last chunk first)
+  // kBatch chunks' loads in flight at once, then the recurrence over them (last chunk first).
+  // The loop counts chunks from the last one upwards (a count-down loop over the same chunks
+  // measured 4x slower: its loads were not kept in flight together)
   constexpr int kBatch = 8;
-  for (int c0 = nchunks - 1; c0 >= 0; c0 -= kBatch) {
+  for (int r0 = 0; r0 < nchunks; r0 += kBatch) {  // r: chunks counted from the last
     float sv[kBatch], lv[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int64_t c = c0 - i;
-      if (c >= 0) {
+      const int r = r0 + i;
+      if (r < nchunks) {
+        const int64_t c = nchunks - 1 - r;
         sv[i] = base[c * cstride];
         lv[i] = last[c * kQ];
       }
     }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int64_t c = c0 - i;
-      if (c >= 0) {
+      const int r = r0 + i;
+      if (r < nchunks) {
+        const int64_t c = nchunks - 1 - r;
         base[c * cstride] = run;
         run = fmaf(expf(lv[i]), run, sv[i]);
       }

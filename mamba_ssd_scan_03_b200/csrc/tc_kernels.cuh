@@ -855,7 +855,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     };
     if (nit > 0) load_dt(0, items_sh[0].k0);
     const float inf = __int_as_float(0x7f800000);
-    // bounded wait by every lane, the same verdict in all of them
+    // bounded wait by every lane, the same result in all of them
     auto wait_all = [&](uint64_t* bar, uint32_t parity, unsigned site) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, site, pl.wait_ns));
     };

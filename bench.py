@@ -323,10 +323,32 @@ def time_backward(c, dev, seed, steps, warmup, hbm):
     tok = c["batch"] * c["seqlen"]
     del t, dy, flush, ws
     torch.cuda.empty_cache()
+    flops = 2 * backward_fmas(c)
+    achieved = flops / (ms * 1e-3) / 1e12
     return {"ms": round(ms, 5), "tokens_per_s": round(tok / (ms * 1e-3), 1),
             "kernels": "float32 CUDA cores (cumsum, chunk states, state pass, adjoint summaries, "
                        "adjoint pass, per-chunk gradients, group and head sums: 8 launches)",
+            "roofline": {"bound": "fp32 fma", "flops": flops, "achieved_tflops": round(achieved, 2),
+                         "peak_tflops": round(FP32_TFLOPS, 1), "frac": round(achieved / FP32_TFLOPS, 4),
+                         "peak_src": "148 SMs x 128 FMA/clk x 2 flops x 1965 MHz (nominal)"},
             "steps": steps, "l2": "flushed before every timed call (256 MB write)"}
+
+
+# float32 FMAs the backward kernels perform (chunks of 64 tokens): the chunk and adjoint summaries
+# (P N Q each), and per chunk the C.B and x.dy tables, the per-token products (M^T dy over
+# tau >= t: about Q/2 + 2 terms, B R, C H) and the dB / dC products (N2^T C and K2 B over about
+# Q/2 + 2 terms, x R, dy H), as the kernels tile them
+FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_fmas(c):
+    Q = 64
+    P, N = c["headdim"], c["dstate"]
+    half = Q // 2 + 2
+    per_chunk = (2 * P * N * Q + Q * Q * N + Q * Q * P + Q * P * half + 2 * Q * P * N +
+                 2 * Q * N * half + 2 * Q * N * P)
+    nc = (c["seqlen"] + Q - 1) // Q
+    return per_chunk * c["batch"] * nc * c["nheads"]
 
 
 def scan_extras(dev, hbm, steps=5, warmup=3):

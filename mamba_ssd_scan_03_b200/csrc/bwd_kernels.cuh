@@ -45,7 +45,6 @@ namespace ssd {
 namespace bwd {
 
 constexpr int kQ = 64;         // tokens per chunk of the backward (the result does not depend on it)
-constexpr int kThreads = 256;
 constexpr int kBwdThreads = 512;  // chunk_bwd: two halves of 256 threads
 
 // ---- 1. adjoint summaries: grid (nchunks, batch * nheads), block 256 ------------------------

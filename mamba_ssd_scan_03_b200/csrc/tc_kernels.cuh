@@ -591,20 +591,6 @@ template <> struct ystage<float> {
       *reinterpret_cast<float4*>(box + swz(t, half * 4 + i)) =
           make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   }
-  // thread (t, head j) writes y[t, p0 .. p0+8) (p0 a multiple of 8)
-  static __device__ __forceinline__ void put8(uint8_t* stage, int t, int j, int p0,
-                                              const float (&v)[8]) {
-    uint8_t* box = stage + (2 * j + (p0 >> 5)) * kTile;
-    const int c = (p0 & 31) >> 2;
-    *reinterpret_cast<float4*>(box + swz(t, c)) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(box + swz(t, c + 1)) = make_float4(v[4], v[5], v[6], v[7]);
-  }
-  static __device__ __forceinline__ void store(const CUtensorMap* map, const uint8_t* stage,
-                                               int h0, int t0, int b) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      tma_store_3d(map, stage + q * kTile, (h0 + q / 2) * kP + (q % 2) * 32, t0, b);
-  }
   // part 0: the boxes over the staging's tiles 0 and 2 (sHh and sHl of head 0); part 1: tiles 1
   // and 3 (head 1)
   static __device__ __forceinline__ void store_part(const CUtensorMap* map, const uint8_t* stage,
@@ -628,17 +614,6 @@ template <> struct ystage<__nv_bfloat16> {
     *reinterpret_cast<uint4*>(box + swz(t, c0 + 1)) =
         make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
                    pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-  }
-  static __device__ __forceinline__ void put8(uint8_t* stage, int t, int j, int p0,
-                                              const float (&v)[8]) {
-    *reinterpret_cast<uint4*>(stage + j * kTile + swz(t, p0 >> 3)) =
-        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                   pack_bf16x2(v[6], v[7]));
-  }
-  static __device__ __forceinline__ void store(const CUtensorMap* map, const uint8_t* stage,
-                                               int h0, int t0, int b) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) tma_store_3d(map, stage + j * kTile, (h0 + j) * kP, t0, b);
   }
   // part j: head j's box, over the staging's tile j
   static __device__ __forceinline__ void store_part(const CUtensorMap* map, const uint8_t* stage,

@@ -151,6 +151,29 @@ def test_walk_plans_agree():
     check_full(inp, *out[0])
 
 
+def test_batch_rows_in_separate_calls():
+    """Each batch row scanned by its own call on views of the same tensors (on its own streams,
+    as bench.py's end-to-end leg does) matches the whole-batch call: rows are independent, only
+    the plan (and so where boundary states are handed over) differs."""
+    inp = small(seed=31, batch=3, seqlen=1500, nheads=4)
+    t = dev_inputs(inp)
+    y, fin = run(inp, t)
+    yr = torch.empty_like(y)
+    fr = torch.empty_like(fin)
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    torch.cuda.synchronize()
+    for r, st in enumerate(streams):
+        with torch.cuda.stream(st):
+            sl = slice(r, r + 1)
+            ssd.chunk_scan_fwd(t["x"][sl], t["dt"][sl], t["A"], t["B"][sl], t["C"][sl], t["D"],
+                               256, init_state=t["init"][sl], out=yr[sl], final_out=fr[sl])
+    torch.cuda.synchronize()
+    assert ssd.device_status() == 0
+    assert rel_err(to_np(yr), to_np(y)) <= TOL["bf16"]
+    assert rel_err(to_np(fr), to_np(fin)) <= TOL["bf16"]
+    check_full(inp, yr, fr)
+
+
 @pytest.mark.parametrize("plan", [1, 2])
 def test_device_timeout_is_reported_and_recovered(plan):
     """A wait that gives up: with no waiting allowed every CTA's first wait on an event that has

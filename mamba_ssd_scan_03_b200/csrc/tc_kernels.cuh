@@ -541,10 +541,11 @@ __global__ void __launch_bounds__(kPassThreads, 4) seg_pass_kernel(
 //               each TMEM lane quarter, so every phase is spread over all 16 warps (a phase's
 //               latency, not only its instructions, bounds the block).  They also load each
 //               item's entering state into TMEM and store its exit state.
-//   warp 16     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block, and x
-//               of the next block into L2; and, with the whole warp, the cumsums: each
-//               block's dt of the two heads and its log2 cumsums in shared memory, up to two
-//               blocks ahead (lane l: rows 4l .. 4l+3).
+//   warp 16     TMA producer (lane 0): B (double buffer), C, x (single buffers) per block; and,
+//               with the whole warp, the cumsums: each block's dt of the two heads and its log2
+//               cumsums in shared memory, up to two blocks ahead (lane l: rows 4l .. 4l+3).
+//               x is not prefetched into L2 ahead of its load: TMA prefetches a block ahead
+//               measured slower, as the C loads of the per-block chain then wait behind them.
 //   warp 17     MMA issuer (lane 0).
 //   warp 18     y writer (lane 0): TMA stores of each block's staged y, in two groups (one per
 //               head) whose halves of the staging buffer are handed back separately.
@@ -791,24 +792,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
     // wait for block j - 2's compute to finish, which comes before block j - 1's C H, so the
     // C and x loads after them are not held back.
     const uint64_t keep = l2_evict_last(), stream = l2_evict_first();  // B/C reread, x once
-    // x of block jj (both heads) into L2, a block ahead: its load into shared memory waits for
-    // the previous block's state MMA, and then hits L2 (two blocks ahead measured slower, three
-    // slower still)
-    auto prefetch_x = [&](int jj) {
-      int acc = 0;
-      for (int i = 0; i < nit; ++i) {
-        const int len = items_sh[i].k1 - items_sh[i].k0;
-        if (jj < acc + len) {
-          const int pb = items_sh[i].seq / pl.npair, ph = (items_sh[i].seq % pl.npair) * 2;
-          const int pt = (items_sh[i].k0 + jj - acc) * kBlk;
-          tma_prefetch_3d(&tm_x, ph * kP, pt, pb);
-          tma_prefetch_3d(&tm_x, (ph + 1) * kP, pt, pb);
-          return;
-        }
-        acc += len;
-      }
-    };
-    constexpr int kAhead = 1;
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_b);
@@ -843,7 +826,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1) scan_walk_kernel(
       const float al[2] = {A[h0] * kLog2e, A[h0 + 1] * kLog2e};
       for (int k = w.k0; k < w.k1; ++k, ++j) {
         const int t0 = k * kBlk;
-        if (lane == 0) prefetch_x(j + kAhead);
         // B of block j into slot j % 2 once block j - 2's G and state MMAs are done
         if (j >= 2 && !wait_all(&bars.b_empty[j & 1], ((j - 2) >> 1) & 1, 33)) {
           ok = false;

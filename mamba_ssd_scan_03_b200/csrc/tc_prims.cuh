@@ -141,15 +141,6 @@ __device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, const 
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
-// Tiled prefetch of a box into L2 (no shared memory, no completion): issued a few blocks ahead so
-// that the later tile load into shared memory hits L2.
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
 // Wait until at most one committed bulk store group has not finished reading its source.
 __device__ __forceinline__ void bulk_wait_read_1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");

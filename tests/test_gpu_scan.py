@@ -204,6 +204,19 @@ def test_slow_decay_stress():
     assert rel_err(to_np(y) - xd, yo) <= 4e-2
 
 
+def test_fast_decay_mix():
+    """Heads whose decay per token ranges from mild to extreme (|A| log-uniform in [0.5, 300]):
+    within one call, 16-token groups whose own decay spans less than 2^-64 sit beside groups that
+    decay past 2^-128, where the mask's exponentials leave the float range unless each is taken
+    over a span that stays in it."""
+    inp = small(seed=23, batch=1, seqlen=512, nheads=8, A_range=(0.5, 300.0))
+    dt, A = inp["dt"].astype(np.float64), inp["A"].astype(np.float64)
+    span = -(dt * A[None, None, :]).reshape(1, -1, 16, 8).sum(axis=2) / math.log(2.0)
+    assert (span < 64).any() and (span > 128).any()  # both kinds of group occur
+    y, fin = run(inp, dev_inputs(inp))
+    check_full(inp, y, fin)
+
+
 def test_initial_state_only():
     """x = 0 with a nonzero initial state: only the state-passing / off-diagonal path acts."""
     inp = small(seed=12, batch=2, seqlen=640, nheads=4)

@@ -206,9 +206,9 @@ def test_slow_decay_stress():
 
 def test_fast_decay_mix():
     """Heads whose decay per token ranges from mild to extreme (|A| log-uniform in [0.5, 300]):
-    within one call, 16-token groups whose own decay spans less than 2^-64 sit beside groups that
-    decay past 2^-128, where the mask's exponentials leave the float range unless each is taken
-    over a span that stays in it."""
+    within one call, 16-token groups that decay by less than a factor 2^64 sit beside groups that
+    decay by more than 2^128, where an exponential taken across the group leaves the float
+    range, so the mask must take each one over the span between its own two tokens."""
     inp = small(seed=23, batch=1, seqlen=512, nheads=8, A_range=(0.5, 300.0))
     dt, A = inp["dt"].astype(np.float64), inp["A"].astype(np.float64)
     span = -(dt * A[None, None, :]).reshape(1, -1, 16, 8).sum(axis=2) / math.log(2.0)

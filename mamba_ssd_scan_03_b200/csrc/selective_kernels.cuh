@@ -10,11 +10,13 @@
 // Unlike the scalar-transition layer there is no matrix form to put on the tensor cores: every
 // (token, channel, state) needs its own exp, so the kernel is bound by the SFU's ex2 rate.
 //
-// Layout of the work: a CTA of WPC warps per batch row and 8 x WPC channels of one group (up to
-// four warps, which share the group's B and C tiles); in a warp, four lanes per channel, each
-// lane holding 4 of the 16 states in registers for the whole sequence.  The inputs arrive as
-// TMA tiles of 32 tokens ({8 WPC channels} of x and dt, {16 states} of B and C) in a two-stage
-// ring, so the loads cost the SM no per-row cache lookups.  Rows past the end of the sequence
+// Layout of the work: a CTA of one warp per batch row and 8 channels; four lanes per channel,
+// each lane holding 4 of the 16 states in registers for the whole sequence.  One warp per CTA
+// makes the most CTAs (2,560 at 4 x 5,120 channels: 17.3 per SM, so no SM holds much more than
+// its share of a grid that runs in one wave); four warps sharing the group's B and C tiles
+// measured 8% slower, as 640 CTAs put five on some SMs and four on most.  The inputs arrive as
+// TMA tiles of 32 tokens ({8 channels} of x and dt, {16 states} of B and C) in a two-stage ring,
+// so the loads cost the SM no per-row cache lookups.  Rows past the end of the sequence
 // are zero-filled by the TMA unit: dt = 0 makes them exact identity steps (decay 1, no input).
 // Per token a lane updates its four states with packed float32 pairs; every four tokens the four
 // lanes of a channel reduce-scatter their partial y sums (three shuffles), so that each lane
@@ -29,14 +31,14 @@ namespace ssd {
 namespace sel {
 
 constexpr int kTok = 32;    // tokens per tile
-constexpr int kCpw = 8;     // channels per warp
+constexpr int kCpw = 8;     // channels per CTA (one warp)
 constexpr int kN = 16;      // states per channel
 constexpr int kSpl = 4;     // states per lane
 constexpr int kStages = 2;  // input tiles in flight
 
-template <typename T, typename TY, int WPC>
+template <typename T, typename TY>
 struct Smem {
-  static constexpr int kCw = kCpw * WPC;                     // channels per CTA
+  static constexpr int kCw = kCpw;                           // channels per CTA
   static constexpr int kX = kTok * kCw * int(sizeof(T));    // x tile   [32][kCw]
   static constexpr int kDt = kTok * kCw * 4;                // dt tile  [32][kCw] float32
   static constexpr int kBC = kTok * kN * int(sizeof(T));    // B, C tiles [32][16]
@@ -76,17 +78,17 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (tc::globaltimer() - t0 > 1000000000ull) return;
 }
 
-// Preconditions (checked on the host): dstate == 16, (dim / ngroups) % (8 WPC) == 0, 16-byte
-// aligned pointers; the tensor maps are 3-D {inner, seqlen, batch} with boxes {8 WPC, 32, 1}
-// (x, dt, y) and {16, 32, 1} (B, C), no swizzle, zero fill.
-template <typename T, typename TY, int WPC>
-__global__ void __launch_bounds__(32 * WPC) selective_scan_kernel(
+// Preconditions (checked on the host): dstate == 16, (dim / ngroups) % 8 == 0, 16-byte aligned
+// pointers; the tensor maps are 3-D {inner, seqlen, batch} with boxes {8, 32, 1} (x, dt, y) and
+// {16, 32, 1} (B, C), no swizzle, zero fill.
+template <typename T, typename TY>
+__global__ void __launch_bounds__(32) selective_scan_kernel(
     const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mdt,
     const __grid_constant__ CUtensorMap mb, const __grid_constant__ CUtensorMap mc,
     const __grid_constant__ CUtensorMap my, const float* __restrict__ A,
     const float* __restrict__ D, const float* __restrict__ init, float* __restrict__ fin,
     int64_t seqlen, int dim, int ngroups) {
-  using S = Smem<T, TY, WPC>;
+  using S = Smem<T, TY>;
   constexpr int CW = S::kCw;
   extern __shared__ uint8_t smraw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 127) &
@@ -94,9 +96,9 @@ __global__ void __launch_bounds__(32 * WPC) selective_scan_kernel(
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + S::kBars);
   __shared__ int abort_flag;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = lane >> 2, q = lane & 3;  // channel within the warp, state quarter
-  const int cw = warp * kCpw + c;         // channel within the CTA's tiles
+  const int tid = threadIdx.x, lane = tid;
+  const int c = lane >> 2, q = lane & 3;  // channel within the CTA, state quarter
+  const int cw = c;                       // channel within the CTA's tiles
   const int cpr = dim / CW;               // CTAs per batch row
   const int b = int(blockIdx.x / cpr);
   const int d0 = int(blockIdx.x % cpr) * CW;

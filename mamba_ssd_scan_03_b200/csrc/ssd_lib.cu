@@ -326,12 +326,9 @@ ssd_status set_smem_attrs() {
           cudaSuccess;
     // the selective scan runs many small CTAs per SM: ask for the largest shared-memory
     // carve-out so that shared memory does not cap them
-#define SSD_SEL_FNS(W)                                                                     \
-  (const void*)ssd::sel::selective_scan_kernel<float, float, W>,                           \
-      (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, float, W>,               \
-      (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, __nv_bfloat16, W>
-    for (auto f : {SSD_SEL_FNS(1), SSD_SEL_FNS(2), SSD_SEL_FNS(4)})
-#undef SSD_SEL_FNS
+    for (auto f : {(const void*)ssd::sel::selective_scan_kernel<float, float>,
+                   (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, float>,
+                   (const void*)ssd::sel::selective_scan_kernel<__nv_bfloat16, __nv_bfloat16>})
       ok &= cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  int(cudaSharedmemCarveoutMaxShared)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(ssd::tc::seg_state_kernel<2>,
@@ -1056,10 +1053,7 @@ ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A
   namespace sel = ssd::sel;
   if (dstate != sel::kN || dim % sel::kCpw != 0 || (dim / ngroups) % sel::kCpw != 0)
     return SSD_ERR_UNSUPPORTED;
-  // warps per CTA: the most (up to four) whose 8-channel slices stay inside one group
-  const int cpg = dim / ngroups;
-  const int wpc = cpg % (4 * sel::kCpw) == 0 ? 4 : (cpg % (2 * sel::kCpw) == 0 ? 2 : 1);
-  const int cw = wpc * sel::kCpw;
+  const int cw = sel::kCpw;  // channels per CTA (one warp)
   for (const void* p : {x, (const void*)dt, (const void*)A, B, C, (const void*)y,
                         (const void*)init_state, (const void*)final_state})
     if (p && !aligned16(p)) return SSD_ERR_UNSUPPORTED;
@@ -1082,19 +1076,12 @@ ssd_status ssd_selective_scan_fwd(const void* x, const float* dt, const float* A
     return SSD_ERR_CUDA;
   if (set_smem_attrs() != SSD_OK) return SSD_ERR_CUDA;
   const unsigned grid = unsigned(ctas);
-#define SSD_SEL(T, TY, W)                                                                   \
-  sel::selective_scan_kernel<T, TY, W><<<grid, 32 * W, sel::Smem<T, TY, W>::kBytes, stream>>>( \
+#define SSD_SEL(T, TY)                                                                  \
+  sel::selective_scan_kernel<T, TY><<<grid, 32, sel::Smem<T, TY>::kBytes, stream>>>(       \
       mx, mdt, mb, mc, my, A, D, init_state, final_state, seqlen, dim, ngroups)
-#define SSD_SEL_W(T, TY)                 \
-  do {                                   \
-    if (wpc == 4) SSD_SEL(T, TY, 4);     \
-    else if (wpc == 2) SSD_SEL(T, TY, 2); \
-    else SSD_SEL(T, TY, 1);              \
-  } while (0)
-  if (!bf) SSD_SEL_W(float, float);
-  else if (!ybf) SSD_SEL_W(__nv_bfloat16, float);
-  else SSD_SEL_W(__nv_bfloat16, __nv_bfloat16);
-#undef SSD_SEL_W
+  if (!bf) SSD_SEL(float, float);
+  else if (!ybf) SSD_SEL(__nv_bfloat16, float);
+  else SSD_SEL(__nv_bfloat16, __nv_bfloat16);
 #undef SSD_SEL
   return launched();
 }

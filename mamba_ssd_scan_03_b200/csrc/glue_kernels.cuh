@@ -55,7 +55,7 @@ __device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.f +
 constexpr int kConvTok = 64, kConvStep = 4;
 
 template <typename T, int K>
-__global__ void __launch_bounds__(128) conv_silu_kernel(const T* __restrict__ u,
+__global__ void __launch_bounds__(32) conv_silu_kernel(const T* __restrict__ u,
                                                         const float* __restrict__ w,
                                                         const float* __restrict__ bias,
                                                         T* __restrict__ out, int64_t seqlen,

@@ -953,9 +953,11 @@ ssd_status ssd_conv_silu(const void* u, const float* w, const float* bias, void*
     return SSD_ERR_UNSUPPORTED;
   const int64_t runs = (seqlen + ssd::glue::kConvTok - 1) / ssd::glue::kConvTok;
   if (runs > 65535 || batch > 65535) return SSD_ERR_UNSUPPORTED;
-  const dim3 grid(unsigned((cdim / vw + 127) / 128), unsigned(runs), unsigned(batch));
+  // one warp per block: the finest split of the grid over the SMs (blocks of 96 and 128 threads
+  // measured 4% and 7% slower at the 2.7B shape)
+  const dim3 grid(unsigned((cdim / vw + 31) / 32), unsigned(runs), unsigned(batch));
 #define SSD_CONV(T, KW)                                                                    \
-  ssd::glue::conv_silu_kernel<T, KW><<<grid, 128, 0, stream>>>(                            \
+  ssd::glue::conv_silu_kernel<T, KW><<<grid, 32, 0, stream>>>(                            \
       static_cast<const T*>(u), w, bias, static_cast<T*>(out), seqlen, cdim)
 #define SSD_CONV_K(T)                                                                      \
   switch (kwidth) {                                                                        \

@@ -111,7 +111,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 // L2 cache policies for TMA copies: evict_last for tiles that other CTAs read again (B, C: a few
-// MB in all), evict_first for data streamed once (x after its prefetch, y).
+// MB in all), evict_first for data streamed once (x, y).
 __device__ __forceinline__ uint64_t l2_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));

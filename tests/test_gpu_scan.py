@@ -60,6 +60,7 @@ def test_tiny_f32_workload():
     dict(batch=1, seqlen=128, nheads=2),
     dict(batch=2, seqlen=300, nheads=4),
     dict(batch=1, seqlen=1000, nheads=8, ngroups=2),
+    dict(batch=2, seqlen=640, nheads=8, ngroups=4),  # one group per head pair
     dict(batch=3, seqlen=777, nheads=6, init="zeros"),
     dict(batch=2, seqlen=1, nheads=2),
     dict(batch=1, seqlen=4500, nheads=4),     # several segments per sequence

@@ -244,6 +244,26 @@ def device_scan_inputs(c, dev, seed):
     return t
 
 
+def timed_after_flush(once, flush, steps):
+    """Device time of `steps` calls of once(), each right behind an L2 flush (a write of
+    `flush`), timed with CUDA events.  Every step is queued before the first is waited for, so
+    the device runs flush, call, flush, call ... back to back and the host's time to validate
+    and launch a call (which a small call does not hide) is not counted; eight more flushes
+    ahead of the first give the host its lead."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for _ in range(8):
+        flush.zero_()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record()
+        once()
+        e1.record()
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in evs]
+
+
 def time_scan(c, dev, seed, y_dtype, steps, warmup, hbm):
     """Mean time of one ssd_chunk_scan_fwd over a device-seeded workload, each call timed alone
     with CUDA events after an L2 flush (a 256 MB write), and its roofline figures."""
@@ -264,15 +284,7 @@ def time_scan(c, dev, seed, y_dtype, steps, warmup, hbm):
 
     for _ in range(warmup):
         once()
-    times = []
-    for _ in range(steps):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        once()
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
+    times = timed_after_flush(once, flush, steps)
     assert ssd.device_status() == 0
     ms = statistics.mean(times)
     nbytes = scan_bytes(c, 2 if y_dtype == torch.bfloat16 else 4)
@@ -309,15 +321,7 @@ def time_backward(c, dev, seed, steps, warmup, hbm):
 
     for _ in range(warmup):
         once()
-    times = []
-    for _ in range(steps):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        once()
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
+    times = timed_after_flush(once, flush, steps)
     assert ssd.device_status() == 0
     ms = statistics.mean(times)
     tok = c["batch"] * c["seqlen"]
